@@ -1,0 +1,341 @@
+"""Throughput of the batched RLT transition engine on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of synthetic
+sequences: reset to H_0, encode the prompt (causal encoder + memory), the
+recurrent prefill (one transition per position per row), then -- for
+workloads with a decode phase -- sampled generation (readout, sample, encode
+the token, one transition), and the final readout.  Inputs are resident on
+the device when the timed region starts.  The metric is transitions per
+second: rows x positions processed, summed over ranks.
+
+With N > 1 (torchrun) every rank runs its own shard of rows (the same
+per-GPU batch: weak scaling); there is no collective on the data path, only
+the barrier and the max-over-ranks reduction of the timing.
+
+--impl reference times the CPU oracle (test infrastructure, float64 numpy)
+on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import rlt_inputs as ri  # noqa: E402
+
+METRIC = "decoder transition tokens/s (batch x steps) at 1 B200"
+DEFAULT_CONFIG = "parity_bf16"
+
+
+def peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+            "fallback"
+
+
+def workload_desc(cfg) -> dict:
+    kind = {0: "RLT-0", 1: "RLT-1", 2: f"RLT-2 (feedback chunk {cfg.chunk})"}[cfg.variant]
+    dt = "bf16" if cfg.dtype == ri.DT_BF16 else "fp32"
+    return {
+        "workload": f"{cfg.name}: {kind} {dt}, vocab {cfg.vocab}, d={cfg.d}, {cfg.heads} heads, "
+                    f"{cfg.n_enc}+{cfg.n_dec} layers{' tied' if cfg.tied else ''}, W={cfg.window}, "
+                    f"G={cfg.groups}, {cfg.token_recipe} tokens, random N(0,0.02) weights",
+        "batch_per_gpu": cfg.batch, "prompt": cfg.prompt, "decode": cfg.decode,
+    }
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle leg
+# ----------------------------------------------------------------------------
+def oracle_sample(cfg, budget_s: float = 15.0):
+    """Time the oracle (float64, as it stands) on rows of the workload until the
+    budget is spent; returns (tokens/s, description, threads)."""
+    from oracle import RLTOracle
+    try:
+        import threadpoolctl
+        threads = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()) \
+            if threadpoolctl.threadpool_info() else 1
+    except Exception:
+        threads = os.cpu_count() or 1
+    W = ri.generate_weights(cfg)
+    orc = RLTOracle(cfg, W, "fp64")
+    T = min(cfg.prompt, 256)
+    done_tok, rows, t0 = 0, 0, time.perf_counter()
+    while True:
+        toks = ri.make_tokens(cfg, 1, T, row0=rows)[0]
+        st = orc.new_state()
+        orc.encode(st, toks)
+        for _ in range(T):
+            orc.transition(st)
+            done_tok += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        orc.readout(st)
+        rows += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    desc = (f"{rows} row(s) of the same workload, prompt {T}: encode + {done_tok} transitions "
+            f"+ readout, float64 numpy oracle, {dt:.1f} s")
+    return done_tok / dt, desc, threads
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    vals = []
+    for _ in range(args.warmup):
+        oracle_sample(cfg, budget_s=2.0)
+    for _ in range(args.steps):
+        v, desc, threads = oracle_sample(cfg, budget_s=max(5.0, 60.0 / max(1, args.steps)))
+        vals.append(v)
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_desc(cfg),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.device = device
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.device}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from tests.conftest import build_library
+    if rank == 0 or world == 1:
+        build_library()
+    if world > 1:
+        dist.barrier()
+    import stateful_decoding_b200 as sd
+
+    B, T, D = cfg.batch, cfg.prompt, cfg.decode
+    W = ri.generate_weights(cfg)
+    model = sd.Model(ri.write_blob(cfg, W), device=local)
+    st = sd.State(model, B, T + D)
+    # each rank runs its own rows: the token substreams start at rank * B
+    toks_h = ri.make_tokens(cfg, B, T, row0=rank * B)
+    toks = torch.from_numpy(toks_h).to(dev)
+    logits = torch.empty(B, cfg.vocab, device=dev)
+    ids = torch.empty(B, dtype=torch.int32, device=dev)
+    am = torch.empty(B, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(tok_in, out_logits, out_ids, out_am):
+        st.reset(stream=stream)
+        st.encode(tok_in, stream=stream)
+        st.prefill(T, stream=stream)
+        for k in range(D):
+            st.readout(sampled=out_ids, seed=ri.SAMPLE_SEED, step=k, stream=stream)
+            st.encode(out_ids.view(B, 1) if hasattr(out_ids, "view") else out_ids.reshape(B, 1),
+                      stream=stream)
+            st.step(stream=stream)
+        st.readout(logits=out_logits, argmax=out_am, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(max(3, args.warmup)):
+        step(toks, logits, ids, am)
+    barrier()
+
+    # ---- device-resident timed region ----
+    launches0 = sd.rlt_kernel_launches()
+    st.profile(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step(toks, logits, ids, am)
+        e1.record(stream)
+        barrier()
+    ms_total = e0.elapsed_time(e1)
+    launches = sd.rlt_kernel_launches() - launches0
+    prof = {name: st.profile_query(cls, stream) for name, cls in
+            (("xattn", sd.PROF_XATTN), ("swa", sd.PROF_SWA), ("step", sd.PROF_STEP),
+             ("enc", sd.PROF_ENC))}
+    st.profile(False)
+    ms_total = max_over_ranks(ms_total)
+    ms_step = ms_total / args.steps
+    tokens_step = B * (T + D) * world
+    value = tokens_step / (ms_step / 1e3)
+
+    # ---- end to end through the C ABI with host buffers ----
+    toks_pin = torch.from_numpy(toks_h).pin_memory()
+    lg_pin = torch.empty(B, cfg.vocab, dtype=torch.float32).pin_memory()
+    am_pin = torch.empty(B, dtype=torch.int32).pin_memory()
+    ids_pin = np.zeros(B, np.int32)
+    barrier()
+    t0 = time.perf_counter()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        step(toks_pin, lg_pin, ids, am_pin)
+    f1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1)) / args.steps
+    e2e_wall = (time.perf_counter() - t0) * 1e3 / args.steps
+    h2d = B * T * 4
+    d2h = B * cfg.vocab * 4 + B * 4
+
+    pk, pk_kind = peaks()
+    dom = "xattn"
+    n, ms, by = prof[dom]
+    achieved = (by / n) / ((ms / n) / 1e3) / 1e9 if n else 0.0
+    n_s, ms_s, by_s = prof["step"]
+    step_gbs = (by_s / ms_s * 1e3 / 1e9) if ms_s else 0.0
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == ri.DT_BF16 else "f32", "data": "synthetic",
+        "config": dict(workload_desc(cfg), global_batch=B * world,
+                       parallelism=f"replicas x{world} (rows sharded, no collective)",
+                       l2="working set per step > L2: caches of all rows (see DESIGN.md)"),
+        "gpu_launches": launches,
+        "e2e": {"value": tokens_step / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms, "wall_ms_per_step": e2e_wall},
+        "roofline": {"bound": "hbm", "kernel": "decoder cross-attention (k_attn_cross)",
+                     "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                     "peak_kind": f"{pk_kind} hbm_gbs", "launches": n,
+                     "avg_launch_us": (ms / n * 1e3) if n else None,
+                     "alg_bytes_per_launch": (by / n) if n else None},
+        "breakdown": {
+            "decoder_step": {"launches": n_s, "avg_us": (ms_s / n_s * 1e3) if n_s else None,
+                             "alg_GBps": step_gbs, "frac_hbm": step_gbs / pk["hbm_gbs"]},
+            "swa": {"launches": prof["swa"][0], "ms": prof["swa"][1]},
+            "encoder_ms_per_step": prof["enc"][1] / args.steps,
+            "decoder_ms_per_step": ms_s / args.steps,
+        },
+    }
+    clk_s = clk.summary()
+    if clk_s:
+        line["clocks"] = clk_s
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, threads = oracle_sample(cfg, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line))
+    st.close()
+    model.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(ri.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = ri.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

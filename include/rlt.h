@@ -1,0 +1,174 @@
+/*
+ * rlt.h -- C ABI of the RLT transition engine (librlt.so, sm_100a).
+ *
+ * The Recurrent Looped Transformer carries a full decoder state
+ * H_t = (s_t, C^D_t) -- the last decoder output and one sliding-window
+ * key/value cache per decoder layer -- across every token, prompt and
+ * response alike, and reads a prefix-restricted memory built by a causal
+ * encoder (jiphyeonjeon.kr review "Recurrent Looped Transformer", §2-§3;
+ * greeksharifa.github.io "Recurrent Looped Transformer 요약 설명", §2.1-§2.7).
+ * This library runs that transition for a batch of independent sequences
+ * ("rows") on one GPU.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Return value: RLT_OK (0) on success, a negative RLT_E_* code otherwise.
+ *   Nothing traps; device-side failures (a bounded wait that gave up) set a
+ *   sticky per-state error word that rlt_state_check() reports.
+ * - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Calls are stream-ordered and asynchronous unless stated.
+ * - Ownership: models and states are library-owned and freed by their
+ *   destroy call.  Caller buffers (tokens, logits, ids) stay caller-owned; the
+ *   library never frees or retains them past the call's stream work.
+ * - Host or device pointers: every caller buffer may be host memory (pageable
+ *   or pinned) or device memory of the state's device; the library checks with
+ *   cudaPointerGetAttributes and stages host buffers through its own device
+ *   copies on `stream`.  Host outputs are valid after `stream` synchronises.
+ * - Rows are independent: row r's results do not depend on the batch size or
+ *   on other rows' tokens, bit for bit (greeksharifa App. C.1, batching
+ *   independent sequences).
+ * - Positions are 1-based; BOS is position 1 (greeksharifa App. I).
+ */
+#ifndef RLT_H
+#define RLT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RLT_OK             0
+#define RLT_E_ARG         -1  /* bad argument (null pointer, size, row index)            */
+#define RLT_E_OOM         -2  /* device or host allocation failed                         */
+#define RLT_E_CAPACITY    -3  /* a row's position would exceed the state's max_len        */
+#define RLT_E_ORDER       -4  /* transition without an encoded token (pos_dec >= pos_enc) */
+#define RLT_E_BLOB        -5  /* weight blob: bad magic, version, manifest or checksum    */
+#define RLT_E_DEVICE      -6  /* a CUDA call failed (no device, launch error, fault)      */
+#define RLT_E_TIMEOUT     -7  /* a bounded device wait gave up                            */
+#define RLT_E_UNSUPPORTED -8  /* configuration this build does not run                    */
+
+#define RLT_DTYPE_F32  0
+#define RLT_DTYPE_BF16 1
+
+typedef struct rlt_model rlt_model;  /* weights on one device + config              */
+typedef struct rlt_state rlt_state;  /* s, R, C^D rings, C^E, memory, e, positions   */
+
+/* Model hyper-parameters as stored in the blob header. */
+typedef struct rlt_config {
+    int32_t vocab, d, heads, n_enc, n_dec, ffn, window, groups, chunk, variant, tied, dtype;
+    double alpha, eps, rope_base;
+} rlt_config;
+
+/* Load a weight blob (host memory, copied; the caller may free it on return)
+ * onto `device`.  Blob = 256-byte header (magic "RLTB", version 1, the
+ * rlt_config fields, seed, tensor count, payload size, checksum) followed by
+ * named tensor records in the fixed manifest order of the config.  Errors:
+ * RLT_E_BLOB (bad magic/version/manifest/checksum), RLT_E_UNSUPPORTED (head
+ * size or shape this build does not run), RLT_E_DEVICE, RLT_E_OOM. */
+int rlt_create(const void* blob, size_t nbytes, int device, rlt_model** out);
+void rlt_destroy(rlt_model* model);
+int rlt_model_config(const rlt_model* model, rlt_config* out);
+
+/* Allocate the per-row state for `batch` rows of up to `max_len` positions:
+ * encoder cache C^E [L_E][2][h][max_len][d_h], memory M [G][2][h][max_len][d_h],
+ * window rings C^D [L_D][2][h][W-1][d_h] (all in the model dtype), e_t
+ * [max_len][d] fp32, s and R [d] fp32 -- the storage bound of the paper's
+ * eq. 3.3 (jiphyeonjeon review §4.2) -- plus scratch for one call.  The
+ * state starts reset (H_0).  Library-owned. */
+int rlt_state_create(rlt_model* model, int batch, int max_len, rlt_state** out);
+void rlt_state_destroy(rlt_state* state);
+
+/* Bytes of the per-row state proper (eq. 3.3 terms) and of everything the
+ * state allocated on the device (state + scratch). */
+int rlt_state_bytes(const rlt_state* state, size_t* per_row_state, size_t* total_device);
+
+/* H_0 = (s_star, empty) for `n` rows listed in host array `rows` (NULL = all
+ * rows): s = R = s_star, caches emptied, positions 0 (jiphyeonjeon review §3.1;
+ * per-document reset, §6.1). */
+int rlt_state_reset(rlt_state* state, const int32_t* rows, int n, void* stream);
+
+/* Encode `n` tokens per row (tokens: int32 [batch][n], host or device) at
+ * positions pos_enc+1..pos_enc+n: appends e_t, C^E and the memory entries
+ * k^g_t = RoPE_t(W^g_K RMSNorm_E(e_t)), v^g_t = W^g_V RMSNorm_E(e_t)
+ * (jiphyeonjeon review §2, eq. 2.1-2.2).  Splitting a prompt over several
+ * calls gives the same result as one call (§3.2).  RLT_E_CAPACITY if a row
+ * would pass max_len; RLT_E_ARG if a token id is outside [0, vocab) when the
+ * tokens are on the host. */
+int rlt_encode(rlt_state* state, const int32_t* tokens, int n, void* stream);
+
+/* One transition per row at t = pos_dec+1: u_t = Merge(e_t, s_{t-1})
+ * (RLT-2: the register R; RLT-0: u_t = e_t), then L_D decoder blocks
+ * (window self-attention over C^D, cross-attention to M_{<=t}, FFN), giving
+ * H_t (greeksharifa §2.3-§2.5; jiphyeonjeon review §3).  RLT_E_ORDER if a row
+ * has no encoded token at t. */
+int rlt_step(rlt_state* state, void* stream);
+
+/* T transitions per row, the recurrent prefill (jiphyeonjeon review §3.2;
+ * greeksharifa App. F.1).  RLT-1 runs T sequential steps; RLT-2 runs the
+ * positions of each chunk together (ceil(T/B) sequential passes when rows
+ * start chunk-aligned, greeksharifa App. I.2); RLT-0 runs blocks of positions
+ * together.  Same results as T calls of rlt_step. */
+int rlt_prefill(rlt_state* state, int T, void* stream);
+
+/* Readout of every row's current s_t: logits = W_out RMSNorm_out(s_t)
+ * (greeksharifa §2.3).  Each output may be NULL.  logits: fp32 [batch][vocab];
+ * argmax: int32 [batch], lowest index among equal maxima; sampled: int32
+ * [batch], first index i with sum_{j<=i} softmax(logits/temperature)_j > u,
+ * u = the SplitMix64 uniform of (rng_seed, row, rng_step):
+ *   key = mix64(rng_seed ^ mix64((row+1)*G)), u = top53(mix64(key + (rng_step+1)*G))
+ * with G = 0x9E3779B97F4A7C15 and mix64 the SplitMix64 finaliser.  No top-k/p
+ * truncation (jiphyeonjeon review §6.2).  temperature > 0. */
+int rlt_readout(rlt_state* state, float* logits, int32_t* argmax, int32_t* sampled,
+                uint64_t rng_seed, uint64_t rng_step, float temperature, void* stream);
+
+/* Host copies of the per-row positions (arrays of `batch` int32; either may
+ * be NULL).  pos_enc = tokens encoded, pos_dec = transitions applied. */
+int rlt_state_positions(const rlt_state* state, int32_t* pos_enc, int32_t* pos_dec);
+
+/* Copy one state component to `dst` (host or device), `nbytes` exactly its
+ * size (query with dst = NULL: *nbytes_out receives the size).  Components:
+ * RLT_PART_S / _R: fp32 [batch][d]; _E: fp32 [batch][max_len][d];
+ * _MEM: model dtype [batch][G][2][h][max_len][d_h]; _RING: model dtype
+ * [batch][L_D][2][h][W-1][d_h]; _ENC: model dtype [batch][L_E][2][h][max_len][d_h].
+ * Synchronises `stream` when dst is host memory. */
+#define RLT_PART_S    0
+#define RLT_PART_R    1
+#define RLT_PART_E    2
+#define RLT_PART_MEM  3
+#define RLT_PART_RING 4
+#define RLT_PART_ENC  5
+int rlt_state_read(rlt_state* state, int part, void* dst, size_t nbytes, size_t* nbytes_out,
+                   void* stream);
+
+/* Synchronise `stream` and report the state's sticky device error word
+ * (RLT_OK, RLT_E_TIMEOUT, ...), clearing it. */
+int rlt_state_check(rlt_state* state, void* stream);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t rlt_kernel_launches(void);
+
+/* Live kernel timing for measurement.  While enabled (on != 0), the library
+ * brackets every launch of the classes below with CUDA events recorded on the
+ * launching stream and counts the algorithmic bytes each launch must move
+ * (keys/values read, cache entries written, activations in and out; weights
+ * excluded).  rlt_profile_query synchronises `stream`, sums the elapsed times
+ * of the class since the last enable, and reports launches, total ms and
+ * bytes.  Enabling resets the counters. */
+#define RLT_PROF_XATTN 0  /* decoder cross-attention over M_{<=t}        */
+#define RLT_PROF_SWA   1  /* decoder window attention over C^D           */
+#define RLT_PROF_STEP  2  /* one whole transition block (merge .. s_t)   */
+#define RLT_PROF_ENC   3  /* one whole encoder block (embed .. memory)   */
+#define RLT_PROF_NCLS  4
+int rlt_profile_enable(rlt_state* state, int on);
+int rlt_profile_query(rlt_state* state, int cls, uint64_t* launches, double* total_ms,
+                      double* bytes, void* stream);
+
+/* Static description of a return code. */
+const char* rlt_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RLT_H */

@@ -1,0 +1,289 @@
+"""Python binding of librlt.so: argument marshalling only.
+
+Every function named ``rlt_*`` here forwards to the C function of the same
+name in ``include/rlt.h``; buffers may be torch tensors (host or CUDA),
+numpy arrays or raw integer addresses, and streams torch.cuda.Stream objects,
+raw handles or None (legacy default stream).  All computation runs in the
+library's CUDA kernels; there is no fallback: if librlt.so is missing or does
+not load, importing this package raises.
+
+``Model`` and ``State`` are small owners that call the same functions.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librlt.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "rlt.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"librlt.so not built at {LIB_PATH}; run `python -m stateful_decoding_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+RLT_OK, RLT_E_ARG, RLT_E_OOM, RLT_E_CAPACITY, RLT_E_ORDER = 0, -1, -2, -3, -4
+RLT_E_BLOB, RLT_E_DEVICE, RLT_E_TIMEOUT, RLT_E_UNSUPPORTED = -5, -6, -7, -8
+PART_S, PART_R, PART_E, PART_MEM, PART_RING, PART_ENC = range(6)
+PROF_XATTN, PROF_SWA, PROF_STEP, PROF_ENC = range(4)
+
+
+class rlt_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("vocab", "d", "heads", "n_enc", "n_dec", "ffn",
+                                               "window", "groups", "chunk", "variant", "tied",
+                                               "dtype")] + \
+               [("alpha", ctypes.c_double), ("eps", ctypes.c_double), ("rope_base", ctypes.c_double)]
+
+
+_vp, _i, _sz, _u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
+_SIGS = {
+    "rlt_create": (_i, [_vp, _sz, _i, ctypes.POINTER(_vp)]),
+    "rlt_destroy": (None, [_vp]),
+    "rlt_model_config": (_i, [_vp, ctypes.POINTER(rlt_config)]),
+    "rlt_state_create": (_i, [_vp, _i, _i, ctypes.POINTER(_vp)]),
+    "rlt_state_destroy": (None, [_vp]),
+    "rlt_state_bytes": (_i, [_vp, ctypes.POINTER(_sz), ctypes.POINTER(_sz)]),
+    "rlt_state_reset": (_i, [_vp, _vp, _i, _vp]),
+    "rlt_encode": (_i, [_vp, _vp, _i, _vp]),
+    "rlt_step": (_i, [_vp, _vp]),
+    "rlt_prefill": (_i, [_vp, _i, _vp]),
+    "rlt_readout": (_i, [_vp, _vp, _vp, _vp, _u64, _u64, ctypes.c_float, _vp]),
+    "rlt_state_positions": (_i, [_vp, _vp, _vp]),
+    "rlt_state_read": (_i, [_vp, _i, _vp, _sz, ctypes.POINTER(_sz), _vp]),
+    "rlt_state_check": (_i, [_vp, _vp]),
+    "rlt_kernel_launches": (_u64, []),
+    "rlt_strerror": (ctypes.c_char_p, [_i]),
+    "rlt_profile_enable": (_i, [_vp, _i]),
+    "rlt_profile_query": (_i, [_vp, _i, ctypes.POINTER(_u64), ctypes.POINTER(ctypes.c_double),
+                               ctypes.POINTER(ctypes.c_double), _vp]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype, _f.argtypes = _res, _args
+
+
+def header_functions() -> list:
+    """Names of the functions include/rlt.h declares."""
+    src = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"\b(rlt_[a-z_]+)\s*\(", src)))
+
+
+class RLTError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {rlt_strerror(code)} ({code})")
+        self.code = code
+
+
+def _check(code: int, what: str) -> int:
+    if code != RLT_OK:
+        raise RLTError(code, what)
+    return code
+
+
+def _ptr(x) -> Optional[int]:
+    """Address of a buffer: torch tensor, numpy array, int, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        if not x.is_contiguous():
+            raise ValueError("buffer must be contiguous")
+        return x.data_ptr()
+    if hasattr(x, "ctypes"):
+        if not x.flags["C_CONTIGUOUS"]:
+            raise ValueError("buffer must be C-contiguous")
+        return x.ctypes.data
+    raise TypeError(f"cannot take the address of {type(x)}")
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+# ---------------------------------------------------------------- C names
+def rlt_strerror(code: int) -> str:
+    return _lib.rlt_strerror(code).decode()
+
+
+def rlt_kernel_launches() -> int:
+    return int(_lib.rlt_kernel_launches())
+
+
+def rlt_create(blob: bytes, device: int = 0):
+    h = _vp()
+    buf = ctypes.create_string_buffer(blob, len(blob))
+    code = _lib.rlt_create(buf, len(blob), device, ctypes.byref(h))
+    return code, h.value
+
+
+def rlt_destroy(model) -> None:
+    _lib.rlt_destroy(model)
+
+
+def rlt_model_config(model):
+    c = rlt_config()
+    return _lib.rlt_model_config(model, ctypes.byref(c)), c
+
+
+def rlt_state_create(model, batch: int, max_len: int):
+    h = _vp()
+    code = _lib.rlt_state_create(model, batch, max_len, ctypes.byref(h))
+    return code, h.value
+
+
+def rlt_state_destroy(state) -> None:
+    _lib.rlt_state_destroy(state)
+
+
+def rlt_state_bytes(state):
+    a, b = _sz(), _sz()
+    return _lib.rlt_state_bytes(state, ctypes.byref(a), ctypes.byref(b)), a.value, b.value
+
+
+def rlt_state_reset(state, rows=None, n: int = 0, stream=None) -> int:
+    return _lib.rlt_state_reset(state, _ptr(rows), n, _stream(stream))
+
+
+def rlt_encode(state, tokens, n: int, stream=None) -> int:
+    return _lib.rlt_encode(state, _ptr(tokens), n, _stream(stream))
+
+
+def rlt_step(state, stream=None) -> int:
+    return _lib.rlt_step(state, _stream(stream))
+
+
+def rlt_prefill(state, T: int, stream=None) -> int:
+    return _lib.rlt_prefill(state, T, _stream(stream))
+
+
+def rlt_readout(state, logits=None, argmax=None, sampled=None, rng_seed: int = 0,
+                rng_step: int = 0, temperature: float = 1.0, stream=None) -> int:
+    return _lib.rlt_readout(state, _ptr(logits), _ptr(argmax), _ptr(sampled), rng_seed, rng_step,
+                            temperature, _stream(stream))
+
+
+def rlt_state_positions(state, pos_enc=None, pos_dec=None) -> int:
+    return _lib.rlt_state_positions(state, _ptr(pos_enc), _ptr(pos_dec))
+
+
+def rlt_state_read(state, part: int, dst=None, nbytes: int = 0, stream=None):
+    out = _sz()
+    code = _lib.rlt_state_read(state, part, _ptr(dst), nbytes, ctypes.byref(out), _stream(stream))
+    return code, out.value
+
+
+def rlt_state_check(state, stream=None) -> int:
+    return _lib.rlt_state_check(state, _stream(stream))
+
+
+def rlt_profile_enable(state, on: bool) -> int:
+    return _lib.rlt_profile_enable(state, int(on))
+
+
+def rlt_profile_query(state, cls: int, stream=None):
+    n, ms, by = _u64(), ctypes.c_double(), ctypes.c_double()
+    code = _lib.rlt_profile_query(state, cls, ctypes.byref(n), ctypes.byref(ms), ctypes.byref(by),
+                                  _stream(stream))
+    return code, n.value, ms.value, by.value
+
+
+# ---------------------------------------------------------------- owners
+class Model:
+    def __init__(self, blob: bytes, device: int = 0):
+        code, self.handle = rlt_create(blob, device)
+        _check(code, "rlt_create")
+        code, self.config = rlt_model_config(self.handle)
+        _check(code, "rlt_model_config")
+        self.device = device
+
+    def close(self):
+        if self.handle:
+            rlt_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class State:
+    def __init__(self, model: Model, batch: int, max_len: int):
+        self.model = model
+        self.batch, self.max_len = batch, max_len
+        code, self.handle = rlt_state_create(model.handle, batch, max_len)
+        _check(code, "rlt_state_create")
+
+    def close(self):
+        if self.handle:
+            rlt_state_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def reset(self, rows: Optional[Sequence[int]] = None, stream=None):
+        if rows is None:
+            return _check(rlt_state_reset(self.handle, None, 0, stream), "rlt_state_reset")
+        import numpy as np
+        r = np.ascontiguousarray(rows, dtype=np.int32)
+        return _check(rlt_state_reset(self.handle, r, len(r), stream), "rlt_state_reset")
+
+    def encode(self, tokens, stream=None):
+        n = tokens.shape[1]
+        return _check(rlt_encode(self.handle, tokens, n, stream), "rlt_encode")
+
+    def step(self, stream=None):
+        return _check(rlt_step(self.handle, stream), "rlt_step")
+
+    def prefill(self, T: int, stream=None):
+        return _check(rlt_prefill(self.handle, T, stream), "rlt_prefill")
+
+    def readout(self, logits=None, argmax=None, sampled=None, seed=0, step=0, temperature=1.0,
+                stream=None):
+        return _check(rlt_readout(self.handle, logits, argmax, sampled, seed, step, temperature,
+                                  stream), "rlt_readout")
+
+    def positions(self):
+        import numpy as np
+        pe = np.zeros(self.batch, np.int32)
+        pd = np.zeros(self.batch, np.int32)
+        _check(rlt_state_positions(self.handle, pe, pd), "rlt_state_positions")
+        return pe, pd
+
+    def read(self, part: int, stream=None):
+        """Copy a state component to a new host numpy array (raw element type)."""
+        import numpy as np
+        code, nbytes = rlt_state_read(self.handle, part)
+        _check(code, "rlt_state_read")
+        buf = np.empty(nbytes, np.uint8)
+        _check(rlt_state_read(self.handle, part, buf, nbytes, stream)[0], "rlt_state_read")
+        return buf
+
+    def check(self, stream=None):
+        return _check(rlt_state_check(self.handle, stream), "rlt_state_check")
+
+    def profile(self, on: bool):
+        return _check(rlt_profile_enable(self.handle, on), "rlt_profile_enable")
+
+    def profile_query(self, cls: int, stream=None):
+        """(launches, total_ms, algorithmic_bytes) of a kernel class since enable."""
+        code, n, ms, by = rlt_profile_query(self.handle, cls, stream)
+        _check(code, "rlt_profile_query")
+        return n, ms, by
+
+    def bytes(self):
+        code, per_row, total = rlt_state_bytes(self.handle)
+        _check(code, "rlt_state_bytes")
+        return per_row, total

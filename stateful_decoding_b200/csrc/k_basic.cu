@@ -1,0 +1,374 @@
+// Row-wise kernels of the RLT path: embedding, RMSNorm, the merge gate
+// (greeksharifa "Recurrent Looped Transformer 요약 설명" §2.5), RoPE scatters
+// into the encoder cache / memory / window chunk, SwiGLU, state hand-off and
+// the window-cache (ring) update of jiphyeonjeon review §3.3.
+#include "kernels.cuh"
+
+namespace rlt {
+
+// ---------------------------------------------------------------- embedding
+template <typename T>
+__global__ void k_embed(const T* __restrict__ E, const int32_t* __restrict__ tok,
+                        float* __restrict__ X, int d, int vocab, int* err) {
+    int r = blockIdx.x;
+    int id = tok[r];
+    bool ok = id >= 0 && id < vocab;
+    if (!ok && threadIdx.x == 0 && err) atomicExch(err, kDevBounds);
+    for (int j = threadIdx.x; j < d; j += blockDim.x)
+        X[(size_t)r * d + j] = ok ? to_f(E[(size_t)id * d + j]) : 0.f;
+}
+template <typename T>
+void launch_embed(const T* E, const int32_t* tok, float* X, int R, int d, int vocab, int* err,
+                  cudaStream_t st) {
+    if (R <= 0) return;
+    k_embed<T><<<R, 128, 0, st>>>(E, tok, X, d, vocab, err);
+    rlt_count_launch();
+}
+
+// ---------------------------------------------------------------- RMSNorm
+// Sum of squares in a fixed order: per-thread strided partials, then a
+// butterfly within warps and a sequential pass over the warp partials.
+__device__ __forceinline__ float block_sum(float v, float* red) {
+    v = warp_sum(v);
+    int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float s = 0.f;
+        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) s += red[i];
+        red[32] = s;
+    }
+    __syncthreads();
+    float out = red[32];
+    __syncthreads();
+    return out;
+}
+
+template <typename T>
+__global__ void k_rmsnorm(const float* __restrict__ X, int ldx, const float* __restrict__ g,
+                          T* __restrict__ Y, int ldy, int d, float eps) {
+    __shared__ float red[33];
+    const float* x = X + (size_t)blockIdx.x * ldx;
+    float ss = 0.f;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) ss += x[j] * x[j];
+    ss = block_sum(ss, red);
+    float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    T* y = Y + (size_t)blockIdx.x * ldy;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) y[j] = from_f<T>(x[j] * inv * g[j]);
+}
+template <typename T>
+void launch_rmsnorm(const float* X, int ldx, const float* gain, T* Y, int ldy, int R, int d,
+                    float eps, cudaStream_t st) {
+    if (R <= 0) return;
+    k_rmsnorm<T><<<R, 128, 0, st>>>(X, ldx, gain, Y, ldy, d, eps);
+    rlt_count_launch();
+}
+
+// ---------------------------------------------------------------- merge
+template <typename T>
+__global__ void k_merge_input(const float* __restrict__ e, int T_cap,
+                              const int32_t* __restrict__ pos_dec, const float* __restrict__ fb,
+                              const float* __restrict__ g, T* __restrict__ Gin, int n, int d,
+                              float eps) {
+    __shared__ float red[33];
+    int r = blockIdx.x, b = r / n, i = r % n;
+    const float* et = e + ((size_t)b * T_cap + pos_dec[b] + i) * d;
+    const float* f = fb + (size_t)b * d;
+    float ss = 0.f;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) ss += f[j] * f[j];
+    ss = block_sum(ss, red);
+    float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    T* out = Gin + (size_t)r * 2 * d;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        out[j] = from_f<T>(et[j]);
+        out[d + j] = from_f<T>(f[j] * inv * g[j]);
+    }
+}
+template <typename T>
+void launch_merge_input(const float* e, int T_cap, const int32_t* pos_dec, const float* fb,
+                        const float* gain, T* Gin, int B, int n, int d, float eps,
+                        cudaStream_t st) {
+    k_merge_input<T><<<B * n, 128, 0, st>>>(e, T_cap, pos_dec, fb, gain, Gin, n, d, eps);
+    rlt_count_launch();
+}
+
+__global__ void k_merge_out(const float* __restrict__ e, int T_cap,
+                            const int32_t* __restrict__ pos_dec, const float* __restrict__ G,
+                            const float* __restrict__ bg, const float* __restrict__ S,
+                            float alpha, float* __restrict__ z, int n, int d) {
+    int r = blockIdx.x, b = r / n, i = r % n;
+    const float* et = e + ((size_t)b * T_cap + pos_dec[b] + i) * d;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        float u = et[j];
+        if (G) {
+            float a = G[(size_t)r * d + j] + bg[j];
+            float gate = 1.0f / (1.0f + expf(-a));
+            u += alpha * gate * S[(size_t)r * d + j];
+        }
+        z[(size_t)r * d + j] = u;
+    }
+}
+void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const float* G,
+                      const float* bg, const float* S, float alpha, float* z, int B, int n, int d,
+                      cudaStream_t st) {
+    k_merge_out<<<B * n, 128, 0, st>>>(e, T_cap, pos_dec, G, bg, S, alpha, z, n, d);
+    rlt_count_launch();
+}
+
+// ---------------------------------------------------------------- RoPE scatters
+// rotate-half: pair (j, j+half) turns by p * base^(-2j/dh)
+__device__ __forceinline__ void rot(float x1, float x2, float c, float s, float& y1, float& y2) {
+    y1 = x1 * c - x2 * s;
+    y2 = x2 * c + x1 * s;
+}
+
+template <typename T>
+__global__ void k_qkv_dec(const float* __restrict__ QKV, const int32_t* __restrict__ pos_dec,
+                          RopeTab rope, float* __restrict__ Q, T* __restrict__ Kc,
+                          T* __restrict__ Vc, int n, int heads, int dh) {
+    int r = blockIdx.x, b = r / n, i = r % n;
+    int d = heads * dh, half = dh / 2;
+    int t = pos_dec[b] + 1 + i;
+    const float* src = QKV + (size_t)r * 3 * d;
+    for (int x = threadIdx.x; x < heads * half; x += blockDim.x) {
+        int h = x / half, j = x % half;
+        float c = rope.cs[(size_t)t * half + j], s = rope.sn[(size_t)t * half + j];
+        int o1 = h * dh + j, o2 = o1 + half;
+        float y1, y2;
+        rot(src[o1], src[o2], c, s, y1, y2);
+        Q[(size_t)r * d + o1] = y1;
+        Q[(size_t)r * d + o2] = y2;
+        rot(src[d + o1], src[d + o2], c, s, y1, y2);
+        Kc[(size_t)r * d + o1] = from_f<T>(y1);
+        Kc[(size_t)r * d + o2] = from_f<T>(y2);
+        Vc[(size_t)r * d + o1] = from_f<T>(src[2 * d + o1]);
+        Vc[(size_t)r * d + o2] = from_f<T>(src[2 * d + o2]);
+    }
+}
+template <typename T>
+void launch_qkv_dec(const float* QKV, const int32_t* pos_dec, RopeTab rope, float* Q, T* Kc,
+                    T* Vc, int B, int n, int heads, int dh, cudaStream_t st) {
+    k_qkv_dec<T><<<B * n, 128, 0, st>>>(QKV, pos_dec, rope, Q, Kc, Vc, n, heads, dh);
+    rlt_count_launch();
+}
+
+// cache layout per sequence: [2][heads][T_cap][dh] starting at cache + b*row_stride
+template <typename T>
+__global__ void k_qkv_enc(const float* __restrict__ QKV, const int32_t* __restrict__ pos_enc,
+                          RopeTab rope, float* __restrict__ Q, T* __restrict__ cache,
+                          size_t row_stride, int T_cap, int n, int heads, int dh) {
+    int r = blockIdx.x, b = r / n, i = r % n;
+    int d = heads * dh, half = dh / 2;
+    int p = pos_enc[b] + 1 + i;
+    const float* src = QKV + (size_t)r * 3 * d;
+    T* kc = cache + (size_t)b * row_stride;
+    T* vc = kc + (size_t)heads * T_cap * dh;
+    for (int x = threadIdx.x; x < heads * half; x += blockDim.x) {
+        int h = x / half, j = x % half;
+        float c = rope.cs[(size_t)p * half + j], s = rope.sn[(size_t)p * half + j];
+        int o1 = h * dh + j, o2 = o1 + half;
+        size_t dst = ((size_t)h * T_cap + (p - 1)) * dh + j;
+        float y1, y2;
+        rot(src[o1], src[o2], c, s, y1, y2);
+        Q[(size_t)r * d + o1] = y1;
+        Q[(size_t)r * d + o2] = y2;
+        rot(src[d + o1], src[d + o2], c, s, y1, y2);
+        kc[dst] = from_f<T>(y1);
+        kc[dst + half] = from_f<T>(y2);
+        vc[dst] = from_f<T>(src[2 * d + o1]);
+        vc[dst + half] = from_f<T>(src[2 * d + o2]);
+    }
+}
+template <typename T>
+void launch_qkv_enc(const float* QKV, const int32_t* pos_enc, RopeTab rope, float* Q, T* cache,
+                    size_t row_stride, int T_cap, int B, int n, int heads, int dh,
+                    cudaStream_t st) {
+    k_qkv_enc<T><<<B * n, 128, 0, st>>>(QKV, pos_enc, rope, Q, cache, row_stride, T_cap, n,
+                                        heads, dh);
+    rlt_count_launch();
+}
+
+template <typename T>
+__global__ void k_mem_scatter(const float* __restrict__ KV, const int32_t* __restrict__ pos_enc,
+                              RopeTab rope, T* __restrict__ mem, size_t row_stride, int T_cap,
+                              int n, int heads, int dh) {
+    int r = blockIdx.x, b = r / n, i = r % n;
+    int d = heads * dh, half = dh / 2;
+    int p = pos_enc[b] + 1 + i;
+    const float* src = KV + (size_t)r * 2 * d;
+    T* mk = mem + (size_t)b * row_stride;
+    T* mv = mk + (size_t)heads * T_cap * dh;
+    for (int x = threadIdx.x; x < heads * half; x += blockDim.x) {
+        int h = x / half, j = x % half;
+        float c = rope.cs[(size_t)p * half + j], s = rope.sn[(size_t)p * half + j];
+        int o1 = h * dh + j, o2 = o1 + half;
+        size_t dst = ((size_t)h * T_cap + (p - 1)) * dh + j;
+        float y1, y2;
+        rot(src[o1], src[o2], c, s, y1, y2);
+        mk[dst] = from_f<T>(y1);
+        mk[dst + half] = from_f<T>(y2);
+        mv[dst] = from_f<T>(src[d + o1]);
+        mv[dst + half] = from_f<T>(src[d + o2]);
+    }
+}
+template <typename T>
+void launch_mem_scatter(const float* KV, const int32_t* pos_enc, RopeTab rope, T* mem,
+                        size_t row_stride, int T_cap, int B, int n, int heads, int dh,
+                        cudaStream_t st) {
+    k_mem_scatter<T><<<B * n, 128, 0, st>>>(KV, pos_enc, rope, mem, row_stride, T_cap, n, heads,
+                                            dh);
+    rlt_count_launch();
+}
+
+__global__ void k_rope_q(float* __restrict__ Q, const int32_t* __restrict__ pos_dec,
+                         RopeTab rope, int n, int heads, int dh) {
+    int r = blockIdx.x, b = r / n, i = r % n;
+    int d = heads * dh, half = dh / 2;
+    int t = pos_dec[b] + 1 + i;
+    for (int x = threadIdx.x; x < heads * half; x += blockDim.x) {
+        int h = x / half, j = x % half;
+        float c = rope.cs[(size_t)t * half + j], s = rope.sn[(size_t)t * half + j];
+        int o1 = h * dh + j, o2 = o1 + half;
+        float y1, y2;
+        rot(Q[(size_t)r * d + o1], Q[(size_t)r * d + o2], c, s, y1, y2);
+        Q[(size_t)r * d + o1] = y1;
+        Q[(size_t)r * d + o2] = y2;
+    }
+}
+void launch_rope_q(float* Q, const int32_t* pos_dec, RopeTab rope, int B, int n, int heads,
+                   int dh, cudaStream_t st) {
+    k_rope_q<<<B * n, 128, 0, st>>>(Q, pos_dec, rope, n, heads, dh);
+    rlt_count_launch();
+}
+
+// ---------------------------------------------------------------- FFN gate
+template <typename T>
+__global__ void k_swiglu(const float* __restrict__ H, int fpad, T* __restrict__ Hd) {
+    int r = blockIdx.x;
+    const float* h = H + (size_t)r * 2 * fpad;
+    for (int j = threadIdx.x; j < fpad; j += blockDim.x) {
+        float a = h[j];
+        float silu = a / (1.0f + expf(-a));
+        Hd[(size_t)r * fpad + j] = from_f<T>(silu * h[fpad + j]);
+    }
+}
+template <typename T>
+void launch_swiglu(const float* H, int fpad, T* Hd, int R, cudaStream_t st) {
+    k_swiglu<T><<<R, 256, 0, st>>>(H, fpad, Hd);
+    rlt_count_launch();
+}
+
+// ---------------------------------------------------------------- state bookkeeping
+__global__ void k_copy_e(const float* __restrict__ X, const int32_t* __restrict__ pos_enc,
+                         float* __restrict__ e, int T_cap, int n, int d) {
+    int r = blockIdx.x, b = r / n, i = r % n;
+    float* dst = e + ((size_t)b * T_cap + pos_enc[b] + i) * d;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) dst[j] = X[(size_t)r * d + j];
+}
+void launch_copy_e(const float* X, const int32_t* pos_enc, float* e, int T_cap, int B, int n,
+                   int d, cudaStream_t st) {
+    k_copy_e<<<B * n, 128, 0, st>>>(X, pos_enc, e, T_cap, n, d);
+    rlt_count_launch();
+}
+
+__global__ void k_set_state(const float* __restrict__ z, float* __restrict__ s,
+                            float* __restrict__ Rr, const int32_t* __restrict__ pos_dec,
+                            int chunk, int n, int d) {
+    int b = blockIdx.x;
+    bool upd = Rr != nullptr && ((pos_dec[b] + n) % chunk) == 0;
+    const float* src = z + ((size_t)b * n + n - 1) * d;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        float v = src[j];
+        s[(size_t)b * d + j] = v;
+        if (upd) Rr[(size_t)b * d + j] = v;
+    }
+}
+void launch_set_state(const float* z, float* s, float* Rreg, const int32_t* pos_dec, int chunk,
+                      int B, int n, int d, cudaStream_t st) {
+    k_set_state<<<B, 128, 0, st>>>(z, s, Rreg, pos_dec, chunk, n, d);
+    rlt_count_launch();
+}
+
+__global__ void k_pos_add(int32_t* pos, int B, int n) {
+    int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < B) pos[b] += n;
+}
+void launch_pos_add(int32_t* pos, int B, int n, cudaStream_t st) {
+    k_pos_add<<<(B + 255) / 256, 256, 0, st>>>(pos, B, n);
+    rlt_count_launch();
+}
+
+__global__ void k_reset_rows(const int32_t* __restrict__ rows, const float* __restrict__ s_star,
+                             float* __restrict__ s, float* __restrict__ Rr,
+                             int32_t* __restrict__ pos_enc, int32_t* __restrict__ pos_dec,
+                             int d) {
+    int b = rows ? rows[blockIdx.x] : blockIdx.x;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        float v = s_star ? s_star[j] : 0.f;
+        s[(size_t)b * d + j] = v;
+        Rr[(size_t)b * d + j] = v;
+    }
+    if (threadIdx.x == 0) {
+        pos_enc[b] = 0;
+        pos_dec[b] = 0;
+    }
+}
+void launch_reset_rows(const int32_t* rows, int nrows, const float* s_star, float* s, float* Rr,
+                       int32_t* pos_enc, int32_t* pos_dec, int d, cudaStream_t st) {
+    if (nrows <= 0) return;
+    k_reset_rows<<<nrows, 128, 0, st>>>(rows, s_star, s, Rr, pos_enc, pos_dec, d);
+    rlt_count_launch();
+}
+
+// ring layout per sequence and layer: [2][heads][W-1][dh]; position p lives in
+// slot (p-1) mod (W-1).  Only the last W-1 positions of a block are written,
+// so no two threads of one launch write the same slot.
+template <typename T>
+__global__ void k_ring_write(const T* __restrict__ Kc, const T* __restrict__ Vc,
+                             const int32_t* __restrict__ pos_dec, T* __restrict__ ring,
+                             size_t row_stride, int W, int n, int heads, int dh) {
+    int r = blockIdx.x, b = r / n, i = r % n;
+    int slots = W - 1;
+    if (i < n - slots) return;
+    int p = pos_dec[b] + 1 + i;
+    int slot = (p - 1) % slots;
+    int d = heads * dh;
+    T* rk = ring + (size_t)b * row_stride;
+    T* rv = rk + (size_t)heads * slots * dh;
+    for (int x = threadIdx.x; x < d; x += blockDim.x) {
+        int h = x / dh, j = x % dh;
+        size_t dst = ((size_t)h * slots + slot) * dh + j;
+        rk[dst] = Kc[(size_t)r * d + x];
+        rv[dst] = Vc[(size_t)r * d + x];
+    }
+}
+template <typename T>
+void launch_ring_write(const T* Kc, const T* Vc, const int32_t* pos_dec, T* ring,
+                       size_t row_stride, int W, int B, int n, int heads, int dh,
+                       cudaStream_t st) {
+    if (W <= 1) return;
+    k_ring_write<T><<<B * n, 128, 0, st>>>(Kc, Vc, pos_dec, ring, row_stride, W, n, heads, dh);
+    rlt_count_launch();
+}
+
+#define RLT_INST(T)                                                                            \
+    template void launch_embed<T>(const T*, const int32_t*, float*, int, int, int, int*,       \
+                                  cudaStream_t);                                               \
+    template void launch_rmsnorm<T>(const float*, int, const float*, T*, int, int, int, float, \
+                                    cudaStream_t);                                             \
+    template void launch_merge_input<T>(const float*, int, const int32_t*, const float*,       \
+                                        const float*, T*, int, int, int, float, cudaStream_t); \
+    template void launch_qkv_dec<T>(const float*, const int32_t*, RopeTab, float*, T*, T*, int,\
+                                    int, int, int, cudaStream_t);                              \
+    template void launch_qkv_enc<T>(const float*, const int32_t*, RopeTab, float*, T*, size_t, \
+                                    int, int, int, int, int, cudaStream_t);                    \
+    template void launch_mem_scatter<T>(const float*, const int32_t*, RopeTab, T*, size_t, int,\
+                                        int, int, int, int, cudaStream_t);                     \
+    template void launch_swiglu<T>(const float*, int, T*, int, cudaStream_t);                  \
+    template void launch_ring_write<T>(const T*, const T*, const int32_t*, T*, size_t, int,    \
+                                       int, int, int, int, cudaStream_t);
+RLT_INST(float)
+RLT_INST(bf16)
+#undef RLT_INST
+
+}  // namespace rlt

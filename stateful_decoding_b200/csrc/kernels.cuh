@@ -1,0 +1,98 @@
+// Launchers of the RLT kernels (host side).  Every launcher enqueues on
+// `st` and counts its launches; none synchronises.
+//
+// Row conventions: a call that handles n positions per sequence for B
+// sequences works on R = B*n "rows" r = b*n + i, position i of sequence b.
+// pos[] arrays are the device copies of the per-sequence counters before the
+// call (positions are 1-based: the i-th new position of sequence b is
+// pos[b] + 1 + i).
+#pragma once
+
+#include "common.cuh"
+
+namespace rlt {
+
+// GEMM epilogues: C (fp32) = acc | C += acc | Ct (storage type) = acc
+enum GemmMode { kStoreF32 = 0, kAddF32 = 1, kStoreT = 2 };
+
+struct RopeTab {          // cos/sin of p * base^(-2i/dh), p = 0..max_pos, i < dh/2
+    const float* cs;      // [max_pos+1][dh/2] cos
+    const float* sn;      // [max_pos+1][dh/2] sin
+    int half;
+};
+
+template <typename T>
+void launch_embed(const T* E, const int32_t* tok, float* X, int R, int d, int vocab, int* err,
+                  cudaStream_t st);
+template <typename T>
+void launch_rmsnorm(const float* X, int ldx, const float* gain, T* Y, int ldy, int R, int d,
+                    float eps, cudaStream_t st);
+// dispatcher: tensor-core kernel where it applies, CUDA-core kernel otherwise
+template <typename T>
+void launch_gemm(const T* A, int lda, const T* W, int ldw, float* C, int ldc, T* Ct, int ldct,
+                 int M, int N, int K, int mode, cudaStream_t st);
+template <typename T>
+void launch_gemm_simt(const T* A, int lda, const T* W, int ldw, float* C, int ldc, T* Ct,
+                      int ldct, int M, int N, int K, int mode, cudaStream_t st);
+
+// merge: Gin[r] = [T(e_t), T(RMSNorm_s(fb[b]))], t = pos_dec[b]+1+i
+template <typename T>
+void launch_merge_input(const float* e, int T_cap, const int32_t* pos_dec, const float* fb,
+                        const float* gain, T* Gin, int B, int n, int d, float eps, cudaStream_t st);
+// z[r] = e_t + alpha * sigmoid(G[r] + bg) * S[r]   (S = W_s r); alpha ignored if G == nullptr
+void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const float* G,
+                      const float* bg, const float* S, float alpha, float* z, int B, int n, int d,
+                      cudaStream_t st);
+
+// decoder q/k/v: QKV fp32 [R][3d] -> Q fp32 [R][d] (RoPE), Kc, Vc storage [R][d] (RoPE on k)
+template <typename T>
+void launch_qkv_dec(const float* QKV, const int32_t* pos_dec, RopeTab rope, float* Q, T* Kc,
+                    T* Vc, int B, int n, int heads, int dh, cudaStream_t st);
+// encoder q/k/v: q -> Q (RoPE); k (RoPE), v -> cache [b][2][h][T_cap][dh] + layer offset
+template <typename T>
+void launch_qkv_enc(const float* QKV, const int32_t* pos_enc, RopeTab rope, float* Q, T* cache,
+                    size_t row_stride, int T_cap, int B, int n, int heads, int dh,
+                    cudaStream_t st);
+// memory: KV fp32 [R][2d] -> memory group g: [b][.. g ..][2][h][T_cap][dh] (RoPE on k)
+template <typename T>
+void launch_mem_scatter(const float* KV, const int32_t* pos_enc, RopeTab rope, T* mem,
+                        size_t row_stride, int T_cap, int B, int n, int heads, int dh,
+                        cudaStream_t st);
+// in-place RoPE on Q fp32 [R][d] at decoder positions
+void launch_rope_q(float* Q, const int32_t* pos_dec, RopeTab rope, int B, int n, int heads,
+                   int dh, cudaStream_t st);
+
+template <typename T>
+void launch_swiglu(const float* H, int fpad, T* Hd, int R, cudaStream_t st);
+void launch_copy_e(const float* X, const int32_t* pos_enc, float* e, int T_cap, int B, int n,
+                   int d, cudaStream_t st);
+// s[b] = z[b*n + n-1]; RLT-2: R[b] = s[b] when (pos_dec[b]+n) % chunk == 0
+void launch_set_state(const float* z, float* s, float* Rreg, const int32_t* pos_dec, int chunk,
+                      int B, int n, int d, cudaStream_t st);
+void launch_pos_add(int32_t* pos, int B, int n, cudaStream_t st);
+void launch_reset_rows(const int32_t* rows, int nrows, const float* s_star, float* s, float* Rr,
+                       int32_t* pos_enc, int32_t* pos_dec, int d, cudaStream_t st);
+template <typename T>
+void launch_ring_write(const T* Kc, const T* Vc, const int32_t* pos_dec, T* ring,
+                       size_t row_stride, int W, int B, int n, int heads, int dh,
+                       cudaStream_t st);
+
+// attention (one warp per row and head); outputs A storage [R][d]
+template <typename T>
+void launch_attn_enc(const float* Q, const T* cache, size_t row_stride, int T_cap,
+                     const int32_t* pos_enc, T* A, int B, int n, int heads, int dh,
+                     cudaStream_t st);
+template <typename T>
+void launch_attn_swa(const float* Q, const T* Kc, const T* Vc, const T* ring, size_t row_stride,
+                     int W, const int32_t* pos_dec, T* A, int B, int n, int heads, int dh,
+                     cudaStream_t st);
+template <typename T>
+void launch_attn_cross(const float* Q, const T* mem, size_t row_stride, int T_cap,
+                       const int32_t* pos_dec, T* A, int B, int n, int heads, int dh,
+                       cudaStream_t st);
+
+// readout sampler: one block per row over logits fp32 [B][V]
+void launch_sample(const float* logits, int V, int B, int32_t* argmax, int32_t* sampled,
+                   uint64_t seed, uint64_t step, float temperature, cudaStream_t st);
+
+}  // namespace rlt

@@ -1,0 +1,989 @@
+// C ABI of the RLT transition engine: weight-blob loading, state allocation
+// and the host-side schedule of the encoder, the transition and the readout.
+//
+// The schedule follows the pages' execution procedures: the prompt is
+// encoded token-parallel, then the decoder runs one transition per position,
+// sequential within a row and batched across rows (jiphyeonjeon review
+// "Recurrent Looped Transformer" §3.2, §5; greeksharifa "Recurrent Looped
+// Transformer 요약 설명" §2.4, App. C.1, F.1-F.2); RLT-2 runs the positions of
+// a chunk together (App. I.2).
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/rlt.h"
+#include "kernels.cuh"
+
+static std::atomic<uint64_t> g_launches{0};
+void rlt_count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+namespace rlt {
+template <typename T>
+void launch_gemm(const T* A, int lda, const T* W, int ldw, float* C, int ldc, T* Ct, int ldct,
+                 int M, int N, int K, int mode, cudaStream_t st);
+}
+
+using rlt::bf16;
+
+// ============================================================================
+// blob
+// ============================================================================
+namespace {
+
+constexpr size_t kHeader = 256, kRecord = 64;
+
+struct TensorSpec {
+    std::string name;
+    int d0, d1, ndim;
+};
+
+std::vector<TensorSpec> expected_manifest(const rlt_config& c) {
+    std::vector<TensorSpec> v;
+    const int d = c.d, f = c.ffn, V = c.vocab;
+    auto mat = [&](const std::string& n, int a, int b) { v.push_back({n, a, b, 2}); };
+    auto vec = [&](const std::string& n, int a) { v.push_back({n, a, 1, 1}); };
+    mat("embed", V, d);
+    if (c.variant != 0) vec("s_star", d);
+    for (int l = 0; l < c.n_enc; ++l) {
+        std::string p = "enc." + std::to_string(l) + ".";
+        vec(p + "attn_norm", d);
+        if (!c.tied) { mat(p + "wq", d, d); mat(p + "wk", d, d); mat(p + "wv", d, d); mat(p + "wo", d, d); }
+        vec(p + "ffn_norm", d);
+        if (!c.tied) { mat(p + "w1", f, d); mat(p + "w3", f, d); mat(p + "w2", d, f); }
+    }
+    if (c.n_dec > 0) {
+        vec("mem_norm", d);
+        for (int g = 0; g < c.groups; ++g) {
+            mat("mem." + std::to_string(g) + ".wk", d, d);
+            mat("mem." + std::to_string(g) + ".wv", d, d);
+        }
+    }
+    if (c.variant != 0) {
+        vec("merge.norm", d); mat("merge.wg", d, 2 * d); vec("merge.bg", d); mat("merge.ws", d, d);
+    }
+    for (int l = 0; l < c.n_dec; ++l) {
+        std::string p = "dec." + std::to_string(l) + ".";
+        vec(p + "swa_norm", d); mat(p + "wq", d, d); mat(p + "wk", d, d); mat(p + "wv", d, d);
+        mat(p + "wo", d, d); vec(p + "x_norm", d); mat(p + "xq", d, d); mat(p + "xo", d, d);
+        vec(p + "ffn_norm", d); mat(p + "w1", f, d); mat(p + "w3", f, d); mat(p + "w2", d, f);
+    }
+    vec("out_norm", d);
+    mat("out", V, d);
+    return v;
+}
+
+uint64_t blob_checksum(const uint8_t* p, size_t n) {
+    uint64_t s = 0;
+    size_t words = n / 8;
+    for (size_t i = 0; i < words; ++i) {
+        uint64_t w;
+        memcpy(&w, p + 8 * i, 8);
+        s += w * (2 * (uint64_t)i + 1);
+    }
+    return s;
+}
+
+float bf16_bits_to_float(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+struct ParsedBlob {
+    rlt_config cfg;
+    std::vector<const uint8_t*> data;   // per manifest entry
+};
+
+int parse_blob(const void* blob, size_t nbytes, ParsedBlob* out) {
+    if (!blob || nbytes < kHeader) return RLT_E_BLOB;
+    const uint8_t* b = (const uint8_t*)blob;
+    if (memcmp(b, "RLTB", 4) != 0) return RLT_E_BLOB;
+    uint32_t ver;
+    memcpy(&ver, b + 4, 4);
+    if (ver != 1) return RLT_E_BLOB;
+    uint32_t u[12];
+    memcpy(u, b + 8, 48);
+    rlt_config c;
+    c.vocab = (int)u[0]; c.d = (int)u[1]; c.heads = (int)u[2]; c.n_enc = (int)u[3];
+    c.n_dec = (int)u[4]; c.ffn = (int)u[5]; c.window = (int)u[6]; c.groups = (int)u[7];
+    c.chunk = (int)u[8]; c.variant = (int)u[9]; c.tied = (int)u[10]; c.dtype = (int)u[11];
+    memcpy(&c.alpha, b + 56, 8);
+    memcpy(&c.eps, b + 64, 8);
+    memcpy(&c.rope_base, b + 72, 8);
+    uint64_t nt, nb, ck;
+    memcpy(&nt, b + 88, 8);
+    memcpy(&nb, b + 96, 8);
+    memcpy(&ck, b + 104, 8);
+    if (nb > nbytes - kHeader) return RLT_E_BLOB;
+    const uint8_t* pay = b + kHeader;
+    if (blob_checksum(pay, nb) != ck) return RLT_E_BLOB;
+    if (c.dtype != RLT_DTYPE_F32 && c.dtype != RLT_DTYPE_BF16) return RLT_E_BLOB;
+    if (c.vocab <= 0 || c.d <= 0 || c.heads <= 0 || c.d % c.heads || c.n_enc < 0 ||
+        c.n_dec < 0 || c.ffn <= 0 || c.window < 1 || c.chunk < 1 || c.variant < 0 ||
+        c.variant > 2 || (c.variant != 2 && c.chunk != 1) ||
+        (c.groups != 1 && c.groups != c.n_dec) || c.groups < 1 ||
+        (c.tied && c.n_enc != c.n_dec) || !(c.eps > 0) || !(c.rope_base > 0))
+        return RLT_E_BLOB;
+    std::vector<TensorSpec> man = expected_manifest(c);
+    if (nt != man.size()) return RLT_E_BLOB;
+    const size_t elt = c.dtype == RLT_DTYPE_BF16 ? 2 : 4;
+    size_t off = 0;
+    out->data.clear();
+    for (const TensorSpec& s : man) {
+        if (off + kRecord > nb) return RLT_E_BLOB;
+        char name[49] = {0};
+        memcpy(name, pay + off, 48);
+        uint32_t r[4];
+        memcpy(r, pay + off + 48, 16);
+        if (s.name != name || (int)r[0] != s.ndim || (int)r[1] != c.dtype || (int)r[2] != s.d0 ||
+            (int)r[3] != s.d1)
+            return RLT_E_BLOB;
+        off += kRecord;
+        size_t bytes = (size_t)s.d0 * s.d1 * elt;
+        if (off + bytes > nb) return RLT_E_BLOB;
+        out->data.push_back(pay + off);
+        off += bytes + ((64 - bytes % 64) % 64);
+    }
+    out->cfg = c;
+    return RLT_OK;
+}
+
+}  // namespace
+
+// ============================================================================
+// model
+// ============================================================================
+struct EncLayerW {
+    float *attn_norm, *ffn_norm;
+    void *wqkv, *wo, *w13, *w2;
+};
+struct DecLayerW {
+    float *swa_norm, *x_norm, *ffn_norm;
+    void *wqkv, *wo, *xq, *xo, *w13, *w2;
+};
+
+struct rlt_model {
+    rlt_config cfg;
+    int device = 0;
+    int dh = 0, fpad = 0;
+    size_t elt = 4;
+    void* arena = nullptr;
+    size_t arena_bytes = 0;
+    void* embed = nullptr;
+    float* s_star = nullptr;
+    std::vector<EncLayerW> enc;
+    float* mem_norm = nullptr;
+    std::vector<void*> wmem;        // per group [2d][d]: K rows then V rows
+    float *merge_norm = nullptr, *bg = nullptr;
+    void *wg = nullptr, *ws = nullptr;
+    std::vector<DecLayerW> dec;
+    float* out_norm = nullptr;
+    void* wout = nullptr;
+};
+
+namespace {
+
+struct Arena {
+    std::vector<uint8_t> host;
+    size_t take(size_t bytes) {
+        size_t off = (host.size() + 255) / 256 * 256;
+        host.resize(off + bytes, 0);
+        return off;
+    }
+};
+
+// copy a stored matrix [rows][cols] into arena rows [row0..] of a [*, ld] matrix
+void put_mat(Arena& a, size_t off, size_t elt, const uint8_t* src, int rows, int cols, int ld,
+             int row0) {
+    for (int r = 0; r < rows; ++r)
+        memcpy(a.host.data() + off + ((size_t)(row0 + r) * ld) * elt, src + (size_t)r * cols * elt,
+               (size_t)cols * elt);
+}
+
+void put_vec_f32(Arena& a, size_t off, size_t elt, const uint8_t* src, int n) {
+    float* dst = (float*)(a.host.data() + off);
+    for (int i = 0; i < n; ++i) {
+        if (elt == 2) {
+            uint16_t h;
+            memcpy(&h, src + 2 * i, 2);
+            dst[i] = bf16_bits_to_float(h);
+        } else {
+            memcpy(dst + i, src + 4 * i, 4);
+        }
+    }
+}
+
+}  // namespace
+
+static int dev_err(cudaError_t e) {
+    if (e == cudaErrorMemoryAllocation) return RLT_E_OOM;
+    return e == cudaSuccess ? RLT_OK : RLT_E_DEVICE;
+}
+
+extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model** out) {
+    if (!out) return RLT_E_ARG;
+    *out = nullptr;
+    ParsedBlob pb;
+    int rc = parse_blob(blob, nbytes, &pb);
+    if (rc) return rc;
+    const rlt_config& c = pb.cfg;
+    const int dh = c.d / c.heads;
+    if (dh != 16 && dh != 32 && dh != 64 && dh != 128) return RLT_E_UNSUPPORTED;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+        cudaGetLastError();
+        return RLT_E_DEVICE;
+    }
+    if (cudaSetDevice(device) != cudaSuccess) return RLT_E_DEVICE;
+
+    rlt_model* m = new rlt_model();
+    m->cfg = c;
+    m->device = device;
+    m->dh = dh;
+    m->fpad = (c.ffn + 63) / 64 * 64;
+    m->elt = c.dtype == RLT_DTYPE_BF16 ? 2 : 4;
+    const size_t elt = m->elt;
+    const int d = c.d, fp = m->fpad;
+
+    // lay the weights out in one arena: fused [3d][d] QKV, [2 fpad][d] W1;W3
+    // (zero rows past ffn), [d][fpad] W2 (zero columns past ffn)
+    Arena a;
+    std::vector<TensorSpec> man = expected_manifest(c);
+    auto idx = [&](const std::string& n) {
+        for (size_t i = 0; i < man.size(); ++i)
+            if (man[i].name == n) return (int)i;
+        return -1;
+    };
+    auto src = [&](const std::string& n) { return pb.data[idx(n)]; };
+    std::vector<std::pair<size_t, void**>> fixups;
+    std::vector<std::pair<size_t, float**>> ffix;
+    auto mat_plain = [&](const std::string& n, int rows, int cols, void** dst) {
+        size_t off = a.take((size_t)rows * cols * elt);
+        put_mat(a, off, elt, src(n), rows, cols, cols, 0);
+        fixups.push_back({off, dst});
+    };
+    auto vecf = [&](const std::string& n, float** dst) {
+        size_t off = a.take((size_t)d * 4);
+        put_vec_f32(a, off, elt, src(n), d);
+        ffix.push_back({off, dst});
+    };
+    auto qkv = [&](const std::string& p, void** dst) {
+        size_t off = a.take((size_t)3 * d * d * elt);
+        put_mat(a, off, elt, src(p + "wq"), d, d, d, 0);
+        put_mat(a, off, elt, src(p + "wk"), d, d, d, d);
+        put_mat(a, off, elt, src(p + "wv"), d, d, d, 2 * d);
+        fixups.push_back({off, dst});
+    };
+    auto ffn = [&](const std::string& p, void** w13, void** w2) {
+        size_t o13 = a.take((size_t)2 * fp * d * elt);
+        put_mat(a, o13, elt, src(p + "w1"), c.ffn, d, d, 0);
+        put_mat(a, o13, elt, src(p + "w3"), c.ffn, d, d, fp);
+        fixups.push_back({o13, w13});
+        size_t o2 = a.take((size_t)d * fp * elt);
+        put_mat(a, o2, elt, src(p + "w2"), d, c.ffn, fp, 0);
+        fixups.push_back({o2, w2});
+    };
+
+    m->enc.resize(c.n_enc);
+    m->dec.resize(c.n_dec);
+    mat_plain("embed", c.vocab, d, &m->embed);
+    if (c.variant != 0) vecf("s_star", &m->s_star);
+    for (int l = 0; l < c.n_dec; ++l) {
+        std::string p = "dec." + std::to_string(l) + ".";
+        DecLayerW& L = m->dec[l];
+        vecf(p + "swa_norm", &L.swa_norm);
+        vecf(p + "x_norm", &L.x_norm);
+        vecf(p + "ffn_norm", &L.ffn_norm);
+        qkv(p, &L.wqkv);
+        mat_plain(p + "wo", d, d, &L.wo);
+        mat_plain(p + "xq", d, d, &L.xq);
+        mat_plain(p + "xo", d, d, &L.xo);
+        ffn(p, &L.w13, &L.w2);
+    }
+    for (int l = 0; l < c.n_enc; ++l) {
+        std::string p = "enc." + std::to_string(l) + ".";
+        EncLayerW& L = m->enc[l];
+        vecf(p + "attn_norm", &L.attn_norm);
+        vecf(p + "ffn_norm", &L.ffn_norm);
+        if (!c.tied) {
+            qkv(p, &L.wqkv);
+            mat_plain(p + "wo", d, d, &L.wo);
+            ffn(p, &L.w13, &L.w2);
+        }
+    }
+    if (c.n_dec > 0) {
+        vecf("mem_norm", &m->mem_norm);
+        m->wmem.resize(c.groups);
+        for (int g = 0; g < c.groups; ++g) {
+            std::string p = "mem." + std::to_string(g) + ".";
+            size_t off = a.take((size_t)2 * d * d * elt);
+            put_mat(a, off, elt, src(p + "wk"), d, d, d, 0);
+            put_mat(a, off, elt, src(p + "wv"), d, d, d, d);
+            fixups.push_back({off, &m->wmem[g]});
+        }
+    }
+    if (c.variant != 0) {
+        vecf("merge.norm", &m->merge_norm);
+        vecf("merge.bg", &m->bg);
+        mat_plain("merge.wg", d, 2 * d, &m->wg);
+        mat_plain("merge.ws", d, d, &m->ws);
+    }
+    vecf("out_norm", &m->out_norm);
+    mat_plain("out", c.vocab, d, &m->wout);
+
+    m->arena_bytes = a.host.size();
+    cudaError_t e = cudaMalloc(&m->arena, m->arena_bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        delete m;
+        return dev_err(e);
+    }
+    e = cudaMemcpy(m->arena, a.host.data(), m->arena_bytes, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        cudaFree(m->arena);
+        delete m;
+        return RLT_E_DEVICE;
+    }
+    uint8_t* base = (uint8_t*)m->arena;
+    for (auto& fx : fixups) *fx.second = base + fx.first;
+    for (auto& fx : ffix) *fx.second = (float*)(base + fx.first);
+    if (c.tied) {
+        for (int l = 0; l < c.n_enc; ++l) {
+            m->enc[l].wqkv = m->dec[l].wqkv;
+            m->enc[l].wo = m->dec[l].wo;
+            m->enc[l].w13 = m->dec[l].w13;
+            m->enc[l].w2 = m->dec[l].w2;
+        }
+    }
+    *out = m;
+    return RLT_OK;
+}
+
+extern "C" void rlt_destroy(rlt_model* m) {
+    if (!m) return;
+    cudaSetDevice(m->device);
+    cudaFree(m->arena);
+    delete m;
+}
+
+extern "C" int rlt_model_config(const rlt_model* m, rlt_config* out) {
+    if (!m || !out) return RLT_E_ARG;
+    *out = m->cfg;
+    return RLT_OK;
+}
+
+// ============================================================================
+// state
+// ============================================================================
+struct rlt_state {
+    rlt_model* m = nullptr;
+    int B = 0, T_cap = 0;
+    int n_enc_blk = 1, n_dec_blk = 1;    // positions per row in one encoder / decoder pass
+    float *s = nullptr, *Rr = nullptr, *e = nullptr;
+    void *enc = nullptr, *mem = nullptr, *ring = nullptr;
+    size_t enc_row = 0, mem_row = 0, ring_row = 0;   // elements per row
+    int32_t *pos_enc = nullptr, *pos_dec = nullptr;
+    std::vector<int32_t> h_pos_enc, h_pos_dec;
+    float *rope_cs = nullptr, *rope_sn = nullptr;
+    int* err = nullptr;
+    // scratch (rows = B * max block)
+    float *X = nullptr, *QKV = nullptr, *Q = nullptr, *H13 = nullptr, *G = nullptr, *S = nullptr;
+    void *Y = nullptr, *Hd = nullptr, *A = nullptr, *Kc = nullptr, *Vc = nullptr;
+    int32_t* tok = nullptr;
+    float* logits = nullptr;
+    int32_t* ids = nullptr;
+    int32_t* rows = nullptr;
+    std::vector<void*> allocs;
+    size_t bytes = 0;
+    // live timing (rlt_profile_*)
+    bool prof = false;
+    struct ProfRec { int cls; cudaEvent_t a, b; double bytes; };
+    std::vector<ProfRec> prof_recs;
+    std::vector<cudaEvent_t> prof_pool;
+};
+
+static cudaEvent_t prof_event(rlt_state* s) {
+    cudaEvent_t e = nullptr;
+    if (!s->prof_pool.empty()) {
+        e = s->prof_pool.back();
+        s->prof_pool.pop_back();
+    } else if (cudaEventCreate(&e) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return e;
+}
+// Bracket a launch sequence with events on `st` when profiling is on.
+struct ProfScope {
+    rlt_state* s;
+    int cls;
+    cudaStream_t st;
+    double bytes;
+    cudaEvent_t a = nullptr;
+    ProfScope(rlt_state* s_, int c, cudaStream_t st_, double b) : s(s_), cls(c), st(st_), bytes(b) {
+        if (s->prof && (a = prof_event(s))) cudaEventRecord(a, st);
+    }
+    ~ProfScope() {
+        if (!a) return;
+        cudaEvent_t b = prof_event(s);
+        if (!b) return;
+        cudaEventRecord(b, st);
+        s->prof_recs.push_back({cls, a, b, bytes});
+    }
+};
+
+static int salloc(rlt_state* s, void** p, size_t bytes) {
+    if (bytes == 0) bytes = 256;
+    cudaError_t e = cudaMalloc(p, bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        *p = nullptr;
+        return dev_err(e);
+    }
+    s->allocs.push_back(*p);
+    s->bytes += bytes;
+    return RLT_OK;
+}
+
+extern "C" void rlt_state_destroy(rlt_state* s) {
+    if (!s) return;
+    cudaSetDevice(s->m->device);
+    cudaDeviceSynchronize();
+    for (auto& r : s->prof_recs) {
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    for (cudaEvent_t e : s->prof_pool) cudaEventDestroy(e);
+    for (void* p : s->allocs) cudaFree(p);
+    delete s;
+}
+
+static size_t max_rows_per_call() {
+    const char* v = getenv("RLT_MAX_ROWS");
+    long x = v ? atol(v) : 65536;
+    return (size_t)std::max(256L, x);
+}
+
+extern "C" int rlt_state_create(rlt_model* m, int batch, int max_len, rlt_state** out) {
+    if (!m || !out || batch <= 0 || max_len <= 0) return RLT_E_ARG;
+    *out = nullptr;
+    if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
+    const rlt_config& c = m->cfg;
+    rlt_state* s = new rlt_state();
+    s->m = m;
+    s->B = batch;
+    s->T_cap = max_len;
+    const size_t elt = m->elt, d = c.d, dh = m->dh, h = c.heads, B = batch, T = max_len;
+    const size_t slots = (size_t)std::max(0, c.window - 1);
+    size_t maxr = max_rows_per_call();
+    s->n_enc_blk = (int)std::max<size_t>(1, std::min<size_t>(T, maxr / B));
+    s->n_dec_blk = c.variant == 2 ? c.chunk : (c.variant == 0 ? std::min(s->n_enc_blk, 256) : 1);
+    const size_t R = B * (size_t)std::max(s->n_enc_blk, s->n_dec_blk);
+    s->enc_row = (size_t)c.n_enc * 2 * h * T * dh;
+    s->mem_row = (size_t)(c.n_dec > 0 ? c.groups : 0) * 2 * h * T * dh;
+    s->ring_row = (size_t)c.n_dec * 2 * h * slots * dh;
+    int rc = RLT_OK;
+    auto take = [&](void** p, size_t bytes) {
+        if (rc == RLT_OK) rc = salloc(s, p, bytes);
+    };
+    const size_t fp = m->fpad;
+    take((void**)&s->s, B * d * 4);
+    take((void**)&s->Rr, B * d * 4);
+    take((void**)&s->e, B * T * d * 4);
+    take(&s->enc, B * s->enc_row * elt);
+    take(&s->mem, B * s->mem_row * elt);
+    take(&s->ring, B * s->ring_row * elt);
+    take((void**)&s->pos_enc, B * 4);
+    take((void**)&s->pos_dec, B * 4);
+    take((void**)&s->rope_cs, (T + 1) * (dh / 2) * 4);
+    take((void**)&s->rope_sn, (T + 1) * (dh / 2) * 4);
+    take((void**)&s->err, 4);
+    take((void**)&s->X, R * d * 4);
+    take((void**)&s->QKV, R * 3 * d * 4);
+    take((void**)&s->Q, R * d * 4);
+    take((void**)&s->H13, R * 2 * fp * 4);
+    take((void**)&s->G, R * d * 4);
+    take((void**)&s->S, R * d * 4);
+    take(&s->Y, R * std::max(2 * d, fp) * elt);
+    take(&s->Hd, R * fp * elt);
+    take(&s->A, R * d * elt);
+    take(&s->Kc, R * d * elt);
+    take(&s->Vc, R * d * elt);
+    take((void**)&s->tok, R * 4);
+    take((void**)&s->logits, B * (size_t)c.vocab * 4);
+    take((void**)&s->ids, 2 * B * 4);
+    take((void**)&s->rows, B * 4);
+    if (rc != RLT_OK) {
+        rlt_state_destroy(s);
+        return rc;
+    }
+    // RoPE table: angle p * base^(-2i/dh) for p = 0..T, computed in double
+    std::vector<float> cs((T + 1) * (dh / 2)), sn((T + 1) * (dh / 2));
+    for (size_t p = 0; p <= T; ++p)
+        for (size_t i = 0; i < dh / 2; ++i) {
+            double ang = (double)p * std::pow(c.rope_base, -2.0 * (double)i / (double)dh);
+            cs[p * (dh / 2) + i] = (float)std::cos(ang);
+            sn[p * (dh / 2) + i] = (float)std::sin(ang);
+        }
+    cudaError_t e1 = cudaMemcpy(s->rope_cs, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice);
+    cudaError_t e2 = cudaMemcpy(s->rope_sn, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice);
+    cudaError_t e3 = cudaMemset(s->err, 0, 4);
+    if (e1 || e2 || e3) {
+        rlt_state_destroy(s);
+        return RLT_E_DEVICE;
+    }
+    s->h_pos_enc.assign(B, 0);
+    s->h_pos_dec.assign(B, 0);
+    rlt::launch_reset_rows(nullptr, batch, m->s_star, s->s, s->Rr, s->pos_enc, s->pos_dec, c.d,
+                           0);
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+        rlt_state_destroy(s);
+        return RLT_E_DEVICE;
+    }
+    *out = s;
+    return RLT_OK;
+}
+
+extern "C" int rlt_state_bytes(const rlt_state* s, size_t* per_row_state, size_t* total) {
+    if (!s) return RLT_E_ARG;
+    const rlt_config& c = s->m->cfg;
+    if (per_row_state)
+        *per_row_state = (s->enc_row + s->mem_row + s->ring_row) * s->m->elt + (size_t)c.d * 4;
+    if (total) *total = s->bytes;
+    return RLT_OK;
+}
+
+// ============================================================================
+// helpers
+// ============================================================================
+static bool is_device_ptr(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+static int launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? RLT_OK : RLT_E_DEVICE;
+}
+
+static rlt::RopeTab rope_of(rlt_state* s) {
+    return rlt::RopeTab{s->rope_cs, s->rope_sn, s->m->dh / 2};
+}
+
+// ============================================================================
+// algorithmic bytes of one launch (what the computation must move at least;
+// weights excluded unless they cannot stay on chip)
+// ============================================================================
+static double kv_bytes(const rlt_state* s) { return 2.0 * s->m->cfg.d * (double)s->m->elt; }
+
+static double xattn_bytes(const rlt_state* s, int n) {   // one cross-attention launch
+    const double d = s->m->cfg.d, elt = (double)s->m->elt;
+    double by = 0;
+    for (int b = 0; b < s->B; ++b)
+        by += (s->h_pos_dec[b] + n) * kv_bytes(s) + n * (d * 4 + d * elt);
+    return by;
+}
+static double swa_bytes(const rlt_state* s, int n) {     // one window-attention launch
+    const double d = s->m->cfg.d, elt = (double)s->m->elt;
+    const int slots = std::max(0, s->m->cfg.window - 1);
+    double by = 0;
+    for (int b = 0; b < s->B; ++b)
+        by += std::min(s->h_pos_dec[b], slots) * kv_bytes(s) + n * (kv_bytes(s) + d * 4 + d * elt);
+    return by;
+}
+static double decoder_weight_bytes(const rlt_model* m) {
+    const double d = m->cfg.d, f = m->cfg.ffn;
+    return (double)m->elt * (m->cfg.n_dec * (6 * d * d + 3 * d * f) + (m->cfg.variant ? 3 * d * d : 0));
+}
+static double step_bytes(const rlt_state* s, int n) {    // one whole transition block
+    const rlt_config& c = s->m->cfg;
+    const int slots = std::max(0, c.window - 1);
+    double by = 0;
+    for (int b = 0; b < s->B; ++b) {
+        const int pd = s->h_pos_dec[b];
+        by += c.n_dec * ((pd + n) * kv_bytes(s) + std::min(pd, slots) * kv_bytes(s) +
+                         std::min(n, slots) * kv_bytes(s));
+        by += n * c.d * 4.0 + 2.0 * c.d * 4.0;            // e_t in, s in and out
+    }
+    // weights re-stream from HBM each step once they exceed what L2 can hold
+    if (decoder_weight_bytes(s->m) > 64e6) by += decoder_weight_bytes(s->m);
+    return by;
+}
+static double enc_bytes(const rlt_state* s, int n) {     // one encoder block
+    const rlt_config& c = s->m->cfg;
+    double by = 0;
+    for (int b = 0; b < s->B; ++b) {
+        const int p0 = s->h_pos_enc[b];
+        // cache and memory written for n positions; cached keys/values re-read
+        by += (c.n_enc + (c.n_dec ? c.groups : 0)) * n * kv_bytes(s) +
+              c.n_enc * (double)p0 * kv_bytes(s) + n * (4.0 + c.d * 4.0);
+    }
+    return by;
+}
+
+// ============================================================================
+// encoder
+// ============================================================================
+template <typename T>
+static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t st) {
+    using namespace rlt;
+    rlt_model* m = s->m;
+    const rlt_config& c = m->cfg;
+    const int B = s->B, d = c.d, h = c.heads, dh = m->dh, fp = m->fpad, R = B * n;
+    const float eps = (float)c.eps;
+    T* Y = (T*)s->Y;
+    T* A = (T*)s->A;
+    T* Hd = (T*)s->Hd;
+    T* enc = (T*)s->enc;
+    const size_t layer_enc = (size_t)2 * h * s->T_cap * dh;
+    launch_embed<T>((const T*)m->embed, tok, s->X, R, d, c.vocab, s->err, st);
+    for (int l = 0; l < c.n_enc; ++l) {
+        const EncLayerW& L = m->enc[l];
+        launch_rmsnorm<T>(s->X, d, L.attn_norm, Y, d, R, d, eps, st);
+        launch_gemm<T>(Y, d, (const T*)L.wqkv, d, s->QKV, 3 * d, nullptr, 0, R, 3 * d, d,
+                       kStoreF32, st);
+        launch_qkv_enc<T>(s->QKV, s->pos_enc, rope_of(s), s->Q, enc + l * layer_enc, s->enc_row,
+                          s->T_cap, B, n, h, dh, st);
+        launch_attn_enc<T>(s->Q, enc + l * layer_enc, s->enc_row, s->T_cap, s->pos_enc, A, B, n,
+                           h, dh, st);
+        launch_gemm<T>(A, d, (const T*)L.wo, d, s->X, d, nullptr, 0, R, d, d, kAddF32, st);
+        launch_rmsnorm<T>(s->X, d, L.ffn_norm, Y, d, R, d, eps, st);
+        launch_gemm<T>(Y, d, (const T*)L.w13, d, s->H13, 2 * fp, nullptr, 0, R, 2 * fp, d,
+                       kStoreF32, st);
+        launch_swiglu<T>(s->H13, fp, Hd, R, st);
+        launch_gemm<T>(Hd, fp, (const T*)L.w2, fp, s->X, d, nullptr, 0, R, d, fp, kAddF32, st);
+    }
+    launch_copy_e(s->X, s->pos_enc, s->e, s->T_cap, B, n, d, st);
+    if (c.n_dec > 0) {
+        launch_rmsnorm<T>(s->X, d, m->mem_norm, Y, d, R, d, eps, st);
+        const size_t layer_mem = (size_t)2 * h * s->T_cap * dh;
+        for (int g = 0; g < c.groups; ++g) {
+            launch_gemm<T>(Y, d, (const T*)m->wmem[g], d, s->QKV, 2 * d, nullptr, 0, R, 2 * d, d,
+                           kStoreF32, st);
+            launch_mem_scatter<T>(s->QKV, s->pos_enc, rope_of(s), (T*)s->mem + g * layer_mem,
+                                  s->mem_row, s->T_cap, B, n, h, dh, st);
+        }
+    }
+    launch_pos_add(s->pos_enc, B, n, st);
+}
+
+extern "C" int rlt_encode(rlt_state* s, const int32_t* tokens, int n, void* stream) {
+    if (!s || !tokens || n < 0) return RLT_E_ARG;
+    if (n == 0) return RLT_OK;
+    rlt_model* m = s->m;
+    if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
+    for (int b = 0; b < s->B; ++b)
+        if (s->h_pos_enc[b] + n > s->T_cap) return RLT_E_CAPACITY;
+    cudaStream_t st = (cudaStream_t)stream;
+    const bool dev = is_device_ptr(tokens);
+    if (!dev) {
+        for (size_t i = 0; i < (size_t)s->B * n; ++i)
+            if (tokens[i] < 0 || tokens[i] >= m->cfg.vocab) return RLT_E_ARG;
+    }
+    // rows of the caller's [B][n] array are split into blocks of n_enc_blk positions
+    for (int j0 = 0; j0 < n; j0 += s->n_enc_blk) {
+        int nb = std::min(s->n_enc_blk, n - j0);
+        cudaError_t e = cudaMemcpy2DAsync(s->tok, (size_t)nb * 4, tokens + j0, (size_t)n * 4,
+                                          (size_t)nb * 4, s->B,
+                                          dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice,
+                                          st);
+        if (e != cudaSuccess) return RLT_E_DEVICE;
+        {
+            ProfScope ps(s, RLT_PROF_ENC, st, s->prof ? enc_bytes(s, nb) : 0.0);
+            if (m->cfg.dtype == RLT_DTYPE_BF16) encode_block<bf16>(s, s->tok, nb, st);
+            else encode_block<float>(s, s->tok, nb, st);
+        }
+        int rc = launch_status();
+        if (rc) return rc;
+    }
+    for (int b = 0; b < s->B; ++b) s->h_pos_enc[b] += n;
+    return RLT_OK;
+}
+
+// ============================================================================
+// transition
+// ============================================================================
+template <typename T>
+static void step_block(rlt_state* s, int n, cudaStream_t st) {
+    using namespace rlt;
+    rlt_model* m = s->m;
+    const rlt_config& c = m->cfg;
+    const int B = s->B, d = c.d, h = c.heads, dh = m->dh, fp = m->fpad, R = B * n;
+    const float eps = (float)c.eps;
+    T* Y = (T*)s->Y;
+    T* A = (T*)s->A;
+    T* Hd = (T*)s->Hd;
+    T* Kc = (T*)s->Kc;
+    T* Vc = (T*)s->Vc;
+    float* z = s->X;
+    if (c.variant == 0) {
+        launch_merge_out(s->e, s->T_cap, s->pos_dec, nullptr, nullptr, nullptr, 0.f, z, B, n, d,
+                         st);
+    } else {
+        const float* fb = c.variant == 2 ? s->Rr : s->s;
+        launch_merge_input<T>(s->e, s->T_cap, s->pos_dec, fb, m->merge_norm, Y, B, n, d, eps, st);
+        launch_gemm<T>(Y, 2 * d, (const T*)m->wg, 2 * d, s->G, d, nullptr, 0, R, d, 2 * d,
+                       kStoreF32, st);
+        launch_gemm<T>(Y + d, 2 * d, (const T*)m->ws, d, s->S, d, nullptr, 0, R, d, d, kStoreF32,
+                       st);
+        launch_merge_out(s->e, s->T_cap, s->pos_dec, s->G, m->bg, s->S, (float)c.alpha, z, B, n,
+                         d, st);
+    }
+    const size_t layer_ring = (size_t)2 * h * std::max(0, c.window - 1) * dh;
+    const size_t layer_mem = (size_t)2 * h * s->T_cap * dh;
+    for (int l = 0; l < c.n_dec; ++l) {
+        const DecLayerW& L = m->dec[l];
+        T* ring = (T*)s->ring + l * layer_ring;
+        launch_rmsnorm<T>(z, d, L.swa_norm, Y, d, R, d, eps, st);
+        launch_gemm<T>(Y, d, (const T*)L.wqkv, d, s->QKV, 3 * d, nullptr, 0, R, 3 * d, d,
+                       kStoreF32, st);
+        launch_qkv_dec<T>(s->QKV, s->pos_dec, rope_of(s), s->Q, Kc, Vc, B, n, h, dh, st);
+        {
+            ProfScope ps(s, RLT_PROF_SWA, st, s->prof ? swa_bytes(s, n) : 0.0);
+            launch_attn_swa<T>(s->Q, Kc, Vc, ring, s->ring_row, c.window, s->pos_dec, A, B, n, h,
+                               dh, st);
+        }
+        launch_ring_write<T>(Kc, Vc, s->pos_dec, ring, s->ring_row, c.window, B, n, h, dh, st);
+        launch_gemm<T>(A, d, (const T*)L.wo, d, z, d, nullptr, 0, R, d, d, kAddF32, st);
+        launch_rmsnorm<T>(z, d, L.x_norm, Y, d, R, d, eps, st);
+        launch_gemm<T>(Y, d, (const T*)L.xq, d, s->Q, d, nullptr, 0, R, d, d, kStoreF32, st);
+        launch_rope_q(s->Q, s->pos_dec, rope_of(s), B, n, h, dh, st);
+        const T* mem = (const T*)s->mem + (c.groups > 1 ? l : 0) * layer_mem;
+        {
+            ProfScope ps(s, RLT_PROF_XATTN, st, s->prof ? xattn_bytes(s, n) : 0.0);
+            launch_attn_cross<T>(s->Q, mem, s->mem_row, s->T_cap, s->pos_dec, A, B, n, h, dh, st);
+        }
+        launch_gemm<T>(A, d, (const T*)L.xo, d, z, d, nullptr, 0, R, d, d, kAddF32, st);
+        launch_rmsnorm<T>(z, d, L.ffn_norm, Y, d, R, d, eps, st);
+        launch_gemm<T>(Y, d, (const T*)L.w13, d, s->H13, 2 * fp, nullptr, 0, R, 2 * fp, d,
+                       kStoreF32, st);
+        launch_swiglu<T>(s->H13, fp, Hd, R, st);
+        launch_gemm<T>(Hd, fp, (const T*)L.w2, fp, z, d, nullptr, 0, R, d, fp, kAddF32, st);
+    }
+    launch_set_state(z, s->s, c.variant == 2 ? s->Rr : nullptr, s->pos_dec, c.chunk, B, n, d, st);
+    launch_pos_add(s->pos_dec, B, n, st);
+}
+
+static int run_block(rlt_state* s, int n, cudaStream_t st) {
+    for (int b = 0; b < s->B; ++b) {
+        if (s->h_pos_dec[b] + n > s->h_pos_enc[b]) return RLT_E_ORDER;
+        if (s->h_pos_dec[b] + n > s->T_cap) return RLT_E_CAPACITY;
+    }
+    {
+        ProfScope ps(s, RLT_PROF_STEP, st, s->prof ? step_bytes(s, n) : 0.0);
+        if (s->m->cfg.dtype == RLT_DTYPE_BF16) step_block<bf16>(s, n, st);
+        else step_block<float>(s, n, st);
+    }
+    int rc = launch_status();
+    if (rc) return rc;
+    for (int b = 0; b < s->B; ++b) s->h_pos_dec[b] += n;
+    return RLT_OK;
+}
+
+extern "C" int rlt_step(rlt_state* s, void* stream) {
+    if (!s) return RLT_E_ARG;
+    if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    return run_block(s, 1, (cudaStream_t)stream);
+}
+
+extern "C" int rlt_prefill(rlt_state* s, int T, void* stream) {
+    if (!s || T < 0) return RLT_E_ARG;
+    if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    const rlt_config& c = s->m->cfg;
+    for (int b = 0; b < s->B; ++b) {
+        if (s->h_pos_dec[b] + T > s->h_pos_enc[b]) return RLT_E_ORDER;
+        if (s->h_pos_dec[b] + T > s->T_cap) return RLT_E_CAPACITY;
+    }
+    int done = 0;
+    while (done < T) {
+        const int pd = s->h_pos_dec[0];
+        bool uniform = true;
+        for (int b = 1; b < s->B; ++b) uniform &= s->h_pos_dec[b] == pd;
+        int n = 1;
+        if (uniform && c.variant == 2) n = std::min(T - done, c.chunk - pd % c.chunk);
+        else if (uniform && c.variant == 0) n = std::min(T - done, s->n_dec_blk);
+        int rc = run_block(s, n, (cudaStream_t)stream);
+        if (rc) return rc;
+        done += n;
+    }
+    return RLT_OK;
+}
+
+// ============================================================================
+// readout
+// ============================================================================
+extern "C" int rlt_readout(rlt_state* s, float* logits, int32_t* argmax, int32_t* sampled,
+                           uint64_t seed, uint64_t step, float temperature, void* stream) {
+    if (!s || !(temperature > 0.f)) return RLT_E_ARG;
+    rlt_model* m = s->m;
+    if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
+    const rlt_config& c = m->cfg;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int B = s->B, d = c.d, V = c.vocab;
+    const bool ld = logits && is_device_ptr(logits);
+    const bool ad = argmax && is_device_ptr(argmax);
+    const bool sd = sampled && is_device_ptr(sampled);
+    float* lbuf = ld ? logits : s->logits;
+    int32_t* abuf = argmax ? (ad ? argmax : s->ids) : nullptr;
+    int32_t* sbuf = sampled ? (sd ? sampled : s->ids + B) : nullptr;
+    if (c.dtype == RLT_DTYPE_BF16) {
+        rlt::launch_rmsnorm<bf16>(s->s, d, m->out_norm, (bf16*)s->Y, d, B, d, (float)c.eps, st);
+        rlt::launch_gemm<bf16>((const bf16*)s->Y, d, (const bf16*)m->wout, d, lbuf, V, nullptr,
+                               0, B, V, d, rlt::kStoreF32, st);
+    } else {
+        rlt::launch_rmsnorm<float>(s->s, d, m->out_norm, (float*)s->Y, d, B, d, (float)c.eps, st);
+        rlt::launch_gemm<float>((const float*)s->Y, d, (const float*)m->wout, d, lbuf, V,
+                                nullptr, 0, B, V, d, rlt::kStoreF32, st);
+    }
+    rlt::launch_sample(lbuf, V, B, abuf, sbuf, seed, step, temperature, st);
+    int rc = launch_status();
+    if (rc) return rc;
+    if (logits && !ld &&
+        cudaMemcpyAsync(logits, lbuf, (size_t)B * V * 4, cudaMemcpyDeviceToHost, st))
+        return RLT_E_DEVICE;
+    if (argmax && !ad &&
+        cudaMemcpyAsync(argmax, abuf, (size_t)B * 4, cudaMemcpyDeviceToHost, st))
+        return RLT_E_DEVICE;
+    if (sampled && !sd &&
+        cudaMemcpyAsync(sampled, sbuf, (size_t)B * 4, cudaMemcpyDeviceToHost, st))
+        return RLT_E_DEVICE;
+    return RLT_OK;
+}
+
+// ============================================================================
+// reset, positions, export, errors
+// ============================================================================
+extern "C" int rlt_state_reset(rlt_state* s, const int32_t* rows, int n, void* stream) {
+    if (!s) return RLT_E_ARG;
+    if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (!rows) {
+        rlt::launch_reset_rows(nullptr, s->B, s->m->s_star, s->s, s->Rr, s->pos_enc, s->pos_dec,
+                               s->m->cfg.d, st);
+        std::fill(s->h_pos_enc.begin(), s->h_pos_enc.end(), 0);
+        std::fill(s->h_pos_dec.begin(), s->h_pos_dec.end(), 0);
+        return launch_status();
+    }
+    if (n < 0 || n > s->B) return RLT_E_ARG;
+    for (int i = 0; i < n; ++i)
+        if (rows[i] < 0 || rows[i] >= s->B) return RLT_E_ARG;
+    if (n == 0) return RLT_OK;
+    if (cudaMemcpyAsync(s->rows, rows, (size_t)n * 4, cudaMemcpyHostToDevice, st))
+        return RLT_E_DEVICE;
+    rlt::launch_reset_rows(s->rows, n, s->m->s_star, s->s, s->Rr, s->pos_enc, s->pos_dec,
+                           s->m->cfg.d, st);
+    // the host copy of `rows` may be reused by the caller once the copy is done
+    if (cudaStreamSynchronize(st) != cudaSuccess) return RLT_E_DEVICE;
+    for (int i = 0; i < n; ++i) s->h_pos_enc[rows[i]] = s->h_pos_dec[rows[i]] = 0;
+    return launch_status();
+}
+
+extern "C" int rlt_state_positions(const rlt_state* s, int32_t* pos_enc, int32_t* pos_dec) {
+    if (!s) return RLT_E_ARG;
+    if (pos_enc) memcpy(pos_enc, s->h_pos_enc.data(), (size_t)s->B * 4);
+    if (pos_dec) memcpy(pos_dec, s->h_pos_dec.data(), (size_t)s->B * 4);
+    return RLT_OK;
+}
+
+extern "C" int rlt_state_read(rlt_state* s, int part, void* dst, size_t nbytes,
+                              size_t* nbytes_out, void* stream) {
+    if (!s) return RLT_E_ARG;
+    const void* src = nullptr;
+    size_t sz = 0;
+    const size_t B = s->B, d = s->m->cfg.d, elt = s->m->elt;
+    switch (part) {
+        case RLT_PART_S: src = s->s; sz = B * d * 4; break;
+        case RLT_PART_R: src = s->Rr; sz = B * d * 4; break;
+        case RLT_PART_E: src = s->e; sz = B * s->T_cap * d * 4; break;
+        case RLT_PART_MEM: src = s->mem; sz = B * s->mem_row * elt; break;
+        case RLT_PART_RING: src = s->ring; sz = B * s->ring_row * elt; break;
+        case RLT_PART_ENC: src = s->enc; sz = B * s->enc_row * elt; break;
+        default: return RLT_E_ARG;
+    }
+    if (nbytes_out) *nbytes_out = sz;
+    if (!dst) return RLT_OK;
+    if (nbytes != sz) return RLT_E_ARG;
+    if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    cudaStream_t st = (cudaStream_t)stream;
+    const bool dev = is_device_ptr(dst);
+    if (cudaMemcpyAsync(dst, src, sz, dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
+                        st))
+        return RLT_E_DEVICE;
+    if (!dev && cudaStreamSynchronize(st)) return RLT_E_DEVICE;
+    return RLT_OK;
+}
+
+extern "C" int rlt_state_check(rlt_state* s, void* stream) {
+    if (!s) return RLT_E_ARG;
+    if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RLT_E_DEVICE;
+    int w = 0;
+    if (cudaMemcpy(&w, s->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return RLT_E_DEVICE;
+    if (w != 0 && cudaMemset(s->err, 0, 4) != cudaSuccess) return RLT_E_DEVICE;
+    if (w == rlt::kDevTimeout) return RLT_E_TIMEOUT;
+    if (w == rlt::kDevBounds) return RLT_E_ARG;
+    return w ? RLT_E_DEVICE : RLT_OK;
+}
+
+extern "C" uint64_t rlt_kernel_launches(void) { return g_launches.load(); }
+
+extern "C" int rlt_profile_enable(rlt_state* s, int on) {
+    if (!s) return RLT_E_ARG;
+    if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    if (cudaDeviceSynchronize() != cudaSuccess) return RLT_E_DEVICE;
+    for (auto& r : s->prof_recs) {
+        s->prof_pool.push_back(r.a);
+        s->prof_pool.push_back(r.b);
+    }
+    s->prof_recs.clear();
+    s->prof = on != 0;
+    return RLT_OK;
+}
+
+extern "C" int rlt_profile_query(rlt_state* s, int cls, uint64_t* launches, double* total_ms,
+                                 double* bytes, void* stream) {
+    if (!s || cls < 0 || cls >= RLT_PROF_NCLS) return RLT_E_ARG;
+    if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RLT_E_DEVICE;
+    uint64_t n = 0;
+    double ms = 0, by = 0;
+    for (auto& r : s->prof_recs) {
+        if (r.cls != cls) continue;
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess ||
+            cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+            return RLT_E_DEVICE;
+        ++n;
+        ms += t;
+        by += r.bytes;
+    }
+    if (launches) *launches = n;
+    if (total_ms) *total_ms = ms;
+    if (bytes) *bytes = by;
+    return RLT_OK;
+}
+
+extern "C" const char* rlt_strerror(int code) {
+    switch (code) {
+        case RLT_OK: return "ok";
+        case RLT_E_ARG: return "invalid argument";
+        case RLT_E_OOM: return "out of memory";
+        case RLT_E_CAPACITY: return "position would exceed the state's max_len";
+        case RLT_E_ORDER: return "transition without an encoded token at that position";
+        case RLT_E_BLOB: return "bad weight blob (magic, version, manifest or checksum)";
+        case RLT_E_DEVICE: return "CUDA error";
+        case RLT_E_TIMEOUT: return "bounded device wait gave up";
+        case RLT_E_UNSUPPORTED: return "unsupported configuration";
+        default: return "unknown error";
+    }
+}

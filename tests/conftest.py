@@ -9,3 +9,14 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200) and the built library")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+def build_library():
+    """Compile librlt.so if a source changed (loads build.py by path, so the
+    package -- which loads the library -- is not imported first)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "rlt_build", os.path.join(ROOT, "stateful_decoding_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()

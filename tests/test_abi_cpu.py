@@ -1,0 +1,99 @@
+"""C ABI checks that need no GPU: the library loads, exports every function
+include/rlt.h declares, and rejects bad input on the host before any CUDA work."""
+import ctypes
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+import rlt_inputs as ri
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tests.conftest import build_library
+    build_library()
+    import stateful_decoding_b200 as sd
+    return sd
+
+
+def test_exports_every_declared_function(lib):
+    declared = lib.header_functions()
+    assert "rlt_create" in declared and "rlt_prefill" in declared
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for name in declared:
+        assert hasattr(raw, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l and l.split()[-1].startswith("rlt_")}
+    assert set(declared) <= exported
+
+
+def test_strerror_covers_codes(lib):
+    for code in range(0, -9, -1):
+        assert lib.rlt_strerror(code) != "unknown error"
+    assert lib.rlt_strerror(-99) == "unknown error"
+
+
+def _blob(name="tiny_fp32", **kw):
+    cfg = ri.CONFIGS[name].replace(**kw) if kw else ri.CONFIGS[name]
+    return cfg, ri.write_blob(cfg, ri.generate_weights(cfg))
+
+
+def test_bad_blobs_rejected_before_device(lib):
+    cfg, blob = _blob()
+    assert lib.rlt_create(b"XXXX" + blob[4:])[0] == lib.RLT_E_BLOB
+    assert lib.rlt_create(blob[:100])[0] == lib.RLT_E_BLOB
+    bad = bytearray(blob)
+    bad[300] ^= 0x40                                  # payload byte: checksum mismatch
+    assert lib.rlt_create(bytes(bad))[0] == lib.RLT_E_BLOB
+    bad = bytearray(blob)
+    bad[4] = 2                                        # version
+    assert lib.rlt_create(bytes(bad))[0] == lib.RLT_E_BLOB
+    # a config whose manifest differs from the records (vocab changed in the header)
+    cfg2 = cfg.replace(vocab=33)
+    hdr = ri.write_blob(cfg2, ri.generate_weights(cfg2))[:256]
+    assert lib.rlt_create(hdr + blob[256:])[0] == lib.RLT_E_BLOB
+
+
+def test_valid_blob_without_gpu_reports_device(lib):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    _, blob = _blob()
+    assert lib.rlt_create(blob)[0] == lib.RLT_E_DEVICE
+
+
+def test_null_arguments(lib):
+    assert lib._lib.rlt_create(None, 0, 0, None) == lib.RLT_E_ARG
+    assert lib._lib.rlt_state_create(None, 1, 1, None) == lib.RLT_E_ARG
+    assert lib._lib.rlt_encode(None, None, 1, None) == lib.RLT_E_ARG
+    assert lib._lib.rlt_step(None, None) == lib.RLT_E_ARG
+    assert lib._lib.rlt_prefill(None, 1, None) == lib.RLT_E_ARG
+    assert lib._lib.rlt_readout(None, None, None, None, 0, 0, 1.0, None) == lib.RLT_E_ARG
+    assert lib._lib.rlt_state_check(None, None) == lib.RLT_E_ARG
+    assert lib.rlt_kernel_launches() >= 0
+
+
+def test_package_fails_loudly_without_library(tmp_path):
+    """The product path has no CPU fallback: without librlt.so the import raises."""
+    pkg = tmp_path / "stateful_decoding_b200"
+    pkg.mkdir()
+    src = open(os.path.join(ROOT, "stateful_decoding_b200", "__init__.py")).read()
+    (pkg / "__init__.py").write_text(src)
+    r = subprocess.run([sys.executable, "-c", "import stateful_decoding_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "librlt.so not built" in r.stderr
+
+
+def test_product_package_never_imports_oracle():
+    pkg = os.path.join(ROOT, "stateful_decoding_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in txt.replace("no fallback", ""), f
