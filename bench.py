@@ -183,10 +183,13 @@ def run_ours(args, cfg):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from tests.conftest import build_library
     if rank == 0 or world == 1:
-        build_library()
+        import importlib.util
+        spec = importlib.util.spec_from_file_location(
+            "rlt_build", os.path.join(ROOT, "stateful_decoding_b200", "build.py"))
+        builder = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(builder)
+        builder.build()
     if world > 1:
         dist.barrier()
     import stateful_decoding_b200 as sd
@@ -236,10 +239,12 @@ def run_ours(args, cfg):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier()
+        torch.cuda.nvtx.range_push("timed")
         e0.record(stream)
         for _ in range(args.steps):
             step(toks, logits, ids, am)
         e1.record(stream)
+        torch.cuda.nvtx.range_pop()
         barrier()
     ms_total = e0.elapsed_time(e1)
     launches = sd.rlt_kernel_launches() - launches0

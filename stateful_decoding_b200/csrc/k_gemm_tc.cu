@@ -1,0 +1,221 @@
+// C[M,N] = A[M,K] . W[N,K]^T on the 5th-generation tensor cores (tcgen05),
+// bf16 operands, fp32 accumulation in tensor memory.
+//
+// One CTA computes a 128 x BN tile.  Warp 0 streams K-slices of A and W into
+// a 4-stage shared-memory ring with TMA (128-byte swizzle); one thread of
+// warp 1 issues the MMAs (4 per 64-wide K-slice) and releases each stage with
+// tcgen05.commit; warps 2-5 wait for the final commit, read the accumulator
+// out of TMEM (each warp its 32-lane quarter) and apply the epilogue.  Every
+// wait is bounded: a wait that gives up records a timeout in the device error
+// word, and the CTA still frees its TMEM and exits.
+//
+// Each output element sums its K products in the same order whatever M, N
+// and the tile position, so a row's result does not depend on its batch.
+#include <cuda.h>
+
+#include "kernels.cuh"
+#include "tc_common.cuh"
+
+namespace rlt {
+
+__device__ int g_dev_error;   // sticky: set by kernels that give up a bounded wait
+
+int read_and_clear_device_error() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(int)) != cudaSuccess) return -1;
+    if (v) {
+        int z = 0;
+        cudaMemcpyToSymbol(g_dev_error, &z, sizeof(int));
+    }
+    return v;
+}
+
+namespace {
+
+constexpr int BM = 128, BK = 64, STAGES = 4, NTHREADS = 192;
+
+template <int BN>
+constexpr uint32_t stage_bytes() { return (uint32_t)(BM * BK * 2 + BN * BK * 2); }
+template <int BN>
+constexpr size_t smem_bytes() { return (size_t)STAGES * stage_bytes<BN>() + 1024; }
+
+template <int BN, int MODE>
+__global__ void __launch_bounds__(NTHREADS, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+          float* __restrict__ C, int ldc, bf16* __restrict__ Ct, int ldct, int M, int N, int K) {
+    using namespace tc;
+    constexpr uint32_t A_BYTES = BM * BK * 2, STAGE = stage_bytes<BN>();
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    __shared__ uint64_t full[STAGES], empty[STAGES], accum;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    const int nk = K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&accum, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_map(&ta);
+        prefetch_map(&tb);
+    }
+    if (warp == 1) tmem_alloc(&tmem_base, BN);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int kt = 0; kt < nk; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
+                if (kt >= STAGES && !mbar_wait(&empty[s], ph ^ 1u)) {
+                    abort_flag = 1;
+                    break;
+                }
+                mbar_expect_tx(&full[s], STAGE);
+                tma_load_2d(smem + s * STAGE, &ta, kt * BK, m0, &full[s]);
+                tma_load_2d(smem + s * STAGE + A_BYTES, &tb, kt * BK, n0, &full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(BM, BN);
+            bool ok = true;
+            for (int kt = 0; kt < nk; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
+                if (!mbar_wait(&full[s], ph)) {
+                    abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                fence_after_sync();
+                const uint32_t a = smem_u32(smem + s * STAGE), b = a + A_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    mma_bf16(tmem, sdesc_k_sw128(a + kk * 32), sdesc_k_sw128(b + kk * 32), idesc,
+                             (kt | kk) != 0);
+                mma_commit(&empty[s]);
+            }
+            if (ok) mma_commit(&accum);
+        }
+    } else {
+        if (mbar_wait(&accum, 0)) {
+            fence_after_sync();
+            const int q = warp & 3;
+            const int row = m0 + 32 * q + lane;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 16) {
+                float v[16];
+                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c, v);
+                if (row < M) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int col = n0 + c + j;
+                        if (col < N) {
+                            if (MODE == kStoreF32) C[(size_t)row * ldc + col] = v[j];
+                            else if (MODE == kAddF32) C[(size_t)row * ldc + col] += v[j];
+                            else Ct[(size_t)row * ldct + col] = __float2bfloat16_rn(v[j]);
+                        }
+                    }
+                }
+            }
+        } else {
+            abort_flag = 1;
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, BN);
+    if (threadIdx.x == 0 && abort_flag) atomicExch(&g_dev_error, kDevTimeout);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// 2-D bf16 map over a row-major [rows][cols] matrix with row pitch `ld`
+// elements; box = 64 columns (128 bytes, swizzled) x box_rows rows.
+bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int MODE>
+bool launch_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
+               int ldct, int M, int N, int K, cudaStream_t st) {
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, A, M, K, lda, BM) || !make_map(&tb, W, N, K, ldw, BN)) return false;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem_bytes<BN>()) != cudaSuccess)
+            return false;
+        attr = true;
+    }
+    dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
+    k_gemm_tc<BN, MODE><<<grid, NTHREADS, smem_bytes<BN>(), st>>>(ta, tb, C, ldc, Ct, ldct, M, N,
+                                                                 K);
+    rlt_count_launch();
+    return true;
+}
+
+template <int BN>
+bool launch_tc_mode(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
+                    int ldct, int M, int N, int K, int mode, cudaStream_t st) {
+    if (mode == kStoreF32) return launch_tc<BN, kStoreF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, st);
+    if (mode == kAddF32) return launch_tc<BN, kAddF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, st);
+    return launch_tc<BN, kStoreT>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, st);
+}
+
+}  // namespace
+
+// Returns false (and launches nothing) when the shape or alignment does not
+// suit the tensor-core kernel; the caller then uses the CUDA-core kernel.
+bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
+                    int ldct, int M, int N, int K, int mode, cudaStream_t st) {
+    if (M <= 0 || N < 16 || K < BK || K % BK) return false;
+    if (lda % 8 || ldw % 8 || ((uintptr_t)A & 15) || ((uintptr_t)W & 15)) return false;
+    // wide tiles when M alone fills the machine, narrow ones (more CTAs) otherwise
+    if (M >= 2048) return launch_tc_mode<256>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, st);
+    return launch_tc_mode<64>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, st);
+}
+
+}  // namespace rlt

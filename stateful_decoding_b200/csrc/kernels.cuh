@@ -95,4 +95,6 @@ void launch_attn_cross(const float* Q, const T* mem, size_t row_stride, int T_ca
 void launch_sample(const float* logits, int V, int B, int32_t* argmax, int32_t* sampled,
                    uint64_t seed, uint64_t step, float temperature, cudaStream_t st);
 
+int read_and_clear_device_error();  // device error word of the bounded-wait kernels
+
 }  // namespace rlt

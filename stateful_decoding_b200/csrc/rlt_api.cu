@@ -930,6 +930,9 @@ extern "C" int rlt_state_check(rlt_state* s, void* stream) {
     int w = 0;
     if (cudaMemcpy(&w, s->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return RLT_E_DEVICE;
     if (w != 0 && cudaMemset(s->err, 0, 4) != cudaSuccess) return RLT_E_DEVICE;
+    const int g = rlt::read_and_clear_device_error();
+    if (g < 0) return RLT_E_DEVICE;
+    if (w == 0) w = g;
     if (w == rlt::kDevTimeout) return RLT_E_TIMEOUT;
     if (w == rlt::kDevBounds) return RLT_E_ARG;
     return w ? RLT_E_DEVICE : RLT_OK;

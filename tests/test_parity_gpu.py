@@ -219,6 +219,24 @@ def test_batch_independence_bitexact(sd):
         np.testing.assert_array_equal(l1[0], lbig[r])
 
 
+def test_batch_independence_across_gemm_tiles(sd):
+    """A batch large enough for the wide GEMM tiles (M = 130 x 16 rows) against
+    the same rows run alone (narrow tiles): bit-identical logits."""
+    cfg = ri.CONFIGS["parity_bf16"]
+    B, T = 130, 16
+    W, model, big = make(sd, cfg, B, T)
+    toks = ri.make_tokens(cfg, B, T)
+    big.encode(toks)
+    big.prefill(T)
+    lbig, _, _ = readout_host(big, cfg)
+    for r in (0, 129):
+        one = sd.State(model, 1, T)
+        one.encode(np.ascontiguousarray(toks[r:r + 1]))
+        one.prefill(T)
+        l1, _, _ = readout_host(one, cfg)
+        np.testing.assert_array_equal(l1[0], lbig[r])
+
+
 def test_causality_bitexact(sd):
     """Prop. B.1: tokens after t do not change the state at t."""
     cfg = ri.CONFIGS["parity_bf16"]
