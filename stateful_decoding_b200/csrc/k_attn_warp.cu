@@ -11,9 +11,30 @@
 // result of a row does not depend on the batch.
 #include <math.h>
 
+#include <cstdlib>
+#include <cstring>
+#include <type_traits>
+
 #include "kernels.cuh"
 
 namespace rlt {
+
+bool launch_attn_cross_fast(const float* Q, const bf16* mem, size_t row_stride, int T_cap,
+                            const int32_t* pos_dec, bf16* A, int B, int n, int heads, int dh,
+                            cudaStream_t st);
+bool launch_attn_swa_fast(const float* Q, const bf16* Kc, const bf16* Vc, const bf16* ring,
+                          size_t row_stride, int W, const int32_t* pos_dec, bf16* A, int B, int n,
+                          int heads, int dh, cudaStream_t st);
+
+// RLT_ATTN=warp keeps the decoder on the warp-per-head kernels (diagnostics)
+static bool fast_attn() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("RLT_ATTN");
+        v = (e && strcmp(e, "warp") == 0) ? 0 : 1;
+    }
+    return v == 1;
+}
 
 namespace {
 
@@ -166,6 +187,13 @@ void launch_attn_enc(const float* Q, const T* cache, size_t row_stride, int T_ca
                      cudaStream_t st) {
     int R = B * n;
     if (R <= 0) return;
+    // the encoder's causal attention is the same prefix read as the memory
+    // read: queries at pos_enc+1+i over cache keys 1..t
+    if constexpr (std::is_same<T, bf16>::value) {
+        if (fast_attn() &&
+            launch_attn_cross_fast(Q, cache, row_stride, T_cap, pos_enc, A, B, n, heads, dh, st))
+            return;
+    }
     RLT_DH_SWITCH(dh, (k_attn_enc<T, DH><<<nblocks(R, heads), 128, 0, st>>>(
                           Q, cache, row_stride, T_cap, pos_enc, A, R, n, heads)));
     rlt_count_launch();
@@ -177,6 +205,11 @@ void launch_attn_swa(const float* Q, const T* Kc, const T* Vc, const T* ring, si
                      cudaStream_t st) {
     int R = B * n;
     if (R <= 0) return;
+    if constexpr (std::is_same<T, bf16>::value) {
+        if (fast_attn() &&
+            launch_attn_swa_fast(Q, Kc, Vc, ring, row_stride, W, pos_dec, A, B, n, heads, dh, st))
+            return;
+    }
     RLT_DH_SWITCH(dh, (k_attn_swa<T, DH><<<nblocks(R, heads), 128, 0, st>>>(
                           Q, Kc, Vc, ring, row_stride, W, pos_dec, A, R, n, heads)));
     rlt_count_launch();
@@ -188,6 +221,11 @@ void launch_attn_cross(const float* Q, const T* mem, size_t row_stride, int T_ca
                        cudaStream_t st) {
     int R = B * n;
     if (R <= 0) return;
+    if constexpr (std::is_same<T, bf16>::value) {
+        if (fast_attn() &&
+            launch_attn_cross_fast(Q, mem, row_stride, T_cap, pos_dec, A, B, n, heads, dh, st))
+            return;
+    }
     RLT_DH_SWITCH(dh, (k_attn_cross<T, DH><<<nblocks(R, heads), 128, 0, st>>>(
                           Q, mem, row_stride, T_cap, pos_dec, A, R, n, heads)));
     rlt_count_launch();
