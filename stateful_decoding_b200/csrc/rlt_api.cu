@@ -14,6 +14,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <string>
+#include <map>
 #include <vector>
 
 #include "../../include/rlt.h"
@@ -406,6 +407,9 @@ struct rlt_state {
     struct ProfRec { int cls; cudaEvent_t a, b; double bytes; };
     std::vector<ProfRec> prof_recs;
     std::vector<cudaEvent_t> prof_pool;
+    // replayable transition blocks, per positions-per-block n
+    struct Graph { cudaGraphExec_t exec; uint64_t launches; };
+    std::map<int, Graph> graphs;
 };
 
 static cudaEvent_t prof_event(rlt_state* s) {
@@ -460,6 +464,7 @@ extern "C" void rlt_state_destroy(rlt_state* s) {
         cudaEventDestroy(r.b);
     }
     for (cudaEvent_t e : s->prof_pool) cudaEventDestroy(e);
+    for (auto& g : s->graphs) cudaGraphExecDestroy(g.second.exec);
     for (void* p : s->allocs) cudaFree(p);
     delete s;
 }
@@ -790,6 +795,73 @@ static int run_block(rlt_state* s, int n, cudaStream_t st) {
     return RLT_OK;
 }
 
+// ---------------------------------------------------------------- graphs
+// A transition block reads its positions from the device counters, so the
+// kernels of kGraphBlocks consecutive blocks of n positions form one CUDA
+// graph that serves every later stretch of the prefill: captured once per
+// (state, n), then replayed.  Needs a stream other than the legacy default.
+static constexpr int kGraphBlocks = 16;
+
+static bool graphs_enabled(cudaStream_t st) {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("RLT_GRAPHS");
+        v = (e && strcmp(e, "0") == 0) ? 0 : 1;
+    }
+    return v == 1 && st != nullptr && st != cudaStreamLegacy && st != cudaStreamPerThread;
+}
+
+static int run_graph(rlt_state* s, int n, cudaStream_t st) {
+    const int span = kGraphBlocks * n;
+    for (int b = 0; b < s->B; ++b) {
+        if (s->h_pos_dec[b] + span > s->h_pos_enc[b]) return RLT_E_ORDER;
+        if (s->h_pos_dec[b] + span > s->T_cap) return RLT_E_CAPACITY;
+    }
+    auto it = s->graphs.find(n);
+    if (it == s->graphs.end()) {
+        const bool prof = s->prof;
+        s->prof = false;                  // no event records inside the capture
+        const uint64_t l0 = rlt_kernel_launches();
+        cudaGraph_t g = nullptr;
+        cudaGraphExec_t ex = nullptr;
+        bool ok = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+        if (ok) {
+            for (int k = 0; k < kGraphBlocks; ++k) {
+                if (s->m->cfg.dtype == RLT_DTYPE_BF16) step_block<bf16>(s, n, st);
+                else step_block<float>(s, n, st);
+            }
+            ok = cudaStreamEndCapture(st, &g) == cudaSuccess && g != nullptr;
+        }
+        ok = ok && cudaGraphInstantiate(&ex, g, 0) == cudaSuccess;
+        if (g) cudaGraphDestroy(g);
+        const uint64_t captured = rlt_kernel_launches() - l0;
+        g_launches.fetch_sub(captured);  // captured, not launched
+        s->prof = prof;
+        if (!ok) {
+            cudaGetLastError();
+            if (ex) cudaGraphExecDestroy(ex);
+            return RLT_E_UNSUPPORTED;     // the caller runs the blocks directly
+        }
+        it = s->graphs.emplace(n, rlt_state::Graph{ex, captured}).first;
+    }
+    double by = 0;
+    if (s->prof) {
+        std::vector<int32_t> saved = s->h_pos_dec;
+        for (int k = 0; k < kGraphBlocks; ++k) {
+            by += step_bytes(s, n);
+            for (int b = 0; b < s->B; ++b) s->h_pos_dec[b] += n;
+        }
+        s->h_pos_dec = saved;
+    }
+    {
+        ProfScope ps(s, RLT_PROF_STEP, st, by);
+        if (cudaGraphLaunch(it->second.exec, st) != cudaSuccess) return RLT_E_DEVICE;
+    }
+    rlt_count_launch((int)it->second.launches);
+    for (int b = 0; b < s->B; ++b) s->h_pos_dec[b] += span;
+    return RLT_OK;
+}
+
 extern "C" int rlt_step(rlt_state* s, void* stream) {
     if (!s) return RLT_E_ARG;
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
@@ -804,6 +876,7 @@ extern "C" int rlt_prefill(rlt_state* s, int T, void* stream) {
         if (s->h_pos_dec[b] + T > s->h_pos_enc[b]) return RLT_E_ORDER;
         if (s->h_pos_dec[b] + T > s->T_cap) return RLT_E_CAPACITY;
     }
+    const cudaStream_t st = (cudaStream_t)stream;
     int done = 0;
     while (done < T) {
         const int pd = s->h_pos_dec[0];
@@ -812,7 +885,18 @@ extern "C" int rlt_prefill(rlt_state* s, int T, void* stream) {
         int n = 1;
         if (uniform && c.variant == 2) n = std::min(T - done, c.chunk - pd % c.chunk);
         else if (uniform && c.variant == 0) n = std::min(T - done, s->n_dec_blk);
-        int rc = run_block(s, n, (cudaStream_t)stream);
+        // whole blocks of the regular shape go through a replayed graph
+        const bool regular = c.variant == 1 || (c.variant == 2 && n == c.chunk) ||
+                             (c.variant == 0 && n == s->n_dec_blk);
+        if (regular && graphs_enabled(st) && T - done >= kGraphBlocks * n) {
+            int rc = run_graph(s, n, st);
+            if (rc == RLT_OK) {
+                done += kGraphBlocks * n;
+                continue;
+            }
+            if (rc != RLT_E_UNSUPPORTED) return rc;
+        }
+        int rc = run_block(s, n, st);
         if (rc) return rc;
         done += n;
     }
