@@ -340,8 +340,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the rows per GPU (small profiling cases only)")
+    ap.add_argument("--prompt", type=int, default=None,
+                    help="override the prompt length (small profiling cases only)")
     args = ap.parse_args()
     cfg = ri.CONFIGS[args.config]
+    if args.batch or args.prompt:
+        cfg = cfg.replace(batch=args.batch or cfg.batch, prompt=args.prompt or cfg.prompt)
     if args.impl == "reference":
         run_reference(args, cfg)
     else:
