@@ -207,6 +207,11 @@ bool launch_tc_mode(const bf16* A, int lda, const bf16* W, int ldw, float* C, in
 
 }  // namespace
 
+bool make_tma_2d_bf16(CUtensorMap* map, const void* base, int rows, int cols, int ld,
+                      int box_rows) {
+    return make_map(map, base, rows, cols, ld, box_rows);
+}
+
 // Returns false (and launches nothing) when the shape or alignment does not
 // suit the tensor-core kernel; the caller then uses the CUDA-core kernel.
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,

@@ -18,6 +18,7 @@
 #include <vector>
 
 #include "../../include/rlt.h"
+#include "fused.cuh"
 #include "kernels.cuh"
 
 static std::atomic<uint64_t> g_launches{0};
@@ -186,7 +187,61 @@ struct rlt_model {
     std::vector<DecLayerW> dec;
     float* out_norm = nullptr;
     void* wout = nullptr;
+    // fused transition kernel: usable for this model, and its weight maps
+    bool fused = false;
+    rlt::fz::FusedParams fp{};
 };
+
+// The fused transition kernel runs bf16 RLT-1 models of width 512 with 8
+// heads and a 1365/1408-wide FFN (the d=512 workloads); RLT_FUSED=0 keeps
+// every model on the per-kernel path.
+static void setup_fused(rlt_model* m) {
+    const rlt_config& c = m->cfg;
+    const char* env = getenv("RLT_FUSED");
+    if (env && strcmp(env, "0") == 0) return;
+    namespace fz = rlt::fz;
+    if (c.dtype != RLT_DTYPE_BF16 || c.d != fz::D || c.heads != fz::H || m->fpad != fz::FP ||
+        c.variant != 1 || c.n_dec < 1 || c.window < 1)
+        return;
+    const size_t elt = 2, d = c.d, fp = m->fpad;
+    // every decoder kind must be one contiguous [L * rows][cols] matrix
+    for (int l = 1; l < c.n_dec; ++l) {
+        auto at = [&](void* p0, size_t per) { return (uint8_t*)p0 + l * per; };
+        if (m->dec[l].wqkv != at(m->dec[0].wqkv, 3 * d * d * elt) ||
+            m->dec[l].wo != at(m->dec[0].wo, d * d * elt) ||
+            m->dec[l].xq != at(m->dec[0].xq, d * d * elt) ||
+            m->dec[l].xo != at(m->dec[0].xo, d * d * elt) ||
+            m->dec[l].w13 != at(m->dec[0].w13, 2 * fp * d * elt) ||
+            m->dec[l].w2 != at(m->dec[0].w2, d * fp * elt) ||
+            m->dec[l].swa_norm != m->dec[0].swa_norm + l * d ||
+            m->dec[l].x_norm != m->dec[0].x_norm + l * d ||
+            m->dec[l].ffn_norm != m->dec[0].ffn_norm + l * d)
+            return;
+    }
+    fz::FusedParams& p = m->fp;
+    const int L = c.n_dec;
+    bool ok = rlt::make_tma_2d_bf16(&p.m_qkv, m->dec[0].wqkv, L * 3 * fz::D, fz::D, fz::D, 64) &&
+              rlt::make_tma_2d_bf16(&p.m_o, m->dec[0].wo, L * fz::D, fz::D, fz::D, 64) &&
+              rlt::make_tma_2d_bf16(&p.m_xq, m->dec[0].xq, L * fz::D, fz::D, fz::D, 64) &&
+              rlt::make_tma_2d_bf16(&p.m_xo, m->dec[0].xo, L * fz::D, fz::D, fz::D, 64) &&
+              rlt::make_tma_2d_bf16(&p.m_13, m->dec[0].w13, L * 2 * fz::FP, fz::D, fz::D, 64) &&
+              rlt::make_tma_2d_bf16(&p.m_2, m->dec[0].w2, L * fz::D, fz::FP, fz::FP, 64) &&
+              rlt::make_tma_2d_bf16(&p.m_g, m->wg, fz::D, 2 * fz::D, 2 * fz::D, 64) &&
+              rlt::make_tma_2d_bf16(&p.m_s, m->ws, fz::D, fz::D, fz::D, 64);
+    if (!ok) return;
+    p.g_swa = m->dec[0].swa_norm;
+    p.g_x = m->dec[0].x_norm;
+    p.g_ffn = m->dec[0].ffn_norm;
+    p.g_merge = m->merge_norm;
+    p.bg = m->bg;
+    p.L = L;
+    p.W = c.window;
+    p.G = c.groups;
+    p.variant = c.variant;
+    p.alpha = (float)c.alpha;
+    p.eps = (float)c.eps;
+    m->fused = true;
+}
 
 namespace {
 
@@ -295,17 +350,30 @@ extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model
     m->dec.resize(c.n_dec);
     mat_plain("embed", c.vocab, d, &m->embed);
     if (c.variant != 0) vecf("s_star", &m->s_star);
-    for (int l = 0; l < c.n_dec; ++l) {
-        std::string p = "dec." + std::to_string(l) + ".";
-        DecLayerW& L = m->dec[l];
-        vecf(p + "swa_norm", &L.swa_norm);
-        vecf(p + "x_norm", &L.x_norm);
-        vecf(p + "ffn_norm", &L.ffn_norm);
-        qkv(p, &L.wqkv);
-        mat_plain(p + "wo", d, d, &L.wo);
-        mat_plain(p + "xq", d, d, &L.xq);
-        mat_plain(p + "xo", d, d, &L.xo);
-        ffn(p, &L.w13, &L.w2);
+    // decoder weights kind by kind, so that each kind is one [L_D * rows][cols]
+    // matrix (every per-layer size is a multiple of the 256-byte arena step):
+    // the fused transition kernel addresses all layers through one tensor map
+    auto dec_p = [&](int l) { return "dec." + std::to_string(l) + "."; };
+    for (int l = 0; l < c.n_dec; ++l) vecf(dec_p(l) + "swa_norm", &m->dec[l].swa_norm);
+    for (int l = 0; l < c.n_dec; ++l) vecf(dec_p(l) + "x_norm", &m->dec[l].x_norm);
+    for (int l = 0; l < c.n_dec; ++l) vecf(dec_p(l) + "ffn_norm", &m->dec[l].ffn_norm);
+    for (int l = 0; l < c.n_dec; ++l) qkv(dec_p(l), &m->dec[l].wqkv);
+    for (int l = 0; l < c.n_dec; ++l) mat_plain(dec_p(l) + "wo", d, d, &m->dec[l].wo);
+    for (int l = 0; l < c.n_dec; ++l) mat_plain(dec_p(l) + "xq", d, d, &m->dec[l].xq);
+    for (int l = 0; l < c.n_dec; ++l) mat_plain(dec_p(l) + "xo", d, d, &m->dec[l].xo);
+    {
+        std::vector<void*> w2s(c.n_dec);
+        for (int l = 0; l < c.n_dec; ++l) {
+            size_t o13 = a.take((size_t)2 * fp * d * elt);
+            put_mat(a, o13, elt, src(dec_p(l) + "w1"), c.ffn, d, d, 0);
+            put_mat(a, o13, elt, src(dec_p(l) + "w3"), c.ffn, d, d, fp);
+            fixups.push_back({o13, &m->dec[l].w13});
+        }
+        for (int l = 0; l < c.n_dec; ++l) {
+            size_t o2 = a.take((size_t)d * fp * elt);
+            put_mat(a, o2, elt, src(dec_p(l) + "w2"), d, c.ffn, fp, 0);
+            fixups.push_back({o2, &m->dec[l].w2});
+        }
     }
     for (int l = 0; l < c.n_enc; ++l) {
         std::string p = "enc." + std::to_string(l) + ".";
@@ -362,6 +430,7 @@ extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model
             m->enc[l].w2 = m->dec[l].w2;
         }
     }
+    setup_fused(m);
     *out = m;
     return RLT_OK;
 }
@@ -862,9 +931,47 @@ static int run_graph(rlt_state* s, int n, cudaStream_t st) {
     return RLT_OK;
 }
 
+// nsteps transitions of every row through the fused kernel (one launch).
+static int run_fused(rlt_state* s, int nsteps, cudaStream_t st) {
+    for (int b = 0; b < s->B; ++b) {
+        if (s->h_pos_dec[b] + nsteps > s->h_pos_enc[b]) return RLT_E_ORDER;
+        if (s->h_pos_dec[b] + nsteps > s->T_cap) return RLT_E_CAPACITY;
+    }
+    rlt::fz::FusedParams p = s->m->fp;
+    p.e = s->e;
+    p.s = s->s;
+    p.pos_dec = s->pos_dec;
+    p.err = s->err;
+    p.mem = (const bf16*)s->mem;
+    p.ring = (bf16*)s->ring;
+    p.rope_cs = s->rope_cs;
+    p.rope_sn = s->rope_sn;
+    p.mem_row = s->mem_row;
+    p.ring_row = s->ring_row;
+    p.B = s->B;
+    p.T_cap = s->T_cap;
+    p.nsteps = nsteps;
+    double by = 0;
+    if (s->prof) {
+        std::vector<int32_t> saved = s->h_pos_dec;
+        for (int k = 0; k < nsteps; ++k) {
+            by += step_bytes(s, 1);
+            for (int b = 0; b < s->B; ++b) s->h_pos_dec[b] += 1;
+        }
+        s->h_pos_dec = saved;
+    }
+    {
+        ProfScope ps(s, RLT_PROF_STEP, st, by);
+        if (!rlt::launch_dec_fused(p, st)) return RLT_E_DEVICE;
+    }
+    for (int b = 0; b < s->B; ++b) s->h_pos_dec[b] += nsteps;
+    return RLT_OK;
+}
+
 extern "C" int rlt_step(rlt_state* s, void* stream) {
     if (!s) return RLT_E_ARG;
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    if (s->m->fused) return run_fused(s, 1, (cudaStream_t)stream);
     return run_block(s, 1, (cudaStream_t)stream);
 }
 
@@ -877,6 +984,7 @@ extern "C" int rlt_prefill(rlt_state* s, int T, void* stream) {
         if (s->h_pos_dec[b] + T > s->T_cap) return RLT_E_CAPACITY;
     }
     const cudaStream_t st = (cudaStream_t)stream;
+    if (s->m->fused) return T > 0 ? run_fused(s, T, st) : RLT_OK;
     int done = 0;
     while (done < T) {
         const int pd = s->h_pos_dec[0];
