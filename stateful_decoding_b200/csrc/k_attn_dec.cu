@@ -1,28 +1,45 @@
 // Decoder attention for bf16 storage: the window self-attention over the
 // ring cache C^D and the cross-attention over the memory prefix M_{<=t}
 // (jiphyeonjeon review "Recurrent Looped Transformer" §2-§3.3; greeksharifa
-// §2.5).  Both are HBM streams: each (sequence, head) reads its keys and
-// values once per call.
+// §2.5); also the encoder's causal attention over its cache prefix.  All are
+// HBM streams: each (sequence, head) reads its keys and values once.
 //
-// One CTA per (sequence, head, group of up to NQ query positions).  The keys
-// of the union of the group's windows are split into blocks of 8*KPL keys,
-// dealt round-robin to 4 warps.  Inside a warp, LPK = DH/8 lanes share one
-// key: each lane loads 16 bytes (8 values) of it, so one warp-wide load
-// brings KPL whole keys; a score is a lane-group dot product reduced with
-// shuffles.  Each warp keeps an online softmax per query; the warps' partial
-// (max, sum, output) are merged in shared memory in warp order.  Key order
-// and reduction order depend only on the positions, never on the batch.
+// One CTA per (sequence, head, group of up to NQ query positions), 4 warps.
+// The keys of the group live in one contiguous run per head: the memory or
+// encoder-cache prefix 1..t, or the ring's occupied slots 0..min(pd, W-1)-1.
+// Thread 0 streams the run through a 2-stage shared-memory pipeline with 1-D
+// bulk copies (64 keys of K and of V per stage, completion counted on an
+// mbarrier); each warp scores its quarter of a stage (d_h/8 lanes per key,
+// 16 bytes each), keeps an online softmax per query, and the warps' partial
+// results are merged in warp order at the end.  The window's keys of the
+// current block (at most NQ positions past the ring) are read directly.
+// Key order and every reduction order depend on positions only, so a row's
+// result does not depend on the batch.  Waits are bounded.
 #include <math.h>
 
 #include "kernels.cuh"
+#include "tc_common.cuh"
 
 namespace rlt {
 
+__device__ int g_attn_error;   // sticky: a bounded wait of these kernels gave up
+
+int read_and_clear_attn_error() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_attn_error, sizeof(int)) != cudaSuccess) return -1;
+    if (v) {
+        int z = 0;
+        cudaMemcpyToSymbol(g_attn_error, &z, sizeof(int));
+    }
+    return v;
+}
+
 namespace {
 
-constexpr int NW = 4;   // warps per CTA
+constexpr int NW = 4;      // warps per CTA
+constexpr int CH = 64;     // keys per pipeline stage
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -32,33 +49,107 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
     }
 }
 
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+        : "memory");
+}
+
+template <int DH, int NQ>
+struct Online {             // per-warp online softmax state of NQ queries
+    float m[NQ], l[NQ], acc[NQ][8];
+};
+
+// Score keys (LPK lanes each; key index from `key_of`) and fold them into the
+// state: KPR keys per round, `rounds` rounds, all scores first, then one max /
+// rescale, then the value accumulation.
+template <int DH, int NQ, int ROUNDS, typename KP, typename VP, typename POS>
+__device__ __forceinline__ void fold_keys(Online<DH, NQ>& st, const float (&q)[NQ][8],
+                                          const int (&lo)[NQ], const int (&hi)[NQ], KP kptr,
+                                          VP vptr, POS pos_of, int lane) {
+    constexpr int LPK = DH / 8, KPR = 32 / LPK;
+    const int seg = lane % LPK, grp = lane / LPK;
+    float s[NQ][ROUNDS];
+#pragma unroll
+    for (int rr = 0; rr < ROUNDS; ++rr) {
+        const int kidx = rr * KPR + grp;
+        const int p = pos_of(kidx);            // 0 when the key does not exist
+        float kf[8] = {};
+        if (p > 0) unpack8(*reinterpret_cast<const uint4*>(kptr(kidx) + seg * 8), kf);
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+            float dot = 0.f;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) dot = fmaf(q[i][x], kf[x], dot);
+#pragma unroll
+            for (int o = LPK / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            s[i][rr] = (p > 0 && p >= lo[i] && p <= hi[i]) ? dot : -INFINITY;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) {
+        float bm = s[i][0];
+#pragma unroll
+        for (int rr = 1; rr < ROUNDS; ++rr) bm = fmaxf(bm, s[i][rr]);
+#pragma unroll
+        for (int o = 16; o >= LPK; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+        const float mn = fmaxf(st.m[i], bm);
+        if (mn == -INFINITY) continue;
+        const float corr = (st.m[i] == -INFINITY) ? 0.f : expf(st.m[i] - mn);
+        float ps = 0.f;
+#pragma unroll
+        for (int rr = 0; rr < ROUNDS; ++rr) {
+            s[i][rr] = (s[i][rr] == -INFINITY) ? 0.f : expf(s[i][rr] - mn);
+            ps += s[i][rr];
+        }
+#pragma unroll
+        for (int o = 16; o >= LPK; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        st.l[i] = st.l[i] * corr + ps;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) st.acc[i][x] *= corr;
+        st.m[i] = mn;
+    }
+#pragma unroll
+    for (int rr = 0; rr < ROUNDS; ++rr) {
+        const int kidx = rr * KPR + grp;
+        if (pos_of(kidx) <= 0) continue;
+        float vf[8];
+        unpack8(*reinterpret_cast<const uint4*>(vptr(kidx) + seg * 8), vf);
+#pragma unroll
+        for (int i = 0; i < NQ; ++i)
+#pragma unroll
+            for (int x = 0; x < 8; ++x) st.acc[i][x] = fmaf(s[i][rr], vf[x], st.acc[i][x]);
+    }
+}
+
 template <int DH, int NQ, bool SWA>
 __global__ void __launch_bounds__(NW * 32)
-k_attn_dec(const float* __restrict__ Q, const bf16* __restrict__ base, size_t row_stride,
-           int span,                          // cross: T_cap; window: W-1 ring slots
-           const bf16* __restrict__ Kc, const bf16* __restrict__ Vc,
-           const int32_t* __restrict__ pos_dec, int W, bf16* __restrict__ A, int n, int heads) {
-    constexpr int LPK = DH / 8;          // lanes per key
-    constexpr int KPL = 32 / LPK;        // keys per warp-wide load
-    constexpr int BLK = 8 * KPL;         // keys per block (8 loads per lane)
+k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t row_stride,
+              int span, const bf16* __restrict__ Kc, const bf16* __restrict__ Vc,
+              const int32_t* __restrict__ pos, int W, bf16* __restrict__ A, int n, int heads) {
+    int* err = &g_attn_error;
+    constexpr int LPK = DH / 8, KPR = 32 / LPK;
+    constexpr int WK = CH / NW;                 // keys per warp per stage
+    constexpr int ROUNDS = WK / KPR;
+    constexpr uint32_t STAGE_BYTES = CH * DH * 2;
+    extern __shared__ __align__(128) uint8_t smem[];
+    bf16* sK = reinterpret_cast<bf16*>(smem);                  // [2][CH][DH]
+    bf16* sV = reinterpret_cast<bf16*>(smem + 2 * STAGE_BYTES);
+    __shared__ uint64_t full[2], empty[2];
     __shared__ float s_m[NW][NQ], s_l[NW][NQ];
     __shared__ float s_o[NW][NQ][DH];
+    __shared__ int s_abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.x, b = bh / heads, h = bh % heads;
     const int q0 = blockIdx.y * NQ;
     const int nq = min(NQ, n - q0);
     const int d = heads * DH;
-    const int pd = pos_dec[b];
-    const int seg = lane % LPK, grp = lane / LPK;
+    const int pd = pos[b];
+    const int seg = lane % LPK;
 
-    // key sources
-    const bf16* kb = base + (size_t)b * row_stride + (size_t)h * span * DH;
-    const bf16* vb = kb + (size_t)heads * span * DH;
-    const bf16* ck = Kc + (size_t)b * n * d + h * DH;
-    const bf16* cv = Vc + (size_t)b * n * d + h * DH;
-
-    // query windows: query i at t_i = pd + 1 + q0 + i
     int lo[NQ], hi[NQ];
     float q[NQ][8];
     const float sc = 1.0f / sqrtf((float)DH);
@@ -71,106 +162,101 @@ k_attn_dec(const float* __restrict__ Q, const bf16* __restrict__ base, size_t ro
 #pragma unroll
         for (int x = 0; x < 8; ++x) q[i][x] = qp[x] * sc;
     }
-    const int u_lo = lo[0], u_hi = hi[nq - 1];     // union of the windows
-    const int nkeys = u_hi - u_lo + 1;
 
-    auto kaddr = [&](int p, bool val) -> const bf16* {
-        if (!SWA) return (val ? vb : kb) + (size_t)(p - 1) * DH;
-        if (p <= pd) return (val ? vb : kb) + (size_t)((p - 1) % span) * DH;
-        return (val ? cv : ck) + (size_t)(p - pd - 1) * d;
+    // the contiguous run: prefix 1..t_last, or the occupied ring slots
+    const bf16* kg = base + (size_t)b * row_stride + (size_t)h * span * DH;
+    const bf16* vg = kg + (size_t)heads * span * DH;
+    const int nreg = SWA ? (W > 1 ? min(pd, span) : 0) : hi[nq - 1];
+    const int nch = (nreg + CH - 1) / CH;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&full[0], 1);
+        tc::mbar_init(&full[1], 1);
+        tc::mbar_init(&empty[0], NW);
+        tc::mbar_init(&empty[1], NW);
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    auto issue = [&](int c) {
+        const int st = c & 1, k0 = c * CH, cnt = min(CH, nreg - k0);
+        const uint32_t bytes = (uint32_t)cnt * DH * 2;
+        tc::mbar_expect_tx(&full[st], 2 * bytes);
+        bulk_load(sK + (size_t)st * CH * DH, kg + (size_t)k0 * DH, bytes, &full[st]);
+        bulk_load(sV + (size_t)st * CH * DH, vg + (size_t)k0 * DH, bytes, &full[st]);
     };
+    if (threadIdx.x == 0 && nch > 0) issue(0);
 
-    float m[NQ], l[NQ], acc[NQ][8];
+    Online<DH, NQ> os;
 #pragma unroll
     for (int i = 0; i < NQ; ++i) {
-        m[i] = -INFINITY;
-        l[i] = 0.f;
+        os.m[i] = -INFINITY;
+        os.l[i] = 0.f;
 #pragma unroll
-        for (int x = 0; x < 8; ++x) acc[i][x] = 0.f;
+        for (int x = 0; x < 8; ++x) os.acc[i][x] = 0.f;
     }
-
-    for (int blk = warp; blk * BLK < nkeys; blk += NW) {
-        const int p0 = u_lo + blk * BLK;
-        uint4 kr[8], vr[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int p = p0 + j * KPL + grp;
-            if (p <= u_hi) {
-                kr[j] = *reinterpret_cast<const uint4*>(kaddr(p, false) + seg * 8);
-                vr[j] = *reinterpret_cast<const uint4*>(kaddr(p, true) + seg * 8);
+    for (int c = 0; c < nch; ++c) {
+        const int st = c & 1;
+        if (threadIdx.x == 0 && c + 1 < nch) {
+            // stage (c+1)&1 was read by chunk c-1: every warp must be done with it
+            if (c >= 1 && !tc::mbar_wait(&empty[(c + 1) & 1], (uint32_t)((c - 1) >> 1) & 1u)) {
+                s_abort = 1;
+                atomicExch(err, kDevTimeout);
             } else {
-                kr[j] = make_uint4(0, 0, 0, 0);
-                vr[j] = make_uint4(0, 0, 0, 0);
+                issue(c + 1);
             }
         }
-        float s[NQ][8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float kf[8];
-            bf16x8_to_f32(kr[j], kf);
-            const int p = p0 + j * KPL + grp;
-#pragma unroll
-            for (int i = 0; i < NQ; ++i) {
-                float dot = 0.f;
-#pragma unroll
-                for (int x = 0; x < 8; ++x) dot = fmaf(q[i][x], kf[x], dot);
-#pragma unroll
-                for (int o = LPK / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-                s[i][j] = (p >= lo[i] && p <= hi[i]) ? dot : -INFINITY;
-            }
+        if (!tc::mbar_wait(&full[st], (uint32_t)(c >> 1) & 1u)) {
+            s_abort = 1;
+            atomicExch(err, kDevTimeout);
+            break;
         }
-#pragma unroll
-        for (int i = 0; i < NQ; ++i) {
-            float bm = s[i][0];
-#pragma unroll
-            for (int j = 1; j < 8; ++j) bm = fmaxf(bm, s[i][j]);
-#pragma unroll
-            for (int o = 16; o >= LPK; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-            const float mn = fmaxf(m[i], bm);
-            if (mn == -INFINITY) continue;          // nothing of this query in the block yet
-            const float corr = (m[i] == -INFINITY) ? 0.f : expf(m[i] - mn);
-            float ps = 0.f, pj[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                pj[j] = (s[i][j] == -INFINITY) ? 0.f : expf(s[i][j] - mn);
-                ps += pj[j];
-            }
-#pragma unroll
-            for (int o = 16; o >= LPK; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-            l[i] = l[i] * corr + ps;
-#pragma unroll
-            for (int x = 0; x < 8; ++x) acc[i][x] *= corr;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float vf[8];
-                bf16x8_to_f32(vr[j], vf);
-#pragma unroll
-                for (int x = 0; x < 8; ++x) acc[i][x] = fmaf(pj[j], vf[x], acc[i][x]);
-            }
-            m[i] = mn;
+        const int k0 = c * CH + warp * WK;     // this warp's first key (index in the run)
+        const bf16* sk = sK + (size_t)st * CH * DH + (size_t)warp * WK * DH;
+        const bf16* sv = sV + (size_t)st * CH * DH + (size_t)warp * WK * DH;
+        auto pos_of = [&](int kidx) -> int {
+            const int j = k0 + kidx;
+            if (j >= nreg) return 0;
+            if (!SWA) return j + 1;
+            return pd - ((pd - 1 - j) % span);   // ring slot j holds this position
+        };
+        fold_keys<DH, NQ, ROUNDS>(os, q, lo, hi, [&](int kidx) { return sk + (size_t)kidx * DH; },
+                                  [&](int kidx) { return sv + (size_t)kidx * DH; }, pos_of, lane);
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&empty[st]);
+        if (s_abort) break;
+    }
+    if (SWA && warp == 0) {   // the block's own positions pd+1 .. pd+q0+nq (this layer's k, v)
+        const bf16* ck = Kc + (size_t)b * n * d + h * DH;
+        const bf16* cv = Vc + (size_t)b * n * d + h * DH;
+        const int nown = q0 + nq;
+        for (int e0 = 0; e0 < nown; e0 += KPR) {
+            fold_keys<DH, NQ, 1>(
+                os, q, lo, hi, [&](int kidx) { return ck + (size_t)(e0 + kidx) * d; },
+                [&](int kidx) { return cv + (size_t)(e0 + kidx) * d; },
+                [&](int kidx) -> int { return e0 + kidx < nown ? pd + 1 + e0 + kidx : 0; }, lane);
         }
     }
-    // reduce the partial outputs over the key groups of the warp
+    // reduce over the key groups of the warp, then merge the warps in order
 #pragma unroll
     for (int i = 0; i < NQ; ++i)
 #pragma unroll
         for (int x = 0; x < 8; ++x)
 #pragma unroll
             for (int o = 16; o >= LPK; o >>= 1)
-                acc[i][x] += __shfl_xor_sync(0xffffffffu, acc[i][x], o);
+                os.acc[i][x] += __shfl_xor_sync(0xffffffffu, os.acc[i][x], o);
     if (lane < LPK) {
 #pragma unroll
         for (int i = 0; i < NQ; ++i) {
 #pragma unroll
-            for (int x = 0; x < 8; ++x) s_o[warp][i][seg * 8 + x] = acc[i][x];
+            for (int x = 0; x < 8; ++x) s_o[warp][i][seg * 8 + x] = os.acc[i][x];
             if (lane == 0) {
-                s_m[warp][i] = m[i];
-                s_l[warp][i] = l[i];
+                s_m[warp][i] = os.m[i];
+                s_l[warp][i] = os.l[i];
             }
         }
     }
     __syncthreads();
-    // merge the warps in order; thread x of the CTA owns output dim x of each query
     for (int e = threadIdx.x; e < nq * DH; e += NW * 32) {
         const int i = e / DH, x = e % DH;
         float M = -INFINITY;
@@ -187,44 +273,56 @@ k_attn_dec(const float* __restrict__ Q, const bf16* __restrict__ base, size_t ro
 }
 
 template <int DH, bool SWA>
-void launch_dec(const float* Q, const bf16* base, size_t row_stride, int span, const bf16* Kc,
-                const bf16* Vc, const int32_t* pos_dec, int W, bf16* A, int B, int n, int heads,
-                cudaStream_t st) {
-    if (n == 1) {
-        k_attn_dec<DH, 1, SWA><<<dim3(B * heads, 1), NW * 32, 0, st>>>(
-            Q, base, row_stride, span, Kc, Vc, pos_dec, W, A, n, heads);
-    } else if (n == 2) {
-        k_attn_dec<DH, 2, SWA><<<dim3(B * heads, 1), NW * 32, 0, st>>>(
-            Q, base, row_stride, span, Kc, Vc, pos_dec, W, A, n, heads);
-    } else {
-        k_attn_dec<DH, 4, SWA><<<dim3(B * heads, (n + 3) / 4), NW * 32, 0, st>>>(
-            Q, base, row_stride, span, Kc, Vc, pos_dec, W, A, n, heads);
-    }
-    rlt_count_launch();
+bool launch_stream(const float* Q, const bf16* base, size_t row_stride, int span, const bf16* Kc,
+                   const bf16* Vc, const int32_t* pos, int W, bf16* A, int B, int n, int heads,
+                   cudaStream_t st) {
+    const size_t smem = 4 * (size_t)CH * DH * 2;
+    auto go = [&](auto kernel, int nqg) {
+        static bool attr = false;
+        if (!attr) {
+            if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem) != cudaSuccess)
+                return false;
+            attr = true;
+        }
+        kernel<<<dim3(B * heads, (n + nqg - 1) / nqg), NW * 32, smem, st>>>(
+            Q, base, row_stride, span, Kc, Vc, pos, W, A, n, heads);
+        rlt_count_launch();
+        return true;
+    };
+    if (n == 1) return go(k_attn_stream<DH, 1, SWA>, 1);
+    if (n == 2) return go(k_attn_stream<DH, 2, SWA>, 2);
+    return go(k_attn_stream<DH, 4, SWA>, 4);
 }
 
 }  // namespace
 
-// bf16 decoder attention with head size 64 or 128; returns false otherwise.
+// bf16 attention with head size 64 or 128; returns false otherwise.
 bool launch_attn_cross_fast(const float* Q, const bf16* mem, size_t row_stride, int T_cap,
-                            const int32_t* pos_dec, bf16* A, int B, int n, int heads, int dh,
+                            const int32_t* pos, bf16* A, int B, int n, int heads, int dh,
                             cudaStream_t st) {
     if (B * n <= 0) return true;
-    if (dh == 64) launch_dec<64, false>(Q, mem, row_stride, T_cap, nullptr, nullptr, pos_dec, 0, A, B, n, heads, st);
-    else if (dh == 128) launch_dec<128, false>(Q, mem, row_stride, T_cap, nullptr, nullptr, pos_dec, 0, A, B, n, heads, st);
-    else return false;
-    return true;
+    if (dh == 64)
+        return launch_stream<64, false>(Q, mem, row_stride, T_cap, nullptr, nullptr, pos, 0, A, B,
+                                        n, heads, st);
+    if (dh == 128)
+        return launch_stream<128, false>(Q, mem, row_stride, T_cap, nullptr, nullptr, pos, 0, A,
+                                         B, n, heads, st);
+    return false;
 }
 
 bool launch_attn_swa_fast(const float* Q, const bf16* Kc, const bf16* Vc, const bf16* ring,
-                          size_t row_stride, int W, const int32_t* pos_dec, bf16* A, int B, int n,
+                          size_t row_stride, int W, const int32_t* pos, bf16* A, int B, int n,
                           int heads, int dh, cudaStream_t st) {
     if (B * n <= 0) return true;
     const int slots = W > 1 ? W - 1 : 1;
-    if (dh == 64) launch_dec<64, true>(Q, ring, row_stride, slots, Kc, Vc, pos_dec, W, A, B, n, heads, st);
-    else if (dh == 128) launch_dec<128, true>(Q, ring, row_stride, slots, Kc, Vc, pos_dec, W, A, B, n, heads, st);
-    else return false;
-    return true;
+    if (dh == 64)
+        return launch_stream<64, true>(Q, ring, row_stride, slots, Kc, Vc, pos, W, A, B, n, heads,
+                                       st);
+    if (dh == 128)
+        return launch_stream<128, true>(Q, ring, row_stride, slots, Kc, Vc, pos, W, A, B, n,
+                                        heads, st);
+    return false;
 }
 
 }  // namespace rlt

@@ -175,6 +175,16 @@ __device__ __forceinline__ TileRef tile_of(const FusedParams& P, int kind, int l
     return r;
 }
 
+// One accumulator per tile.  (Measured on B200: spreading a tile's K range
+// over several partial accumulators, or interleaving tiles chunk by chunk,
+// made the MMA issue slower, not faster; so did releasing weight slots in
+// batches.  A 64-wide K chunk costs ~0.4 us of issue time at N = 16.)
+__device__ __forceinline__ int nsplit(int) { return 1; }
+__device__ __forceinline__ int kfirst(int kind, int t) { return (kind == J_MERGE && t == 1) ? 8 : 0; }
+__device__ __forceinline__ int nch_max(int kind, int c) {
+    return kind == J_MERGE ? 2 * D / 64 : (kind == J_W2 ? nhid(c) : D / 64);
+}
+
 __device__ __forceinline__ int njobs(const FusedParams& P) { return 1 + 6 * P.L; }
 __device__ __forceinline__ void job_kind(int j, int& kind, int& l) {
     if (j == 0) { kind = J_MERGE; l = 0; }
@@ -371,6 +381,20 @@ __device__ __forceinline__ void attend_row(const float* q_s, const bf16* kb, con
     for (int x = 0; x < 8; ++x) out[x] = acc[x] * inv;
 }
 
+// Tile t's accumulator for this warp's lane quarter: the sum, in order, of
+// its ns partial accumulators (TMEM columns (t*ns + s) * 16).
+__device__ __forceinline__ void acc_sum(uint32_t tmem, int quarter, int t, int ns,
+                                        float (&v)[16]) {
+    const uint32_t base = tmem + ((uint32_t)(32 * quarter) << 16);
+    tmem_ld16(base + (uint32_t)(t * ns * RB), v);
+    for (int s = 1; s < ns; ++s) {
+        float w[16];
+        tmem_ld16(base + (uint32_t)((t * ns + s) * RB), w);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] += w[i];
+    }
+}
+
 // ---------------------------------------------------------------- the kernel
 __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 1)
 k_dec_fused(const __grid_constant__ FusedParams P) {
@@ -429,17 +453,17 @@ k_dec_fused(const __grid_constant__ FusedParams P) {
                     int kind, l;
                     job_kind(j, kind, l);
                     const int nt = ntiles(kind, c);
-                    for (int t = 0; t < nt && !ctl.abort; ++t) {
-                        const TileRef tr = tile_of(P, kind, l, t, c);
-                        for (int k = 0; k < tr.nch; ++k, ++ld) {
+                    for (int t = 0; t < nt && !ctl.abort; ++t)
+                        for (int kl = 0; kl < tile_of(P, kind, l, t, c).nch && !ctl.abort; ++kl) {
+                            const TileRef tr = tile_of(P, kind, l, t, c);
                             const int s = ld % NSLOT;
                             const uint32_t ph = (ld / NSLOT) & 1u;
                             if (ld >= NSLOT && !waitb(&ctl.empty[s], ph ^ 1u, &ctl, P.err)) break;
                             mbar_expect_tx(&ctl.full[s], SLOT);
-                            tma_load_2d(stage + s * SLOT, tr.map, tr.kx0 + k * tr.kstep, tr.row,
+                            tma_load_2d(stage + s * SLOT, tr.map, tr.kx0 + kl * tr.kstep, tr.row,
                                         &ctl.full[s]);
+                            ++ld;
                         }
-                    }
                 }
         }
     } else if (warp == 1) {
@@ -453,24 +477,38 @@ k_dec_fused(const __grid_constant__ FusedParams P) {
                     job_kind(j, kind, l);
                     if (!waitb(&ctl.op_full, job & 1u, &ctl, P.err)) continue;
                     fence_after_sync();
-                    const int nt = ntiles(kind, c);
+                    const int nt = ntiles(kind, c), nk = nch_max(kind, c), ns = nsplit(kind);
+                    (void)nk;
+                    // slot releases are batched: a commit per consumed box costs a
+                    // pipe round trip, so up to kBatch boxes are released together
+                    constexpr int kBatch = 1;
+                    int pend[kBatch], np = 0;
                     for (int t = 0; t < nt; ++t) {
                         const TileRef tr = tile_of(P, kind, l, t, c);
-                        for (int k = 0; k < tr.nch; ++k, ++ld) {
+                        for (int kl = 0; kl < tr.nch; ++kl) {
                             const int s = ld % NSLOT;
                             const uint32_t ph = (ld / NSLOT) & 1u;
+                            ++ld;
+                            // TMA data is ordered by the barrier's transaction count:
+                            // no tcgen05 fence is needed between the wait and the MMA
                             if (!waitb(&ctl.full[s], ph, &ctl, P.err)) continue;
-                            fence_after_sync();
                             const uint32_t a = smem_u32(stage + s * SLOT);
-                            const uint32_t b =
-                                smem_u32((tr.hid ? hidb : opnd) + (tr.op0 + k) * CHUNK_BYTES);
+                            const uint32_t bsm =
+                                smem_u32((tr.hid ? hidb : opnd) + (tr.op0 + kl) * CHUNK_BYTES);
+                            const uint32_t col = (uint32_t)((t * ns + kl % ns) * RB);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
-                                mma_bf16(tmem + (uint32_t)(t * RB), sdesc_k_sw128(a + kk * 32),
-                                         sdesc_k_sw128(b + kk * 32), idesc, (k | kk) != 0);
-                            mma_commit(&ctl.empty[s]);
+                                mma_bf16(tmem + col, sdesc_k_sw128(a + kk * 32),
+                                         sdesc_k_sw128(bsm + kk * 32), idesc,
+                                         (kl < ns && kk == 0) ? 0u : 1u);
+                            pend[np++] = s;
+                            if (np == kBatch) {
+                                for (int i = 0; i < kBatch; ++i) mma_commit(&ctl.empty[pend[i]]);
+                                np = 0;
+                            }
                         }
                     }
+                    for (int i = 0; i < np; ++i) mma_commit(&ctl.empty[pend[i]]);
                     mma_commit(&ctl.acc_full);
                 }
         }
@@ -548,8 +586,8 @@ k_dec_fused(const __grid_constant__ FusedParams P) {
                 wait_acc();
                 if (epi_a) {
                     float g[16], w[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16) + 0, g);
-                    tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16) + RB, w);
+                    acc_sum(tmem, quarter, 0, nsplit(J_MERGE), g);
+                    acc_sum(tmem, quarter, 1, nsplit(J_MERGE), w);
                     const float bgf = P.bg[c * 64 + f_epi];
 #pragma unroll
                     for (int rr = 0; rr < RB; ++rr) {
@@ -578,14 +616,14 @@ k_dec_fused(const __grid_constant__ FusedParams P) {
                     float v[16];
                     // pair a: tiles 0 (q) and 2 (v); pair b: tile 1 (k)
                     if (epi_a) {
-                        tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16) + 0, v);
+                        acc_sum(tmem, quarter, 0, nsplit(J_QKV), v);
 #pragma unroll
                         for (int rr = 0; rr < RB; ++rr) qs[rr * 64 + f_epi] = v[rr];
-                        tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16) + 2 * RB, v);
+                        acc_sum(tmem, quarter, 2, nsplit(J_QKV), v);
 #pragma unroll
                         for (int rr = 0; rr < RB; ++rr) vs[rr * 64 + f_epi] = bf16r(v[rr]);
                     } else {
-                        tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16) + RB, v);
+                        acc_sum(tmem, quarter, 1, nsplit(J_QKV), v);
 #pragma unroll
                         for (int rr = 0; rr < RB; ++rr) ks[rr * 64 + f_epi] = v[rr];
                     }
@@ -652,7 +690,7 @@ k_dec_fused(const __grid_constant__ FusedParams P) {
                 wait_acc();
                 if (epi_a) {
                     float v[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16), v);
+                    acc_sum(tmem, quarter, 0, nsplit(J_WO), v);
 #pragma unroll
                     for (int rr = 0; rr < RB; ++rr) zs[rr * 64 + f_epi] += v[rr];
                 }
@@ -666,7 +704,7 @@ k_dec_fused(const __grid_constant__ FusedParams P) {
                 wait_acc();
                 if (epi_a) {
                     float v[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16), v);
+                    acc_sum(tmem, quarter, 0, nsplit(J_WO), v);
 #pragma unroll
                     for (int rr = 0; rr < RB; ++rr) qs[rr * 64 + f_epi] = v[rr];
                 }
@@ -715,7 +753,7 @@ k_dec_fused(const __grid_constant__ FusedParams P) {
                 wait_acc();
                 if (epi_a) {
                     float v[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16), v);
+                    acc_sum(tmem, quarter, 0, nsplit(J_WO), v);
 #pragma unroll
                     for (int rr = 0; rr < RB; ++rr) zs[rr * 64 + f_epi] += v[rr];
                 }

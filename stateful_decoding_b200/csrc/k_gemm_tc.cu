@@ -100,7 +100,6 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                     ok = false;
                     break;
                 }
-                fence_after_sync();
                 const uint32_t a = smem_u32(smem + s * STAGE), b = a + A_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)

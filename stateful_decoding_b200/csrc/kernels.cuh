@@ -96,5 +96,6 @@ void launch_sample(const float* logits, int V, int B, int32_t* argmax, int32_t* 
                    uint64_t seed, uint64_t step, float temperature, cudaStream_t st);
 
 int read_and_clear_device_error();  // device error word of the bounded-wait kernels
+int read_and_clear_attn_error();    // same, for the streaming attention kernels
 
 }  // namespace rlt

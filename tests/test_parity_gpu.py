@@ -154,6 +154,27 @@ def test_large_config_slice(sd):
     run_stepwise_and_compare(sd, cfg, 2, 12, n_decode=2)
 
 
+def test_fused_transition_kernel(sd, monkeypatch):
+    """The opt-in fused cluster kernel (RLT_FUSED=1) against the oracle on a
+    ragged batch (20 rows: one full and one partial 16-row cluster), stepwise
+    and through one prefill launch."""
+    monkeypatch.setenv("RLT_FUSED", "1")
+    cfg = ri.CONFIGS["parity_bf16"]
+    run_stepwise_and_compare(sd, cfg, 20, 21, n_decode=1)
+    B, T = 20, 33
+    W, model, st = make(sd, cfg, B, T)
+    toks = ri.make_tokens(cfg, B, T)
+    st.encode(toks)
+    st.prefill(T)
+    lg, _, _ = readout_host(st, cfg)
+    orc = RLTOracle(cfg, W, "bf16")
+    for b in (0, 17, 19):
+        r = orc.new_state()
+        orc.encode(r, toks[b])
+        orc.prefill(r, T)
+        assert np.max(np.abs(lg[b] - orc.readout(r))) <= 3e-2
+
+
 def test_full_size_bench_config_sampled_rows(sd):
     """parity_bf16 at its full size (256 rows x 256) in the bench's launch
     configuration (one encode call, one prefill call); rows 0, 131 and 255
