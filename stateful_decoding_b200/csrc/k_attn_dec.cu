@@ -272,27 +272,36 @@ k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t
     }
 }
 
+// One launcher per kernel instance, so that each instance gets its own
+// shared-memory attribute (the instances share a function-pointer type).
+template <int DH, int NQ, bool SWA>
+bool launch_one(const float* Q, const bf16* base, size_t row_stride, int span, const bf16* Kc,
+                const bf16* Vc, const int32_t* pos, int W, bf16* A, int B, int n, int heads,
+                cudaStream_t st) {
+    constexpr size_t smem = 4 * (size_t)CH * DH * 2;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(k_attn_stream<DH, NQ, SWA>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return false;
+        attr = true;
+    }
+    k_attn_stream<DH, NQ, SWA><<<dim3(B * heads, (n + NQ - 1) / NQ), NW * 32, smem, st>>>(
+        Q, base, row_stride, span, Kc, Vc, pos, W, A, n, heads);
+    rlt_count_launch();
+    return true;
+}
+
 template <int DH, bool SWA>
 bool launch_stream(const float* Q, const bf16* base, size_t row_stride, int span, const bf16* Kc,
                    const bf16* Vc, const int32_t* pos, int W, bf16* A, int B, int n, int heads,
                    cudaStream_t st) {
-    const size_t smem = 4 * (size_t)CH * DH * 2;
-    auto go = [&](auto kernel, int nqg) {
-        static bool attr = false;
-        if (!attr) {
-            if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)smem) != cudaSuccess)
-                return false;
-            attr = true;
-        }
-        kernel<<<dim3(B * heads, (n + nqg - 1) / nqg), NW * 32, smem, st>>>(
-            Q, base, row_stride, span, Kc, Vc, pos, W, A, n, heads);
-        rlt_count_launch();
-        return true;
-    };
-    if (n == 1) return go(k_attn_stream<DH, 1, SWA>, 1);
-    if (n == 2) return go(k_attn_stream<DH, 2, SWA>, 2);
-    return go(k_attn_stream<DH, 4, SWA>, 4);
+    if (n == 1)
+        return launch_one<DH, 1, SWA>(Q, base, row_stride, span, Kc, Vc, pos, W, A, B, n, heads, st);
+    if (n == 2)
+        return launch_one<DH, 2, SWA>(Q, base, row_stride, span, Kc, Vc, pos, W, A, B, n, heads, st);
+    return launch_one<DH, 4, SWA>(Q, base, row_stride, span, Kc, Vc, pos, W, A, B, n, heads, st);
 }
 
 }  // namespace
