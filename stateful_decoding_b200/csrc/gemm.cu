@@ -10,7 +10,8 @@
 namespace rlt {
 
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
-                    int ldct, int M, int N, int K, int mode, cudaStream_t st);
+                    int ldct, int M, int N, int K, int mode, int splits, size_t slab,
+                    cudaStream_t st);
 
 static bool tc_enabled() {
     static int v = -1;
@@ -30,9 +31,34 @@ void launch_gemm<float>(const float* A, int lda, const float* W, int ldw, float*
 template <>
 void launch_gemm<bf16>(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc,
                        bf16* Ct, int ldct, int M, int N, int K, int mode, cudaStream_t st) {
-    if (tc_enabled() && launch_gemm_tc(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, st))
+    if (tc_enabled() && launch_gemm_tc(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, 1, 0, st))
         return;
     launch_gemm_simt<bf16>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, st);
+}
+
+// Split-K partial sums: with `splits` > 1, slab z = C + z*slab holds the sum
+// over the z-th run of K-chunks; the consumer adds the slabs in order.  The
+// split count must depend on N and K only, never on M, so that a row's result
+// does not depend on its batch.  Returns the number of slabs written.
+template <>
+int launch_gemm_split<float>(const float* A, int lda, const float* W, int ldw, float* C, int ldc,
+                             int M, int N, int K, int splits, size_t slab, cudaStream_t st) {
+    (void)splits;
+    (void)slab;
+    launch_gemm_simt<float>(A, lda, W, ldw, C, ldc, nullptr, 0, M, N, K, kStoreF32, st);
+    return 1;
+}
+
+template <>
+int launch_gemm_split<bf16>(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc,
+                            int M, int N, int K, int splits, size_t slab, cudaStream_t st) {
+    if (tc_enabled() && splits > 1 && K % 64 == 0) {
+        const int nk = K / 64, cps = (nk + splits - 1) / splits, s = (nk + cps - 1) / cps;
+        if (launch_gemm_tc(A, lda, W, ldw, C, ldc, nullptr, 0, M, N, K, kStoreF32, s, slab, st))
+            return s;
+    }
+    launch_gemm<bf16>(A, lda, W, ldw, C, ldc, nullptr, 0, M, N, K, kStoreF32, st);
+    return 1;
 }
 
 }  // namespace rlt

@@ -6,6 +6,14 @@
 
 namespace rlt {
 
+// Sum of S split-K partial slabs (slab z at P + z*slab), in slab order.
+__device__ __forceinline__ float slab_sum(const float* __restrict__ P, int S, size_t slab,
+                                          size_t i) {
+    float v = P[i];
+    for (int z = 1; z < S; ++z) v += P[(size_t)z * slab + i];
+    return v;
+}
+
 // ---------------------------------------------------------------- embedding
 template <typename T>
 __global__ void k_embed(const T* __restrict__ E, const int32_t* __restrict__ tok,
@@ -64,6 +72,35 @@ void launch_rmsnorm(const float* X, int ldx, const float* gain, T* Y, int ldy, i
     rlt_count_launch();
 }
 
+// z += sum of the residual partial slabs P (if any), then Y = RMSNorm(z).
+template <typename T>
+__global__ void k_add_rmsnorm(float* __restrict__ Z, const float* __restrict__ P, int S,
+                              size_t slab, const float* __restrict__ g, T* __restrict__ Y, int d,
+                              float eps) {
+    __shared__ float red[33];
+    float* z = Z + (size_t)blockIdx.x * d;
+    float ss = 0.f;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        float v = z[j];
+        if (P) {
+            v += slab_sum(P, S, slab, (size_t)blockIdx.x * d + j);
+            z[j] = v;
+        }
+        ss += v * v;
+    }
+    ss = block_sum(ss, red);
+    float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    T* y = Y + (size_t)blockIdx.x * d;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) y[j] = from_f<T>(z[j] * inv * g[j]);
+}
+template <typename T>
+void launch_add_rmsnorm(float* Z, const float* P, int S, size_t slab, const float* gain, T* Y,
+                        int R, int d, float eps, cudaStream_t st) {
+    if (R <= 0) return;
+    k_add_rmsnorm<T><<<R, 128, 0, st>>>(Z, P, S, slab, gain, Y, d, eps);
+    rlt_count_launch();
+}
+
 // ---------------------------------------------------------------- merge
 template <typename T>
 __global__ void k_merge_input(const float* __restrict__ e, int T_cap,
@@ -94,24 +131,26 @@ void launch_merge_input(const float* e, int T_cap, const int32_t* pos_dec, const
 
 __global__ void k_merge_out(const float* __restrict__ e, int T_cap,
                             const int32_t* __restrict__ pos_dec, const float* __restrict__ G,
-                            const float* __restrict__ bg, const float* __restrict__ S,
-                            float alpha, float* __restrict__ z, int n, int d) {
+                            int nG, size_t slabG, const float* __restrict__ bg,
+                            const float* __restrict__ S, int nS, size_t slabS, float alpha,
+                            float* __restrict__ z, int n, int d) {
     int r = blockIdx.x, b = r / n, i = r % n;
     const float* et = e + ((size_t)b * T_cap + pos_dec[b] + i) * d;
     for (int j = threadIdx.x; j < d; j += blockDim.x) {
         float u = et[j];
         if (G) {
-            float a = G[(size_t)r * d + j] + bg[j];
+            float a = slab_sum(G, nG, slabG, (size_t)r * d + j) + bg[j];
             float gate = 1.0f / (1.0f + expf(-a));
-            u += alpha * gate * S[(size_t)r * d + j];
+            u += alpha * gate * slab_sum(S, nS, slabS, (size_t)r * d + j);
         }
         z[(size_t)r * d + j] = u;
     }
 }
-void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const float* G,
-                      const float* bg, const float* S, float alpha, float* z, int B, int n, int d,
-                      cudaStream_t st) {
-    k_merge_out<<<B * n, 128, 0, st>>>(e, T_cap, pos_dec, G, bg, S, alpha, z, n, d);
+void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const float* G, int nG,
+                      size_t slabG, const float* bg, const float* S, int nS, size_t slabS,
+                      float alpha, float* z, int B, int n, int d, cudaStream_t st) {
+    k_merge_out<<<B * n, 128, 0, st>>>(e, T_cap, pos_dec, G, nG, slabG, bg, S, nS, slabS, alpha,
+                                       z, n, d);
     rlt_count_launch();
 }
 
@@ -123,32 +162,34 @@ __device__ __forceinline__ void rot(float x1, float x2, float c, float s, float&
 }
 
 template <typename T>
-__global__ void k_qkv_dec(const float* __restrict__ QKV, const int32_t* __restrict__ pos_dec,
-                          RopeTab rope, float* __restrict__ Q, T* __restrict__ Kc,
-                          T* __restrict__ Vc, int n, int heads, int dh) {
+__global__ void k_qkv_dec(const float* __restrict__ QKV, int S, size_t slab,
+                          const int32_t* __restrict__ pos_dec, RopeTab rope,
+                          float* __restrict__ Q, T* __restrict__ Kc, T* __restrict__ Vc, int n,
+                          int heads, int dh) {
     int r = blockIdx.x, b = r / n, i = r % n;
     int d = heads * dh, half = dh / 2;
     int t = pos_dec[b] + 1 + i;
-    const float* src = QKV + (size_t)r * 3 * d;
+    const size_t base = (size_t)r * 3 * d;
     for (int x = threadIdx.x; x < heads * half; x += blockDim.x) {
         int h = x / half, j = x % half;
         float c = rope.cs[(size_t)t * half + j], s = rope.sn[(size_t)t * half + j];
         int o1 = h * dh + j, o2 = o1 + half;
         float y1, y2;
-        rot(src[o1], src[o2], c, s, y1, y2);
+        rot(slab_sum(QKV, S, slab, base + o1), slab_sum(QKV, S, slab, base + o2), c, s, y1, y2);
         Q[(size_t)r * d + o1] = y1;
         Q[(size_t)r * d + o2] = y2;
-        rot(src[d + o1], src[d + o2], c, s, y1, y2);
+        rot(slab_sum(QKV, S, slab, base + d + o1), slab_sum(QKV, S, slab, base + d + o2), c, s, y1,
+            y2);
         Kc[(size_t)r * d + o1] = from_f<T>(y1);
         Kc[(size_t)r * d + o2] = from_f<T>(y2);
-        Vc[(size_t)r * d + o1] = from_f<T>(src[2 * d + o1]);
-        Vc[(size_t)r * d + o2] = from_f<T>(src[2 * d + o2]);
+        Vc[(size_t)r * d + o1] = from_f<T>(slab_sum(QKV, S, slab, base + 2 * d + o1));
+        Vc[(size_t)r * d + o2] = from_f<T>(slab_sum(QKV, S, slab, base + 2 * d + o2));
     }
 }
 template <typename T>
-void launch_qkv_dec(const float* QKV, const int32_t* pos_dec, RopeTab rope, float* Q, T* Kc,
-                    T* Vc, int B, int n, int heads, int dh, cudaStream_t st) {
-    k_qkv_dec<T><<<B * n, 128, 0, st>>>(QKV, pos_dec, rope, Q, Kc, Vc, n, heads, dh);
+void launch_qkv_dec(const float* QKV, int S, size_t slab, const int32_t* pos_dec, RopeTab rope,
+                    float* Q, T* Kc, T* Vc, int B, int n, int heads, int dh, cudaStream_t st) {
+    k_qkv_dec<T><<<B * n, 128, 0, st>>>(QKV, S, slab, pos_dec, rope, Q, Kc, Vc, n, heads, dh);
     rlt_count_launch();
 }
 
@@ -220,7 +261,8 @@ void launch_mem_scatter(const float* KV, const int32_t* pos_enc, RopeTab rope, T
     rlt_count_launch();
 }
 
-__global__ void k_rope_q(float* __restrict__ Q, const int32_t* __restrict__ pos_dec,
+__global__ void k_rope_q(const float* __restrict__ P, int S, size_t slab,
+                         float* __restrict__ Q, const int32_t* __restrict__ pos_dec,
                          RopeTab rope, int n, int heads, int dh) {
     int r = blockIdx.x, b = r / n, i = r % n;
     int d = heads * dh, half = dh / 2;
@@ -230,31 +272,33 @@ __global__ void k_rope_q(float* __restrict__ Q, const int32_t* __restrict__ pos_
         float c = rope.cs[(size_t)t * half + j], s = rope.sn[(size_t)t * half + j];
         int o1 = h * dh + j, o2 = o1 + half;
         float y1, y2;
-        rot(Q[(size_t)r * d + o1], Q[(size_t)r * d + o2], c, s, y1, y2);
+        rot(slab_sum(P, S, slab, (size_t)r * d + o1), slab_sum(P, S, slab, (size_t)r * d + o2), c,
+            s, y1, y2);
         Q[(size_t)r * d + o1] = y1;
         Q[(size_t)r * d + o2] = y2;
     }
 }
-void launch_rope_q(float* Q, const int32_t* pos_dec, RopeTab rope, int B, int n, int heads,
-                   int dh, cudaStream_t st) {
-    k_rope_q<<<B * n, 128, 0, st>>>(Q, pos_dec, rope, n, heads, dh);
+void launch_rope_q(const float* P, int S, size_t slab, float* Q, const int32_t* pos_dec,
+                   RopeTab rope, int B, int n, int heads, int dh, cudaStream_t st) {
+    k_rope_q<<<B * n, 128, 0, st>>>(P, S, slab, Q, pos_dec, rope, n, heads, dh);
     rlt_count_launch();
 }
 
 // ---------------------------------------------------------------- FFN gate
 template <typename T>
-__global__ void k_swiglu(const float* __restrict__ H, int fpad, T* __restrict__ Hd) {
+__global__ void k_swiglu(const float* __restrict__ H, int S, size_t slab, int fpad,
+                         T* __restrict__ Hd) {
     int r = blockIdx.x;
-    const float* h = H + (size_t)r * 2 * fpad;
+    const size_t base = (size_t)r * 2 * fpad;
     for (int j = threadIdx.x; j < fpad; j += blockDim.x) {
-        float a = h[j];
+        float a = slab_sum(H, S, slab, base + j);
         float silu = a / (1.0f + expf(-a));
-        Hd[(size_t)r * fpad + j] = from_f<T>(silu * h[fpad + j]);
+        Hd[(size_t)r * fpad + j] = from_f<T>(silu * slab_sum(H, S, slab, base + fpad + j));
     }
 }
 template <typename T>
-void launch_swiglu(const float* H, int fpad, T* Hd, int R, cudaStream_t st) {
-    k_swiglu<T><<<R, 256, 0, st>>>(H, fpad, Hd);
+void launch_swiglu(const float* H, int S, size_t slab, int fpad, T* Hd, int R, cudaStream_t st) {
+    k_swiglu<T><<<R, 256, 0, st>>>(H, S, slab, fpad, Hd);
     rlt_count_launch();
 }
 
@@ -271,21 +315,22 @@ void launch_copy_e(const float* X, const int32_t* pos_enc, float* e, int T_cap, 
     rlt_count_launch();
 }
 
-__global__ void k_set_state(const float* __restrict__ z, float* __restrict__ s,
-                            float* __restrict__ Rr, const int32_t* __restrict__ pos_dec,
-                            int chunk, int n, int d) {
+__global__ void k_set_state(const float* __restrict__ z, const float* __restrict__ P, int S,
+                            size_t slab, float* __restrict__ s, float* __restrict__ Rr,
+                            const int32_t* __restrict__ pos_dec, int chunk, int n, int d) {
     int b = blockIdx.x;
     bool upd = Rr != nullptr && ((pos_dec[b] + n) % chunk) == 0;
-    const float* src = z + ((size_t)b * n + n - 1) * d;
+    const size_t row = ((size_t)b * n + n - 1) * d;
     for (int j = threadIdx.x; j < d; j += blockDim.x) {
-        float v = src[j];
+        float v = z[row + j];
+        if (P) v += slab_sum(P, S, slab, row + j);
         s[(size_t)b * d + j] = v;
         if (upd) Rr[(size_t)b * d + j] = v;
     }
 }
-void launch_set_state(const float* z, float* s, float* Rreg, const int32_t* pos_dec, int chunk,
-                      int B, int n, int d, cudaStream_t st) {
-    k_set_state<<<B, 128, 0, st>>>(z, s, Rreg, pos_dec, chunk, n, d);
+void launch_set_state(const float* z, const float* P, int S, size_t slab, float* s, float* Rreg,
+                      const int32_t* pos_dec, int chunk, int B, int n, int d, cudaStream_t st) {
+    k_set_state<<<B, 128, 0, st>>>(z, P, S, slab, s, Rreg, pos_dec, chunk, n, d);
     rlt_count_launch();
 }
 
@@ -358,13 +403,15 @@ void launch_ring_write(const T* Kc, const T* Vc, const int32_t* pos_dec, T* ring
                                     cudaStream_t);                                             \
     template void launch_merge_input<T>(const float*, int, const int32_t*, const float*,       \
                                         const float*, T*, int, int, int, float, cudaStream_t); \
-    template void launch_qkv_dec<T>(const float*, const int32_t*, RopeTab, float*, T*, T*, int,\
-                                    int, int, int, cudaStream_t);                              \
+    template void launch_qkv_dec<T>(const float*, int, size_t, const int32_t*, RopeTab, float*, \
+                                    T*, T*, int, int, int, int, cudaStream_t);                 \
+    template void launch_add_rmsnorm<T>(float*, const float*, int, size_t, const float*, T*,   \
+                                        int, int, float, cudaStream_t);                        \
     template void launch_qkv_enc<T>(const float*, const int32_t*, RopeTab, float*, T*, size_t, \
                                     int, int, int, int, int, cudaStream_t);                    \
     template void launch_mem_scatter<T>(const float*, const int32_t*, RopeTab, T*, size_t, int,\
                                         int, int, int, int, cudaStream_t);                     \
-    template void launch_swiglu<T>(const float*, int, T*, int, cudaStream_t);                  \
+    template void launch_swiglu<T>(const float*, int, size_t, int, T*, int, cudaStream_t);     \
     template void launch_ring_write<T>(const T*, const T*, const int32_t*, T*, size_t, int,    \
                                        int, int, int, int, cudaStream_t);
 RLT_INST(float)

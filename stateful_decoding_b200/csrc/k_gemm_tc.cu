@@ -42,7 +42,8 @@ constexpr size_t smem_bytes() { return (size_t)STAGES * stage_bytes<BN>() + 1024
 template <int BN, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
-          float* __restrict__ C, int ldc, bf16* __restrict__ Ct, int ldct, int M, int N, int K) {
+          float* __restrict__ C, int ldc, bf16* __restrict__ Ct, int ldct, int M, int N, int K,
+          int cps, size_t slab) {
     using namespace tc;
     constexpr uint32_t A_BYTES = BM * BK * 2, STAGE = stage_bytes<BN>();
     extern __shared__ uint8_t smem_raw[];
@@ -53,7 +54,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-    const int nk = K / BK;
+    // split-K: this CTA sums K-chunks [kbeg, kbeg+nk) and, with several
+    // splits, writes its partial sums to slab blockIdx.z of C
+    const int kbeg = blockIdx.z * cps;
+    const int nk = min(K / BK - kbeg, cps);
+    C += (size_t)blockIdx.z * slab;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -84,8 +89,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                     break;
                 }
                 mbar_expect_tx(&full[s], STAGE);
-                tma_load_2d(smem + s * STAGE, &ta, kt * BK, m0, &full[s]);
-                tma_load_2d(smem + s * STAGE + A_BYTES, &tb, kt * BK, n0, &full[s]);
+                tma_load_2d(smem + s * STAGE, &ta, (kbeg + kt) * BK, m0, &full[s]);
+                tma_load_2d(smem + s * STAGE + A_BYTES, &tb, (kbeg + kt) * BK, n0, &full[s]);
             }
         }
     } else if (warp == 1) {
@@ -179,7 +184,7 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int ld, in
 
 template <int BN, int MODE>
 bool launch_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
-               int ldct, int M, int N, int K, cudaStream_t st) {
+               int ldct, int M, int N, int K, int splits, size_t slab, cudaStream_t st) {
     CUtensorMap ta, tb;
     if (!make_map(&ta, A, M, K, lda, BM) || !make_map(&tb, W, N, K, ldw, BN)) return false;
     static bool attr = false;
@@ -189,19 +194,24 @@ bool launch_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc
             return false;
         attr = true;
     }
-    dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
+    const int nk = K / BK, cps = (nk + splits - 1) / splits;
+    dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, (nk + cps - 1) / cps);
     k_gemm_tc<BN, MODE><<<grid, NTHREADS, smem_bytes<BN>(), st>>>(ta, tb, C, ldc, Ct, ldct, M, N,
-                                                                 K);
+                                                                 K, cps, slab);
     rlt_count_launch();
     return true;
 }
 
 template <int BN>
 bool launch_tc_mode(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
-                    int ldct, int M, int N, int K, int mode, cudaStream_t st) {
-    if (mode == kStoreF32) return launch_tc<BN, kStoreF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, st);
-    if (mode == kAddF32) return launch_tc<BN, kAddF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, st);
-    return launch_tc<BN, kStoreT>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, st);
+                    int ldct, int M, int N, int K, int mode, int splits, size_t slab,
+                    cudaStream_t st) {
+    if (mode == kStoreF32)
+        return launch_tc<BN, kStoreF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, splits, slab, st);
+    if (splits != 1) return false;          // partial sums only go to fp32 slabs
+    if (mode == kAddF32)
+        return launch_tc<BN, kAddF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, 1, 0, st);
+    return launch_tc<BN, kStoreT>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, 1, 0, st);
 }
 
 }  // namespace
@@ -214,12 +224,14 @@ bool make_tma_2d_bf16(CUtensorMap* map, const void* base, int rows, int cols, in
 // Returns false (and launches nothing) when the shape or alignment does not
 // suit the tensor-core kernel; the caller then uses the CUDA-core kernel.
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
-                    int ldct, int M, int N, int K, int mode, cudaStream_t st) {
-    if (M <= 0 || N < 16 || K < BK || K % BK) return false;
+                    int ldct, int M, int N, int K, int mode, int splits, size_t slab,
+                    cudaStream_t st) {
+    if (M <= 0 || N < 16 || K < BK || K % BK || splits < 1) return false;
     if (lda % 8 || ldw % 8 || ((uintptr_t)A & 15) || ((uintptr_t)W & 15)) return false;
     // wide tiles when M alone fills the machine, narrow ones (more CTAs) otherwise
-    if (M >= 2048) return launch_tc_mode<256>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, st);
-    return launch_tc_mode<64>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, st);
+    if (M >= 2048)
+        return launch_tc_mode<256>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, splits, slab, st);
+    return launch_tc_mode<64>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, splits, slab, st);
 }
 
 }  // namespace rlt

@@ -32,6 +32,9 @@ template <typename T>
 void launch_gemm(const T* A, int lda, const T* W, int ldw, float* C, int ldc, T* Ct, int ldct,
                  int M, int N, int K, int mode, cudaStream_t st);
 template <typename T>
+int launch_gemm_split(const T* A, int lda, const T* W, int ldw, float* C, int ldc, int M, int N,
+                      int K, int splits, size_t slab, cudaStream_t st);
+template <typename T>
 void launch_gemm_simt(const T* A, int lda, const T* W, int ldw, float* C, int ldc, T* Ct,
                       int ldct, int M, int N, int K, int mode, cudaStream_t st);
 
@@ -39,15 +42,20 @@ void launch_gemm_simt(const T* A, int lda, const T* W, int ldw, float* C, int ld
 template <typename T>
 void launch_merge_input(const float* e, int T_cap, const int32_t* pos_dec, const float* fb,
                         const float* gain, T* Gin, int B, int n, int d, float eps, cudaStream_t st);
-// z[r] = e_t + alpha * sigmoid(G[r] + bg) * S[r]   (S = W_s r); alpha ignored if G == nullptr
-void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const float* G,
-                      const float* bg, const float* S, float alpha, float* z, int B, int n, int d,
-                      cudaStream_t st);
+// z[r] = e_t + alpha * sigmoid(G[r] + bg) * S[r]   (S = W_s r); alpha ignored if G == nullptr.
+// G and S may be split-K partial slabs (nG / nS slabs, slabG / slabS apart).
+void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const float* G, int nG,
+                      size_t slabG, const float* bg, const float* S, int nS, size_t slabS,
+                      float alpha, float* z, int B, int n, int d, cudaStream_t st);
+// z += sum of residual partial slabs P (P may be null), then Y = RMSNorm(z)
+template <typename T>
+void launch_add_rmsnorm(float* Z, const float* P, int S, size_t slab, const float* gain, T* Y,
+                        int R, int d, float eps, cudaStream_t st);
 
 // decoder q/k/v: QKV fp32 [R][3d] -> Q fp32 [R][d] (RoPE), Kc, Vc storage [R][d] (RoPE on k)
 template <typename T>
-void launch_qkv_dec(const float* QKV, const int32_t* pos_dec, RopeTab rope, float* Q, T* Kc,
-                    T* Vc, int B, int n, int heads, int dh, cudaStream_t st);
+void launch_qkv_dec(const float* QKV, int S, size_t slab, const int32_t* pos_dec, RopeTab rope,
+                    float* Q, T* Kc, T* Vc, int B, int n, int heads, int dh, cudaStream_t st);
 // encoder q/k/v: q -> Q (RoPE); k (RoPE), v -> cache [b][2][h][T_cap][dh] + layer offset
 template <typename T>
 void launch_qkv_enc(const float* QKV, const int32_t* pos_enc, RopeTab rope, float* Q, T* cache,
@@ -58,17 +66,18 @@ template <typename T>
 void launch_mem_scatter(const float* KV, const int32_t* pos_enc, RopeTab rope, T* mem,
                         size_t row_stride, int T_cap, int B, int n, int heads, int dh,
                         cudaStream_t st);
-// in-place RoPE on Q fp32 [R][d] at decoder positions
-void launch_rope_q(float* Q, const int32_t* pos_dec, RopeTab rope, int B, int n, int heads,
-                   int dh, cudaStream_t st);
+// Q fp32 [R][d] = RoPE(sum of the partial slabs P) at decoder positions
+void launch_rope_q(const float* P, int S, size_t slab, float* Q, const int32_t* pos_dec,
+                   RopeTab rope, int B, int n, int heads, int dh, cudaStream_t st);
 
 template <typename T>
-void launch_swiglu(const float* H, int fpad, T* Hd, int R, cudaStream_t st);
+void launch_swiglu(const float* H, int S, size_t slab, int fpad, T* Hd, int R, cudaStream_t st);
 void launch_copy_e(const float* X, const int32_t* pos_enc, float* e, int T_cap, int B, int n,
                    int d, cudaStream_t st);
-// s[b] = z[b*n + n-1]; RLT-2: R[b] = s[b] when (pos_dec[b]+n) % chunk == 0
-void launch_set_state(const float* z, float* s, float* Rreg, const int32_t* pos_dec, int chunk,
-                      int B, int n, int d, cudaStream_t st);
+// s[b] = z[b*n + n-1] (+ its residual partial slabs); RLT-2: R[b] = s[b] when
+// (pos_dec[b]+n) % chunk == 0
+void launch_set_state(const float* z, const float* P, int S, size_t slab, float* s, float* Rreg,
+                      const int32_t* pos_dec, int chunk, int B, int n, int d, cudaStream_t st);
 void launch_pos_add(int32_t* pos, int B, int n, cudaStream_t st);
 void launch_reset_rows(const int32_t* rows, int nrows, const float* s_star, float* s, float* Rr,
                        int32_t* pos_enc, int32_t* pos_dec, int d, cudaStream_t st);

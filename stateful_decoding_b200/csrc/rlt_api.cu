@@ -471,6 +471,9 @@ struct rlt_state {
     float* logits = nullptr;
     int32_t* ids = nullptr;
     int32_t* rows = nullptr;
+    float* P = nullptr;             // split-K partial slabs of the transition's projections
+    size_t p_cols = 0;              // columns of one slab row (the widest projection)
+    int p_slabs = 1;                // slabs allocated
     std::vector<void*> allocs;
     size_t bytes = 0;
     // live timing (rlt_profile_*)
@@ -540,6 +543,8 @@ extern "C" void rlt_state_destroy(rlt_state* s) {
     delete s;
 }
 
+static int max_dec_splits(const rlt_config& c, int fp);
+
 static size_t max_rows_per_call() {
     const char* v = getenv("RLT_MAX_ROWS");
     long x = v ? atol(v) : 65536;
@@ -559,7 +564,7 @@ extern "C" int rlt_state_create(rlt_model* m, int batch, int max_len, rlt_state*
     const size_t slots = (size_t)std::max(0, c.window - 1);
     size_t maxr = max_rows_per_call();
     s->n_enc_blk = (int)std::max<size_t>(1, std::min<size_t>(T, maxr / B));
-    s->n_dec_blk = c.variant == 2 ? c.chunk : (c.variant == 0 ? std::min(s->n_enc_blk, 256) : 1);
+    s->n_dec_blk = c.variant == 2 ? c.chunk : (c.variant == 0 ? std::min(s->n_enc_blk, 16) : 1);
     const size_t R = B * (size_t)std::max(s->n_enc_blk, s->n_dec_blk);
     s->enc_row = (size_t)c.n_enc * 2 * h * T * dh;
     s->mem_row = (size_t)(c.n_dec > 0 ? c.groups : 0) * 2 * h * T * dh;
@@ -595,6 +600,12 @@ extern "C" int rlt_state_create(rlt_model* m, int batch, int max_len, rlt_state*
     take((void**)&s->logits, B * (size_t)c.vocab * 4);
     take((void**)&s->ids, 2 * B * 4);
     take((void**)&s->rows, B * 4);
+    {   // split-K slabs for the transition: widest projection x most splits
+        const size_t Rd = B * (size_t)s->n_dec_blk;
+        s->p_cols = std::max<size_t>(3 * d, 2 * fp);
+        s->p_slabs = max_dec_splits(c, (int)fp);
+        take((void**)&s->P, (size_t)s->p_slabs * Rd * s->p_cols * 4);
+    }
     if (rc != RLT_OK) {
         rlt_state_destroy(s);
         return rc;
@@ -707,6 +718,30 @@ static double enc_bytes(const rlt_state* s, int n) {     // one encoder block
     return by;
 }
 
+// Split-K factor of a transition projection (N outputs, K inputs): enough
+// CTAs for the machine when M = 256 rows, a function of N and K only (never of
+// the batch), at least two 64-wide K-chunks per split.  1 for fp32 models.
+static int dec_splits_for(const rlt_config& c, int N, int K) {
+    if (c.dtype != RLT_DTYPE_BF16 || K % 64) return 1;
+    const int tiles = 2 * ((N + 63) / 64);            // output tiles at M = 256
+    const int nk = K / 64;
+    int want = std::max(1, (148 + tiles - 1) / tiles);
+    want = std::min(want, std::max(1, nk / 2));
+    const int cps = (nk + want - 1) / want;
+    return (nk + cps - 1) / cps;
+}
+static int dec_splits(const rlt_state* s, int N, int K) {
+    return std::min(s->p_slabs, dec_splits_for(s->m->cfg, N, K));
+}
+// the most slabs any transition projection of this model uses
+static int max_dec_splits(const rlt_config& c, int fp) {
+    const int d = c.d;
+    const int shapes[6][2] = {{3 * d, d}, {d, d}, {2 * fp, d}, {d, fp}, {d, 2 * d}, {d, d}};
+    int m = 1;
+    for (auto& sh : shapes) m = std::max(m, dec_splits_for(c, sh[0], sh[1]));
+    return m;
+}
+
 // ============================================================================
 // encoder
 // ============================================================================
@@ -736,7 +771,7 @@ static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t s
         launch_rmsnorm<T>(s->X, d, L.ffn_norm, Y, d, R, d, eps, st);
         launch_gemm<T>(Y, d, (const T*)L.w13, d, s->H13, 2 * fp, nullptr, 0, R, 2 * fp, d,
                        kStoreF32, st);
-        launch_swiglu<T>(s->H13, fp, Hd, R, st);
+        launch_swiglu<T>(s->H13, 1, 0, fp, Hd, R, st);
         launch_gemm<T>(Hd, fp, (const T*)L.w2, fp, s->X, d, nullptr, 0, R, d, fp, kAddF32, st);
     }
     launch_copy_e(s->X, s->pos_enc, s->e, s->T_cap, B, n, d, st);
@@ -802,51 +837,60 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
     T* Kc = (T*)s->Kc;
     T* Vc = (T*)s->Vc;
     float* z = s->X;
+    // Split-K partial slabs of each projection land in s->P; the kernel that
+    // consumes the projection adds them in slab order (residual projections:
+    // the next RMSNorm, or the state hand-off).
+    float* P = s->P;
+    const size_t slab = (size_t)R * s->p_cols;
+    auto gemm_p = [&](const T* Ain, int lda, const T* Wt, int N, int K, float* dst) {
+        return launch_gemm_split<T>(Ain, lda, Wt, K, dst, N, R, N, K, dec_splits(s, N, K), slab,
+                                    st);
+    };
     if (c.variant == 0) {
-        launch_merge_out(s->e, s->T_cap, s->pos_dec, nullptr, nullptr, nullptr, 0.f, z, B, n, d,
-                         st);
+        launch_merge_out(s->e, s->T_cap, s->pos_dec, nullptr, 0, 0, nullptr, nullptr, 0, 0, 0.f, z,
+                         B, n, d, st);
     } else {
         const float* fb = c.variant == 2 ? s->Rr : s->s;
         launch_merge_input<T>(s->e, s->T_cap, s->pos_dec, fb, m->merge_norm, Y, B, n, d, eps, st);
-        launch_gemm<T>(Y, 2 * d, (const T*)m->wg, 2 * d, s->G, d, nullptr, 0, R, d, 2 * d,
-                       kStoreF32, st);
-        launch_gemm<T>(Y + d, 2 * d, (const T*)m->ws, d, s->S, d, nullptr, 0, R, d, d, kStoreF32,
-                       st);
-        launch_merge_out(s->e, s->T_cap, s->pos_dec, s->G, m->bg, s->S, (float)c.alpha, z, B, n,
-                         d, st);
+        // gate partials in P, projection partials in a second region P2 of the same slabs
+        float* P2 = P + (size_t)R * d;
+        const int nG = gemm_p(Y, 2 * d, (const T*)m->wg, d, 2 * d, P);
+        const int nS = gemm_p(Y + d, 2 * d, (const T*)m->ws, d, d, P2);
+        launch_merge_out(s->e, s->T_cap, s->pos_dec, P, nG, slab, m->bg, P2, nS, slab,
+                         (float)c.alpha, z, B, n, d, st);
     }
     const size_t layer_ring = (size_t)2 * h * std::max(0, c.window - 1) * dh;
     const size_t layer_mem = (size_t)2 * h * s->T_cap * dh;
+    int nres = 0;                       // pending residual partial slabs in P
     for (int l = 0; l < c.n_dec; ++l) {
         const DecLayerW& L = m->dec[l];
         T* ring = (T*)s->ring + l * layer_ring;
-        launch_rmsnorm<T>(z, d, L.swa_norm, Y, d, R, d, eps, st);
-        launch_gemm<T>(Y, d, (const T*)L.wqkv, d, s->QKV, 3 * d, nullptr, 0, R, 3 * d, d,
-                       kStoreF32, st);
-        launch_qkv_dec<T>(s->QKV, s->pos_dec, rope_of(s), s->Q, Kc, Vc, B, n, h, dh, st);
+        launch_add_rmsnorm<T>(z, nres ? P : nullptr, nres, slab, L.swa_norm, Y, R, d, eps, st);
+        int np = gemm_p(Y, d, (const T*)L.wqkv, 3 * d, d, P);
+        launch_qkv_dec<T>(P, np, slab, s->pos_dec, rope_of(s), s->Q, Kc, Vc, B, n, h, dh, st);
         {
             ProfScope ps(s, RLT_PROF_SWA, st, s->prof ? swa_bytes(s, n) : 0.0);
             launch_attn_swa<T>(s->Q, Kc, Vc, ring, s->ring_row, c.window, s->pos_dec, A, B, n, h,
                                dh, st);
         }
         launch_ring_write<T>(Kc, Vc, s->pos_dec, ring, s->ring_row, c.window, B, n, h, dh, st);
-        launch_gemm<T>(A, d, (const T*)L.wo, d, z, d, nullptr, 0, R, d, d, kAddF32, st);
-        launch_rmsnorm<T>(z, d, L.x_norm, Y, d, R, d, eps, st);
-        launch_gemm<T>(Y, d, (const T*)L.xq, d, s->Q, d, nullptr, 0, R, d, d, kStoreF32, st);
-        launch_rope_q(s->Q, s->pos_dec, rope_of(s), B, n, h, dh, st);
+        nres = gemm_p(A, d, (const T*)L.wo, d, d, P);
+        launch_add_rmsnorm<T>(z, P, nres, slab, L.x_norm, Y, R, d, eps, st);
+        np = gemm_p(Y, d, (const T*)L.xq, d, d, P);
+        launch_rope_q(P, np, slab, s->Q, s->pos_dec, rope_of(s), B, n, h, dh, st);
         const T* mem = (const T*)s->mem + (c.groups > 1 ? l : 0) * layer_mem;
         {
             ProfScope ps(s, RLT_PROF_XATTN, st, s->prof ? xattn_bytes(s, n) : 0.0);
             launch_attn_cross<T>(s->Q, mem, s->mem_row, s->T_cap, s->pos_dec, A, B, n, h, dh, st);
         }
-        launch_gemm<T>(A, d, (const T*)L.xo, d, z, d, nullptr, 0, R, d, d, kAddF32, st);
-        launch_rmsnorm<T>(z, d, L.ffn_norm, Y, d, R, d, eps, st);
-        launch_gemm<T>(Y, d, (const T*)L.w13, d, s->H13, 2 * fp, nullptr, 0, R, 2 * fp, d,
-                       kStoreF32, st);
-        launch_swiglu<T>(s->H13, fp, Hd, R, st);
-        launch_gemm<T>(Hd, fp, (const T*)L.w2, fp, z, d, nullptr, 0, R, d, fp, kAddF32, st);
+        nres = gemm_p(A, d, (const T*)L.xo, d, d, P);
+        launch_add_rmsnorm<T>(z, P, nres, slab, L.ffn_norm, Y, R, d, eps, st);
+        np = gemm_p(Y, d, (const T*)L.w13, 2 * fp, d, P);
+        launch_swiglu<T>(P, np, slab, fp, Hd, R, st);
+        nres = gemm_p(Hd, fp, (const T*)L.w2, d, fp, P);
     }
-    launch_set_state(z, s->s, c.variant == 2 ? s->Rr : nullptr, s->pos_dec, c.chunk, B, n, d, st);
+    launch_set_state(z, nres ? P : nullptr, nres, slab, s->s, c.variant == 2 ? s->Rr : nullptr,
+                     s->pos_dec, c.chunk, B, n, d, st);
     launch_pos_add(s->pos_dec, B, n, st);
 }
 
