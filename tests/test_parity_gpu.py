@@ -11,7 +11,7 @@ import pytest
 
 import rlt_inputs as ri
 from oracle import RLTOracle
-from tests.rlt_testlib import Tally, check_argmax, check_sample, oracle_mode, tol_for
+from tests.rlt_testlib import TOL_BF16, Tally, check_argmax, check_sample, oracle_mode, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -223,8 +223,9 @@ def test_serving_split_bitexact(sd, name):
     if cfg.variant == 2:
         # RLT-2: the one-shot prefill runs whole chunks in one block while the
         # split schedule steps token by token, so the window attention folds
-        # its keys in another order: equal up to rounding
-        np.testing.assert_allclose(la, lb, atol=2e-3, rtol=0)
+        # its keys in another order: equal up to rounding, which bf16 storage
+        # amplifies to its noise floor (the bf16 tolerance)
+        np.testing.assert_allclose(la, lb, atol=TOL_BF16, rtol=0)
     else:
         np.testing.assert_array_equal(la, lb)
         np.testing.assert_array_equal(a.read(sd.PART_S), b_.read(sd.PART_S))
