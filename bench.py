@@ -94,6 +94,32 @@ def oracle_sample(cfg, budget_s: float = 15.0):
     return done_tok / dt, desc, threads
 
 
+# ----------------------------------------------------------------------------
+# rank bookkeeping (weak scaling: every rank runs its own rows, no collective
+# on the data path)
+# ----------------------------------------------------------------------------
+def shard_tokens(cfg, rank: int, batch: int, length: int) -> np.ndarray:
+    """This rank's prompts: rows rank*batch .. rank*batch+batch-1 of the one
+    global token stream (each row has its own substream)."""
+    return ri.make_tokens(cfg, batch, length, row0=rank * batch)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's time: the job's time."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(batch: int, positions: int, world: int, ms_per_step: float) -> float:
+    """Transitions of all ranks in one step over the slowest rank's time."""
+    return batch * positions * world / (ms_per_step / 1e3)
+
+
 def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -199,7 +225,7 @@ def run_ours(args, cfg):
     model = sd.Model(ri.write_blob(cfg, W), device=local)
     st = sd.State(model, B, T + D)
     # each rank runs its own rows: the token substreams start at rank * B
-    toks_h = ri.make_tokens(cfg, B, T, row0=rank * B)
+    toks_h = shard_tokens(cfg, rank, B, T)
     toks = torch.from_numpy(toks_h).to(dev)
     logits = torch.empty(B, cfg.vocab, device=dev)
     ids = torch.empty(B, dtype=torch.int32, device=dev)
@@ -225,13 +251,6 @@ def run_ours(args, cfg):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     for _ in range(max(3, args.warmup)):
         step(toks, logits, ids, am)
     barrier()
@@ -255,10 +274,10 @@ def run_ours(args, cfg):
             (("xattn", sd.PROF_XATTN), ("swa", sd.PROF_SWA), ("step", sd.PROF_STEP),
              ("enc", sd.PROF_ENC))}
     st.profile(False)
-    ms_total = max_over_ranks(ms_total)
+    ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / args.steps
     tokens_step = B * (T + D) * world
-    value = tokens_step / (ms_step / 1e3)
+    value = job_tokens_per_s(B, T + D, world, ms_step)
 
     # ---- end to end through the C ABI with host buffers ----
     toks_pin = torch.from_numpy(toks_h).pin_memory()
@@ -274,7 +293,7 @@ def run_ours(args, cfg):
         step(toks_pin, lg_pin, ids, am_pin)
     f1.record(stream)
     barrier()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1)) / args.steps
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev) / args.steps
     e2e_wall = (time.perf_counter() - t0) * 1e3 / args.steps
     h2d = B * T * 4
     d2h = B * cfg.vocab * 4 + B * 4
@@ -298,7 +317,7 @@ def run_ours(args, cfg):
                        parallelism=f"replicas x{world} (rows sharded, no collective)",
                        l2="working set per step > L2: caches of all rows (see DESIGN.md)"),
         "gpu_launches": launches,
-        "e2e": {"value": tokens_step / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(B, T + D, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms, "wall_ms_per_step": e2e_wall},
         "roofline": {"bound": "hbm", "kernel": kname,
