@@ -155,7 +155,10 @@ uint64_t rlt_kernel_launches(void);
  * (keys/values read, cache entries written, activations in and out; weights
  * excluded).  rlt_profile_query synchronises `stream`, sums the elapsed times
  * of the class since the last enable, and reports launches, total ms and
- * bytes.  Enabling resets the counters. */
+ * bytes.  Enabling resets the counters.  on = 1 keeps replaying transition
+ * blocks as CUDA graphs (then only whole blocks are timed, as RLT_PROF_STEP);
+ * on = 2 runs them launch by launch so that the attention launches are timed
+ * one by one too (for measurement: slower than the graph replay). */
 #define RLT_PROF_XATTN 0  /* decoder cross-attention over M_{<=t}        */
 #define RLT_PROF_SWA   1  /* decoder window attention over C^D           */
 #define RLT_PROF_STEP  2  /* one whole transition block (merge .. s_t)   */

@@ -274,8 +274,11 @@ class State:
     def check(self, stream=None):
         return _check(rlt_state_check(self.handle, stream), "rlt_state_check")
 
-    def profile(self, on: bool):
-        return _check(rlt_profile_enable(self.handle, on), "rlt_profile_enable")
+    def profile(self, on: int):
+        """0: off; 1: time kernel classes, transition blocks still replayed as
+        graphs (timed as whole blocks); 2: blocks run launch by launch so that
+        every attention launch is timed."""
+        return _check(rlt_profile_enable(self.handle, int(on)), "rlt_profile_enable")
 
     def profile_query(self, cls: int, stream=None):
         """(launches, total_ms, algorithmic_bytes) of a kernel class since enable."""

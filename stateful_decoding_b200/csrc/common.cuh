@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace rlt {
 
 typedef __nv_bfloat16 bf16;
@@ -44,3 +46,40 @@ enum DevError : int { kDevOk = 0, kDevTimeout = 1, kDevBounds = 2 };
 
 // Launch bookkeeping (defined in rlt_api.cu).
 void rlt_count_launch(int n = 1);
+
+// Programmatic dependent launch.  Every kernel of the library starts with
+// pdl_wait() (before it reads or writes anything an earlier kernel of the
+// stream touches) and then lets the next kernel of the stream begin its own
+// launch and prologue.  Both are no-ops in a kernel launched without the
+// attribute.
+namespace rlt {
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_enter() {
+    pdl_wait();
+    pdl_trigger();
+}
+
+// True unless RLT_PDL=0 (defined in rlt_api.cu).
+bool pdl_enabled();
+
+// kernel<<<grid, block, smem, st>>>(args...) with the programmatic-serialisation
+// attribute set when PDL is enabled.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+}  // namespace rlt

@@ -57,6 +57,19 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
         : "memory");
 }
 
+__device__ __forceinline__ float slab_sum(const float* __restrict__ P, int S, size_t slab,
+                                          size_t i) {
+    float v = P[i];
+    for (int z = 1; z < S; ++z) v += P[(size_t)z * slab + i];
+    return v;
+}
+// rotate-half RoPE of one pair (j, j + d_h/2)
+__device__ __forceinline__ void rope_rot(float x1, float x2, float c, float s, float& y1,
+                                         float& y2) {
+    y1 = x1 * c - x2 * s;
+    y2 = x2 * c + x1 * s;
+}
+
 template <int DH, int NQ>
 struct Online {             // per-warp online softmax state of NQ queries
     float m[NQ], l[NQ], acc[NQ][8];
@@ -124,11 +137,13 @@ __device__ __forceinline__ void fold_keys(Online<DH, NQ>& st, const float (&q)[N
     }
 }
 
-template <int DH, int NQ, bool SWA>
+template <int DH, int NQ, bool SWA, bool PRO>
 __global__ void __launch_bounds__(NW * 32)
 k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t row_stride,
               int span, const bf16* __restrict__ Kc, const bf16* __restrict__ Vc,
-              const int32_t* __restrict__ pos, int W, bf16* __restrict__ A, int n, int heads) {
+              const int32_t* __restrict__ pos, int W, bf16* __restrict__ A, int n, int heads,
+              ProjIn pin) {
+    pdl_enter();
     int* err = &g_attn_error;
     constexpr int LPK = DH / 8, KPR = 32 / LPK;
     constexpr int WK = CH / NW;                 // keys per warp per stage
@@ -150,6 +165,37 @@ k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t
     const int pd = pos[b];
     const int seg = lane % LPK;
 
+    // PRO: q (and, for the window attention, this block's own k and v) are
+    // formed here from the projection's partial slabs: summed in slab order,
+    // RoPE at the query's position, k and v rounded to the storage type.
+    __shared__ __align__(16) float s_q[PRO ? NQ : 1][DH];
+    __shared__ __align__(16) bf16 s_k[PRO && SWA ? NQ : 1][DH];
+    __shared__ __align__(16) bf16 s_v[PRO && SWA ? NQ : 1][DH];
+    if (PRO) {
+        constexpr int HALF = DH / 2;
+        for (int e = threadIdx.x; e < nq * HALF; e += NW * 32) {
+            const int i = e / HALF, j = e % HALF;
+            const int t = pd + 1 + q0 + i;
+            const float c = pin.rope.cs[(size_t)t * HALF + j], sn = pin.rope.sn[(size_t)t * HALF + j];
+            const size_t rb = (size_t)(b * n + q0 + i) * pin.ldp + h * DH + j;
+            float y1, y2;
+            rope_rot(slab_sum(pin.P, pin.S, pin.slab, rb), slab_sum(pin.P, pin.S, pin.slab, rb + HALF),
+                     c, sn, y1, y2);
+            s_q[i][j] = y1;
+            s_q[i][j + HALF] = y2;
+            if (SWA) {
+                rope_rot(slab_sum(pin.P, pin.S, pin.slab, rb + d),
+                         slab_sum(pin.P, pin.S, pin.slab, rb + d + HALF), c, sn, y1, y2);
+                s_k[i][j] = __float2bfloat16_rn(y1);
+                s_k[i][j + HALF] = __float2bfloat16_rn(y2);
+                s_v[i][j] = __float2bfloat16_rn(slab_sum(pin.P, pin.S, pin.slab, rb + 2 * d));
+                s_v[i][j + HALF] =
+                    __float2bfloat16_rn(slab_sum(pin.P, pin.S, pin.slab, rb + 2 * d + HALF));
+            }
+        }
+        __syncthreads();
+    }
+
     int lo[NQ], hi[NQ];
     float q[NQ][8];
     const float sc = 1.0f / sqrtf((float)DH);
@@ -158,7 +204,8 @@ k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t
         const int t = pd + 1 + q0 + min(i, nq - 1);
         hi[i] = i < nq ? t : 0;
         lo[i] = SWA ? max(1, t - W + 1) : 1;
-        const float* qp = Q + (size_t)(b * n + q0 + min(i, nq - 1)) * d + h * DH + seg * 8;
+        const float* qp = PRO ? &s_q[min(i, nq - 1)][seg * 8]
+                              : Q + (size_t)(b * n + q0 + min(i, nq - 1)) * d + h * DH + seg * 8;
 #pragma unroll
         for (int x = 0; x < 8; ++x) q[i][x] = qp[x] * sc;
     }
@@ -227,13 +274,15 @@ k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t
         if (s_abort) break;
     }
     if (SWA && warp == 0) {   // the block's own positions pd+1 .. pd+q0+nq (this layer's k, v)
-        const bf16* ck = Kc + (size_t)b * n * d + h * DH;
-        const bf16* cv = Vc + (size_t)b * n * d + h * DH;
+        // (with PRO the grid has one query group, so all of them are in s_k / s_v)
+        const bf16* ck = PRO ? &s_k[0][0] : Kc + (size_t)b * n * d + h * DH;
+        const bf16* cv = PRO ? &s_v[0][0] : Vc + (size_t)b * n * d + h * DH;
+        const int ld = PRO ? DH : d;
         const int nown = q0 + nq;
         for (int e0 = 0; e0 < nown; e0 += KPR) {
             fold_keys<DH, NQ, 1>(
-                os, q, lo, hi, [&](int kidx) { return ck + (size_t)(e0 + kidx) * d; },
-                [&](int kidx) { return cv + (size_t)(e0 + kidx) * d; },
+                os, q, lo, hi, [&](int kidx) { return ck + (size_t)(e0 + kidx) * ld; },
+                [&](int kidx) { return cv + (size_t)(e0 + kidx) * ld; },
                 [&](int kidx) -> int { return e0 + kidx < nown ? pd + 1 + e0 + kidx : 0; }, lane);
         }
     }
@@ -270,38 +319,55 @@ k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t
         }
         A[(size_t)(b * n + q0 + i) * d + h * DH + x] = __float2bfloat16_rn(O / L);
     }
+    if (PRO && SWA && W > 1 && !s_abort) {
+        // every read of this head's ring has landed (all stages were waited
+        // for): move the block's last min(n, W-1) positions into their slots
+        const int slots = span;
+        bf16* rk = const_cast<bf16*>(kg);
+        bf16* rv = const_cast<bf16*>(vg);
+        for (int e = threadIdx.x; e < nq * DH; e += NW * 32) {
+            const int i = e / DH, x = e % DH;
+            if (i < n - slots) continue;
+            const int slot = (pd + i) % slots;     // position pd+1+i
+            rk[(size_t)slot * DH + x] = s_k[i][x];
+            rv[(size_t)slot * DH + x] = s_v[i][x];
+        }
+    }
 }
 
 // One launcher per kernel instance, so that each instance gets its own
 // shared-memory attribute (the instances share a function-pointer type).
-template <int DH, int NQ, bool SWA>
+template <int DH, int NQ, bool SWA, bool PRO>
 bool launch_one(const float* Q, const bf16* base, size_t row_stride, int span, const bf16* Kc,
                 const bf16* Vc, const int32_t* pos, int W, bf16* A, int B, int n, int heads,
-                cudaStream_t st) {
+                const ProjIn& pin, cudaStream_t st) {
     constexpr size_t smem = 4 * (size_t)CH * DH * 2;
     static bool attr = false;
     if (!attr) {
-        if (cudaFuncSetAttribute(k_attn_stream<DH, NQ, SWA>,
+        if (cudaFuncSetAttribute(k_attn_stream<DH, NQ, SWA, PRO>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return false;
         attr = true;
     }
-    k_attn_stream<DH, NQ, SWA><<<dim3(B * heads, (n + NQ - 1) / NQ), NW * 32, smem, st>>>(
-        Q, base, row_stride, span, Kc, Vc, pos, W, A, n, heads);
+    launch(k_attn_stream<DH, NQ, SWA, PRO>, dim3(B * heads, (n + NQ - 1) / NQ), NW * 32, smem, st,
+           Q, base, row_stride, span, Kc, Vc, pos, W, A, n, heads, pin);
     rlt_count_launch();
     return true;
 }
 
-template <int DH, bool SWA>
+template <int DH, bool SWA, bool PRO>
 bool launch_stream(const float* Q, const bf16* base, size_t row_stride, int span, const bf16* Kc,
                    const bf16* Vc, const int32_t* pos, int W, bf16* A, int B, int n, int heads,
-                   cudaStream_t st) {
+                   const ProjIn& pin, cudaStream_t st) {
     if (n == 1)
-        return launch_one<DH, 1, SWA>(Q, base, row_stride, span, Kc, Vc, pos, W, A, B, n, heads, st);
+        return launch_one<DH, 1, SWA, PRO>(Q, base, row_stride, span, Kc, Vc, pos, W, A, B, n,
+                                           heads, pin, st);
     if (n == 2)
-        return launch_one<DH, 2, SWA>(Q, base, row_stride, span, Kc, Vc, pos, W, A, B, n, heads, st);
-    return launch_one<DH, 4, SWA>(Q, base, row_stride, span, Kc, Vc, pos, W, A, B, n, heads, st);
+        return launch_one<DH, 2, SWA, PRO>(Q, base, row_stride, span, Kc, Vc, pos, W, A, B, n,
+                                           heads, pin, st);
+    return launch_one<DH, 4, SWA, PRO>(Q, base, row_stride, span, Kc, Vc, pos, W, A, B, n, heads,
+                                       pin, st);
 }
 
 }  // namespace
@@ -312,11 +378,11 @@ bool launch_attn_cross_fast(const float* Q, const bf16* mem, size_t row_stride, 
                             cudaStream_t st) {
     if (B * n <= 0) return true;
     if (dh == 64)
-        return launch_stream<64, false>(Q, mem, row_stride, T_cap, nullptr, nullptr, pos, 0, A, B,
-                                        n, heads, st);
+        return launch_stream<64, false, false>(Q, mem, row_stride, T_cap, nullptr, nullptr, pos, 0,
+                                               A, B, n, heads, ProjIn{}, st);
     if (dh == 128)
-        return launch_stream<128, false>(Q, mem, row_stride, T_cap, nullptr, nullptr, pos, 0, A,
-                                         B, n, heads, st);
+        return launch_stream<128, false, false>(Q, mem, row_stride, T_cap, nullptr, nullptr, pos,
+                                                0, A, B, n, heads, ProjIn{}, st);
     return false;
 }
 
@@ -326,12 +392,39 @@ bool launch_attn_swa_fast(const float* Q, const bf16* Kc, const bf16* Vc, const 
     if (B * n <= 0) return true;
     const int slots = W > 1 ? W - 1 : 1;
     if (dh == 64)
-        return launch_stream<64, true>(Q, ring, row_stride, slots, Kc, Vc, pos, W, A, B, n, heads,
-                                       st);
+        return launch_stream<64, true, false>(Q, ring, row_stride, slots, Kc, Vc, pos, W, A, B, n,
+                                              heads, ProjIn{}, st);
     if (dh == 128)
-        return launch_stream<128, true>(Q, ring, row_stride, slots, Kc, Vc, pos, W, A, B, n,
-                                        heads, st);
+        return launch_stream<128, true, false>(Q, ring, row_stride, slots, Kc, Vc, pos, W, A, B,
+                                               n, heads, ProjIn{}, st);
     return false;
+}
+
+bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int W,
+                          const int32_t* pos, bf16* A, int B, int n, int heads, int dh,
+                          cudaStream_t st) {
+    // one query group per (sequence, head): the kernel then owns every read
+    // and write of that head's ring for the block
+    if (!fast_attn_enabled() || n > 4 || (dh != 64 && dh != 128)) return false;
+    if (B * n <= 0) return true;
+    const int slots = W > 1 ? W - 1 : 1;
+    if (dh == 64)
+        return launch_stream<64, true, true>(nullptr, ring, row_stride, slots, nullptr, nullptr,
+                                             pos, W, A, B, n, heads, pin, st);
+    return launch_stream<128, true, true>(nullptr, ring, row_stride, slots, nullptr, nullptr, pos,
+                                          W, A, B, n, heads, pin, st);
+}
+
+bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_stride, int T_cap,
+                            const int32_t* pos, bf16* A, int B, int n, int heads, int dh,
+                            cudaStream_t st) {
+    if (!fast_attn_enabled() || (dh != 64 && dh != 128)) return false;
+    if (B * n <= 0) return true;
+    if (dh == 64)
+        return launch_stream<64, false, true>(nullptr, mem, row_stride, T_cap, nullptr, nullptr,
+                                              pos, 0, A, B, n, heads, pin, st);
+    return launch_stream<128, false, true>(nullptr, mem, row_stride, T_cap, nullptr, nullptr, pos,
+                                           0, A, B, n, heads, pin, st);
 }
 
 }  // namespace rlt

@@ -27,7 +27,7 @@ bool launch_attn_swa_fast(const float* Q, const bf16* Kc, const bf16* Vc, const 
                           int heads, int dh, cudaStream_t st);
 
 // RLT_ATTN=warp keeps the decoder on the warp-per-head kernels (diagnostics)
-static bool fast_attn() {
+bool fast_attn_enabled() {
     static int v = -1;
     if (v < 0) {
         const char* e = getenv("RLT_ATTN");
@@ -101,6 +101,7 @@ template <typename T, int DH>
 __global__ void k_attn_enc(const float* __restrict__ Q, const T* __restrict__ cache,
                            size_t row_stride, int T_cap, const int32_t* __restrict__ pos_enc,
                            T* __restrict__ A, int R, int n, int heads) {
+    pdl_enter();
     __shared__ float sm[4 * DH];
     int item = blockIdx.x * 4 + (threadIdx.x >> 5);
     if (item >= R * heads) return;
@@ -121,6 +122,7 @@ __global__ void k_attn_swa(const float* __restrict__ Q, const T* __restrict__ Kc
                            const T* __restrict__ Vc, const T* __restrict__ ring,
                            size_t row_stride, int W, const int32_t* __restrict__ pos_dec,
                            T* __restrict__ A, int R, int n, int heads) {
+    pdl_enter();
     __shared__ float sm[4 * DH];
     int item = blockIdx.x * 4 + (threadIdx.x >> 5);
     if (item >= R * heads) return;
@@ -153,6 +155,7 @@ template <typename T, int DH>
 __global__ void k_attn_cross(const float* __restrict__ Q, const T* __restrict__ mem,
                              size_t row_stride, int T_cap, const int32_t* __restrict__ pos_dec,
                              T* __restrict__ A, int R, int n, int heads) {
+    pdl_enter();
     __shared__ float sm[4 * DH];
     int item = blockIdx.x * 4 + (threadIdx.x >> 5);
     if (item >= R * heads) return;
@@ -190,11 +193,11 @@ void launch_attn_enc(const float* Q, const T* cache, size_t row_stride, int T_ca
     // the encoder's causal attention is the same prefix read as the memory
     // read: queries at pos_enc+1+i over cache keys 1..t
     if constexpr (std::is_same<T, bf16>::value) {
-        if (fast_attn() &&
+        if (fast_attn_enabled() &&
             launch_attn_cross_fast(Q, cache, row_stride, T_cap, pos_enc, A, B, n, heads, dh, st))
             return;
     }
-    RLT_DH_SWITCH(dh, (k_attn_enc<T, DH><<<nblocks(R, heads), 128, 0, st>>>(
+    RLT_DH_SWITCH(dh, (launch(k_attn_enc<T, DH>, nblocks(R, heads), 128, 0, st,
                           Q, cache, row_stride, T_cap, pos_enc, A, R, n, heads)));
     rlt_count_launch();
 }
@@ -206,11 +209,11 @@ void launch_attn_swa(const float* Q, const T* Kc, const T* Vc, const T* ring, si
     int R = B * n;
     if (R <= 0) return;
     if constexpr (std::is_same<T, bf16>::value) {
-        if (fast_attn() &&
+        if (fast_attn_enabled() &&
             launch_attn_swa_fast(Q, Kc, Vc, ring, row_stride, W, pos_dec, A, B, n, heads, dh, st))
             return;
     }
-    RLT_DH_SWITCH(dh, (k_attn_swa<T, DH><<<nblocks(R, heads), 128, 0, st>>>(
+    RLT_DH_SWITCH(dh, (launch(k_attn_swa<T, DH>, nblocks(R, heads), 128, 0, st,
                           Q, Kc, Vc, ring, row_stride, W, pos_dec, A, R, n, heads)));
     rlt_count_launch();
 }
@@ -222,11 +225,11 @@ void launch_attn_cross(const float* Q, const T* mem, size_t row_stride, int T_ca
     int R = B * n;
     if (R <= 0) return;
     if constexpr (std::is_same<T, bf16>::value) {
-        if (fast_attn() &&
+        if (fast_attn_enabled() &&
             launch_attn_cross_fast(Q, mem, row_stride, T_cap, pos_dec, A, B, n, heads, dh, st))
             return;
     }
-    RLT_DH_SWITCH(dh, (k_attn_cross<T, DH><<<nblocks(R, heads), 128, 0, st>>>(
+    RLT_DH_SWITCH(dh, (launch(k_attn_cross<T, DH>, nblocks(R, heads), 128, 0, st,
                           Q, mem, row_stride, T_cap, pos_dec, A, R, n, heads)));
     rlt_count_launch();
 }

@@ -18,6 +18,7 @@ __device__ __forceinline__ float slab_sum(const float* __restrict__ P, int S, si
 template <typename T>
 __global__ void k_embed(const T* __restrict__ E, const int32_t* __restrict__ tok,
                         float* __restrict__ X, int d, int vocab, int* err) {
+    pdl_enter();
     int r = blockIdx.x;
     int id = tok[r];
     bool ok = id >= 0 && id < vocab;
@@ -29,7 +30,7 @@ template <typename T>
 void launch_embed(const T* E, const int32_t* tok, float* X, int R, int d, int vocab, int* err,
                   cudaStream_t st) {
     if (R <= 0) return;
-    k_embed<T><<<R, 128, 0, st>>>(E, tok, X, d, vocab, err);
+    launch(k_embed<T>, R, 128, 0, st, E, tok, X, d, vocab, err);
     rlt_count_launch();
 }
 
@@ -55,6 +56,7 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 template <typename T>
 __global__ void k_rmsnorm(const float* __restrict__ X, int ldx, const float* __restrict__ g,
                           T* __restrict__ Y, int ldy, int d, float eps) {
+    pdl_enter();
     __shared__ float red[33];
     const float* x = X + (size_t)blockIdx.x * ldx;
     float ss = 0.f;
@@ -68,7 +70,7 @@ template <typename T>
 void launch_rmsnorm(const float* X, int ldx, const float* gain, T* Y, int ldy, int R, int d,
                     float eps, cudaStream_t st) {
     if (R <= 0) return;
-    k_rmsnorm<T><<<R, 128, 0, st>>>(X, ldx, gain, Y, ldy, d, eps);
+    launch(k_rmsnorm<T>, R, 128, 0, st, X, ldx, gain, Y, ldy, d, eps);
     rlt_count_launch();
 }
 
@@ -77,6 +79,7 @@ template <typename T>
 __global__ void k_add_rmsnorm(float* __restrict__ Z, const float* __restrict__ P, int S,
                               size_t slab, const float* __restrict__ g, T* __restrict__ Y, int d,
                               float eps) {
+    pdl_enter();
     __shared__ float red[33];
     float* z = Z + (size_t)blockIdx.x * d;
     float ss = 0.f;
@@ -97,7 +100,7 @@ template <typename T>
 void launch_add_rmsnorm(float* Z, const float* P, int S, size_t slab, const float* gain, T* Y,
                         int R, int d, float eps, cudaStream_t st) {
     if (R <= 0) return;
-    k_add_rmsnorm<T><<<R, 128, 0, st>>>(Z, P, S, slab, gain, Y, d, eps);
+    launch(k_add_rmsnorm<T>, R, 128, 0, st, Z, P, S, slab, gain, Y, d, eps);
     rlt_count_launch();
 }
 
@@ -107,6 +110,7 @@ __global__ void k_merge_input(const float* __restrict__ e, int T_cap,
                               const int32_t* __restrict__ pos_dec, const float* __restrict__ fb,
                               const float* __restrict__ g, T* __restrict__ Gin, int n, int d,
                               float eps) {
+    pdl_enter();
     __shared__ float red[33];
     int r = blockIdx.x, b = r / n, i = r % n;
     const float* et = e + ((size_t)b * T_cap + pos_dec[b] + i) * d;
@@ -125,17 +129,24 @@ template <typename T>
 void launch_merge_input(const float* e, int T_cap, const int32_t* pos_dec, const float* fb,
                         const float* gain, T* Gin, int B, int n, int d, float eps,
                         cudaStream_t st) {
-    k_merge_input<T><<<B * n, 128, 0, st>>>(e, T_cap, pos_dec, fb, gain, Gin, n, d, eps);
+    launch(k_merge_input<T>, B * n, 128, 0, st, e, T_cap, pos_dec, fb, gain, Gin, n, d, eps);
     rlt_count_launch();
 }
 
+// z = e_t + alpha * sigma(gate) * projection; with a gain, also Y = RMSNorm(z)
+// (the first decoder block's input norm, same arithmetic as k_add_rmsnorm).
+template <typename T>
 __global__ void k_merge_out(const float* __restrict__ e, int T_cap,
                             const int32_t* __restrict__ pos_dec, const float* __restrict__ G,
                             int nG, size_t slabG, const float* __restrict__ bg,
                             const float* __restrict__ S, int nS, size_t slabS, float alpha,
-                            float* __restrict__ z, int n, int d) {
+                            float* __restrict__ z, int n, int d, const float* __restrict__ g,
+                            T* __restrict__ Y, float eps) {
+    pdl_enter();
+    __shared__ float red[33];
     int r = blockIdx.x, b = r / n, i = r % n;
     const float* et = e + ((size_t)b * T_cap + pos_dec[b] + i) * d;
+    float ss = 0.f;
     for (int j = threadIdx.x; j < d; j += blockDim.x) {
         float u = et[j];
         if (G) {
@@ -144,13 +155,22 @@ __global__ void k_merge_out(const float* __restrict__ e, int T_cap,
             u += alpha * gate * slab_sum(S, nS, slabS, (size_t)r * d + j);
         }
         z[(size_t)r * d + j] = u;
+        ss += u * u;
     }
+    if (!g) return;
+    ss = block_sum(ss, red);
+    float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    T* y = Y + (size_t)r * d;
+    for (int j = threadIdx.x; j < d; j += blockDim.x)
+        y[j] = from_f<T>(z[(size_t)r * d + j] * inv * g[j]);
 }
+template <typename T>
 void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const float* G, int nG,
                       size_t slabG, const float* bg, const float* S, int nS, size_t slabS,
-                      float alpha, float* z, int B, int n, int d, cudaStream_t st) {
-    k_merge_out<<<B * n, 128, 0, st>>>(e, T_cap, pos_dec, G, nG, slabG, bg, S, nS, slabS, alpha,
-                                       z, n, d);
+                      float alpha, float* z, const float* gain, T* Y, float eps, int B, int n,
+                      int d, cudaStream_t st) {
+    launch(k_merge_out<T>, B * n, 128, 0, st, e, T_cap, pos_dec, G, nG, slabG, bg, S, nS, slabS,
+           alpha, z, n, d, gain, Y, eps);
     rlt_count_launch();
 }
 
@@ -166,6 +186,7 @@ __global__ void k_qkv_dec(const float* __restrict__ QKV, int S, size_t slab,
                           const int32_t* __restrict__ pos_dec, RopeTab rope,
                           float* __restrict__ Q, T* __restrict__ Kc, T* __restrict__ Vc, int n,
                           int heads, int dh) {
+    pdl_enter();
     int r = blockIdx.x, b = r / n, i = r % n;
     int d = heads * dh, half = dh / 2;
     int t = pos_dec[b] + 1 + i;
@@ -189,7 +210,7 @@ __global__ void k_qkv_dec(const float* __restrict__ QKV, int S, size_t slab,
 template <typename T>
 void launch_qkv_dec(const float* QKV, int S, size_t slab, const int32_t* pos_dec, RopeTab rope,
                     float* Q, T* Kc, T* Vc, int B, int n, int heads, int dh, cudaStream_t st) {
-    k_qkv_dec<T><<<B * n, 128, 0, st>>>(QKV, S, slab, pos_dec, rope, Q, Kc, Vc, n, heads, dh);
+    launch(k_qkv_dec<T>, B * n, 128, 0, st, QKV, S, slab, pos_dec, rope, Q, Kc, Vc, n, heads, dh);
     rlt_count_launch();
 }
 
@@ -198,6 +219,7 @@ template <typename T>
 __global__ void k_qkv_enc(const float* __restrict__ QKV, const int32_t* __restrict__ pos_enc,
                           RopeTab rope, float* __restrict__ Q, T* __restrict__ cache,
                           size_t row_stride, int T_cap, int n, int heads, int dh) {
+    pdl_enter();
     int r = blockIdx.x, b = r / n, i = r % n;
     int d = heads * dh, half = dh / 2;
     int p = pos_enc[b] + 1 + i;
@@ -224,7 +246,7 @@ template <typename T>
 void launch_qkv_enc(const float* QKV, const int32_t* pos_enc, RopeTab rope, float* Q, T* cache,
                     size_t row_stride, int T_cap, int B, int n, int heads, int dh,
                     cudaStream_t st) {
-    k_qkv_enc<T><<<B * n, 128, 0, st>>>(QKV, pos_enc, rope, Q, cache, row_stride, T_cap, n,
+    launch(k_qkv_enc<T>, B * n, 128, 0, st, QKV, pos_enc, rope, Q, cache, row_stride, T_cap, n,
                                         heads, dh);
     rlt_count_launch();
 }
@@ -233,6 +255,7 @@ template <typename T>
 __global__ void k_mem_scatter(const float* __restrict__ KV, const int32_t* __restrict__ pos_enc,
                               RopeTab rope, T* __restrict__ mem, size_t row_stride, int T_cap,
                               int n, int heads, int dh) {
+    pdl_enter();
     int r = blockIdx.x, b = r / n, i = r % n;
     int d = heads * dh, half = dh / 2;
     int p = pos_enc[b] + 1 + i;
@@ -256,7 +279,7 @@ template <typename T>
 void launch_mem_scatter(const float* KV, const int32_t* pos_enc, RopeTab rope, T* mem,
                         size_t row_stride, int T_cap, int B, int n, int heads, int dh,
                         cudaStream_t st) {
-    k_mem_scatter<T><<<B * n, 128, 0, st>>>(KV, pos_enc, rope, mem, row_stride, T_cap, n, heads,
+    launch(k_mem_scatter<T>, B * n, 128, 0, st, KV, pos_enc, rope, mem, row_stride, T_cap, n, heads,
                                             dh);
     rlt_count_launch();
 }
@@ -264,6 +287,7 @@ void launch_mem_scatter(const float* KV, const int32_t* pos_enc, RopeTab rope, T
 __global__ void k_rope_q(const float* __restrict__ P, int S, size_t slab,
                          float* __restrict__ Q, const int32_t* __restrict__ pos_dec,
                          RopeTab rope, int n, int heads, int dh) {
+    pdl_enter();
     int r = blockIdx.x, b = r / n, i = r % n;
     int d = heads * dh, half = dh / 2;
     int t = pos_dec[b] + 1 + i;
@@ -280,7 +304,7 @@ __global__ void k_rope_q(const float* __restrict__ P, int S, size_t slab,
 }
 void launch_rope_q(const float* P, int S, size_t slab, float* Q, const int32_t* pos_dec,
                    RopeTab rope, int B, int n, int heads, int dh, cudaStream_t st) {
-    k_rope_q<<<B * n, 128, 0, st>>>(P, S, slab, Q, pos_dec, rope, n, heads, dh);
+    launch(k_rope_q, B * n, 128, 0, st, P, S, slab, Q, pos_dec, rope, n, heads, dh);
     rlt_count_launch();
 }
 
@@ -288,6 +312,7 @@ void launch_rope_q(const float* P, int S, size_t slab, float* Q, const int32_t* 
 template <typename T>
 __global__ void k_swiglu(const float* __restrict__ H, int S, size_t slab, int fpad,
                          T* __restrict__ Hd) {
+    pdl_enter();
     int r = blockIdx.x;
     const size_t base = (size_t)r * 2 * fpad;
     for (int j = threadIdx.x; j < fpad; j += blockDim.x) {
@@ -298,26 +323,30 @@ __global__ void k_swiglu(const float* __restrict__ H, int S, size_t slab, int fp
 }
 template <typename T>
 void launch_swiglu(const float* H, int S, size_t slab, int fpad, T* Hd, int R, cudaStream_t st) {
-    k_swiglu<T><<<R, 256, 0, st>>>(H, S, slab, fpad, Hd);
+    launch(k_swiglu<T>, R, 256, 0, st, H, S, slab, fpad, Hd);
     rlt_count_launch();
 }
 
 // ---------------------------------------------------------------- state bookkeeping
 __global__ void k_copy_e(const float* __restrict__ X, const int32_t* __restrict__ pos_enc,
                          float* __restrict__ e, int T_cap, int n, int d) {
+    pdl_enter();
     int r = blockIdx.x, b = r / n, i = r % n;
     float* dst = e + ((size_t)b * T_cap + pos_enc[b] + i) * d;
     for (int j = threadIdx.x; j < d; j += blockDim.x) dst[j] = X[(size_t)r * d + j];
 }
 void launch_copy_e(const float* X, const int32_t* pos_enc, float* e, int T_cap, int B, int n,
                    int d, cudaStream_t st) {
-    k_copy_e<<<B * n, 128, 0, st>>>(X, pos_enc, e, T_cap, n, d);
+    launch(k_copy_e, B * n, 128, 0, st, X, pos_enc, e, T_cap, n, d);
     rlt_count_launch();
 }
 
+// s <- last row of z (+ residual slabs); RLT-2 register when the chunk ends;
+// with `bump`, also pos_dec += n once every thread has read it.
 __global__ void k_set_state(const float* __restrict__ z, const float* __restrict__ P, int S,
                             size_t slab, float* __restrict__ s, float* __restrict__ Rr,
-                            const int32_t* __restrict__ pos_dec, int chunk, int n, int d) {
+                            int32_t* __restrict__ pos_dec, int chunk, int n, int d, int bump) {
+    pdl_enter();
     int b = blockIdx.x;
     bool upd = Rr != nullptr && ((pos_dec[b] + n) % chunk) == 0;
     const size_t row = ((size_t)b * n + n - 1) * d;
@@ -327,19 +356,25 @@ __global__ void k_set_state(const float* __restrict__ z, const float* __restrict
         s[(size_t)b * d + j] = v;
         if (upd) Rr[(size_t)b * d + j] = v;
     }
+    if (bump) {
+        __syncthreads();
+        if (threadIdx.x == 0) pos_dec[b] += n;
+    }
 }
 void launch_set_state(const float* z, const float* P, int S, size_t slab, float* s, float* Rreg,
-                      const int32_t* pos_dec, int chunk, int B, int n, int d, cudaStream_t st) {
-    k_set_state<<<B, 128, 0, st>>>(z, P, S, slab, s, Rreg, pos_dec, chunk, n, d);
+                      int32_t* pos_dec, int chunk, int B, int n, int d, bool bump,
+                      cudaStream_t st) {
+    launch(k_set_state, B, 128, 0, st, z, P, S, slab, s, Rreg, pos_dec, chunk, n, d, (int)bump);
     rlt_count_launch();
 }
 
 __global__ void k_pos_add(int32_t* pos, int B, int n) {
+    pdl_enter();
     int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b < B) pos[b] += n;
 }
 void launch_pos_add(int32_t* pos, int B, int n, cudaStream_t st) {
-    k_pos_add<<<(B + 255) / 256, 256, 0, st>>>(pos, B, n);
+    launch(k_pos_add, (B + 255) / 256, 256, 0, st, pos, B, n);
     rlt_count_launch();
 }
 
@@ -347,6 +382,7 @@ __global__ void k_reset_rows(const int32_t* __restrict__ rows, const float* __re
                              float* __restrict__ s, float* __restrict__ Rr,
                              int32_t* __restrict__ pos_enc, int32_t* __restrict__ pos_dec,
                              int d) {
+    pdl_enter();
     int b = rows ? rows[blockIdx.x] : blockIdx.x;
     for (int j = threadIdx.x; j < d; j += blockDim.x) {
         float v = s_star ? s_star[j] : 0.f;
@@ -361,7 +397,7 @@ __global__ void k_reset_rows(const int32_t* __restrict__ rows, const float* __re
 void launch_reset_rows(const int32_t* rows, int nrows, const float* s_star, float* s, float* Rr,
                        int32_t* pos_enc, int32_t* pos_dec, int d, cudaStream_t st) {
     if (nrows <= 0) return;
-    k_reset_rows<<<nrows, 128, 0, st>>>(rows, s_star, s, Rr, pos_enc, pos_dec, d);
+    launch(k_reset_rows, nrows, 128, 0, st, rows, s_star, s, Rr, pos_enc, pos_dec, d);
     rlt_count_launch();
 }
 
@@ -372,6 +408,7 @@ template <typename T>
 __global__ void k_ring_write(const T* __restrict__ Kc, const T* __restrict__ Vc,
                              const int32_t* __restrict__ pos_dec, T* __restrict__ ring,
                              size_t row_stride, int W, int n, int heads, int dh) {
+    pdl_enter();
     int r = blockIdx.x, b = r / n, i = r % n;
     int slots = W - 1;
     if (i < n - slots) return;
@@ -392,7 +429,7 @@ void launch_ring_write(const T* Kc, const T* Vc, const int32_t* pos_dec, T* ring
                        size_t row_stride, int W, int B, int n, int heads, int dh,
                        cudaStream_t st) {
     if (W <= 1) return;
-    k_ring_write<T><<<B * n, 128, 0, st>>>(Kc, Vc, pos_dec, ring, row_stride, W, n, heads, dh);
+    launch(k_ring_write<T>, B * n, 128, 0, st, Kc, Vc, pos_dec, ring, row_stride, W, n, heads, dh);
     rlt_count_launch();
 }
 
@@ -401,6 +438,10 @@ void launch_ring_write(const T* Kc, const T* Vc, const int32_t* pos_dec, T* ring
                                   cudaStream_t);                                               \
     template void launch_rmsnorm<T>(const float*, int, const float*, T*, int, int, int, float, \
                                     cudaStream_t);                                             \
+    template void launch_merge_out<T>(const float*, int, const int32_t*, const float*, int,    \
+                                      size_t, const float*, const float*, int, size_t, float,  \
+                                      float*, const float*, T*, float, int, int, int,          \
+                                      cudaStream_t);                                           \
     template void launch_merge_input<T>(const float*, int, const int32_t*, const float*,       \
                                         const float*, T*, int, int, int, float, cudaStream_t); \
     template void launch_qkv_dec<T>(const float*, int, size_t, const int32_t*, RopeTab, float*, \

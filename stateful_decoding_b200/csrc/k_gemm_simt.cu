@@ -15,6 +15,7 @@ template <typename T, int MODE>
 __global__ void __launch_bounds__(NT)
 k_gemm_simt(const T* __restrict__ A, int lda, const T* __restrict__ W, int ldw,
             float* __restrict__ C, int ldc, T* __restrict__ Ct, int ldct, int M, int N, int K) {
+    pdl_enter();
     __shared__ float As[BK][BM + 4];
     __shared__ float Ws[BK][BN + 4];
     int tid = threadIdx.x;
@@ -68,11 +69,11 @@ void launch_gemm_simt(const T* A, int lda, const T* W, int ldw, float* C, int ld
     if (M <= 0 || N <= 0) return;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
     if (mode == kStoreF32)
-        k_gemm_simt<T, kStoreF32><<<grid, NT, 0, st>>>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K);
+        launch(k_gemm_simt<T, kStoreF32>, grid, NT, 0, st, A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K);
     else if (mode == kAddF32)
-        k_gemm_simt<T, kAddF32><<<grid, NT, 0, st>>>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K);
+        launch(k_gemm_simt<T, kAddF32>, grid, NT, 0, st, A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K);
     else
-        k_gemm_simt<T, kStoreT><<<grid, NT, 0, st>>>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K);
+        launch(k_gemm_simt<T, kStoreT>, grid, NT, 0, st, A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K);
     rlt_count_launch();
 }
 

@@ -78,6 +78,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tmem_base;
+    // the set-up above touches no global memory: it overlaps the previous
+    // kernel of the stream; operands are read only after it has finished
+    pdl_enter();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -119,18 +122,56 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
             fence_after_sync();
             const int q = warp & 3;
             const int row = m0 + 32 * q + lane;
+            const bool vec = MODE == kStoreT
+                                 ? ((ldct & 7) == 0 && ((uintptr_t)Ct & 15) == 0)
+                                 : ((ldc & 3) == 0 && ((uintptr_t)C & 15) == 0);
 #pragma unroll 1
             for (int c = 0; c < BN; c += 16) {
                 float v[16];
                 tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c, v);
                 if (row < M) {
+                    const int col0 = n0 + c;
+                    if (vec && col0 + 16 <= N) {
+                        // 16 consecutive outputs of this row: 16-byte stores
+                        if (MODE == kStoreT) {
+                            uint4* dst = reinterpret_cast<uint4*>(Ct + (size_t)row * ldct + col0);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int col = n0 + c + j;
-                        if (col < N) {
-                            if (MODE == kStoreF32) C[(size_t)row * ldc + col] = v[j];
-                            else if (MODE == kAddF32) C[(size_t)row * ldc + col] += v[j];
-                            else Ct[(size_t)row * ldct + col] = __float2bfloat16_rn(v[j]);
+                            for (int u = 0; u < 2; ++u) {
+                                uint4 w;
+                                uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    __nv_bfloat162 p2 =
+                                        __floats2bfloat162_rn(v[8 * u + 2 * k], v[8 * u + 2 * k + 1]);
+                                    wp[k] = *reinterpret_cast<uint32_t*>(&p2);
+                                }
+                                dst[u] = w;
+                            }
+                        } else {
+                            float4* dst = reinterpret_cast<float4*>(C + (size_t)row * ldc + col0);
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                float4 w = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2],
+                                                       v[4 * u + 3]);
+                                if (MODE == kAddF32) {
+                                    const float4 o = dst[u];
+                                    w.x += o.x;
+                                    w.y += o.y;
+                                    w.z += o.z;
+                                    w.w += o.w;
+                                }
+                                dst[u] = w;
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int col = col0 + j;
+                            if (col < N) {
+                                if (MODE == kStoreF32) C[(size_t)row * ldc + col] = v[j];
+                                else if (MODE == kAddF32) C[(size_t)row * ldc + col] += v[j];
+                                else Ct[(size_t)row * ldct + col] = __float2bfloat16_rn(v[j]);
+                            }
                         }
                     }
                 }
@@ -196,7 +237,7 @@ bool launch_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc
     }
     const int nk = K / BK, cps = (nk + splits - 1) / splits;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, (nk + cps - 1) / cps);
-    k_gemm_tc<BN, MODE><<<grid, NTHREADS, smem_bytes<BN>(), st>>>(ta, tb, C, ldc, Ct, ldct, M, N,
+    launch(k_gemm_tc<BN, MODE>, grid, NTHREADS, smem_bytes<BN>(), st, ta, tb, C, ldc, Ct, ldct, M, N,
                                                                  K, cps, slab);
     rlt_count_launch();
     return true;

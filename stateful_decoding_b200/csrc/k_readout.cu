@@ -25,6 +25,7 @@ __device__ __forceinline__ double sampler_uniform(uint64_t seed, uint64_t row, u
 __global__ void __launch_bounds__(NT)
 k_sample(const float* __restrict__ logits, int V, int32_t* __restrict__ argmax_out,
          int32_t* __restrict__ sampled_out, uint64_t seed, uint64_t step, float temperature) {
+    pdl_enter();
     __shared__ float s_val[NT];
     __shared__ int s_idx[NT];
     __shared__ double s_sum[NT];
@@ -99,7 +100,7 @@ k_sample(const float* __restrict__ logits, int V, int32_t* __restrict__ argmax_o
 void launch_sample(const float* logits, int V, int B, int32_t* argmax, int32_t* sampled,
                    uint64_t seed, uint64_t step, float temperature, cudaStream_t st) {
     if (B <= 0 || (!argmax && !sampled)) return;
-    k_sample<<<B, NT, 0, st>>>(logits, V, argmax, sampled, seed, step, temperature);
+    launch(k_sample, B, NT, 0, st, logits, V, argmax, sampled, seed, step, temperature);
     rlt_count_launch();
 }
 

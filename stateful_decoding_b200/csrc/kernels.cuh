@@ -44,9 +44,12 @@ void launch_merge_input(const float* e, int T_cap, const int32_t* pos_dec, const
                         const float* gain, T* Gin, int B, int n, int d, float eps, cudaStream_t st);
 // z[r] = e_t + alpha * sigmoid(G[r] + bg) * S[r]   (S = W_s r); alpha ignored if G == nullptr.
 // G and S may be split-K partial slabs (nG / nS slabs, slabG / slabS apart).
+// With a gain (non-null), also Y[r] = RMSNorm(z[r]) * gain.
+template <typename T>
 void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const float* G, int nG,
                       size_t slabG, const float* bg, const float* S, int nS, size_t slabS,
-                      float alpha, float* z, int B, int n, int d, cudaStream_t st);
+                      float alpha, float* z, const float* gain, T* Y, float eps, int B, int n,
+                      int d, cudaStream_t st);
 // z += sum of residual partial slabs P (P may be null), then Y = RMSNorm(z)
 template <typename T>
 void launch_add_rmsnorm(float* Z, const float* P, int S, size_t slab, const float* gain, T* Y,
@@ -75,9 +78,10 @@ void launch_swiglu(const float* H, int S, size_t slab, int fpad, T* Hd, int R, c
 void launch_copy_e(const float* X, const int32_t* pos_enc, float* e, int T_cap, int B, int n,
                    int d, cudaStream_t st);
 // s[b] = z[b*n + n-1] (+ its residual partial slabs); RLT-2: R[b] = s[b] when
-// (pos_dec[b]+n) % chunk == 0
+// (pos_dec[b]+n) % chunk == 0; with bump, then pos_dec[b] += n
 void launch_set_state(const float* z, const float* P, int S, size_t slab, float* s, float* Rreg,
-                      const int32_t* pos_dec, int chunk, int B, int n, int d, cudaStream_t st);
+                      int32_t* pos_dec, int chunk, int B, int n, int d, bool bump,
+                      cudaStream_t st);
 void launch_pos_add(int32_t* pos, int B, int n, cudaStream_t st);
 void launch_reset_rows(const int32_t* rows, int nrows, const float* s_star, float* s, float* Rr,
                        int32_t* pos_enc, int32_t* pos_dec, int d, cudaStream_t st);
@@ -105,6 +109,26 @@ void launch_sample(const float* logits, int V, int B, int32_t* argmax, int32_t* 
                    uint64_t seed, uint64_t step, float temperature, cudaStream_t st);
 
 int read_and_clear_device_error();  // device error word of the bounded-wait kernels
-int read_and_clear_attn_error();    // same, for the streaming attention kernels
+int read_and_clear_attn_error();
+// Partial-sum slabs of a projection, consumed directly by an attention kernel.
+struct ProjIn {
+    const float* P;   // slab 0 of the fp32 partial sums, [R][ldp]
+    int S;            // number of slabs, summed in slab order
+    size_t slab;      // elements from one slab to the next
+    int ldp;          // row pitch: 3d for the fused q|k|v projection, d for q alone
+    RopeTab rope;
+};
+// bf16 decoder attention that forms q (and, for the window attention, the
+// block's own k and v, which it then writes into the ring) from the
+// projection slabs.  They return false, launching nothing, for shapes they do
+// not handle; the caller then runs the RoPE scatter and the plain kernels.
+bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int W,
+                          const int32_t* pos_dec, bf16* A, int B, int n, int heads, int dh,
+                          cudaStream_t st);
+bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_stride, int T_cap,
+                            const int32_t* pos_dec, bf16* A, int B, int n, int heads, int dh,
+                            cudaStream_t st);
+bool fast_attn_enabled();           // false when RLT_ATTN=warp
+    // same, for the streaming attention kernels
 
 }  // namespace rlt

@@ -25,6 +25,15 @@ static std::atomic<uint64_t> g_launches{0};
 void rlt_count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 namespace rlt {
+// Programmatic dependent launch between consecutive kernels of a stream
+// (and of a captured graph); RLT_PDL=0 launches them plainly.
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char* e = getenv("RLT_PDL");
+        return !(e && strcmp(e, "0") == 0);
+    }();
+    return on;
+}
 template <typename T>
 void launch_gemm(const T* A, int lda, const T* W, int ldw, float* C, int ldc, T* Ct, int ldct,
                  int M, int N, int K, int mode, cudaStream_t st);
@@ -478,6 +487,7 @@ struct rlt_state {
     size_t bytes = 0;
     // live timing (rlt_profile_*)
     bool prof = false;
+    int prof_level = 0;               // 2: transition blocks run launch by launch
     struct ProfRec { int cls; cudaEvent_t a, b; double bytes; };
     std::vector<ProfRec> prof_recs;
     std::vector<cudaEvent_t> prof_pool;
@@ -846,9 +856,11 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
         return launch_gemm_split<T>(Ain, lda, Wt, K, dst, N, R, N, K, dec_splits(s, N, K), slab,
                                     st);
     };
+    // the merge kernel also applies the first decoder block's input RMSNorm
+    const float* norm0 = c.n_dec > 0 ? m->dec[0].swa_norm : nullptr;
     if (c.variant == 0) {
-        launch_merge_out(s->e, s->T_cap, s->pos_dec, nullptr, 0, 0, nullptr, nullptr, 0, 0, 0.f, z,
-                         B, n, d, st);
+        launch_merge_out<T>(s->e, s->T_cap, s->pos_dec, nullptr, 0, 0, nullptr, nullptr, 0, 0, 0.f,
+                            z, norm0, Y, eps, B, n, d, st);
     } else {
         const float* fb = c.variant == 2 ? s->Rr : s->s;
         launch_merge_input<T>(s->e, s->T_cap, s->pos_dec, fb, m->merge_norm, Y, B, n, d, eps, st);
@@ -856,8 +868,8 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
         float* P2 = P + (size_t)R * d;
         const int nG = gemm_p(Y, 2 * d, (const T*)m->wg, d, 2 * d, P);
         const int nS = gemm_p(Y + d, 2 * d, (const T*)m->ws, d, d, P2);
-        launch_merge_out(s->e, s->T_cap, s->pos_dec, P, nG, slab, m->bg, P2, nS, slab,
-                         (float)c.alpha, z, B, n, d, st);
+        launch_merge_out<T>(s->e, s->T_cap, s->pos_dec, P, nG, slab, m->bg, P2, nS, slab,
+                            (float)c.alpha, z, norm0, Y, eps, B, n, d, st);
     }
     const size_t layer_ring = (size_t)2 * h * std::max(0, c.window - 1) * dh;
     const size_t layer_mem = (size_t)2 * h * s->T_cap * dh;
@@ -865,23 +877,41 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
     for (int l = 0; l < c.n_dec; ++l) {
         const DecLayerW& L = m->dec[l];
         T* ring = (T*)s->ring + l * layer_ring;
-        launch_add_rmsnorm<T>(z, nres ? P : nullptr, nres, slab, L.swa_norm, Y, R, d, eps, st);
+        if (l > 0)
+            launch_add_rmsnorm<T>(z, nres ? P : nullptr, nres, slab, L.swa_norm, Y, R, d, eps, st);
         int np = gemm_p(Y, d, (const T*)L.wqkv, 3 * d, d, P);
-        launch_qkv_dec<T>(P, np, slab, s->pos_dec, rope_of(s), s->Q, Kc, Vc, B, n, h, dh, st);
         {
+            // bf16: the attention kernel forms q, k, v from the slabs and
+            // updates the ring itself; otherwise scatter, attend, write
             ProfScope ps(s, RLT_PROF_SWA, st, s->prof ? swa_bytes(s, n) : 0.0);
-            launch_attn_swa<T>(s->Q, Kc, Vc, ring, s->ring_row, c.window, s->pos_dec, A, B, n, h,
-                               dh, st);
+            bool done = false;
+            if constexpr (std::is_same<T, bf16>::value)
+                done = launch_attn_swa_proj(ProjIn{P, np, slab, 3 * d, rope_of(s)}, ring,
+                                            s->ring_row, c.window, s->pos_dec, A, B, n, h, dh, st);
+            if (!done) {
+                launch_qkv_dec<T>(P, np, slab, s->pos_dec, rope_of(s), s->Q, Kc, Vc, B, n, h, dh,
+                                  st);
+                launch_attn_swa<T>(s->Q, Kc, Vc, ring, s->ring_row, c.window, s->pos_dec, A, B, n,
+                                   h, dh, st);
+                launch_ring_write<T>(Kc, Vc, s->pos_dec, ring, s->ring_row, c.window, B, n, h, dh,
+                                     st);
+            }
         }
-        launch_ring_write<T>(Kc, Vc, s->pos_dec, ring, s->ring_row, c.window, B, n, h, dh, st);
         nres = gemm_p(A, d, (const T*)L.wo, d, d, P);
         launch_add_rmsnorm<T>(z, P, nres, slab, L.x_norm, Y, R, d, eps, st);
         np = gemm_p(Y, d, (const T*)L.xq, d, d, P);
-        launch_rope_q(P, np, slab, s->Q, s->pos_dec, rope_of(s), B, n, h, dh, st);
         const T* mem = (const T*)s->mem + (c.groups > 1 ? l : 0) * layer_mem;
         {
             ProfScope ps(s, RLT_PROF_XATTN, st, s->prof ? xattn_bytes(s, n) : 0.0);
-            launch_attn_cross<T>(s->Q, mem, s->mem_row, s->T_cap, s->pos_dec, A, B, n, h, dh, st);
+            bool done = false;
+            if constexpr (std::is_same<T, bf16>::value)
+                done = launch_attn_cross_proj(ProjIn{P, np, slab, d, rope_of(s)}, mem, s->mem_row,
+                                              s->T_cap, s->pos_dec, A, B, n, h, dh, st);
+            if (!done) {
+                launch_rope_q(P, np, slab, s->Q, s->pos_dec, rope_of(s), B, n, h, dh, st);
+                launch_attn_cross<T>(s->Q, mem, s->mem_row, s->T_cap, s->pos_dec, A, B, n, h, dh,
+                                     st);
+            }
         }
         nres = gemm_p(A, d, (const T*)L.xo, d, d, P);
         launch_add_rmsnorm<T>(z, P, nres, slab, L.ffn_norm, Y, R, d, eps, st);
@@ -890,8 +920,7 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
         nres = gemm_p(Hd, fp, (const T*)L.w2, d, fp, P);
     }
     launch_set_state(z, nres ? P : nullptr, nres, slab, s->s, c.variant == 2 ? s->Rr : nullptr,
-                     s->pos_dec, c.chunk, B, n, d, st);
-    launch_pos_add(s->pos_dec, B, n, st);
+                     s->pos_dec, c.chunk, B, n, d, /*bump=*/true, st);
 }
 
 static int run_block(rlt_state* s, int n, cudaStream_t st) {
@@ -1042,7 +1071,7 @@ extern "C" int rlt_prefill(rlt_state* s, int T, void* stream) {
         // whole blocks of the regular shape go through a replayed graph
         const bool regular = c.variant == 1 || (c.variant == 2 && n == c.chunk) ||
                              (c.variant == 0 && n == s->n_dec_blk);
-        if (regular && graphs_enabled(st) && T - done >= kGraphBlocks * n) {
+        if (regular && graphs_enabled(st) && s->prof_level < 2 && T - done >= kGraphBlocks * n) {
             int rc = run_graph(s, n, st);
             if (rc == RLT_OK) {
                 done += kGraphBlocks * n;
@@ -1189,6 +1218,7 @@ extern "C" int rlt_profile_enable(rlt_state* s, int on) {
     }
     s->prof_recs.clear();
     s->prof = on != 0;
+    s->prof_level = on < 0 ? 0 : on;
     return RLT_OK;
 }
 
