@@ -123,6 +123,30 @@ int rlt_prefill(rlt_state* state, int T, void* stream);
 int rlt_readout(rlt_state* state, float* logits, int32_t* argmax, int32_t* sampled,
                 uint64_t rng_seed, uint64_t rng_step, float temperature, void* stream);
 
+/* Readout of caller-supplied state vectors that allocates nothing (no
+ * counterpart in the method: a serving convenience for callers that hold a
+ * model but no state, and may not allocate device memory).  s_rows: device
+ * fp32 [rows][d]; row r is read out exactly as rlt_readout reads out row r of
+ * a state whose s_t equals it (same logits, argmax and sampled id for the
+ * same rng_seed, rng_step, temperature).  Outputs as in rlt_readout: each may
+ * be NULL, device or host memory.
+ * Scratch: a file-scope device array of RLT_READOUT_ROWS_SCRATCH_BYTES (16 MiB)
+ * per device.  A call needs rows*d*(2 for bf16, 4 for fp32) bytes, plus
+ * rows*vocab*4 when `logits` is not a device pointer, plus rows*8, each rounded
+ * up to 256; a call needing more returns RLT_E_ARG and launches nothing (e.g.
+ * vocab 32000, d 2048, bf16, host logits: at most 127 rows).  Nothing in the scratch
+ * has to start at zero.  The first call on a device looks the array's address
+ * up (cudaGetSymbolAddress), which may load the module: make that first call
+ * before any stream capture on the device begins.  All calls on one device
+ * share the one array: calls in flight at the same time (other streams, other
+ * threads) race on it; order them on one stream.
+ * RLT_E_ARG also for a null model or s_rows, s_rows not in device memory,
+ * rows < 0, temperature <= 0.  rows == 0 does nothing. */
+#define RLT_READOUT_ROWS_SCRATCH_BYTES (16u << 20)
+int rlt_readout_rows(const rlt_model* model, const float* s_rows, int rows, float* logits,
+                     int32_t* argmax, int32_t* sampled, uint64_t rng_seed, uint64_t rng_step,
+                     float temperature, void* stream);
+
 /* Host copies of the per-row positions (arrays of `batch` int32; either may
  * be NULL).  pos_enc = tokens encoded, pos_dec = transitions applied. */
 int rlt_state_positions(const rlt_state* state, int32_t* pos_enc, int32_t* pos_dec);

@@ -28,6 +28,7 @@ RLT_OK, RLT_E_ARG, RLT_E_OOM, RLT_E_CAPACITY, RLT_E_ORDER = 0, -1, -2, -3, -4
 RLT_E_BLOB, RLT_E_DEVICE, RLT_E_TIMEOUT, RLT_E_UNSUPPORTED = -5, -6, -7, -8
 PART_S, PART_R, PART_E, PART_MEM, PART_RING, PART_ENC = range(6)
 PROF_XATTN, PROF_SWA, PROF_STEP, PROF_ENC = range(4)
+READOUT_ROWS_SCRATCH_BYTES = 16 << 20      # RLT_READOUT_ROWS_SCRATCH_BYTES
 
 
 class rlt_config(ctypes.Structure):
@@ -50,6 +51,7 @@ _SIGS = {
     "rlt_step": (_i, [_vp, _vp]),
     "rlt_prefill": (_i, [_vp, _i, _vp]),
     "rlt_readout": (_i, [_vp, _vp, _vp, _vp, _u64, _u64, ctypes.c_float, _vp]),
+    "rlt_readout_rows": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _u64, _u64, ctypes.c_float, _vp]),
     "rlt_state_positions": (_i, [_vp, _vp, _vp]),
     "rlt_state_read": (_i, [_vp, _i, _vp, _sz, ctypes.POINTER(_sz), _vp]),
     "rlt_state_check": (_i, [_vp, _vp]),
@@ -169,6 +171,22 @@ def rlt_readout(state, logits=None, argmax=None, sampled=None, rng_seed: int = 0
                             temperature, _stream(stream))
 
 
+def rlt_readout_rows(model, s_rows, rows: int, logits=None, argmax=None, sampled=None,
+                     rng_seed: int = 0, rng_step: int = 0, temperature: float = 1.0,
+                     stream=None) -> int:
+    return _lib.rlt_readout_rows(model, _ptr(s_rows), rows, _ptr(logits), _ptr(argmax),
+                                 _ptr(sampled), rng_seed, rng_step, temperature, _stream(stream))
+
+
+def readout_rows_scratch_bytes(rows: int, d: int, vocab: int, bf16: bool,
+                               host_logits: bool) -> int:
+    """Static scratch a rlt_readout_rows call needs (its limit is
+    READOUT_ROWS_SCRATCH_BYTES)."""
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    return (up(rows * d * (2 if bf16 else 4)) + (up(rows * vocab * 4) if host_logits else 0)
+            + up(rows * 8))
+
+
 def rlt_state_positions(state, pos_enc=None, pos_dec=None) -> int:
     return _lib.rlt_state_positions(state, _ptr(pos_enc), _ptr(pos_dec))
 
@@ -202,6 +220,23 @@ class Model:
         code, self.config = rlt_model_config(self.handle)
         _check(code, "rlt_model_config")
         self.device = device
+
+    def readout_rows(self, s_rows, logits=None, argmax=None, sampled=None, seed=0, step=0,
+                     temperature=1.0, stream=None):
+        """Readout of caller-supplied state vectors (device fp32 [rows][d])
+        with no allocation: the scratch is a static device array."""
+        rows = int(s_rows.shape[0])
+        code = rlt_readout_rows(self.handle, s_rows, rows, logits, argmax, sampled, seed, step,
+                                temperature, stream)
+        if code == RLT_E_ARG:
+            c = self.config
+            host_logits = logits is not None and not getattr(logits, "is_cuda", False)
+            need = readout_rows_scratch_bytes(rows, c.d, c.vocab, c.dtype == 1, host_logits)
+            if need > READOUT_ROWS_SCRATCH_BYTES:
+                raise ValueError(
+                    f"rlt_readout_rows: {rows} rows need {need} bytes of static scratch, more "
+                    f"than its {READOUT_ROWS_SCRATCH_BYTES} bytes; split the rows over calls")
+        return _check(code, "rlt_readout_rows")
 
     def close(self):
         if self.handle:

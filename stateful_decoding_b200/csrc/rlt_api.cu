@@ -15,6 +15,7 @@
 #include <cstring>
 #include <string>
 #include <map>
+#include <mutex>
 #include <vector>
 
 #include "../../include/rlt.h"
@@ -1258,4 +1259,91 @@ extern "C" const char* rlt_strerror(int code) {
         case RLT_E_UNSUPPORTED: return "unsupported configuration";
         default: return "unknown error";
     }
+}
+
+// ============================================================================
+// readout of caller-supplied state vectors, without allocating
+// ============================================================================
+// rlt_readout keeps its scratch (normalised rows, logits, ids) in the state.
+// A caller that holds only a model -- scoring state vectors it exported with
+// rlt_state_read, or candidates of its own -- has no state to lend, and some
+// such callers must not allocate at all: a serving process whose memory pool
+// already owns the rest of the device (a cudaMalloc there fails or evicts),
+// or one whose other streams are in flight (cudaMalloc / cudaFree may
+// synchronise the device and stall them).  This entry point therefore keeps
+// its scratch in a file-scope device array, sized once at build time, and
+// runs the same three kernels as rlt_readout on it.
+namespace {
+static __device__ __align__(256) unsigned char g_rows_scratch[RLT_READOUT_ROWS_SCRATCH_BYTES];
+constexpr int kScratchDevices = 64;
+void* g_rows_scratch_at[kScratchDevices];    // device address, looked up once per device
+std::mutex g_rows_scratch_mu;
+
+void* rows_scratch(int device) {
+    std::lock_guard<std::mutex> lk(g_rows_scratch_mu);
+    if (!g_rows_scratch_at[device]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_rows_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        g_rows_scratch_at[device] = p;
+    }
+    return g_rows_scratch_at[device];
+}
+}  // namespace
+
+extern "C" int rlt_readout_rows(const rlt_model* m, const float* s_rows, int rows, float* logits,
+                                int32_t* argmax, int32_t* sampled, uint64_t seed, uint64_t step,
+                                float temperature, void* stream) {
+    if (!m || !s_rows || rows < 0 || !(temperature > 0.f)) return RLT_E_ARG;
+    if (m->device < 0 || m->device >= kScratchDevices) return RLT_E_DEVICE;
+    if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
+    if (rows == 0) return RLT_OK;
+    if (!is_device_ptr(s_rows)) return RLT_E_ARG;
+    const rlt_config& c = m->cfg;
+    const int d = c.d, V = c.vocab;
+    const bool bf = c.dtype == RLT_DTYPE_BF16;
+    const bool ld = logits && is_device_ptr(logits);
+    const bool ad = argmax && is_device_ptr(argmax);
+    const bool sd = sampled && is_device_ptr(sampled);
+    // scratch: [normalised rows, storage type][logits fp32, unless the
+    // caller's are on the device][argmax, sampled int32], each 256-aligned;
+    // every byte read is written earlier in the same call
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t off_l = up((size_t)rows * d * (bf ? 2 : 4));
+    const size_t off_i = off_l + (ld ? 0 : up((size_t)rows * V * 4));
+    const size_t need = off_i + up((size_t)rows * 2 * 4);
+    if (need > (size_t)RLT_READOUT_ROWS_SCRATCH_BYTES) return RLT_E_ARG;
+    unsigned char* base = (unsigned char*)rows_scratch(m->device);
+    if (!base) return RLT_E_DEVICE;
+    cudaStream_t st = (cudaStream_t)stream;
+    float* lbuf = ld ? logits : (float*)(base + off_l);
+    int32_t* ids = (int32_t*)(base + off_i);
+    int32_t* abuf = argmax ? (ad ? argmax : ids) : nullptr;
+    int32_t* sbuf = sampled ? (sd ? sampled : ids + rows) : nullptr;
+    if (bf) {
+        bf16* Y = (bf16*)base;
+        rlt::launch_rmsnorm<bf16>(s_rows, d, m->out_norm, Y, d, rows, d, (float)c.eps, st);
+        rlt::launch_gemm<bf16>(Y, d, (const bf16*)m->wout, d, lbuf, V, nullptr, 0, rows, V, d,
+                               rlt::kStoreF32, st);
+    } else {
+        float* Y = (float*)base;
+        rlt::launch_rmsnorm<float>(s_rows, d, m->out_norm, Y, d, rows, d, (float)c.eps, st);
+        rlt::launch_gemm<float>(Y, d, (const float*)m->wout, d, lbuf, V, nullptr, 0, rows, V, d,
+                                rlt::kStoreF32, st);
+    }
+    rlt::launch_sample(lbuf, V, rows, abuf, sbuf, seed, step, temperature, st);
+    int rc = launch_status();
+    if (rc) return rc;
+    if (logits && !ld &&
+        cudaMemcpyAsync(logits, lbuf, (size_t)rows * V * 4, cudaMemcpyDeviceToHost, st))
+        return RLT_E_DEVICE;
+    if (argmax && !ad &&
+        cudaMemcpyAsync(argmax, abuf, (size_t)rows * 4, cudaMemcpyDeviceToHost, st))
+        return RLT_E_DEVICE;
+    if (sampled && !sd &&
+        cudaMemcpyAsync(sampled, sbuf, (size_t)rows * 4, cudaMemcpyDeviceToHost, st))
+        return RLT_E_DEVICE;
+    return RLT_OK;
 }

@@ -98,3 +98,19 @@ def test_product_package_never_imports_oracle():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in txt.replace("no fallback", ""), f
 
+
+def test_readout_rows_scratch_limit_matches_header():
+    """The binding's copy of the static scratch size and its size rule agree
+    with the header (and its worked example: vocab 32000, d 2048, bf16, host
+    logits -> at most 127 rows)."""
+    import re
+    hdr = open(os.path.join(ROOT, "include", "rlt.h")).read()
+    m = re.search(r"#define RLT_READOUT_ROWS_SCRATCH_BYTES \((\d+)u << (\d+)\)", hdr)
+    assert m, "scratch size define not found"
+    import importlib
+    sd = importlib.import_module("stateful_decoding_b200")
+    assert sd.READOUT_ROWS_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+    fits = [r for r in range(1, 200)
+            if sd.readout_rows_scratch_bytes(r, 2048, 32000, True, True)
+            <= sd.READOUT_ROWS_SCRATCH_BYTES]
+    assert max(fits) == 127 and "at most 127 rows" in hdr

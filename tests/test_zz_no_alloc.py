@@ -1,0 +1,93 @@
+"""rlt_readout_rows: the readout of caller-supplied state vectors whose scratch
+is a static device array (no allocation in the call), against rlt_readout on
+the same s_t.  Named to be collected last: it must pass alone and after every
+other test of the session has used the device.
+"""
+import numpy as np
+import pytest
+
+import rlt_inputs as ri
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-6      # same kernels on the same inputs: equal in practice
+
+
+@pytest.fixture(scope="module")
+def sd():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from tests.conftest import build_library
+    build_library()
+    import stateful_decoding_b200 as sd
+    return sd
+
+
+@pytest.mark.parametrize("name,B,T", [("parity_bf16", 7, 20), ("tiny_fp32", 3, 9)])
+def test_readout_rows_matches_readout(sd, name, B, T):
+    import torch
+    cfg = ri.CONFIGS[name]
+    W = ri.generate_weights(cfg)
+    model = sd.Model(ri.write_blob(cfg, W))
+    st = sd.State(model, B, T)
+    st.encode(ri.make_tokens(cfg, B, T))
+    st.prefill(T)
+    seed, step, temp = ri.SAMPLE_SEED, 3, 0.8
+    lg = np.zeros((B, cfg.vocab), np.float32)
+    am = np.zeros(B, np.int32)
+    sp = np.zeros(B, np.int32)
+    st.readout(lg, am, sp, seed=seed, step=step, temperature=temp)
+    torch.cuda.synchronize()
+    s_rows = torch.from_numpy(st.read(sd.PART_S).view(np.float32).reshape(B, cfg.d).copy()).cuda()
+
+    stream = torch.cuda.Stream()
+    for call in range(2):          # two calls in a row reuse the one scratch
+        # device outputs
+        lg_d = torch.full((B, cfg.vocab), float("nan"), device="cuda")
+        am_d = torch.full((B,), -1, dtype=torch.int32, device="cuda")
+        sp_d = torch.full((B,), -1, dtype=torch.int32, device="cuda")
+        model.readout_rows(s_rows, lg_d, am_d, sp_d, seed=seed, step=step, temperature=temp,
+                           stream=stream)
+        stream.synchronize()
+        np.testing.assert_allclose(lg_d.cpu().numpy(), lg, atol=TOL, rtol=0)
+        np.testing.assert_array_equal(am_d.cpu().numpy(), am)
+        np.testing.assert_array_equal(sp_d.cpu().numpy(), sp)
+        # host outputs: logits and ids pass through the scratch
+        lg_h = np.full((B, cfg.vocab), np.nan, np.float32)
+        am_h = np.full(B, -1, np.int32)
+        sp_h = np.full(B, -1, np.int32)
+        model.readout_rows(s_rows, lg_h, am_h, sp_h, seed=seed, step=step, temperature=temp,
+                           stream=stream)
+        stream.synchronize()
+        np.testing.assert_allclose(lg_h, lg, atol=TOL, rtol=0)
+        np.testing.assert_array_equal(am_h, am)
+        np.testing.assert_array_equal(sp_h, sp)
+    st.close()
+    model.close()
+
+
+def test_readout_rows_rejects_oversize_and_bad_args(sd):
+    import torch
+    cfg = ri.CONFIGS["parity_bf16"]
+    model = sd.Model(ri.write_blob(cfg, ri.generate_weights(cfg)))
+    limit = sd.READOUT_ROWS_SCRATCH_BYTES
+    fits = max(r for r in range(15000, 17000)
+               if sd.readout_rows_scratch_bytes(r, cfg.d, cfg.vocab, True, False) <= limit)
+    s_big = torch.zeros(fits + 1, cfg.d, device="cuda")
+    am = torch.empty(fits + 1, dtype=torch.int32, device="cuda")
+    lg = torch.empty(fits + 1, cfg.vocab, device="cuda")
+    with pytest.raises(ValueError, match="static scratch"):
+        model.readout_rows(s_big, lg, am)
+    # the largest request that fits runs
+    model.readout_rows(s_big[:fits], lg[:fits], am[:fits])
+    torch.cuda.synchronize()
+    assert (am[:fits].cpu().numpy() >= 0).all()
+    # host input, non-positive temperature
+    code = sd.rlt_readout_rows(model.handle, np.zeros((2, cfg.d), np.float32), 2, None, None,
+                               None)
+    assert code == sd.RLT_E_ARG
+    code = sd.rlt_readout_rows(model.handle, s_big, 2, None, am, None, 0, 0, 0.0)
+    assert code == sd.RLT_E_ARG
+    assert sd.rlt_readout_rows(model.handle, s_big, 0) == 0
+    model.close()
