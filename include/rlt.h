@@ -66,7 +66,8 @@ typedef struct rlt_config {
  * rlt_config fields, seed, tensor count, payload size, checksum) followed by
  * named tensor records in the fixed manifest order of the config.  Errors:
  * RLT_E_BLOB (bad magic/version/manifest/checksum), RLT_E_UNSUPPORTED (head
- * size or shape this build does not run), RLT_E_DEVICE, RLT_E_OOM. */
+ * size other than 16, 32, 64, 128, or width d above 2048), RLT_E_DEVICE,
+ * RLT_E_OOM. */
 int rlt_create(const void* blob, size_t nbytes, int device, rlt_model** out);
 void rlt_destroy(rlt_model* model);
 int rlt_model_config(const rlt_model* model, rlt_config* out);
@@ -179,10 +180,11 @@ uint64_t rlt_kernel_launches(void);
  * (keys/values read, cache entries written, activations in and out; weights
  * excluded).  rlt_profile_query synchronises `stream`, sums the elapsed times
  * of the class since the last enable, and reports launches, total ms and
- * bytes.  Enabling resets the counters.  on = 1 keeps replaying transition
- * blocks as CUDA graphs (then only whole blocks are timed, as RLT_PROF_STEP);
- * on = 2 runs them launch by launch so that the attention launches are timed
- * one by one too (for measurement: slower than the graph replay). */
+ * bytes.  Enabling resets the counters.  on = 1: transition blocks replayed
+ * as CUDA graphs are timed as whole blocks (RLT_PROF_STEP) only; on = 2: they
+ * replay a twin graph with event nodes around each attention launch (those
+ * launches then lose their overlap with the kernel before them) and each
+ * replay is followed by a stream synchronisation: for measurement only. */
 #define RLT_PROF_XATTN 0  /* decoder cross-attention over M_{<=t}        */
 #define RLT_PROF_SWA   1  /* decoder window attention over C^D           */
 #define RLT_PROF_STEP  2  /* one whole transition block (merge .. s_t)   */

@@ -310,9 +310,8 @@ class State:
         return _check(rlt_state_check(self.handle, stream), "rlt_state_check")
 
     def profile(self, on: int):
-        """0: off; 1: time kernel classes, transition blocks still replayed as
-        graphs (timed as whole blocks); 2: blocks run launch by launch so that
-        every attention launch is timed."""
+        """0: off; 1: time kernel classes (graph-replayed transition blocks
+        as whole blocks); 2: also every attention launch inside the graphs."""
         return _check(rlt_profile_enable(self.handle, int(on)), "rlt_profile_enable")
 
     def profile_query(self, cls: int, stream=None):

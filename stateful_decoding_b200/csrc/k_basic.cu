@@ -2,6 +2,8 @@
 // (greeksharifa "Recurrent Looped Transformer 요약 설명" §2.5), RoPE scatters
 // into the encoder cache / memory / window chunk, SwiGLU, state hand-off and
 // the window-cache (ring) update of jiphyeonjeon review §3.3.
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace rlt {
@@ -12,6 +14,59 @@ __device__ __forceinline__ float slab_sum(const float* __restrict__ P, int S, si
     float v = P[i];
     for (int z = 1; z < S; ++z) v += P[(size_t)z * slab + i];
     return v;
+}
+
+// ---------------------------------------------------------------- row kernels
+// The decoder's row kernels give each thread one group of 4 consecutive
+// features (blockDim = d/4 rounded up to a warp), so that every load a thread
+// needs -- the row and each split-K partial slab -- is issued before the
+// first is used: one memory latency per kernel instead of a chain of them.
+constexpr int kMaxSlabs = 8;       // split-K slabs a consumer sums (the splitter caps at this)
+
+__device__ __forceinline__ float4 ld4(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+}
+__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ float4 add4(float4 a, float4 b) {
+    return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+__device__ __forceinline__ float dot4(float4 a) { return a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w; }
+// sum of S partial slabs at element i (4 wide), in slab order
+__device__ __forceinline__ float4 slab_sum4(const float* __restrict__ P, int S, size_t slab,
+                                            size_t i) {
+    float4 t[kMaxSlabs];
+#pragma unroll
+    for (int z = 0; z < kMaxSlabs; ++z)
+        if (z < S) t[z] = ld4(P + (size_t)z * slab + i);
+    float4 v = t[0];
+#pragma unroll
+    for (int z = 1; z < kMaxSlabs; ++z)
+        if (z < S) v = add4(v, t[z]);
+    return v;
+}
+template <typename T> __device__ __forceinline__ void store4(T* p, float4 v);
+template <> __device__ __forceinline__ void store4<float>(float* p, float4 v) { st4(p, v); }
+template <> __device__ __forceinline__ void store4<bf16>(bf16* p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+// Block-wide sum with a fixed order (warp butterfly, then the warp partials
+// in warp order, summed by every thread alike).
+__device__ __forceinline__ float row_sum(float v, float* red) {
+    v = warp_sum(v);
+    const int w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+    if ((threadIdx.x & 31) == 0) red[w] = v;
+    __syncthreads();
+    float s = 0.f;
+    for (int i = 0; i < nw; ++i) s += red[i];
+    return s;
+}
+__host__ __forceinline__ int row_threads(int groups) { return ((groups + 31) / 32) * 32; }
+__device__ __forceinline__ float4 scale4(float4 v, float inv, float4 g) {
+    return make_float4(v.x * inv * g.x, v.y * inv * g.y, v.z * inv * g.z, v.w * inv * g.w);
 }
 
 // ---------------------------------------------------------------- embedding
@@ -76,101 +131,110 @@ void launch_rmsnorm(const float* X, int ldx, const float* gain, T* Y, int ldy, i
 
 // z += sum of the residual partial slabs P (if any), then Y = RMSNorm(z).
 template <typename T>
-__global__ void k_add_rmsnorm(float* __restrict__ Z, const float* __restrict__ P, int S,
+__global__ void __launch_bounds__(512) k_add_rmsnorm(float* __restrict__ Z, const float* __restrict__ P, int S,
                               size_t slab, const float* __restrict__ g, T* __restrict__ Y, int d,
                               float eps) {
     pdl_enter();
-    __shared__ float red[33];
-    float* z = Z + (size_t)blockIdx.x * d;
-    float ss = 0.f;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) {
-        float v = z[j];
+    __shared__ float red[32];
+    const int j = 4 * threadIdx.x;
+    const size_t i = (size_t)blockIdx.x * d + j;
+    const bool act = j < d;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f), gv = v;
+    if (act) {
+        gv = ld4(g + j);
+        v = ld4(Z + i);
         if (P) {
-            v += slab_sum(P, S, slab, (size_t)blockIdx.x * d + j);
-            z[j] = v;
+            v = add4(v, slab_sum4(P, S, slab, i));
+            st4(Z + i, v);
         }
-        ss += v * v;
     }
-    ss = block_sum(ss, red);
-    float inv = 1.0f / sqrtf(ss / (float)d + eps);
-    T* y = Y + (size_t)blockIdx.x * d;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) y[j] = from_f<T>(z[j] * inv * g[j]);
+    const float ss = row_sum(act ? dot4(v) : 0.f, red);
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    if (act) store4<T>(Y + i, scale4(v, inv, gv));
 }
 template <typename T>
 void launch_add_rmsnorm(float* Z, const float* P, int S, size_t slab, const float* gain, T* Y,
                         int R, int d, float eps, cudaStream_t st) {
     if (R <= 0) return;
-    launch(k_add_rmsnorm<T>, R, 128, 0, st, Z, P, S, slab, gain, Y, d, eps);
+    launch(k_add_rmsnorm<T>, R, row_threads(d / 4), 0, st, Z, P, S, slab, gain, Y, d, eps);
     rlt_count_launch();
 }
 
 // ---------------------------------------------------------------- merge
 template <typename T>
-__global__ void k_merge_input(const float* __restrict__ e, int T_cap,
+__global__ void __launch_bounds__(512) k_merge_input(const float* __restrict__ e, int T_cap,
                               const int32_t* __restrict__ pos_dec, const float* __restrict__ fb,
                               const float* __restrict__ g, T* __restrict__ Gin, int n, int d,
                               float eps) {
     pdl_enter();
-    __shared__ float red[33];
-    int r = blockIdx.x, b = r / n, i = r % n;
-    const float* et = e + ((size_t)b * T_cap + pos_dec[b] + i) * d;
-    const float* f = fb + (size_t)b * d;
-    float ss = 0.f;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) ss += f[j] * f[j];
-    ss = block_sum(ss, red);
-    float inv = 1.0f / sqrtf(ss / (float)d + eps);
-    T* out = Gin + (size_t)r * 2 * d;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) {
-        out[j] = from_f<T>(et[j]);
-        out[d + j] = from_f<T>(f[j] * inv * g[j]);
+    __shared__ float red[32];
+    const int r = blockIdx.x, b = r / n, i = r % n;
+    const int j = 4 * threadIdx.x;
+    const bool act = j < d;
+    float4 ev = make_float4(0.f, 0.f, 0.f, 0.f), f = ev, gv = ev;
+    if (act) {
+        ev = ld4(e + ((size_t)b * T_cap + pos_dec[b] + i) * d + j);
+        f = ld4(fb + (size_t)b * d + j);
+        gv = ld4(g + j);
+    }
+    const float ss = row_sum(act ? dot4(f) : 0.f, red);
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    if (act) {
+        T* out = Gin + (size_t)r * 2 * d;
+        store4<T>(out + j, ev);
+        store4<T>(out + d + j, scale4(f, inv, gv));
     }
 }
 template <typename T>
 void launch_merge_input(const float* e, int T_cap, const int32_t* pos_dec, const float* fb,
                         const float* gain, T* Gin, int B, int n, int d, float eps,
                         cudaStream_t st) {
-    launch(k_merge_input<T>, B * n, 128, 0, st, e, T_cap, pos_dec, fb, gain, Gin, n, d, eps);
+    launch(k_merge_input<T>, B * n, row_threads(d / 4), 0, st, e, T_cap, pos_dec, fb, gain, Gin,
+           n, d, eps);
     rlt_count_launch();
 }
 
 // z = e_t + alpha * sigma(gate) * projection; with a gain, also Y = RMSNorm(z)
 // (the first decoder block's input norm, same arithmetic as k_add_rmsnorm).
 template <typename T>
-__global__ void k_merge_out(const float* __restrict__ e, int T_cap,
+__global__ void __launch_bounds__(512) k_merge_out(const float* __restrict__ e, int T_cap,
                             const int32_t* __restrict__ pos_dec, const float* __restrict__ G,
                             int nG, size_t slabG, const float* __restrict__ bg,
                             const float* __restrict__ S, int nS, size_t slabS, float alpha,
                             float* __restrict__ z, int n, int d, const float* __restrict__ g,
                             T* __restrict__ Y, float eps) {
     pdl_enter();
-    __shared__ float red[33];
-    int r = blockIdx.x, b = r / n, i = r % n;
-    const float* et = e + ((size_t)b * T_cap + pos_dec[b] + i) * d;
-    float ss = 0.f;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) {
-        float u = et[j];
+    __shared__ float red[32];
+    const int r = blockIdx.x, b = r / n, i = r % n;
+    const int j = 4 * threadIdx.x;
+    const bool act = j < d;
+    const size_t o = (size_t)r * d + j;
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f), gv = u;
+    if (act) {
+        u = ld4(e + ((size_t)b * T_cap + pos_dec[b] + i) * d + j);
+        if (g) gv = ld4(g + j);
         if (G) {
-            float a = slab_sum(G, nG, slabG, (size_t)r * d + j) + bg[j];
-            float gate = 1.0f / (1.0f + expf(-a));
-            u += alpha * gate * slab_sum(S, nS, slabS, (size_t)r * d + j);
+            const float4 a = add4(slab_sum4(G, nG, slabG, o), ld4(bg + j));
+            const float4 p = slab_sum4(S, nS, slabS, o);
+            u.x += alpha * (1.0f / (1.0f + expf(-a.x))) * p.x;
+            u.y += alpha * (1.0f / (1.0f + expf(-a.y))) * p.y;
+            u.z += alpha * (1.0f / (1.0f + expf(-a.z))) * p.z;
+            u.w += alpha * (1.0f / (1.0f + expf(-a.w))) * p.w;
         }
-        z[(size_t)r * d + j] = u;
-        ss += u * u;
+        st4(z + o, u);
     }
     if (!g) return;
-    ss = block_sum(ss, red);
-    float inv = 1.0f / sqrtf(ss / (float)d + eps);
-    T* y = Y + (size_t)r * d;
-    for (int j = threadIdx.x; j < d; j += blockDim.x)
-        y[j] = from_f<T>(z[(size_t)r * d + j] * inv * g[j]);
+    const float ss = row_sum(act ? dot4(u) : 0.f, red);
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    if (act) store4<T>(Y + o, scale4(u, inv, gv));
 }
 template <typename T>
 void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const float* G, int nG,
                       size_t slabG, const float* bg, const float* S, int nS, size_t slabS,
                       float alpha, float* z, const float* gain, T* Y, float eps, int B, int n,
                       int d, cudaStream_t st) {
-    launch(k_merge_out<T>, B * n, 128, 0, st, e, T_cap, pos_dec, G, nG, slabG, bg, S, nS, slabS,
-           alpha, z, n, d, gain, Y, eps);
+    launch(k_merge_out<T>, B * n, row_threads(d / 4), 0, st, e, T_cap, pos_dec, G, nG, slabG, bg,
+           S, nS, slabS, alpha, z, n, d, gain, Y, eps);
     rlt_count_launch();
 }
 
@@ -309,21 +373,29 @@ void launch_rope_q(const float* P, int S, size_t slab, float* Q, const int32_t* 
 }
 
 // ---------------------------------------------------------------- FFN gate
+// grid (rows, ceil(fpad/4 / 256)): one group of 4 hidden units per thread
 template <typename T>
-__global__ void k_swiglu(const float* __restrict__ H, int S, size_t slab, int fpad,
-                         T* __restrict__ Hd) {
+__global__ void __launch_bounds__(256) k_swiglu(const float* __restrict__ H, int S, size_t slab,
+                                                int fpad, T* __restrict__ Hd) {
     pdl_enter();
-    int r = blockIdx.x;
-    const size_t base = (size_t)r * 2 * fpad;
-    for (int j = threadIdx.x; j < fpad; j += blockDim.x) {
-        float a = slab_sum(H, S, slab, base + j);
-        float silu = a / (1.0f + expf(-a));
-        Hd[(size_t)r * fpad + j] = from_f<T>(silu * slab_sum(H, S, slab, base + fpad + j));
-    }
+    const int r = blockIdx.x;
+    const int j = 4 * (blockIdx.y * blockDim.x + threadIdx.x);
+    if (j >= fpad) return;
+    // interleaved W1;W3 (w13_gate_col): 4 consecutive units share a 64-block
+    const size_t base = (size_t)r * 2 * fpad + w13_gate_col(j);
+    const float4 a = slab_sum4(H, S, slab, base);
+    const float4 u = slab_sum4(H, S, slab, base + 64);
+    float4 y;
+    y.x = a.x / (1.0f + expf(-a.x)) * u.x;
+    y.y = a.y / (1.0f + expf(-a.y)) * u.y;
+    y.z = a.z / (1.0f + expf(-a.z)) * u.z;
+    y.w = a.w / (1.0f + expf(-a.w)) * u.w;
+    store4<T>(Hd + (size_t)r * fpad + j, y);
 }
 template <typename T>
 void launch_swiglu(const float* H, int S, size_t slab, int fpad, T* Hd, int R, cudaStream_t st) {
-    launch(k_swiglu<T>, R, 256, 0, st, H, S, slab, fpad, Hd);
+    if (R <= 0) return;
+    launch(k_swiglu<T>, dim3(R, (fpad / 4 + 255) / 256), 256, 0, st, H, S, slab, fpad, Hd);
     rlt_count_launch();
 }
 
@@ -343,18 +415,19 @@ void launch_copy_e(const float* X, const int32_t* pos_enc, float* e, int T_cap, 
 
 // s <- last row of z (+ residual slabs); RLT-2 register when the chunk ends;
 // with `bump`, also pos_dec += n once every thread has read it.
-__global__ void k_set_state(const float* __restrict__ z, const float* __restrict__ P, int S,
+__global__ void __launch_bounds__(512) k_set_state(const float* __restrict__ z, const float* __restrict__ P, int S,
                             size_t slab, float* __restrict__ s, float* __restrict__ Rr,
                             int32_t* __restrict__ pos_dec, int chunk, int n, int d, int bump) {
     pdl_enter();
-    int b = blockIdx.x;
-    bool upd = Rr != nullptr && ((pos_dec[b] + n) % chunk) == 0;
-    const size_t row = ((size_t)b * n + n - 1) * d;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) {
-        float v = z[row + j];
-        if (P) v += slab_sum(P, S, slab, row + j);
-        s[(size_t)b * d + j] = v;
-        if (upd) Rr[(size_t)b * d + j] = v;
+    const int b = blockIdx.x;
+    const bool upd = Rr != nullptr && ((pos_dec[b] + n) % chunk) == 0;
+    const int j = 4 * threadIdx.x;
+    if (j < d) {
+        const size_t row = ((size_t)b * n + n - 1) * d;
+        float4 v = ld4(z + row + j);
+        if (P) v = add4(v, slab_sum4(P, S, slab, row + j));
+        st4(s + (size_t)b * d + j, v);
+        if (upd) st4(Rr + (size_t)b * d + j, v);
     }
     if (bump) {
         __syncthreads();
@@ -364,7 +437,8 @@ __global__ void k_set_state(const float* __restrict__ z, const float* __restrict
 void launch_set_state(const float* z, const float* P, int S, size_t slab, float* s, float* Rreg,
                       int32_t* pos_dec, int chunk, int B, int n, int d, bool bump,
                       cudaStream_t st) {
-    launch(k_set_state, B, 128, 0, st, z, P, S, slab, s, Rreg, pos_dec, chunk, n, d, (int)bump);
+    launch(k_set_state, B, row_threads(d / 4), 0, st, z, P, S, slab, s, Rreg, pos_dec, chunk, n, d,
+           (int)bump);
     rlt_count_launch();
 }
 

@@ -159,7 +159,7 @@ __device__ __forceinline__ TileRef tile_of(const FusedParams& P, int kind, int l
         case J_W13: {
             const int i = t >> 1, which = t & 1, j = c + CL * i;
             r.map = &P.m_13;
-            r.row = l * 2 * FP + which * FP + j * 64;
+            r.row = l * 2 * FP + j * 128 + which * 64;     // interleaved W1;W3 blocks
             break;
         }
         default: {  // J_W2: output rows t*64.., K over this CTA's hidden chunks c, c+8, c+16

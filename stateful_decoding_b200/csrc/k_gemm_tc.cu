@@ -78,8 +78,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tmem_base;
-    // the set-up above touches no global memory: it overlaps the previous
-    // kernel of the stream; operands are read only after it has finished
+    // The set-up above and the first stages' weight tiles (weights are never
+    // written by a kernel) overlap the previous kernel of the stream; the
+    // activations are read only after it has finished.
+    const int pre = min(nk, STAGES);
+    if (warp == 0 && lane == 0) {
+        for (int kt = 0; kt < pre; ++kt) {
+            mbar_expect_tx(&full[kt], STAGE);
+            tma_load_2d(smem + kt * STAGE + A_BYTES, &tb, (kbeg + kt) * BK, n0, &full[kt]);
+        }
+    }
     pdl_enter();
 
     if (warp == 0) {
@@ -91,9 +99,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                     abort_flag = 1;
                     break;
                 }
-                mbar_expect_tx(&full[s], STAGE);
+                if (kt >= pre) {
+                    mbar_expect_tx(&full[s], STAGE);
+                    tma_load_2d(smem + s * STAGE + A_BYTES, &tb, (kbeg + kt) * BK, n0, &full[s]);
+                }
                 tma_load_2d(smem + s * STAGE, &ta, (kbeg + kt) * BK, m0, &full[s]);
-                tma_load_2d(smem + s * STAGE + A_BYTES, &tb, (kbeg + kt) * BK, n0, &full[s]);
             }
         }
     } else if (warp == 1) {
@@ -118,7 +128,46 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
             if (ok) mma_commit(&accum);
         }
     } else {
-        if (mbar_wait(&accum, 0)) {
+        if (MODE == kSwiGLU) {
+            // columns come in 128-wide groups: 64 gates, then the 64 matching
+            // up projections; unit u of group g0 goes to Ct column (n0+g0)/2+u
+            if (mbar_wait(&accum, 0)) {
+                fence_after_sync();
+                const int q = warp & 3;
+                const int row = m0 + 32 * q + lane;
+                const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+#pragma unroll 1
+                for (int g0 = 0; g0 < BN; g0 += 128) {
+#pragma unroll 1
+                    for (int c = 0; c < 64; c += 16) {
+                        float a[16], u[16];
+                        tmem_ld16(tq + (uint32_t)(g0 + c), a);
+                        tmem_ld16(tq + (uint32_t)(g0 + 64 + c), u);
+                        if (row < M && n0 + g0 + 128 <= N) {
+                            uint4* dst = reinterpret_cast<uint4*>(
+                                Ct + (size_t)row * ldct + (n0 + g0) / 2 + c);
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                uint4 w;
+                                uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const int e = 8 * h + 2 * k;
+                                    const float y0 = a[e] / (1.0f + expf(-a[e])) * u[e];
+                                    const float y1 =
+                                        a[e + 1] / (1.0f + expf(-a[e + 1])) * u[e + 1];
+                                    __nv_bfloat162 p2 = __floats2bfloat162_rn(y0, y1);
+                                    wp[k] = *reinterpret_cast<uint32_t*>(&p2);
+                                }
+                                dst[h] = w;
+                            }
+                        }
+                    }
+                }
+            } else {
+                abort_flag = 1;
+            }
+        } else if (mbar_wait(&accum, 0)) {
             fence_after_sync();
             const int q = warp & 3;
             const int row = m0 + 32 * q + lane;
@@ -250,6 +299,11 @@ bool launch_tc_mode(const bf16* A, int lda, const bf16* W, int ldw, float* C, in
     if (mode == kStoreF32)
         return launch_tc<BN, kStoreF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, splits, slab, st);
     if (splits != 1) return false;          // partial sums only go to fp32 slabs
+    if (mode == kSwiGLU) {
+        if constexpr (BN % 128 == 0)
+            return launch_tc<BN, kSwiGLU>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, 1, 0, st);
+        return false;
+    }
     if (mode == kAddF32)
         return launch_tc<BN, kAddF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, 1, 0, st);
     return launch_tc<BN, kStoreT>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, 1, 0, st);
@@ -268,10 +322,16 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, in
                     int ldct, int M, int N, int K, int mode, int splits, size_t slab,
                     cudaStream_t st) {
     if (M <= 0 || N < 16 || K < BK || K % BK || splits < 1) return false;
+    if (mode == kSwiGLU && (N % 128 || (ldct % 8) || ((uintptr_t)Ct & 15))) return false;
     if (lda % 8 || ldw % 8 || ((uintptr_t)A & 15) || ((uintptr_t)W & 15)) return false;
-    // wide tiles when M alone fills the machine, narrow ones (more CTAs) otherwise
+    // wide tiles when M alone fills the machine, narrow ones (more CTAs)
+    // otherwise; the SwiGLU epilogue needs whole 128-column gate/up groups
     if (M >= 2048)
         return launch_tc_mode<256>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, splits, slab, st);
+    if (mode == kSwiGLU) {
+        if (N % 128 || (ldct % 8) || ((uintptr_t)Ct & 15)) return false;
+        return launch_tc_mode<128>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, 1, 0, st);
+    }
     return launch_tc_mode<64>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, splits, slab, st);
 }
 

@@ -13,7 +13,11 @@
 namespace rlt {
 
 // GEMM epilogues: C (fp32) = acc | C += acc | Ct (storage type) = acc
-enum GemmMode { kStoreF32 = 0, kAddF32 = 1, kStoreT = 2 };
+enum GemmMode { kStoreF32 = 0, kAddF32 = 1, kStoreT = 2, kSwiGLU = 3 };
+// The fused FFN input projection stores W1 and W3 interleaved in blocks of
+// 64 rows: packed rows [128k, 128k+64) are W1 rows [64k, 64k+64) (gates),
+// rows [128k+64, 128k+128) the W3 rows of the same units.
+__host__ __device__ __forceinline__ int w13_gate_col(int j) { return (j / 64) * 128 + j % 64; }
 
 struct RopeTab {          // cos/sin of p * base^(-2i/dh), p = 0..max_pos, i < dh/2
     const float* cs;      // [max_pos+1][dh/2] cos
@@ -31,6 +35,10 @@ void launch_rmsnorm(const float* X, int ldx, const float* gain, T* Y, int ldy, i
 template <typename T>
 void launch_gemm(const T* A, int lda, const T* W, int ldw, float* C, int ldc, T* Ct, int ldct,
                  int M, int N, int K, int mode, cudaStream_t st);
+// Hd[M, N/2] = SwiGLU of A . W13^T (interleaved W13, N = 2 f_pad) in the
+// tensor-core GEMM's epilogue; false (nothing launched) where unsupported.
+bool launch_gemm_swiglu(const bf16* A, int lda, const bf16* W13, int ldw, bf16* Hd, int ldh, int M,
+                        int N, int K, cudaStream_t st);
 template <typename T>
 int launch_gemm_split(const T* A, int lda, const T* W, int ldw, float* C, int ldc, int M, int N,
                       int K, int splits, size_t slab, cudaStream_t st);

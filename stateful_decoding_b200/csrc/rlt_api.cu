@@ -303,6 +303,7 @@ extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model
     const rlt_config& c = pb.cfg;
     const int dh = c.d / c.heads;
     if (dh != 16 && dh != 32 && dh != 64 && dh != 128) return RLT_E_UNSUPPORTED;
+    if (c.d > 2048) return RLT_E_UNSUPPORTED;      // row kernels: one thread per 4 features
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
         cudaGetLastError();
@@ -348,10 +349,18 @@ extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model
         put_mat(a, off, elt, src(p + "wv"), d, d, d, 2 * d);
         fixups.push_back({off, dst});
     };
+    // W1 and W3 interleaved in blocks of 64 rows (w13_gate_col), so that a
+    // 128-column output tile holds 64 gates and their up projections
+    auto put_w13 = [&](Arena& ar, size_t o13, const uint8_t* w1, const uint8_t* w3) {
+        for (int r = 0; r < c.ffn; ++r) {
+            const int gr = rlt::w13_gate_col(r);
+            put_mat(ar, o13, elt, w1 + (size_t)r * d * elt, 1, d, d, gr);
+            put_mat(ar, o13, elt, w3 + (size_t)r * d * elt, 1, d, d, gr + 64);
+        }
+    };
     auto ffn = [&](const std::string& p, void** w13, void** w2) {
         size_t o13 = a.take((size_t)2 * fp * d * elt);
-        put_mat(a, o13, elt, src(p + "w1"), c.ffn, d, d, 0);
-        put_mat(a, o13, elt, src(p + "w3"), c.ffn, d, d, fp);
+        put_w13(a, o13, src(p + "w1"), src(p + "w3"));
         fixups.push_back({o13, w13});
         size_t o2 = a.take((size_t)d * fp * elt);
         put_mat(a, o2, elt, src(p + "w2"), d, c.ffn, fp, 0);
@@ -377,8 +386,7 @@ extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model
         std::vector<void*> w2s(c.n_dec);
         for (int l = 0; l < c.n_dec; ++l) {
             size_t o13 = a.take((size_t)2 * fp * d * elt);
-            put_mat(a, o13, elt, src(dec_p(l) + "w1"), c.ffn, d, d, 0);
-            put_mat(a, o13, elt, src(dec_p(l) + "w3"), c.ffn, d, d, fp);
+            put_w13(a, o13, src(dec_p(l) + "w1"), src(dec_p(l) + "w3"));
             fixups.push_back({o13, &m->dec[l].w13});
         }
         for (int l = 0; l < c.n_dec; ++l) {
@@ -488,13 +496,22 @@ struct rlt_state {
     size_t bytes = 0;
     // live timing (rlt_profile_*)
     bool prof = false;
-    int prof_level = 0;               // 2: transition blocks run launch by launch
-    struct ProfRec { int cls; cudaEvent_t a, b; double bytes; };
+    int prof_level = 0;               // 2: also time each attention launch inside the graphs
+    // a record holds its events until queried, or (events owned by a graph)
+    // the elapsed time read right after the replay
+    struct ProfRec { int cls; cudaEvent_t a, b; double bytes; float ms; };
     std::vector<ProfRec> prof_recs;
     std::vector<cudaEvent_t> prof_pool;
-    // replayable transition blocks, per positions-per-block n
-    struct Graph { cudaGraphExec_t exec; uint64_t launches; };
-    std::map<int, Graph> graphs;
+    // event pairs captured into a graph (cudaEventRecordExternal nodes), with
+    // the index of the block they bracket
+    struct CapRec { int cls; cudaEvent_t a, b; int block; };
+    bool prof_capture = false;
+    int prof_block = 0;
+    std::vector<CapRec> cap_recs;
+    // replayable transition blocks, per positions-per-block n; graphs_prof
+    // carries event nodes around the attention launches (profiling level 2)
+    struct Graph { cudaGraphExec_t exec; uint64_t launches; std::vector<CapRec> caps; };
+    std::map<int, Graph> graphs, graphs_prof;
 };
 
 static cudaEvent_t prof_event(rlt_state* s) {
@@ -515,15 +532,37 @@ struct ProfScope {
     cudaStream_t st;
     double bytes;
     cudaEvent_t a = nullptr;
+    bool cap = false;
     ProfScope(rlt_state* s_, int c, cudaStream_t st_, double b) : s(s_), cls(c), st(st_), bytes(b) {
-        if (s->prof && (a = prof_event(s))) cudaEventRecord(a, st);
+        if (s->prof_capture) {          // becomes an event node of the graph being captured
+            if (cudaEventCreate(&a) != cudaSuccess) {
+                cudaGetLastError();
+                a = nullptr;
+                return;
+            }
+            cap = true;
+            cudaEventRecordWithFlags(a, st, cudaEventRecordExternal);
+        } else if (s->prof && (a = prof_event(s))) {
+            cudaEventRecord(a, st);
+        }
     }
     ~ProfScope() {
         if (!a) return;
+        if (cap) {
+            cudaEvent_t b = nullptr;
+            if (cudaEventCreate(&b) != cudaSuccess) {
+                cudaGetLastError();
+                cudaEventDestroy(a);
+                return;
+            }
+            cudaEventRecordWithFlags(b, st, cudaEventRecordExternal);
+            s->cap_recs.push_back({cls, a, b, s->prof_block});
+            return;
+        }
         cudaEvent_t b = prof_event(s);
         if (!b) return;
         cudaEventRecord(b, st);
-        s->prof_recs.push_back({cls, a, b, bytes});
+        s->prof_recs.push_back({cls, a, b, bytes, -1.f});
     }
 };
 
@@ -545,11 +584,18 @@ extern "C" void rlt_state_destroy(rlt_state* s) {
     cudaSetDevice(s->m->device);
     cudaDeviceSynchronize();
     for (auto& r : s->prof_recs) {
-        cudaEventDestroy(r.a);
-        cudaEventDestroy(r.b);
+        if (r.a) cudaEventDestroy(r.a);
+        if (r.b) cudaEventDestroy(r.b);
     }
     for (cudaEvent_t e : s->prof_pool) cudaEventDestroy(e);
-    for (auto& g : s->graphs) cudaGraphExecDestroy(g.second.exec);
+    for (auto* gm : {&s->graphs, &s->graphs_prof})
+        for (auto& g : *gm) {
+            cudaGraphExecDestroy(g.second.exec);
+            for (auto& c : g.second.caps) {
+                cudaEventDestroy(c.a);
+                cudaEventDestroy(c.b);
+            }
+        }
     for (void* p : s->allocs) cudaFree(p);
     delete s;
 }
@@ -737,7 +783,7 @@ static int dec_splits_for(const rlt_config& c, int N, int K) {
     const int tiles = 2 * ((N + 63) / 64);            // output tiles at M = 256
     const int nk = K / 64;
     int want = std::max(1, (148 + tiles - 1) / tiles);
-    want = std::min(want, std::max(1, nk / 2));
+    want = std::min({want, std::max(1, nk / 2), 8});      // consumers sum at most 8 slabs
     const int cps = (nk + want - 1) / want;
     return (nk + cps - 1) / cps;
 }
@@ -780,9 +826,14 @@ static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t s
                            h, dh, st);
         launch_gemm<T>(A, d, (const T*)L.wo, d, s->X, d, nullptr, 0, R, d, d, kAddF32, st);
         launch_rmsnorm<T>(s->X, d, L.ffn_norm, Y, d, R, d, eps, st);
-        launch_gemm<T>(Y, d, (const T*)L.w13, d, s->H13, 2 * fp, nullptr, 0, R, 2 * fp, d,
-                       kStoreF32, st);
-        launch_swiglu<T>(s->H13, 1, 0, fp, Hd, R, st);
+        bool ffn_done = false;
+        if constexpr (std::is_same<T, bf16>::value)
+            ffn_done = launch_gemm_swiglu(Y, d, (const bf16*)L.w13, d, Hd, fp, R, 2 * fp, d, st);
+        if (!ffn_done) {
+            launch_gemm<T>(Y, d, (const T*)L.w13, d, s->H13, 2 * fp, nullptr, 0, R, 2 * fp, d,
+                           kStoreF32, st);
+            launch_swiglu<T>(s->H13, 1, 0, fp, Hd, R, st);
+        }
         launch_gemm<T>(Hd, fp, (const T*)L.w2, fp, s->X, d, nullptr, 0, R, d, fp, kAddF32, st);
     }
     launch_copy_e(s->X, s->pos_enc, s->e, s->T_cap, B, n, d, st);
@@ -916,8 +967,13 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
         }
         nres = gemm_p(A, d, (const T*)L.xo, d, d, P);
         launch_add_rmsnorm<T>(z, P, nres, slab, L.ffn_norm, Y, R, d, eps, st);
-        np = gemm_p(Y, d, (const T*)L.w13, 2 * fp, d, P);
-        launch_swiglu<T>(P, np, slab, fp, Hd, R, st);
+        bool ffn_done = false;
+        if constexpr (std::is_same<T, bf16>::value)
+            ffn_done = launch_gemm_swiglu(Y, d, (const bf16*)L.w13, d, Hd, fp, R, 2 * fp, d, st);
+        if (!ffn_done) {
+            np = gemm_p(Y, d, (const T*)L.w13, 2 * fp, d, P);
+            launch_swiglu<T>(P, np, slab, fp, Hd, R, st);
+        }
         nres = gemm_p(Hd, fp, (const T*)L.w2, d, fp, P);
     }
     launch_set_state(z, nres ? P : nullptr, nres, slab, s->s, c.variant == 2 ? s->Rr : nullptr,
@@ -962,16 +1018,23 @@ static int run_graph(rlt_state* s, int n, cudaStream_t st) {
         if (s->h_pos_dec[b] + span > s->h_pos_enc[b]) return RLT_E_ORDER;
         if (s->h_pos_dec[b] + span > s->T_cap) return RLT_E_CAPACITY;
     }
-    auto it = s->graphs.find(n);
-    if (it == s->graphs.end()) {
+    // profiling level 2 replays a twin graph whose attention launches are
+    // bracketed by event nodes
+    const bool timed = s->prof && s->prof_level >= 2;
+    auto& gmap = timed ? s->graphs_prof : s->graphs;
+    auto it = gmap.find(n);
+    if (it == gmap.end()) {
         const bool prof = s->prof;
-        s->prof = false;                  // no event records inside the capture
+        s->prof = false;                  // no stream event records inside the capture
+        s->prof_capture = timed;
+        s->cap_recs.clear();
         const uint64_t l0 = rlt_kernel_launches();
         cudaGraph_t g = nullptr;
         cudaGraphExec_t ex = nullptr;
         bool ok = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
         if (ok) {
             for (int k = 0; k < kGraphBlocks; ++k) {
+                s->prof_block = k;
                 if (s->m->cfg.dtype == RLT_DTYPE_BF16) step_block<bf16>(s, n, st);
                 else step_block<float>(s, n, st);
             }
@@ -982,12 +1045,19 @@ static int run_graph(rlt_state* s, int n, cudaStream_t st) {
         const uint64_t captured = rlt_kernel_launches() - l0;
         g_launches.fetch_sub(captured);  // captured, not launched
         s->prof = prof;
+        s->prof_capture = false;
+        std::vector<rlt_state::CapRec> caps;
+        caps.swap(s->cap_recs);
         if (!ok) {
             cudaGetLastError();
             if (ex) cudaGraphExecDestroy(ex);
+            for (auto& c : caps) {
+                cudaEventDestroy(c.a);
+                cudaEventDestroy(c.b);
+            }
             return RLT_E_UNSUPPORTED;     // the caller runs the blocks directly
         }
-        it = s->graphs.emplace(n, rlt_state::Graph{ex, captured}).first;
+        it = gmap.emplace(n, rlt_state::Graph{ex, captured, std::move(caps)}).first;
     }
     double by = 0;
     if (s->prof) {
@@ -1003,6 +1073,23 @@ static int run_graph(rlt_state* s, int n, cudaStream_t st) {
         if (cudaGraphLaunch(it->second.exec, st) != cudaSuccess) return RLT_E_DEVICE;
     }
     rlt_count_launch((int)it->second.launches);
+    if (timed && !it->second.caps.empty()) {
+        // the next replay re-records these events: read them now
+        if (cudaStreamSynchronize(st) != cudaSuccess) return RLT_E_DEVICE;
+        std::vector<int32_t> saved = s->h_pos_dec;
+        for (auto& c : it->second.caps) {
+            float t = 0.f;
+            if (cudaEventElapsedTime(&t, c.a, c.b) != cudaSuccess) {
+                cudaGetLastError();
+                continue;
+            }
+            for (int b = 0; b < s->B; ++b) s->h_pos_dec[b] = saved[b] + c.block * n;
+            const double cb = c.cls == RLT_PROF_XATTN ? xattn_bytes(s, n)
+                              : c.cls == RLT_PROF_SWA ? swa_bytes(s, n) : 0.0;
+            s->prof_recs.push_back({c.cls, nullptr, nullptr, cb, t});
+        }
+        s->h_pos_dec = saved;
+    }
     for (int b = 0; b < s->B; ++b) s->h_pos_dec[b] += span;
     return RLT_OK;
 }
@@ -1072,7 +1159,7 @@ extern "C" int rlt_prefill(rlt_state* s, int T, void* stream) {
         // whole blocks of the regular shape go through a replayed graph
         const bool regular = c.variant == 1 || (c.variant == 2 && n == c.chunk) ||
                              (c.variant == 0 && n == s->n_dec_blk);
-        if (regular && graphs_enabled(st) && s->prof_level < 2 && T - done >= kGraphBlocks * n) {
+        if (regular && graphs_enabled(st) && T - done >= kGraphBlocks * n) {
             int rc = run_graph(s, n, st);
             if (rc == RLT_OK) {
                 done += kGraphBlocks * n;
@@ -1214,8 +1301,8 @@ extern "C" int rlt_profile_enable(rlt_state* s, int on) {
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
     if (cudaDeviceSynchronize() != cudaSuccess) return RLT_E_DEVICE;
     for (auto& r : s->prof_recs) {
-        s->prof_pool.push_back(r.a);
-        s->prof_pool.push_back(r.b);
+        if (r.a) s->prof_pool.push_back(r.a);
+        if (r.b) s->prof_pool.push_back(r.b);
     }
     s->prof_recs.clear();
     s->prof = on != 0;
@@ -1232,7 +1319,13 @@ extern "C" int rlt_profile_query(rlt_state* s, int cls, uint64_t* launches, doub
     double ms = 0, by = 0;
     for (auto& r : s->prof_recs) {
         if (r.cls != cls) continue;
-        float t = 0.f;
+        float t = r.ms;
+        if (!r.a) {                      // resolved right after its graph replay
+            ++n;
+            ms += t;
+            by += r.bytes;
+            continue;
+        }
         if (cudaEventSynchronize(r.b) != cudaSuccess ||
             cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
             return RLT_E_DEVICE;
