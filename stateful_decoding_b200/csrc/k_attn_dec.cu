@@ -372,324 +372,172 @@ k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t
     }
 }
 
-// ---------------------------------------------------------------- persistent decode
-// One position per row (n = 1), the decode-time shape: a persistent grid of
-// about two CTAs per SM loops over the (row, head) items; a producer warp
-// streams, for item after item, the item's projection slabs (q; for the
-// window attention also k and v) and its keys and values through a 4-stage
-// ring of 1-D bulk copies, so that the copies of the next items are in flight
-// while 4 consumer warps fold the current one.  Same arithmetic per key as
-// k_attn_stream (the fold is shared), so results match it exactly.
-constexpr int PW = 4;        // consumer warps
-constexpr int PNS = 2;       // key/value stages
-constexpr int PMAXS = 8;     // split-K slabs of a projection (the splitter caps at 8)
-
-template <int DH>
-struct PCfg {
-    static constexpr int CH = 4096 / DH;            // keys per stage: 8 KB of K, 8 KB of V
-    static constexpr int LPK = DH / 8, KPR = 32 / LPK;
-    static constexpr int WK = CH / PW;
-    static constexpr int ROUNDS = WK / KPR;
-    static constexpr uint32_t STAGE = CH * DH * 2;  // bytes of K (or V) per stage
-    // item header: slabs [3][PMAXS][DH] (q, k, v), then the RoPE row of t (cos, sin)
-    static constexpr int HFLOATS = 3 * PMAXS * DH + DH;
-    static constexpr uint32_t HDR = HFLOATS * 4;
-    static constexpr size_t SMEM = 2 * PNS * (size_t)STAGE + 2 * (size_t)HDR;
-};
-
-__device__ __forceinline__ void consumer_sync() {
-    asm volatile("bar.sync 1, %0;" ::"r"(PW * 32) : "memory");
-}
+// ---------------------------------------------------------------- one-position decode
+// One position per row (n = 1, the decode shape): one warp per (row, head),
+// four items per CTA, no shared pipeline and no cross-warp merge.  The warp
+// forms q (and, for the window attention, the position's own k and v) from
+// the projection slabs, then walks the keys in batches of DRB rounds: the K
+// and V loads of a batch (16 bytes per lane, d_h/8 lanes per key) are all
+// issued before the first is used, then scores, one max and rescale per
+// batch, and the value accumulation.  Every occupied ring slot lies inside
+// the window and every memory key up to t is visible, so the only mask is
+// the run's length.  The keys of the first batch are requested before the
+// wait for the previous kernel (ring and memory are written two or more
+// kernels back).
+constexpr int DWARPS = 4;      // items (warps) per CTA
+constexpr int DRB = 8;         // rounds per batch
 
 template <int DH, bool SWA>
-__global__ void __launch_bounds__((PW + 1) * 32)
-k_attn_persist(const bf16* __restrict__ base, size_t row_stride, int span,
-               const int32_t* __restrict__ pos, int W, bf16* __restrict__ A, int B, int heads,
-               ProjIn pin) {
-    using C = PCfg<DH>;
-    int* err = &g_attn_error;
-    extern __shared__ __align__(128) uint8_t smem[];
-    bf16* sK = reinterpret_cast<bf16*>(smem);                          // [PNS][CH][DH]
-    bf16* sV = reinterpret_cast<bf16*>(smem + PNS * C::STAGE);
-    float* sH = reinterpret_cast<float*>(smem + 2 * PNS * C::STAGE);    // [2][HFLOATS]
-    __shared__ uint64_t full[PNS], empty[PNS], hfull[2], hempty[2];
-    __shared__ float s_m[PW], s_l[PW];
-    __shared__ float s_o[PW][DH];
-    __shared__ __align__(16) bf16 own_k[DH];
-    __shared__ __align__(16) bf16 own_v[DH];
-    __shared__ volatile int s_abort;
-    __shared__ int s_stop;
-
+__global__ void __launch_bounds__(DWARPS * 32)
+k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
+            const int32_t* __restrict__ pos, int W, bf16* __restrict__ A, int B, int heads,
+            ProjIn pin) {
+    constexpr int LPK = DH / 8, KPR = 32 / LPK, HALF = DH / 2;
+    __shared__ __align__(16) float s_q[DWARPS][DH];
+    __shared__ __align__(16) bf16 s_k[DWARPS][DH];
+    __shared__ __align__(16) bf16 s_v[DWARPS][DH];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int items = B * heads, d = heads * DH, S = pin.S;
-    const uint32_t hbytes = (uint32_t)S * DH * 4 * (SWA ? 3 : 1) + DH * 4;
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < PNS; ++i) {
-            tc::mbar_init(&full[i], 1);
-            tc::mbar_init(&empty[i], PW);
-        }
-        for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&hfull[i], 1);
-            tc::mbar_init(&hempty[i], PW);
-        }
-        s_abort = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
+    const int it = blockIdx.x * DWARPS + warp;
+    const bool live = it < B * heads;
+    const int b = live ? it / heads : 0, h = live ? it % heads : 0;
+    const int d = heads * DH, seg = lane % LPK, grp = lane / LPK;
+    const int pd = live ? __ldcg(pos + b) : 0, t = pd + 1;
+    const int nreg = !live ? 0 : (SWA ? (W > 1 ? min(pd, span) : 0) : t);
+    const bf16* kg = base + (size_t)b * row_stride + (size_t)h * span * DH + seg * 8;
+    const bf16* vg = kg + (size_t)heads * span * DH;
 
-    // per-item geometry, identical in producer and consumers
-    auto geom = [&](int it, int& b, int& h, int& pd, int& nreg) {
-        b = it / heads;
-        h = it % heads;
-        pd = __ldcg(pos + b);
-        nreg = SWA ? (W > 1 ? min(pd, span) : 0) : pd + 1;
+    uint4 kb[DRB], vb[DRB];
+    auto load_batch = [&](int j0) {
+#pragma unroll
+        for (int r = 0; r < DRB; ++r) {
+            const int j = j0 + r * KPR + grp;
+            if (j < nreg) {
+                kb[r] = __ldcs(reinterpret_cast<const uint4*>(kg + (size_t)j * DH));
+                vb[r] = __ldcs(reinterpret_cast<const uint4*>(vg + (size_t)j * DH));
+            }
+        }
     };
-
-    if (warp == PW) {
-        // ------------------------------------------------ producer
-        uint32_t nf = 0;          // stage fills issued
-        int nh = 0;               // headers issued
-        if (lane == 0) {
-            bool waited = false;
-            for (int it = blockIdx.x; it < items && !s_abort; it += gridDim.x) {
-                int b, h, pd, nreg;
-                geom(it, b, h, pd, nreg);
-                const bf16* kg = base + (size_t)b * row_stride + (size_t)h * span * DH;
-                const bf16* vg = kg + (size_t)heads * span * DH;
-                const int nch = (nreg + C::CH - 1) / C::CH;
-                auto chunk = [&](int c) -> bool {
-                    const int st = nf % PNS;
-                    if (nf >= PNS && !tc::mbar_wait(&empty[st], ((nf / PNS) & 1u) ^ 1u))
-                        return false;
-                    const int k0 = c * C::CH, cnt = min(C::CH, nreg - k0);
-                    const uint32_t bytes = (uint32_t)cnt * DH * 2;
-                    tc::mbar_expect_tx(&full[st], 2 * bytes);
-                    bulk_load(sK + (size_t)st * C::CH * DH, kg + (size_t)k0 * DH, bytes, &full[st]);
-                    bulk_load(sV + (size_t)st * C::CH * DH, vg + (size_t)k0 * DH, bytes, &full[st]);
-                    ++nf;
-                    return true;
-                };
-                int c = 0;
-                if (!waited) {
-                    // the first item's keys need nothing from the previous kernel
-                    for (; c < min(nch, PNS); ++c)
-                        if (!chunk(c)) break;
-                    pdl_wait();
-                    waited = true;
-                }
-                // header: this item's projection slabs (written by the kernel before)
-                const int hb = nh & 1;
-                if (nh >= 2 && !tc::mbar_wait(&hempty[hb], ((nh >> 1) & 1) ^ 1)) {
-                    s_abort = 1;
-                    atomicExch(err, kDevTimeout);
-                    break;
-                }
-                tc::mbar_expect_tx(&hfull[hb], hbytes);
-                float* hdst = sH + (size_t)hb * C::HFLOATS;
-                const size_t rowo = (size_t)b * pin.ldp + h * DH;
-                for (int z = 0; z < S; ++z)
-                    for (int part = 0; part < (SWA ? 3 : 1); ++part)
-                        bulk_load(hdst + ((size_t)part * PMAXS + z) * DH,
-                                  pin.P + (size_t)z * pin.slab + rowo + (size_t)part * d,
-                                  DH * 4, &hfull[hb]);
-                const size_t ro = (size_t)(pd + 1) * (DH / 2);
-                bulk_load(hdst + 3 * PMAXS * DH, pin.rope.cs + ro, DH * 2, &hfull[hb]);
-                bulk_load(hdst + 3 * PMAXS * DH + DH / 2, pin.rope.sn + ro, DH * 2, &hfull[hb]);
-                ++nh;
-                bool ok = true;
-                for (; c < nch; ++c)
-                    if (!chunk(c)) { ok = false; break; }
-                if (!ok) {
-                    s_abort = 1;
-                    atomicExch(err, kDevTimeout);
-                    break;
-                }
-            }
-            if (!waited) pdl_wait();
-        }
-        __syncwarp();
-        pdl_trigger();
-        __syncthreads();            // consumers are done with every stage they waited for
-        if (lane == 0 && s_abort) {
-            // copies in flight must land before the CTA exits: wait (bounded)
-            // for the last fill of every stage and of every header buffer
-            for (uint32_t i = 0; i < PNS && i < nf; ++i) {
-                const uint32_t last = nf - 1 - ((nf - 1 - i) % PNS);
-                tc::mbar_wait(&full[i], (last / PNS) & 1u, 1u << 20);
-            }
-            for (int i = 0; i < 2 && i < nh; ++i) {
-                const int last = nh - 1 - ((nh - 1 - i) % 2);
-                tc::mbar_wait(&hfull[i], (uint32_t)(last >> 1) & 1u, 1u << 20);
-            }
-        }
-        return;
-    }
-
-    // ---------------------------------------------------- consumers
+    load_batch(0);
     pdl_enter();
-    constexpr int LPK = C::LPK, HALF = DH / 2;
-    const int seg = lane % LPK;
-    const float sc = 1.0f / sqrtf((float)DH);
-    uint32_t f = 0;
-    int k = 0;
-    for (int it = blockIdx.x; it < items; it += gridDim.x, ++k) {
-        int b, h, pd, nreg;
-        geom(it, b, h, pd, nreg);
-        const int t = pd + 1, nch = (nreg + C::CH - 1) / C::CH;
-        const int hb = k & 1;
-        bool ok = !s_abort && tc::mbar_wait(&hfull[hb], (k >> 1) & 1);
-        if (!ok && !s_abort) {
-            s_abort = 1;
-            atomicExch(err, kDevTimeout);
-        }
-        const float* hq = sH + (size_t)hb * C::HFLOATS;
-        const float* hcs = hq + 3 * PMAXS * DH;      // RoPE row of t
-        const float* hsn = hcs + HALF;
-        float q[1][8];
-        int lo[1], hi[1];
-        hi[0] = t;
-        lo[0] = SWA ? max(1, t - W + 1) : 1;
-        if (ok) {
-            // q: slab sums in slab order, RoPE at t (rotate-half pairs), scale
-#pragma unroll
-            for (int x8 = 0; x8 < 8; ++x8) {
-                const int x = seg * 8 + x8, j = x % HALF;
-                float a = hq[x], p = hq[x < HALF ? x + HALF : x - HALF];
-                for (int z = 1; z < S; ++z) {
-                    a += hq[z * DH + x];
-                    p += hq[z * DH + (x < HALF ? x + HALF : x - HALF)];
-                }
-                const float c = hcs[j], sn = hsn[j];
-                const float y = x < HALF ? a * c - p * sn : a * c + p * sn;
-                q[0][x8] = y * sc;
-            }
-            if (SWA && warp == 0) {
-                // this position's own key and value (rounded like the stored ones)
-                const float* hk = hq + PMAXS * DH;
-                const float* hv = hq + 2 * PMAXS * DH;
-                for (int x = lane; x < DH; x += 32) {
-                    const int j = x % HALF, xp = x < HALF ? x + HALF : x - HALF;
-                    float a = hk[x], p = hk[xp], v = hv[x];
-                    for (int z = 1; z < S; ++z) {
-                        a += hk[z * DH + x];
-                        p += hk[z * DH + xp];
-                        v += hv[z * DH + x];
-                    }
-                    const float c = hcs[j], sn = hsn[j];
-                    own_k[x] = __float2bfloat16_rn(x < HALF ? a * c - p * sn : a * c + p * sn);
-                    own_v[x] = __float2bfloat16_rn(v);
-                }
-                __syncwarp();
-            }
-        }
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&hempty[hb]);
 
-        Online<DH, 1> os;
-        os.m[0] = -INFINITY;
-        os.l[0] = 0.f;
-#pragma unroll
-        for (int x = 0; x < 8; ++x) os.acc[0][x] = 0.f;
-        const int pdv = pd;
-        for (int c = 0; c < nch; ++c, ++f) {
-            const int st = f % PNS;
-            const bool got = ok && !s_abort && tc::mbar_wait(&full[st], (f / PNS) & 1u);
-            if (!got && ok) {
-                s_abort = 1;
-                atomicExch(err, kDevTimeout);
-            }
-            if (got) {
-                const int k0 = c * C::CH + warp * C::WK;
-                const bf16* sk = sK + (size_t)st * C::CH * DH + (size_t)warp * C::WK * DH;
-                const bf16* sv = sV + (size_t)st * C::CH * DH + (size_t)warp * C::WK * DH;
-                auto pos_of = [&](int kidx) -> int {
-                    const int j = k0 + kidx;
-                    if (j >= nreg) return 0;
-                    if (!SWA) return j + 1;
-                    return pdv - ((pdv - 1 - j) % span);
-                };
-                fold_keys<DH, 1, C::ROUNDS>(os, q, lo, hi,
-                                             [&](int kidx) { return sk + (size_t)kidx * DH; },
-                                             [&](int kidx) { return sv + (size_t)kidx * DH; },
-                                             pos_of, lane);
-            }
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&empty[st]);
-        }
-        if (SWA && warp == 0 && ok) {       // the current position itself
-            fold_keys<DH, 1, 1>(os, q, lo, hi, [&](int) { return (const bf16*)own_k; },
-                                [&](int) { return (const bf16*)own_v; },
-                                [&](int kidx) -> int { return kidx == 0 ? t : 0; }, lane);
-        }
-        // merge the warps' partial results in warp order
-#pragma unroll
-        for (int x = 0; x < 8; ++x)
-#pragma unroll
-            for (int o = 16; o >= LPK; o >>= 1)
-                os.acc[0][x] += __shfl_xor_sync(0xffffffffu, os.acc[0][x], o);
-        if (lane < LPK) {
-#pragma unroll
-            for (int x = 0; x < 8; ++x) s_o[warp][seg * 8 + x] = os.acc[0][x];
-            if (lane == 0) {
-                s_m[warp] = os.m[0];
-                s_l[warp] = os.l[0];
+    // q, and the own k, v: lane j forms the rotate-half pairs (j, j + HALF)
+    if (live) {
+        const size_t rb = (size_t)b * pin.ldp + h * DH;
+        const float* cs = pin.rope.cs + (size_t)t * HALF;
+        const float* sn = pin.rope.sn + (size_t)t * HALF;
+        for (int j = lane; j < HALF; j += 32) {
+            const float c = cs[j], s_ = sn[j];
+            float y1, y2;
+            rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + j),
+                     slab_sum8(pin.P, pin.S, pin.slab, rb + j + HALF), c, s_, y1, y2);
+            s_q[warp][j] = y1;
+            s_q[warp][j + HALF] = y2;
+            if (SWA) {
+                rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + d + j),
+                         slab_sum8(pin.P, pin.S, pin.slab, rb + d + j + HALF), c, s_, y1, y2);
+                s_k[warp][j] = __float2bfloat16_rn(y1);
+                s_k[warp][j + HALF] = __float2bfloat16_rn(y2);
+                s_v[warp][j] = __float2bfloat16_rn(slab_sum8(pin.P, pin.S, pin.slab, rb + 2 * d + j));
+                s_v[warp][j + HALF] =
+                    __float2bfloat16_rn(slab_sum8(pin.P, pin.S, pin.slab, rb + 2 * d + j + HALF));
             }
         }
-        // one decision for all consumer warps (s_abort may change at any time)
-        if (threadIdx.x == 0) s_stop = s_abort;
-        consumer_sync();
-        const bool abort_now = s_stop;
-        if (!abort_now) {
-            for (int x = threadIdx.x; x < DH; x += PW * 32) {
-                float M = -INFINITY;
-                for (int w = 0; w < PW; ++w) M = fmaxf(M, s_m[w]);
-                float L = 0.f, O = 0.f;
-                for (int w = 0; w < PW; ++w) {
-                    if (s_m[w] == -INFINITY) continue;
-                    const float e = expf(s_m[w] - M);
-                    L += s_l[w] * e;
-                    O += s_o[w][x] * e;
-                }
-                A[(size_t)b * d + h * DH + x] = __float2bfloat16_rn(O / L);
-                if (SWA && W > 1) {
-                    // every key of this item has been read: the position enters its slot
-                    bf16* rk = const_cast<bf16*>(base) + (size_t)b * row_stride +
-                               (size_t)h * span * DH;
-                    const int slot = pd % span;
-                    rk[(size_t)slot * DH + x] = own_k[x];
-                    rk[(size_t)heads * span * DH + (size_t)slot * DH + x] = own_v[x];
-                }
-            }
-        }
-        consumer_sync();
-        if (abort_now) break;
     }
-    __syncthreads();
+    __syncwarp();
+    const float sc = 1.0f / sqrtf((float)DH);
+    float q[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) q[x] = s_q[warp][seg * 8 + x] * sc;
+
+    float m = -INFINITY, l = 0.f, acc[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+    // fold DRB rounds whose K, V sit in kb, vb; `valid(r)`: this lane's key exists
+    auto fold = [&](auto valid) {
+        float s[DRB];
+#pragma unroll
+        for (int r = 0; r < DRB; ++r) {
+            float kf[8] = {};
+            if (valid(r)) unpack8(kb[r], kf);
+            float dot = 0.f;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) dot = fmaf(q[x], kf[x], dot);
+#pragma unroll
+            for (int o = LPK / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            s[r] = valid(r) ? dot : -INFINITY;
+        }
+        float bm = s[0];
+#pragma unroll
+        for (int r = 1; r < DRB; ++r) bm = fmaxf(bm, s[r]);
+#pragma unroll
+        for (int o = 16; o >= LPK; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+        const float mn = fmaxf(m, bm);
+        if (mn == -INFINITY) return;
+        const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);
+        float ps = 0.f;
+#pragma unroll
+        for (int r = 0; r < DRB; ++r) {
+            s[r] = (s[r] == -INFINITY) ? 0.f : expf(s[r] - mn);
+            ps += s[r];
+        }
+#pragma unroll
+        for (int o = 16; o >= LPK; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        l = l * corr + ps;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc[x] *= corr;
+        m = mn;
+#pragma unroll
+        for (int r = 0; r < DRB; ++r) {
+            if (!valid(r)) continue;
+            float vf[8];
+            unpack8(vb[r], vf);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) acc[x] = fmaf(s[r], vf[x], acc[x]);
+        }
+    };
+    constexpr int BATCH = DRB * KPR;             // keys per batch
+    for (int j0 = 0; j0 < nreg; j0 += BATCH) {
+        if (j0 > 0) load_batch(j0);
+        fold([&](int r) { return j0 + r * KPR + grp < nreg; });
+    }
+    if (SWA && live) {                           // the current position itself
+        if (grp == 0) {
+            kb[0] = *reinterpret_cast<const uint4*>(&s_k[warp][seg * 8]);
+            vb[0] = *reinterpret_cast<const uint4*>(&s_v[warp][seg * 8]);
+        }
+        fold([&](int r) { return r == 0 && grp == 0; });
+    }
+    // reduce over the key groups; lanes of group 0 hold the head's output
+#pragma unroll
+    for (int x = 0; x < 8; ++x)
+#pragma unroll
+        for (int o = 16; o >= LPK; o >>= 1) acc[x] += __shfl_xor_sync(0xffffffffu, acc[x], o);
+    if (live && grp == 0) {
+        const float inv = 1.0f / l;
+        uint4 w;
+        uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            __nv_bfloat162 p2 = __floats2bfloat162_rn(acc[2 * x] * inv, acc[2 * x + 1] * inv);
+            wp[x] = *reinterpret_cast<uint32_t*>(&p2);
+        }
+        *reinterpret_cast<uint4*>(A + (size_t)b * d + h * DH + seg * 8) = w;
+        if (SWA && W > 1) {
+            // all of this head's ring has been read: the position enters slot pd mod (W-1)
+            const size_t slot = (size_t)(pd % span) * DH;
+            *reinterpret_cast<uint4*>(const_cast<bf16*>(kg) + slot) =
+                *reinterpret_cast<const uint4*>(&s_k[warp][seg * 8]);
+            *reinterpret_cast<uint4*>(const_cast<bf16*>(vg) + slot) =
+                *reinterpret_cast<const uint4*>(&s_v[warp][seg * 8]);
+        }
+    }
 }
 
-// One launcher per kernel instance, so that each instance gets its own
-// shared-memory attribute (the instances share a function-pointer type).
 template <int DH, bool SWA>
-bool launch_persist(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W,
-                    bf16* A, int B, int heads, const ProjIn& pin, cudaStream_t st) {
-    constexpr size_t smem = PCfg<DH>::SMEM;
-    static int grid_cap = 0;
-    if (!grid_cap) {
-        if (cudaFuncSetAttribute(k_attn_persist<DH, SWA>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return false;
-        int dev = 0, sms = 0, per_sm = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_attn_persist<DH, SWA>,
-                                                          (PW + 1) * 32, smem) != cudaSuccess ||
-            per_sm < 1)
-            return false;
-        grid_cap = per_sm * sms;
-    }
+bool launch_dec1(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W, bf16* A,
+                 int B, int heads, const ProjIn& pin, cudaStream_t st) {
     const int items = B * heads;
-    launch(k_attn_persist<DH, SWA>, std::min(items, grid_cap), (PW + 1) * 32, smem, st, base,
+    launch(k_attn_dec1<DH, SWA>, (items + DWARPS - 1) / DWARPS, DWARPS * 32, 0, st, base,
            row_stride, span, pos, W, A, B, heads, pin);
     rlt_count_launch();
     return true;
@@ -772,16 +620,6 @@ bool launch_attn_swa_fast(const float* Q, const bf16* Kc, const bf16* Vc, const 
     return false;
 }
 
-// RLT_ATTN_PERSIST=1 runs decode steps on the persistent kernel (measured
-// slower than the per-item kernel on B200 so far, so not the default)
-static bool persist_enabled() {
-    static const bool on = [] {
-        const char* e = getenv("RLT_ATTN_PERSIST");
-        return e && strcmp(e, "1") == 0;
-    }();
-    return on;
-}
-
 bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int W,
                           const int32_t* pos, bf16* A, int B, int n, int heads, int dh,
                           cudaStream_t st) {
@@ -790,9 +628,9 @@ bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int 
     if (!fast_attn_enabled() || n > 4 || (dh != 64 && dh != 128)) return false;
     if (B * n <= 0) return true;
     const int slots = W > 1 ? W - 1 : 1;
-    if (n == 1 && pin.S <= PMAXS && persist_enabled())
-        return dh == 64 ? launch_persist<64, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st)
-                        : launch_persist<128, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st);
+    if (n == 1 && pin.S <= 8)
+        return dh == 64 ? launch_dec1<64, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st)
+                        : launch_dec1<128, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st);
     if (dh == 64)
         return launch_stream<64, true, true>(nullptr, ring, row_stride, slots, nullptr, nullptr,
                                              pos, W, A, B, n, heads, pin, st);
@@ -805,9 +643,9 @@ bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_strid
                             cudaStream_t st) {
     if (!fast_attn_enabled() || (dh != 64 && dh != 128)) return false;
     if (B * n <= 0) return true;
-    if (n == 1 && pin.S <= PMAXS && persist_enabled())
-        return dh == 64 ? launch_persist<64, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st)
-                        : launch_persist<128, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st);
+    if (n == 1 && pin.S <= 8)
+        return dh == 64 ? launch_dec1<64, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st)
+                        : launch_dec1<128, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st);
     if (dh == 64)
         return launch_stream<64, false, true>(nullptr, mem, row_stride, T_cap, nullptr, nullptr,
                                               pos, 0, A, B, n, heads, pin, st);

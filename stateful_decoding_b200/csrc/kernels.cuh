@@ -137,6 +137,12 @@ bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_strid
                             const int32_t* pos_dec, bf16* A, int B, int n, int heads, int dh,
                             cudaStream_t st);
 bool fast_attn_enabled();           // false when RLT_ATTN=warp
+// Encoder causal attention on the tensor cores (k_attn_enc_tc.cu) for d_h = 64
+// and at most 256 keys per row (max_keys = max over rows of pos_enc + n);
+// false (nothing launched) otherwise.  err: the state's device error word.
+bool launch_attn_enc_tc(const float* Q, const bf16* cache, size_t row_stride, int T_cap,
+                        const int32_t* pos, bf16* A, int B, int n, int heads, int dh, int max_keys,
+                        int* err, cudaStream_t st);
     // same, for the streaming attention kernels
 
 }  // namespace rlt

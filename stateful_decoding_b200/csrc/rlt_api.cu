@@ -815,6 +815,8 @@ static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t s
     T* enc = (T*)s->enc;
     const size_t layer_enc = (size_t)2 * h * s->T_cap * dh;
     launch_embed<T>((const T*)m->embed, tok, s->X, R, d, c.vocab, s->err, st);
+    int max_keys = 0;                        // longest cache prefix any row attends to
+    for (int b = 0; b < B; ++b) max_keys = std::max(max_keys, s->h_pos_enc[b] + n);
     for (int l = 0; l < c.n_enc; ++l) {
         const EncLayerW& L = m->enc[l];
         launch_rmsnorm<T>(s->X, d, L.attn_norm, Y, d, R, d, eps, st);
@@ -822,8 +824,14 @@ static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t s
                        kStoreF32, st);
         launch_qkv_enc<T>(s->QKV, s->pos_enc, rope_of(s), s->Q, enc + l * layer_enc, s->enc_row,
                           s->T_cap, B, n, h, dh, st);
-        launch_attn_enc<T>(s->Q, enc + l * layer_enc, s->enc_row, s->T_cap, s->pos_enc, A, B, n,
-                           h, dh, st);
+        bool attn_done = false;
+        if constexpr (std::is_same<T, bf16>::value)
+            attn_done = fast_attn_enabled() &&
+                        launch_attn_enc_tc(s->Q, enc + l * layer_enc, s->enc_row, s->T_cap,
+                                           s->pos_enc, A, B, n, h, dh, max_keys, s->err, st);
+        if (!attn_done)
+            launch_attn_enc<T>(s->Q, enc + l * layer_enc, s->enc_row, s->T_cap, s->pos_enc, A, B,
+                               n, h, dh, st);
         launch_gemm<T>(A, d, (const T*)L.wo, d, s->X, d, nullptr, 0, R, d, d, kAddF32, st);
         launch_rmsnorm<T>(s->X, d, L.ffn_norm, Y, d, R, d, eps, st);
         bool ffn_done = false;
