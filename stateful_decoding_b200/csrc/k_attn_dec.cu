@@ -385,7 +385,7 @@ k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t
 // wait for the previous kernel (ring and memory are written two or more
 // kernels back).
 constexpr int DWARPS = 4;      // items (warps) per CTA
-constexpr int DRB = 8;         // rounds per batch
+constexpr int DRB = 4;         // rounds per batch (two batches in flight)
 
 template <int DH, bool SWA>
 __global__ void __launch_bounds__(DWARPS * 32)
@@ -406,8 +406,9 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
     const bf16* kg = base + (size_t)b * row_stride + (size_t)h * span * DH + seg * 8;
     const bf16* vg = kg + (size_t)heads * span * DH;
 
-    uint4 kb[DRB], vb[DRB];
-    auto load_batch = [&](int j0) {
+    // two batch buffers: the loads of batch i+1 are in flight while batch i is folded
+    uint4 kb0[DRB], vb0[DRB], kb1[DRB], vb1[DRB];
+    auto load_batch = [&](int j0, uint4 (&kb)[DRB], uint4 (&vb)[DRB]) {
 #pragma unroll
         for (int r = 0; r < DRB; ++r) {
             const int j = j0 + r * KPR + grp;
@@ -417,7 +418,9 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
             }
         }
     };
-    load_batch(0);
+    constexpr int BATCH = DRB * KPR;             // keys per batch
+    load_batch(0, kb0, vb0);
+    if (BATCH < nreg) load_batch(BATCH, kb1, vb1);
     pdl_enter();
 
     // q, and the own k, v: lane j forms the rotate-half pairs (j, j + HALF)
@@ -452,27 +455,27 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
     float m = -INFINITY, l = 0.f, acc[8];
 #pragma unroll
     for (int x = 0; x < 8; ++x) acc[x] = 0.f;
-    // fold DRB rounds whose K, V sit in kb, vb; `valid(r)`: this lane's key exists
-    auto fold = [&](auto valid) {
+    // fold the batch of keys j0.. held in kb, vb
+    auto fold = [&](int j0, const uint4 (&kb)[DRB], const uint4 (&vb)[DRB]) {
         float s[DRB];
 #pragma unroll
         for (int r = 0; r < DRB; ++r) {
+            const bool v = j0 + r * KPR + grp < nreg;
             float kf[8] = {};
-            if (valid(r)) unpack8(kb[r], kf);
+            if (v) unpack8(kb[r], kf);
             float dot = 0.f;
 #pragma unroll
             for (int x = 0; x < 8; ++x) dot = fmaf(q[x], kf[x], dot);
 #pragma unroll
             for (int o = LPK / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-            s[r] = valid(r) ? dot : -INFINITY;
+            s[r] = v ? dot : -INFINITY;
         }
         float bm = s[0];
 #pragma unroll
         for (int r = 1; r < DRB; ++r) bm = fmaxf(bm, s[r]);
 #pragma unroll
         for (int o = 16; o >= LPK; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-        const float mn = fmaxf(m, bm);
-        if (mn == -INFINITY) return;
+        const float mn = fmaxf(m, bm);          // finite: the batch holds a key
         const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);
         float ps = 0.f;
 #pragma unroll
@@ -488,24 +491,38 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
         m = mn;
 #pragma unroll
         for (int r = 0; r < DRB; ++r) {
-            if (!valid(r)) continue;
+            if (!(j0 + r * KPR + grp < nreg)) continue;
             float vf[8];
             unpack8(vb[r], vf);
 #pragma unroll
             for (int x = 0; x < 8; ++x) acc[x] = fmaf(s[r], vf[x], acc[x]);
         }
     };
-    constexpr int BATCH = DRB * KPR;             // keys per batch
-    for (int j0 = 0; j0 < nreg; j0 += BATCH) {
-        if (j0 > 0) load_batch(j0);
-        fold([&](int r) { return j0 + r * KPR + grp < nreg; });
+    for (int j0 = 0; j0 < nreg; j0 += 2 * BATCH) {
+        fold(j0, kb0, vb0);
+        if (j0 + 2 * BATCH < nreg) load_batch(j0 + 2 * BATCH, kb0, vb0);
+        if (j0 + BATCH >= nreg) break;
+        fold(j0 + BATCH, kb1, vb1);
+        if (j0 + 3 * BATCH < nreg) load_batch(j0 + 3 * BATCH, kb1, vb1);
     }
-    if (SWA && live) {                           // the current position itself
-        if (grp == 0) {
-            kb[0] = *reinterpret_cast<const uint4*>(&s_k[warp][seg * 8]);
-            vb[0] = *reinterpret_cast<const uint4*>(&s_v[warp][seg * 8]);
-        }
-        fold([&](int r) { return r == 0 && grp == 0; });
+    if (SWA && live) {
+        // the current position itself: one key, every lane group scores it,
+        // group 0 accumulates its value
+        float kf[8], vf[8];
+        unpack8(*reinterpret_cast<const uint4*>(&s_k[warp][seg * 8]), kf);
+        unpack8(*reinterpret_cast<const uint4*>(&s_v[warp][seg * 8]), vf);
+        float dot = 0.f;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) dot = fmaf(q[x], kf[x], dot);
+#pragma unroll
+        for (int o = LPK / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        const float mn = fmaxf(m, dot);
+        const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);
+        const float p = expf(dot - mn);
+        l = l * corr + p;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc[x] = acc[x] * corr + (grp == 0 ? p * vf[x] : 0.f);
+        m = mn;
     }
     // reduce over the key groups; lanes of group 0 hold the head's output
 #pragma unroll

@@ -975,9 +975,13 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
         }
         nres = gemm_p(A, d, (const T*)L.xo, d, d, P);
         launch_add_rmsnorm<T>(z, P, nres, slab, L.ffn_norm, Y, R, d, eps, st);
+        // SwiGLU in the GEMM epilogue only when the rows alone fill the
+        // machine: at a few hundred rows the split-K GEMM plus a row kernel
+        // is faster (measured on B200)
         bool ffn_done = false;
         if constexpr (std::is_same<T, bf16>::value)
-            ffn_done = launch_gemm_swiglu(Y, d, (const bf16*)L.w13, d, Hd, fp, R, 2 * fp, d, st);
+            ffn_done = R >= 2048 &&
+                       launch_gemm_swiglu(Y, d, (const bf16*)L.w13, d, Hd, fp, R, 2 * fp, d, st);
         if (!ffn_done) {
             np = gemm_p(Y, d, (const T*)L.w13, 2 * fp, d, P);
             launch_swiglu<T>(P, np, slab, fp, Hd, R, st);
