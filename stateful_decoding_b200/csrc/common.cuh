@@ -64,6 +64,10 @@ __device__ __forceinline__ void pdl_enter() {
 
 // True unless RLT_PDL=0 (defined in rlt_api.cu).
 bool pdl_enabled();
+// Once per kernel: the same preferred shared-memory carveout (all shared)
+// for every kernel of the library, so that consecutive kernels never make an
+// SM switch its L1 / shared-memory split (defined in rlt_api.cu).
+void set_carveout_once(const void* kernel);
 
 // kernel<<<grid, block, smem, st>>>(args...) with the programmatic-serialisation
 // attribute set when PDL is enabled.
@@ -80,6 +84,7 @@ inline cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    set_carveout_once(reinterpret_cast<const void*>(kernel));
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 }  // namespace rlt

@@ -373,6 +373,7 @@ k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t
 }
 
 // ---------------------------------------------------------------- one-position decode
+// Softmax exponentials use the fast exp2-based intrinsic (bf16 storage only).
 // One position per row (n = 1, the decode shape): one warp per (row, head),
 // four items per CTA, no shared pipeline and no cross-warp merge.  The warp
 // forms q (and, for the window attention, the position's own k and v) from
@@ -385,6 +386,22 @@ k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t
 // wait for the previous kernel (ring and memory are written two or more
 // kernels back).
 constexpr int DWARPS = 4;      // items (warps) per CTA
+
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// 16 bytes of cached keys/values: kept in L2 (KEEP) or streamed (evict-first)
+template <bool KEEP>
+__device__ __forceinline__ uint4 ld_kv(const bf16* p, uint64_t pol) {
+    if (!KEEP) return __ldcs(reinterpret_cast<const uint4*>(p));
+    uint4 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
 constexpr int DRB = 4;         // rounds per batch (two batches in flight)
 
 template <int DH, bool SWA>
@@ -406,6 +423,11 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
     const bf16* kg = base + (size_t)b * row_stride + (size_t)h * span * DH + seg * 8;
     const bf16* vg = kg + (size_t)heads * span * DH;
 
+    // The memory is read by every decoder block of the step (one group shared
+    // by all blocks): its lines are kept in L2 (evict-last) so that the next
+    // blocks' cross-attention can find them there; the window ring, read once
+    // per step, streams through (evict-first).
+    const uint64_t l2pol = SWA ? 0 : l2_evict_last_policy();
     // two batch buffers: the loads of batch i+1 are in flight while batch i is folded
     uint4 kb0[DRB], vb0[DRB], kb1[DRB], vb1[DRB];
     auto load_batch = [&](int j0, uint4 (&kb)[DRB], uint4 (&vb)[DRB]) {
@@ -413,8 +435,8 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
         for (int r = 0; r < DRB; ++r) {
             const int j = j0 + r * KPR + grp;
             if (j < nreg) {
-                kb[r] = __ldcs(reinterpret_cast<const uint4*>(kg + (size_t)j * DH));
-                vb[r] = __ldcs(reinterpret_cast<const uint4*>(vg + (size_t)j * DH));
+                kb[r] = ld_kv<!SWA>(kg + (size_t)j * DH, l2pol);
+                vb[r] = ld_kv<!SWA>(vg + (size_t)j * DH, l2pol);
             }
         }
     };
@@ -423,27 +445,17 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
     if (BATCH < nreg) load_batch(BATCH, kb1, vb1);
     pdl_enter();
 
-    // q, and the own k, v: lane j forms the rotate-half pairs (j, j + HALF)
+    // q: lane j forms the rotate-half pair (j, j + HALF)
+    const size_t rb = (size_t)b * pin.ldp + h * DH;
+    const float* cs = pin.rope.cs + (size_t)t * HALF;
+    const float* sn = pin.rope.sn + (size_t)t * HALF;
     if (live) {
-        const size_t rb = (size_t)b * pin.ldp + h * DH;
-        const float* cs = pin.rope.cs + (size_t)t * HALF;
-        const float* sn = pin.rope.sn + (size_t)t * HALF;
         for (int j = lane; j < HALF; j += 32) {
-            const float c = cs[j], s_ = sn[j];
             float y1, y2;
             rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + j),
-                     slab_sum8(pin.P, pin.S, pin.slab, rb + j + HALF), c, s_, y1, y2);
+                     slab_sum8(pin.P, pin.S, pin.slab, rb + j + HALF), cs[j], sn[j], y1, y2);
             s_q[warp][j] = y1;
             s_q[warp][j + HALF] = y2;
-            if (SWA) {
-                rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + d + j),
-                         slab_sum8(pin.P, pin.S, pin.slab, rb + d + j + HALF), c, s_, y1, y2);
-                s_k[warp][j] = __float2bfloat16_rn(y1);
-                s_k[warp][j + HALF] = __float2bfloat16_rn(y2);
-                s_v[warp][j] = __float2bfloat16_rn(slab_sum8(pin.P, pin.S, pin.slab, rb + 2 * d + j));
-                s_v[warp][j + HALF] =
-                    __float2bfloat16_rn(slab_sum8(pin.P, pin.S, pin.slab, rb + 2 * d + j + HALF));
-            }
         }
     }
     __syncwarp();
@@ -476,11 +488,11 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
 #pragma unroll
         for (int o = 16; o >= LPK; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
         const float mn = fmaxf(m, bm);          // finite: the batch holds a key
-        const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);
+        const float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
         float ps = 0.f;
 #pragma unroll
         for (int r = 0; r < DRB; ++r) {
-            s[r] = (s[r] == -INFINITY) ? 0.f : expf(s[r] - mn);
+            s[r] = (s[r] == -INFINITY) ? 0.f : __expf(s[r] - mn);
             ps += s[r];
         }
 #pragma unroll
@@ -506,6 +518,19 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
         if (j0 + 3 * BATCH < nreg) load_batch(j0 + 3 * BATCH, kb1, vb1);
     }
     if (SWA && live) {
+        // the current position's own k and v (formed after the loop, when the
+        // batch registers are free), rounded like the stored ones
+        for (int j = lane; j < HALF; j += 32) {
+            float y1, y2;
+            rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + d + j),
+                     slab_sum8(pin.P, pin.S, pin.slab, rb + d + j + HALF), cs[j], sn[j], y1, y2);
+            s_k[warp][j] = __float2bfloat16_rn(y1);
+            s_k[warp][j + HALF] = __float2bfloat16_rn(y2);
+            s_v[warp][j] = __float2bfloat16_rn(slab_sum8(pin.P, pin.S, pin.slab, rb + 2 * d + j));
+            s_v[warp][j + HALF] =
+                __float2bfloat16_rn(slab_sum8(pin.P, pin.S, pin.slab, rb + 2 * d + j + HALF));
+        }
+        __syncwarp();
         // the current position itself: one key, every lane group scores it,
         // group 0 accumulates its value
         float kf[8], vf[8];
@@ -517,8 +542,8 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
 #pragma unroll
         for (int o = LPK / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
         const float mn = fmaxf(m, dot);
-        const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);
-        const float p = expf(dot - mn);
+        const float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
+        const float p = __expf(dot - mn);
         l = l * corr + p;
 #pragma unroll
         for (int x = 0; x < 8; ++x) acc[x] = acc[x] * corr + (grp == 0 ? p * vf[x] : 0.f);

@@ -90,42 +90,42 @@ void launch_embed(const T* E, const int32_t* tok, float* X, int R, int d, int vo
 }
 
 // ---------------------------------------------------------------- RMSNorm
-// Sum of squares in a fixed order: per-thread strided partials, then a
-// butterfly within warps and a sequential pass over the warp partials.
-__device__ __forceinline__ float block_sum(float v, float* red) {
-    v = warp_sum(v);
-    int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    if (l == 0) red[w] = v;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float s = 0.f;
-        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) s += red[i];
-        red[32] = s;
-    }
-    __syncthreads();
-    float out = red[32];
-    __syncthreads();
-    return out;
-}
-
+// One warp per row (d <= 2048: at most 16 float4 groups per lane), 8 rows
+// per block; the row is loaded once, squares summed per lane then across
+// the warp in a fixed order.
 template <typename T>
-__global__ void k_rmsnorm(const float* __restrict__ X, int ldx, const float* __restrict__ g,
-                          T* __restrict__ Y, int ldy, int d, float eps) {
+__global__ void __launch_bounds__(256) k_rmsnorm(const float* __restrict__ X, int ldx,
+                                                 const float* __restrict__ g, T* __restrict__ Y,
+                                                 int ldy, int R, int d, float eps) {
     pdl_enter();
-    __shared__ float red[33];
-    const float* x = X + (size_t)blockIdx.x * ldx;
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (row >= R) return;
+    const float* x = X + (size_t)row * ldx;
+    const int d4 = d / 4;
+    float4 v[16];
     float ss = 0.f;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) ss += x[j] * x[j];
-    ss = block_sum(ss, red);
-    float inv = 1.0f / sqrtf(ss / (float)d + eps);
-    T* y = Y + (size_t)blockIdx.x * ldy;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) y[j] = from_f<T>(x[j] * inv * g[j]);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        const int j4 = lane + 32 * c;
+        if (j4 < d4) {
+            v[c] = ld4(x + 4 * j4);
+            ss += dot4(v[c]);
+        }
+    }
+    ss = warp_sum(ss);
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    T* y = Y + (size_t)row * ldy;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        const int j4 = lane + 32 * c;
+        if (j4 < d4) store4<T>(y + 4 * j4, scale4(v[c], inv, ld4(g + 4 * j4)));
+    }
 }
 template <typename T>
 void launch_rmsnorm(const float* X, int ldx, const float* gain, T* Y, int ldy, int R, int d,
                     float eps, cudaStream_t st) {
     if (R <= 0) return;
-    launch(k_rmsnorm<T>, R, 128, 0, st, X, ldx, gain, Y, ldy, d, eps);
+    launch(k_rmsnorm<T>, (R + 7) / 8, 256, 0, st, X, ldx, gain, Y, ldy, R, d, eps);
     rlt_count_launch();
 }
 
@@ -200,9 +200,9 @@ template <typename T>
 __global__ void __launch_bounds__(512) k_merge_out(const float* __restrict__ e, int T_cap,
                             const int32_t* __restrict__ pos_dec, const float* __restrict__ G,
                             int nG, size_t slabG, const float* __restrict__ bg,
-                            const float* __restrict__ S, int nS, size_t slabS, float alpha,
-                            float* __restrict__ z, int n, int d, const float* __restrict__ g,
-                            T* __restrict__ Y, float eps) {
+                            const float* __restrict__ S, int nS, size_t slabS, int ldg,
+                            float alpha, float* __restrict__ z, int n, int d,
+                            const float* __restrict__ g, T* __restrict__ Y, float eps) {
     pdl_enter();
     __shared__ float red[32];
     const int r = blockIdx.x, b = r / n, i = r % n;
@@ -214,8 +214,9 @@ __global__ void __launch_bounds__(512) k_merge_out(const float* __restrict__ e, 
         u = ld4(e + ((size_t)b * T_cap + pos_dec[b] + i) * d + j);
         if (g) gv = ld4(g + j);
         if (G) {
-            const float4 a = add4(slab_sum4(G, nG, slabG, o), ld4(bg + j));
-            const float4 p = slab_sum4(S, nS, slabS, o);
+            const size_t og = (size_t)r * ldg + j;      // G and S rows have pitch ldg
+            const float4 a = add4(slab_sum4(G, nG, slabG, og), ld4(bg + j));
+            const float4 p = slab_sum4(S, nS, slabS, og);
             u.x += alpha * (1.0f / (1.0f + expf(-a.x))) * p.x;
             u.y += alpha * (1.0f / (1.0f + expf(-a.y))) * p.y;
             u.z += alpha * (1.0f / (1.0f + expf(-a.z))) * p.z;
@@ -231,10 +232,10 @@ __global__ void __launch_bounds__(512) k_merge_out(const float* __restrict__ e, 
 template <typename T>
 void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const float* G, int nG,
                       size_t slabG, const float* bg, const float* S, int nS, size_t slabS,
-                      float alpha, float* z, const float* gain, T* Y, float eps, int B, int n,
-                      int d, cudaStream_t st) {
+                      int ldg, float alpha, float* z, const float* gain, T* Y, float eps, int B,
+                      int n, int d, cudaStream_t st) {
     launch(k_merge_out<T>, B * n, row_threads(d / 4), 0, st, e, T_cap, pos_dec, G, nG, slabG, bg,
-           S, nS, slabS, alpha, z, n, d, gain, Y, eps);
+           S, nS, slabS, ldg, alpha, z, n, d, gain, Y, eps);
     rlt_count_launch();
 }
 
@@ -513,8 +514,8 @@ void launch_ring_write(const T* Kc, const T* Vc, const int32_t* pos_dec, T* ring
     template void launch_rmsnorm<T>(const float*, int, const float*, T*, int, int, int, float, \
                                     cudaStream_t);                                             \
     template void launch_merge_out<T>(const float*, int, const int32_t*, const float*, int,    \
-                                      size_t, const float*, const float*, int, size_t, float,  \
-                                      float*, const float*, T*, float, int, int, int,          \
+                                      size_t, const float*, const float*, int, size_t, int,    \
+                                      float, float*, const float*, T*, float, int, int, int,   \
                                       cudaStream_t);                                           \
     template void launch_merge_input<T>(const float*, int, const int32_t*, const float*,       \
                                         const float*, T*, int, int, int, float, cudaStream_t); \

@@ -123,7 +123,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                 for (int kk = 0; kk < BK / 16; ++kk)
                     mma_bf16(tmem, sdesc_k_sw128(a + kk * 32), sdesc_k_sw128(b + kk * 32), idesc,
                              (kt | kk) != 0);
-                mma_commit(&empty[s]);
+                // release the stage only if the producer will refill it
+                if (kt + STAGES < nk) mma_commit(&empty[s]);
             }
             if (ok) mma_commit(&accum);
         }
@@ -167,13 +168,65 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
             } else {
                 abort_flag = 1;
             }
-        } else if (mbar_wait(&accum, 0)) {
+        } else {
+            const bool got = mbar_wait(&accum, 0);
+            if (!got) abort_flag = 1;
             fence_after_sync();
             const int q = warp & 3;
             const int row = m0 + 32 * q + lane;
             const bool vec = MODE == kStoreT
                                  ? ((ldct & 7) == 0 && ((uintptr_t)Ct & 15) == 0)
                                  : ((ldc & 3) == 0 && ((uintptr_t)C & 15) == 0);
+            if (BN <= 128 && vec && n0 + BN <= N) {
+                // Whole-width narrow tile (the decoder's few-hundred-row
+                // projections): stage the accumulator in shared memory (the
+                // pipeline stages are free once the last MMA has completed), then
+                // write it out row-contiguously, consecutive threads on
+                // consecutive 16-byte pieces of a row.
+                constexpr int SP = BN + 4;          // row pitch in floats (conflict-free)
+                float* stg = reinterpret_cast<float*>(smem);
+                const int r = 32 * q + lane;
+                if (__all_sync(0xffffffffu, got)) {
+#pragma unroll 1
+                    for (int c = 0; c < BN; c += 64) {
+                        float v[64];
+                        tmem_ld64(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c, v);
+                        float4* d4 = reinterpret_cast<float4*>(stg + (size_t)r * SP + c);
+#pragma unroll
+                        for (int u = 0; u < 16; ++u)
+                            d4[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                    }
+                }
+                // the four epilogue warps meet here whatever their waits said
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (abort_flag) goto epilogue_done;
+                constexpr int C4 = BN / 4;
+                const int et = threadIdx.x - 64;
+#pragma unroll 4
+                for (int i = et; i < BM * C4; i += 128) {
+                    const int rr = i / C4, c4 = i % C4, grow = m0 + rr;
+                    if (grow >= M) continue;
+                    float4 w = *reinterpret_cast<const float4*>(stg + (size_t)rr * SP + 4 * c4);
+                    if (MODE == kStoreT) {
+                        __nv_bfloat162 a = __floats2bfloat162_rn(w.x, w.y);
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(w.z, w.w);
+                        uint2 u2;
+                        u2.x = *reinterpret_cast<uint32_t*>(&a);
+                        u2.y = *reinterpret_cast<uint32_t*>(&b2);
+                        *reinterpret_cast<uint2*>(Ct + (size_t)grow * ldct + n0 + 4 * c4) = u2;
+                    } else {
+                        float4* dst = reinterpret_cast<float4*>(C + (size_t)grow * ldc + n0 + 4 * c4);
+                        if (MODE == kAddF32) {
+                            const float4 o = *dst;
+                            w.x += o.x;
+                            w.y += o.y;
+                            w.z += o.z;
+                            w.w += o.w;
+                        }
+                        *dst = w;
+                    }
+                }
+            } else if (__all_sync(0xffffffffu, got))
 #pragma unroll 1
             for (int c = 0; c < BN; c += 16) {
                 float v[16];
@@ -225,10 +278,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                     }
                 }
             }
-        } else {
-            abort_flag = 1;
         }
     }
+epilogue_done:
     fence_before_sync();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, BN);

@@ -51,13 +51,13 @@ template <typename T>
 void launch_merge_input(const float* e, int T_cap, const int32_t* pos_dec, const float* fb,
                         const float* gain, T* Gin, int B, int n, int d, float eps, cudaStream_t st);
 // z[r] = e_t + alpha * sigmoid(G[r] + bg) * S[r]   (S = W_s r); alpha ignored if G == nullptr.
-// G and S may be split-K partial slabs (nG / nS slabs, slabG / slabS apart).
-// With a gain (non-null), also Y[r] = RMSNorm(z[r]) * gain.
+// G and S may be split-K partial slabs (nG / nS slabs, slabG / slabS apart),
+// rows ldg floats apart.  With a gain (non-null), also Y[r] = RMSNorm(z[r]) * gain.
 template <typename T>
 void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const float* G, int nG,
                       size_t slabG, const float* bg, const float* S, int nS, size_t slabS,
-                      float alpha, float* z, const float* gain, T* Y, float eps, int B, int n,
-                      int d, cudaStream_t st);
+                      int ldg, float alpha, float* z, const float* gain, T* Y, float eps, int B,
+                      int n, int d, cudaStream_t st);
 // z += sum of residual partial slabs P (P may be null), then Y = RMSNorm(z)
 template <typename T>
 void launch_add_rmsnorm(float* Z, const float* P, int S, size_t slab, const float* gain, T* Y,

@@ -16,6 +16,7 @@
 #include <string>
 #include <map>
 #include <mutex>
+#include <set>
 #include <vector>
 
 #include "../../include/rlt.h"
@@ -34,6 +35,15 @@ bool pdl_enabled() {
         return !(e && strcmp(e, "0") == 0);
     }();
     return on;
+}
+void set_carveout_once(const void* kernel) {
+    static std::mutex mu;
+    static std::set<const void*> done;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!done.insert(kernel).second) return;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+        cudaGetLastError();        // a preference only: launching works without it
 }
 template <typename T>
 void launch_gemm(const T* A, int lda, const T* W, int ldw, float* C, int ldc, T* Ct, int ldct,
@@ -193,7 +203,7 @@ struct rlt_model {
     float* mem_norm = nullptr;
     std::vector<void*> wmem;        // per group [2d][d]: K rows then V rows
     float *merge_norm = nullptr, *bg = nullptr;
-    void *wg = nullptr, *ws = nullptr;
+    void *wg = nullptr, *ws = nullptr, *wgs = nullptr;
     std::vector<DecLayerW> dec;
     float* out_norm = nullptr;
     void* wout = nullptr;
@@ -422,6 +432,15 @@ extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model
         vecf("merge.bg", &m->bg);
         mat_plain("merge.wg", d, 2 * d, &m->wg);
         mat_plain("merge.ws", d, d, &m->ws);
+        // both merge projections as one [2d][2d] matrix over [e_t; r]: rows
+        // 0..d-1 are W_g, rows d..2d-1 are [0 | W_s] (one GEMM launch)
+        size_t og = a.take((size_t)4 * d * d * elt);
+        put_mat(a, og, elt, src("merge.wg"), d, 2 * d, 2 * d, 0);
+        const uint8_t* wsrc = src("merge.ws");
+        for (int r = 0; r < d; ++r)
+            memcpy(a.host.data() + og + ((size_t)(d + r) * 2 * d + d) * elt,
+                   wsrc + (size_t)r * d * elt, (size_t)d * elt);
+        fixups.push_back({og, &m->wgs});
     }
     vecf("out_norm", &m->out_norm);
     mat_plain("out", c.vocab, d, &m->wout);
@@ -775,14 +794,15 @@ static double enc_bytes(const rlt_state* s, int n) {     // one encoder block
     return by;
 }
 
-// Split-K factor of a transition projection (N outputs, K inputs): enough
-// CTAs for the machine when M = 256 rows, a function of N and K only (never of
-// the batch), at least two 64-wide K-chunks per split.  1 for fp32 models.
+// Split-K factor of a transition projection (N outputs, K inputs): as many
+// CTAs as fit one wave on the machine when M = 256 rows (a second wave costs
+// more than the longer K run), a function of N and K only (never of the
+// batch), at least two 64-wide K-chunks per split.  1 for fp32 models.
 static int dec_splits_for(const rlt_config& c, int N, int K) {
     if (c.dtype != RLT_DTYPE_BF16 || K % 64) return 1;
     const int tiles = 2 * ((N + 63) / 64);            // output tiles at M = 256
     const int nk = K / 64;
-    int want = std::max(1, (148 + tiles - 1) / tiles);
+    int want = std::max(1, 148 / tiles);
     want = std::min({want, std::max(1, nk / 2), 8});      // consumers sum at most 8 slabs
     const int cps = (nk + want - 1) / want;
     return (nk + cps - 1) / cps;
@@ -793,7 +813,7 @@ static int dec_splits(const rlt_state* s, int N, int K) {
 // the most slabs any transition projection of this model uses
 static int max_dec_splits(const rlt_config& c, int fp) {
     const int d = c.d;
-    const int shapes[6][2] = {{3 * d, d}, {d, d}, {2 * fp, d}, {d, fp}, {d, 2 * d}, {d, d}};
+    const int shapes[6][2] = {{3 * d, d}, {d, d}, {2 * fp, d}, {d, fp}, {2 * d, 2 * d}, {d, d}};
     int m = 1;
     for (auto& sh : shapes) m = std::max(m, dec_splits_for(c, sh[0], sh[1]));
     return m;
@@ -919,17 +939,16 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
     // the merge kernel also applies the first decoder block's input RMSNorm
     const float* norm0 = c.n_dec > 0 ? m->dec[0].swa_norm : nullptr;
     if (c.variant == 0) {
-        launch_merge_out<T>(s->e, s->T_cap, s->pos_dec, nullptr, 0, 0, nullptr, nullptr, 0, 0, 0.f,
-                            z, norm0, Y, eps, B, n, d, st);
+        launch_merge_out<T>(s->e, s->T_cap, s->pos_dec, nullptr, 0, 0, nullptr, nullptr, 0, 0, d,
+                            0.f, z, norm0, Y, eps, B, n, d, st);
     } else {
         const float* fb = c.variant == 2 ? s->Rr : s->s;
         launch_merge_input<T>(s->e, s->T_cap, s->pos_dec, fb, m->merge_norm, Y, B, n, d, eps, st);
-        // gate partials in P, projection partials in a second region P2 of the same slabs
-        float* P2 = P + (size_t)R * d;
-        const int nG = gemm_p(Y, 2 * d, (const T*)m->wg, d, 2 * d, P);
-        const int nS = gemm_p(Y + d, 2 * d, (const T*)m->ws, d, d, P2);
-        launch_merge_out<T>(s->e, s->T_cap, s->pos_dec, P, nG, slab, m->bg, P2, nS, slab,
-                            (float)c.alpha, z, norm0, Y, eps, B, n, d, st);
+        // one GEMM for both projections: gate pre-activations in columns
+        // 0..d-1 of the slabs, W_s r in columns d..2d-1
+        const int nGS = gemm_p(Y, 2 * d, (const T*)m->wgs, 2 * d, 2 * d, P);
+        launch_merge_out<T>(s->e, s->T_cap, s->pos_dec, P, nGS, slab, m->bg, P + d, nGS, slab,
+                            2 * d, (float)c.alpha, z, norm0, Y, eps, B, n, d, st);
     }
     const size_t layer_ring = (size_t)2 * h * std::max(0, c.window - 1) * dh;
     const size_t layer_mem = (size_t)2 * h * s->T_cap * dh;
