@@ -35,6 +35,11 @@ void launch_rmsnorm(const float* X, int ldx, const float* gain, T* Y, int ldy, i
 template <typename T>
 void launch_gemm(const T* A, int lda, const T* W, int ldw, float* C, int ldc, T* Ct, int ldct,
                  int M, int N, int K, int mode, cudaStream_t st);
+// z[M, N] += A . W^T and Y = RMSNorm(z) * gain in one kernel (k_gemm_norm.cu;
+// N = d, a cluster of CTAs spans each row block); false (nothing launched)
+// for shapes it does not handle.  err: the state's device error word.
+bool launch_gemm_norm(const bf16* A, int lda, const bf16* W, int ldw, float* Z, const float* gain,
+                      bf16* Y, int M, int N, int K, float eps, int* err, cudaStream_t st);
 // Hd[M, N/2] = SwiGLU of A . W13^T (interleaved W13, N = 2 f_pad) in the
 // tensor-core GEMM's epilogue; false (nothing launched) where unsupported.
 bool launch_gemm_swiglu(const bf16* A, int lda, const bf16* W13, int ldw, bf16* Hd, int ldh, int M,

@@ -514,6 +514,7 @@ struct rlt_state {
     std::vector<void*> allocs;
     size_t bytes = 0;
     // live timing (rlt_profile_*)
+    int norm_fuse = 0;                // see norm_fuse_from_env
     bool prof = false;
     int prof_level = 0;               // 2: also time each attention launch inside the graphs
     // a record holds its events until queried, or (events owned by a graph)
@@ -620,6 +621,7 @@ extern "C" void rlt_state_destroy(rlt_state* s) {
 }
 
 static int max_dec_splits(const rlt_config& c, int fp);
+static int norm_fuse_from_env();
 
 static size_t max_rows_per_call() {
     const char* v = getenv("RLT_MAX_ROWS");
@@ -636,6 +638,7 @@ extern "C" int rlt_state_create(rlt_model* m, int batch, int max_len, rlt_state*
     s->m = m;
     s->B = batch;
     s->T_cap = max_len;
+    s->norm_fuse = norm_fuse_from_env();
     const size_t elt = m->elt, d = c.d, dh = m->dh, h = c.heads, B = batch, T = max_len;
     const size_t slots = (size_t)std::max(0, c.window - 1);
     size_t maxr = max_rows_per_call();
@@ -914,6 +917,15 @@ extern "C" int rlt_encode(rlt_state* s, const int32_t* tokens, int n, void* stre
 // ============================================================================
 // transition
 // ============================================================================
+// RLT_NORM_FUSE (read when a state is created): 0 (default) = split-K GEMM
+// and a row kernel for each residual projection and the RMSNorm after it;
+// 1 = one clustered kernel (k_gemm_norm.cu) for the attention output
+// projections; 2 = also for W_2.  Measured on B200 at 256 rows the clustered
+// kernel is slower (16 CTAs each running the whole K range), so it is opt-in.
+static int norm_fuse_from_env() {
+    const char* e = getenv("RLT_NORM_FUSE");
+    return e ? atoi(e) : 0;
+}
 template <typename T>
 static void step_block(rlt_state* s, int n, cudaStream_t st) {
     using namespace rlt;
@@ -952,12 +964,22 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
     }
     const size_t layer_ring = (size_t)2 * h * std::max(0, c.window - 1) * dh;
     const size_t layer_mem = (size_t)2 * h * s->T_cap * dh;
+    // residual projection + the RMSNorm after it in one clustered kernel
+    // (level 1: attention output projections; level 2: also W_2)
+    const int fuse = s->norm_fuse;
+    auto proj_norm = [&](const T* Ain, int lda, const T* Wt, int K, const float* gain) -> bool {
+        if constexpr (std::is_same<T, bf16>::value)
+            return launch_gemm_norm(Ain, lda, Wt, K, z, gain, Y, R, d, K, eps, s->err, st);
+        return false;
+    };
     int nres = 0;                       // pending residual partial slabs in P
+    bool normed = false;                // Y already holds this block's input norm
     for (int l = 0; l < c.n_dec; ++l) {
         const DecLayerW& L = m->dec[l];
         T* ring = (T*)s->ring + l * layer_ring;
-        if (l > 0)
+        if (l > 0 && !normed)
             launch_add_rmsnorm<T>(z, nres ? P : nullptr, nres, slab, L.swa_norm, Y, R, d, eps, st);
+        normed = false;
         int np = gemm_p(Y, d, (const T*)L.wqkv, 3 * d, d, P);
         {
             // bf16: the attention kernel forms q, k, v from the slabs and
@@ -976,8 +998,10 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
                                      st);
             }
         }
-        nres = gemm_p(A, d, (const T*)L.wo, d, d, P);
-        launch_add_rmsnorm<T>(z, P, nres, slab, L.x_norm, Y, R, d, eps, st);
+        if (!(fuse >= 1 && proj_norm(A, d, (const T*)L.wo, d, L.x_norm))) {
+            nres = gemm_p(A, d, (const T*)L.wo, d, d, P);
+            launch_add_rmsnorm<T>(z, P, nres, slab, L.x_norm, Y, R, d, eps, st);
+        }
         np = gemm_p(Y, d, (const T*)L.xq, d, d, P);
         const T* mem = (const T*)s->mem + (c.groups > 1 ? l : 0) * layer_mem;
         {
@@ -992,8 +1016,10 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
                                      st);
             }
         }
-        nres = gemm_p(A, d, (const T*)L.xo, d, d, P);
-        launch_add_rmsnorm<T>(z, P, nres, slab, L.ffn_norm, Y, R, d, eps, st);
+        if (!(fuse >= 1 && proj_norm(A, d, (const T*)L.xo, d, L.ffn_norm))) {
+            nres = gemm_p(A, d, (const T*)L.xo, d, d, P);
+            launch_add_rmsnorm<T>(z, P, nres, slab, L.ffn_norm, Y, R, d, eps, st);
+        }
         // SwiGLU in the GEMM epilogue only when the rows alone fill the
         // machine: at a few hundred rows the split-K GEMM plus a row kernel
         // is faster (measured on B200)
@@ -1005,7 +1031,12 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
             np = gemm_p(Y, d, (const T*)L.w13, 2 * fp, d, P);
             launch_swiglu<T>(P, np, slab, fp, Hd, R, st);
         }
-        nres = gemm_p(Hd, fp, (const T*)L.w2, d, fp, P);
+        nres = 0;
+        if (fuse >= 2 && l + 1 < c.n_dec &&
+            proj_norm(Hd, fp, (const T*)L.w2, fp, m->dec[l + 1].swa_norm))
+            normed = true;              // the next block's input norm is done
+        else
+            nres = gemm_p(Hd, fp, (const T*)L.w2, d, fp, P);
     }
     launch_set_state(z, nres ? P : nullptr, nres, slab, s->s, c.variant == 2 ? s->Rr : nullptr,
                      s->pos_dec, c.chunk, B, n, d, /*bump=*/true, st);

@@ -175,6 +175,29 @@ def test_fused_transition_kernel(sd, monkeypatch):
         assert np.max(np.abs(lg[b] - orc.readout(r))) <= 3e-2
 
 
+@pytest.mark.parametrize("level", [1, 2])
+def test_fused_projection_norm_kernel(sd, monkeypatch, level):
+    """The opt-in clustered projection + RMSNorm kernel (RLT_NORM_FUSE=1: the
+    attention output projections; 2: also W_2) against the oracle, stepwise
+    on a ragged batch (two 128-row tiles, the second partial) and through
+    one prefill."""
+    monkeypatch.setenv("RLT_NORM_FUSE", str(level))
+    cfg = ri.CONFIGS["parity_bf16"]
+    run_stepwise_and_compare(sd, cfg, 3, 13, n_decode=1)
+    B, T = 130, 9
+    W, model, st = make(sd, cfg, B, T)
+    toks = ri.make_tokens(cfg, B, T)
+    st.encode(toks)
+    st.prefill(T)
+    lg, _, _ = readout_host(st, cfg)
+    orc = RLTOracle(cfg, W, "bf16")
+    for b in (0, 129):
+        r = orc.new_state()
+        orc.encode(r, toks[b])
+        orc.prefill(r, T)
+        assert np.max(np.abs(lg[b] - orc.readout(r))) <= 3e-2
+
+
 def test_full_size_bench_config_sampled_rows(sd):
     """parity_bf16 at its full size (256 rows x 256) in the bench's launch
     configuration (one encode call, one prefill call); rows 0, 131 and 255
