@@ -162,36 +162,39 @@ k_attn_enc_tc(const float* __restrict__ Q, const bf16* __restrict__ cache, size_
     const int nvis = r < nq ? min(qpos, NK) : 0;
     const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
     const float sc = 1.0f / sqrtf((float)EDH);
+    // 64 columns of S per TMEM load (one wait each)
     float m = -INFINITY;
     if (ok) {
 #pragma unroll 1
-        for (int c = 0; c < NK; c += 16) {
-            float v[16];
-            tmem_ld16(trow + (uint32_t)c, v);
+        for (int c = 0; c < NK; c += 64) {
+            float v[64];
+            tmem_ld64(trow + (uint32_t)c, v);
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
+            for (int j = 0; j < 64; ++j)
                 if (c + j < nvis) m = fmaxf(m, v[j] * sc);
         }
     }
     float sum = 0.f;
     if (ok) {
 #pragma unroll 1
-        for (int c = 0; c < NK; c += 16) {
-            float v[16];
-            tmem_ld16(trow + (uint32_t)c, v);
-            uint32_t w[8];
-#pragma unroll
-            for (int j = 0; j < 16; j += 2) {
-                const float e0 = (c + j < nvis) ? expf(v[j] * sc - m) : 0.f;
-                const float e1 = (c + j + 1 < nvis) ? expf(v[j + 1] * sc - m) : 0.f;
-                __nv_bfloat162 p2 = __floats2bfloat162_rn(e0, e1);
-                sum += __low2float(p2) + __high2float(p2);
-                w[j / 2] = *reinterpret_cast<uint32_t*>(&p2);
-            }
+        for (int c = 0; c < NK; c += 64) {
+            float v[64];
+            tmem_ld64(trow + (uint32_t)c, v);
             uint8_t* pb = sP + (c >> 6) * P_BLOCK;
-            const int ch = (c & 63) >> 3;
-            *reinterpret_cast<uint4*>(pb + sw128(r, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4*>(pb + sw128(r, ch + 1)) = make_uint4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {          // 8 keys per 16-byte chunk
+                uint32_t w[4];
+#pragma unroll
+                for (int j = 0; j < 8; j += 2) {
+                    const int k = 8 * ch + j;
+                    const float e0 = (c + k < nvis) ? __expf(v[k] * sc - m) : 0.f;
+                    const float e1 = (c + k + 1 < nvis) ? __expf(v[k + 1] * sc - m) : 0.f;
+                    __nv_bfloat162 p2 = __floats2bfloat162_rn(e0, e1);
+                    sum += __low2float(p2) + __high2float(p2);
+                    w[j / 2] = *reinterpret_cast<uint32_t*>(&p2);
+                }
+                *reinterpret_cast<uint4*>(pb + sw128(r, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
         }
     }
     proxy_fence();
@@ -219,17 +222,15 @@ k_attn_enc_tc(const float* __restrict__ Q, const bf16* __restrict__ cache, size_
         // all lanes load (warp-collective); rows past the block store nothing
         const float inv = r < nq ? 1.0f / sum : 0.f;
         bf16* dst = A + (size_t)(b * n + q0 + min(r, nq - 1)) * d + h * EDH;
-#pragma unroll 1
-        for (int c = 0; c < EDH; c += 16) {
-            float v[16];
-            tmem_ld16(trow + (uint32_t)c, v);
-            if (r >= nq) continue;
-            uint4 w0 = make_uint4(pack2(v[0] * inv, v[1] * inv), pack2(v[2] * inv, v[3] * inv),
-                                  pack2(v[4] * inv, v[5] * inv), pack2(v[6] * inv, v[7] * inv));
-            uint4 w1 = make_uint4(pack2(v[8] * inv, v[9] * inv), pack2(v[10] * inv, v[11] * inv),
-                                  pack2(v[12] * inv, v[13] * inv), pack2(v[14] * inv, v[15] * inv));
-            *reinterpret_cast<uint4*>(dst + c) = w0;
-            *reinterpret_cast<uint4*>(dst + c + 8) = w1;
+        float v[64];
+        tmem_ld64(trow, v);                       // the whole output row (d_h = 64)
+        if (r < nq) {
+#pragma unroll
+            for (int c = 0; c < EDH; c += 8) {
+                *reinterpret_cast<uint4*>(dst + c) =
+                    make_uint4(pack2(v[c] * inv, v[c + 1] * inv), pack2(v[c + 2] * inv, v[c + 3] * inv),
+                               pack2(v[c + 4] * inv, v[c + 5] * inv), pack2(v[c + 6] * inv, v[c + 7] * inv));
+            }
         }
     }
     if (!ok && threadIdx.x == 0) atomicExch(err, kDevTimeout);

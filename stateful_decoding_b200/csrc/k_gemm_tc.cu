@@ -139,16 +139,17 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                 const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
                 for (int g0 = 0; g0 < BN; g0 += 128) {
+                    // the group's 64 gates, then its 64 up projections: 16 at a time
 #pragma unroll 1
-                    for (int c = 0; c < 64; c += 16) {
-                        float a[16], u[16];
-                        tmem_ld16(tq + (uint32_t)(g0 + c), a);
-                        tmem_ld16(tq + (uint32_t)(g0 + 64 + c), u);
+                    for (int c = 0; c < 64; c += 32) {
+                        float a[32], u[32];
+                        tmem_ld32(tq + (uint32_t)(g0 + c), a);
+                        tmem_ld32(tq + (uint32_t)(g0 + 64 + c), u);
                         if (row < M && n0 + g0 + 128 <= N) {
                             uint4* dst = reinterpret_cast<uint4*>(
                                 Ct + (size_t)row * ldct + (n0 + g0) / 2 + c);
 #pragma unroll
-                            for (int h = 0; h < 2; ++h) {
+                            for (int h = 0; h < 4; ++h) {
                                 uint4 w;
                                 uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
@@ -228,9 +229,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                 }
             } else if (__all_sync(0xffffffffu, got))
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 16) {
-                float v[16];
-                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c, v);
+            for (int c64 = 0; c64 < BN; c64 += 64) {
+            float v64[64];
+            tmem_ld64(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c64, v64);
+#pragma unroll
+            for (int c = c64; c < c64 + 64; c += 16) {
+                const float* v = v64 + (c - c64);
                 if (row < M) {
                     const int col0 = n0 + c;
                     if (vec && col0 + 16 <= N) {
@@ -277,6 +281,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                         }
                     }
                 }
+            }
             }
         }
     }
