@@ -1,0 +1,254 @@
+// Large-M GEMM on the tensor cores (the encoder's projections over B·T rows):
+// C[M,N] = A[M,K] . W[N,K]^T with a persistent grid and two accumulators.
+//
+// One CTA per SM loops over 128 x 256 output tiles (tile t: rows
+// 128·(t / tiles_n), columns 256·(t % tiles_n)).  Warp 0 streams K-slices of
+// A and W through a 4-stage TMA ring that runs on across tiles; one thread of
+// warp 1 issues the MMAs of tile j into TMEM accumulator j % 2 (512 columns
+// in all) and commits it; warps 2-5 drain accumulator j % 2 and apply the
+// epilogue while the MMAs of tile j+1 already run into the other one.  The
+// epilogues are those of k_gemm_tc (fp32 store, fp32 accumulate, SwiGLU over
+// interleaved W1/W3 columns).  Each output element sums its K products in the
+// same order as k_gemm_tc, whatever the tile's position.  Waits are bounded:
+// a wait that gives up records a timeout in the device error word, the roles
+// stop, and the CTA still frees its tensor memory.
+#include <cuda.h>
+
+#include "fused.cuh"
+#include "kernels.cuh"
+#include "tc_common.cuh"
+
+namespace rlt {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, NTHREADS = 192;
+constexpr uint32_t A_BYTES = BM * BK * 2, STAGE = BM * BK * 2 + BN * BK * 2;
+constexpr size_t SMEM = (size_t)STAGES * STAGE + 1024;
+
+__device__ int g_persist_error;
+
+template <int MODE>
+__global__ void __launch_bounds__(NTHREADS, 1)
+k_gemm_persist(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+               float* __restrict__ C, int ldc, bf16* __restrict__ Ct, int ldct, int M, int N,
+               int K) {
+    using namespace tc;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    __shared__ uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2];
+    __shared__ uint32_t tmem_base;
+    __shared__ volatile int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles_n = N / BN, tiles = ((M + BM - 1) / BM) * tiles_n;
+    const int nk = K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);          // one arrival per epilogue warp
+        }
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_map(&ta);
+        prefetch_map(&tb);
+    }
+    if (warp == 1) tmem_alloc(&tmem_base, 2 * BN);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tmem_base;
+    pdl_enter();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int t = blockIdx.x; t < tiles && !abort_flag; t += gridDim.x) {
+                const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+                for (int kt = 0; kt < nk; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (it >= STAGES && !mbar_wait(&empty[s], ph ^ 1u)) {
+                        abort_flag = 1;
+                        break;
+                    }
+                    mbar_expect_tx(&full[s], STAGE);
+                    tma_load_2d(smem + s * STAGE, &ta, kt * BK, m0, &full[s]);
+                    tma_load_2d(smem + s * STAGE + A_BYTES, &tb, kt * BK, n0, &full[s]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(BM, BN);
+            uint32_t it = 0;
+            int j = 0;
+            for (int t = blockIdx.x; t < tiles && !abort_flag; t += gridDim.x, ++j) {
+                const int acc = j & 1;
+                // the epilogue has drained this accumulator (tile j-2)
+                if (j >= 2 && !mbar_wait(&tempty[acc], ((uint32_t)(j >> 1) & 1u) ^ 1u)) {
+                    abort_flag = 1;
+                    break;
+                }
+                fence_after_sync();
+                const uint32_t d = tmem + (uint32_t)(acc * BN);
+                bool ok = true;
+                for (int kt = 0; kt < nk; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait(&full[s], ph)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a = smem_u32(smem + s * STAGE), b = a + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_bf16(d, sdesc_k_sw128(a + kk * 32), sdesc_k_sw128(b + kk * 32), idesc,
+                                 (kt | kk) != 0);
+                    mma_commit(&empty[s]);
+                }
+                if (!ok) {
+                    abort_flag = 1;
+                    break;
+                }
+                mma_commit(&tfull[acc]);
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        int j = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+            const int acc = j & 1;
+            const bool got = __all_sync(0xffffffffu, !abort_flag &&
+                                                          mbar_wait(&tfull[acc], (j >> 1) & 1u));
+            if (!got) {
+                abort_flag = 1;
+                break;
+            }
+            fence_after_sync();
+            const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+            const int row = m0 + 32 * q + lane;
+            const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
+            if (MODE == kSwiGLU) {
+#pragma unroll 1
+                for (int g0 = 0; g0 < BN; g0 += 128) {
+#pragma unroll 1
+                    for (int c = 0; c < 64; c += 32) {
+                        float a[32], u[32];
+                        tmem_ld32(tq + (uint32_t)(g0 + c), a);
+                        tmem_ld32(tq + (uint32_t)(g0 + 64 + c), u);
+                        if (row < M) {
+                            uint4* dst = reinterpret_cast<uint4*>(
+                                Ct + (size_t)row * ldct + (n0 + g0) / 2 + c);
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                uint4 w;
+                                uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const int e = 8 * h + 2 * k;
+                                    const float y0 = a[e] / (1.0f + expf(-a[e])) * u[e];
+                                    const float y1 =
+                                        a[e + 1] / (1.0f + expf(-a[e + 1])) * u[e + 1];
+                                    __nv_bfloat162 p2 = __floats2bfloat162_rn(y0, y1);
+                                    wp[k] = *reinterpret_cast<uint32_t*>(&p2);
+                                }
+                                dst[h] = w;
+                            }
+                        }
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 64) {
+                    float v[64];
+                    tmem_ld64(tq + (uint32_t)c, v);
+                    if (row < M) {
+                        float4* dst = reinterpret_cast<float4*>(C + (size_t)row * ldc + n0 + c);
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) {
+                            float4 w = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2],
+                                                   v[4 * u + 3]);
+                            if (MODE == kAddF32) {
+                                const float4 o = dst[u];
+                                w.x += o.x;
+                                w.y += o.y;
+                                w.z += o.z;
+                                w.w += o.w;
+                            }
+                            dst[u] = w;
+                        }
+                    }
+                }
+            }
+            // this accumulator may take the MMAs of tile j+2
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 2 * BN);
+    if (threadIdx.x == 0 && abort_flag) atomicExch(&g_persist_error, kDevTimeout);
+}
+
+template <int MODE>
+bool launch_mode(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
+                 int ldct, int M, int N, int K, cudaStream_t st) {
+    CUtensorMap ta, tb;
+    if (!make_tma_2d_bf16(&ta, A, M, K, lda, BM) || !make_tma_2d_bf16(&tb, W, N, K, ldw, BN))
+        return false;
+    static int sms = 0;
+    if (!sms) {
+        if (cudaFuncSetAttribute(k_gemm_persist<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)SMEM) != cudaSuccess)
+            return false;
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return false;
+    }
+    const int tiles = ((M + BM - 1) / BM) * (N / BN);
+    launch(k_gemm_persist<MODE>, std::min(tiles, sms), NTHREADS, SMEM, st, ta, tb, C, ldc, Ct,
+           ldct, M, N, K);
+    rlt_count_launch();
+    return true;
+}
+
+}  // namespace
+
+int read_and_clear_persist_error() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_persist_error, sizeof(int)) != cudaSuccess) return -1;
+    if (v) {
+        int z = 0;
+        cudaMemcpyToSymbol(g_persist_error, &z, sizeof(int));
+    }
+    return v;
+}
+
+// Returns false (nothing launched) for shapes or modes it does not handle.
+bool launch_gemm_persist(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc,
+                         bf16* Ct, int ldct, int M, int N, int K, int mode, cudaStream_t st) {
+    if (M < 2048 || N % BN || K < BK || K % BK) return false;
+    if (lda % 8 || ldw % 8 || ((uintptr_t)A & 15) || ((uintptr_t)W & 15)) return false;
+    if (mode == kSwiGLU) {
+        if (ldct % 8 || ((uintptr_t)Ct & 15)) return false;
+        return launch_mode<kSwiGLU>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, st);
+    }
+    if (ldc % 4 || ((uintptr_t)C & 15)) return false;
+    if (mode == kStoreF32)
+        return launch_mode<kStoreF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, st);
+    if (mode == kAddF32)
+        return launch_mode<kAddF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, st);
+    return false;
+}
+
+}  // namespace rlt

@@ -13,6 +13,9 @@
 // and the tile position, so a row's result does not depend on its batch.
 #include <cuda.h>
 
+#include <cstdlib>
+#include <cstring>
+
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -373,6 +376,16 @@ bool make_tma_2d_bf16(CUtensorMap* map, const void* base, int rows, int cols, in
     return make_map(map, base, rows, cols, ld, box_rows);
 }
 
+bool launch_gemm_persist(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc,
+                         bf16* Ct, int ldct, int M, int N, int K, int mode, cudaStream_t st);
+static bool persist_enabled() {
+    static const bool on = [] {
+        const char* e = getenv("RLT_GEMM_PERSIST");
+        return !(e && strcmp(e, "0") == 0);
+    }();
+    return on;
+}
+
 // Returns false (and launches nothing) when the shape or alignment does not
 // suit the tensor-core kernel; the caller then uses the CUDA-core kernel.
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
@@ -381,6 +394,11 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, in
     if (M <= 0 || N < 16 || K < BK || K % BK || splits < 1) return false;
     if (mode == kSwiGLU && (N % 128 || (ldct % 8) || ((uintptr_t)Ct & 15))) return false;
     if (lda % 8 || ldw % 8 || ((uintptr_t)A & 15) || ((uintptr_t)W & 15)) return false;
+    // many rows: the persistent kernel with two accumulators (epilogue of one
+    // tile under the MMAs of the next); RLT_GEMM_PERSIST=0 turns it off
+    if (M >= 2048 && splits == 1 && persist_enabled() &&
+        launch_gemm_persist(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, st))
+        return true;
     // wide tiles when M alone fills the machine, narrow ones (more CTAs)
     // otherwise; the SwiGLU epilogue needs whole 128-column gate/up groups
     if (M >= 2048)

@@ -123,6 +123,7 @@ void launch_sample(const float* logits, int V, int B, int32_t* argmax, int32_t* 
 
 int read_and_clear_device_error();  // device error word of the bounded-wait kernels
 int read_and_clear_attn_error();
+int read_and_clear_persist_error();  // same, for the persistent GEMM
 // Partial-sum slabs of a projection, consumed directly by an attention kernel.
 struct ProjIn {
     const float* P;   // slab 0 of the fp32 partial sums, [R][ldp]

@@ -1349,8 +1349,9 @@ extern "C" int rlt_state_check(rlt_state* s, void* stream) {
     if (w != 0 && cudaMemset(s->err, 0, 4) != cudaSuccess) return RLT_E_DEVICE;
     const int g = rlt::read_and_clear_device_error();
     const int ga = rlt::read_and_clear_attn_error();
-    if (g < 0 || ga < 0) return RLT_E_DEVICE;
-    if (w == 0) w = g ? g : ga;
+    const int gp = rlt::read_and_clear_persist_error();
+    if (g < 0 || ga < 0 || gp < 0) return RLT_E_DEVICE;
+    if (w == 0) w = g ? g : (ga ? ga : gp);
     if (w == rlt::kDevTimeout) return RLT_E_TIMEOUT;
     if (w == rlt::kDevBounds) return RLT_E_ARG;
     return w ? RLT_E_DEVICE : RLT_OK;
