@@ -47,6 +47,22 @@ def peaks():
             "fallback"
 
 
+def kernel_traffic(alg_bytes_per_launch: float):
+    """DRAM bytes per launch of the dominant kernel from its committed ncu
+    capture (profiles/dominant_kernel_traffic.json), scaled from the captured
+    launch to the average launch by the algorithmic bytes.  None when there is
+    no capture or the kernel's source changed since it was taken."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "dominant_kernel_traffic.json")))
+        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+        if hashlib.sha256(src).hexdigest() != rec["source_sha256"]:
+            return None
+        return rec["dram_bytes"] * alg_bytes_per_launch / rec["alg_bytes"]
+    except Exception:
+        return None
+
+
 def workload_desc(cfg) -> dict:
     kind = {0: "RLT-0", 1: "RLT-1", 2: f"RLT-2 (feedback chunk {cfg.chunk})"}[cfg.variant]
     dt = "bf16" if cfg.dtype == ri.DT_BF16 else "fp32"
@@ -311,7 +327,8 @@ def run_ours(args, cfg):
     n_s, ms_s, by_s = prof["step"]
     step_gbs = (by_s / ms_s * 1e3 / 1e9) if ms_s else 0.0
     n, ms, by = kprof["xattn"]
-    kname = "decoder cross-attention (k_attn_stream, window=false, q from projection slabs)"
+    kname = "decoder cross-attention (k_attn_dec1: one warp per (row, head), q from the projection slabs)"
+    xattn_timed = bool(n)
     if not n:       # no per-launch records: fall back to whole transition blocks
         n, ms, by = prof["step"]
         kname = "decoder transition block (graph of the block's kernels)"
@@ -333,7 +350,8 @@ def run_ours(args, cfg):
                 "ms_per_step": e2e_ms, "wall_ms_per_step": e2e_wall},
         "roofline": {"bound": "hbm", "kernel": kname,
                      "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                     "frac": achieved / pk["hbm_gbs"],
+                     "traffic": kernel_traffic(by / n) if xattn_timed else None,
                      "peak_kind": f"{pk_kind} hbm_gbs", "launches": n,
                      "avg_launch_us": (ms / n * 1e3) if n else None,
                      "alg_bytes_per_launch": (by / n) if n else None},
