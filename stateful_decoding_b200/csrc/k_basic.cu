@@ -443,6 +443,56 @@ void launch_set_state(const float* z, const float* P, int S, size_t slab, float*
     rlt_count_launch();
 }
 
+// One position per row: the state hand-off of this transition and the
+// merge input of the next, in one kernel (rows of a replayed run of blocks):
+// s <- z (+ residual slabs), RLT-2 register at a chunk end, pos_dec += 1, then
+// Gin = [T(e at the new position), T(RMSNorm(s or R) * gain)].  Same
+// arithmetic as k_set_state followed by k_merge_input.
+template <typename T>
+__global__ void __launch_bounds__(512)
+k_state_merge(const float* __restrict__ z, const float* __restrict__ P, int S, size_t slab,
+              float* __restrict__ s, float* __restrict__ Rr, int32_t* __restrict__ pos_dec,
+              int chunk, const float* __restrict__ e, int T_cap, const float* __restrict__ g,
+              T* __restrict__ Gin, int d, float eps) {
+    pdl_enter();
+    __shared__ float red[32];
+    const int b = blockIdx.x;
+    const int pd = pos_dec[b];
+    const bool upd = Rr != nullptr && ((pd + 1) % chunk) == 0;
+    const int j = 4 * threadIdx.x;
+    const bool act = j < d;
+    float4 fb = make_float4(0.f, 0.f, 0.f, 0.f), ev = fb, gv = fb;
+    if (act) {
+        const size_t row = (size_t)b * d + j;
+        float4 v = ld4(z + row);
+        if (P) v = add4(v, slab_sum4(P, S, slab, row));
+        st4(s + row, v);
+        fb = v;
+        if (Rr) {
+            if (upd) st4(Rr + row, v);
+            else fb = ld4(Rr + row);
+        }
+        ev = ld4(e + ((size_t)b * T_cap + pd + 1) * d + j);
+        gv = ld4(g + j);
+    }
+    const float ss = row_sum(act ? dot4(fb) : 0.f, red);   // every thread read pd before this
+    if (threadIdx.x == 0) pos_dec[b] = pd + 1;
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    if (act) {
+        T* out = Gin + (size_t)b * 2 * d;
+        store4<T>(out + j, ev);
+        store4<T>(out + d + j, scale4(fb, inv, gv));
+    }
+}
+template <typename T>
+void launch_state_merge(const float* z, const float* P, int S, size_t slab, float* s, float* Rreg,
+                        int32_t* pos_dec, int chunk, const float* e, int T_cap, const float* gain,
+                        T* Gin, int B, int d, float eps, cudaStream_t st) {
+    launch(k_state_merge<T>, B, row_threads(d / 4), 0, st, z, P, S, slab, s, Rreg, pos_dec, chunk,
+           e, T_cap, gain, Gin, d, eps);
+    rlt_count_launch();
+}
+
 __global__ void k_pos_add(int32_t* pos, int B, int n) {
     pdl_enter();
     int b = blockIdx.x * blockDim.x + threadIdx.x;
@@ -517,6 +567,9 @@ void launch_ring_write(const T* Kc, const T* Vc, const int32_t* pos_dec, T* ring
                                       size_t, const float*, const float*, int, size_t, int,    \
                                       float, float*, const float*, T*, float, int, int, int,   \
                                       cudaStream_t);                                           \
+    template void launch_state_merge<T>(const float*, const float*, int, size_t, float*,      \
+                                        float*, int32_t*, int, const float*, int, const float*, \
+                                        T*, int, int, float, cudaStream_t);                    \
     template void launch_merge_input<T>(const float*, int, const int32_t*, const float*,       \
                                         const float*, T*, int, int, int, float, cudaStream_t); \
     template void launch_qkv_dec<T>(const float*, int, size_t, const int32_t*, RopeTab, float*, \

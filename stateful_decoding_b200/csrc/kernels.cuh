@@ -96,6 +96,11 @@ void launch_set_state(const float* z, const float* P, int S, size_t slab, float*
                       int32_t* pos_dec, int chunk, int B, int n, int d, bool bump,
                       cudaStream_t st);
 void launch_pos_add(int32_t* pos, int B, int n, cudaStream_t st);
+// one position per row: launch_set_state(bump) and the next launch_merge_input
+template <typename T>
+void launch_state_merge(const float* z, const float* P, int S, size_t slab, float* s, float* Rreg,
+                        int32_t* pos_dec, int chunk, const float* e, int T_cap, const float* gain,
+                        T* Gin, int B, int d, float eps, cudaStream_t st);
 void launch_reset_rows(const int32_t* rows, int nrows, const float* s_star, float* s, float* Rr,
                        int32_t* pos_enc, int32_t* pos_dec, int d, cudaStream_t st);
 template <typename T>

@@ -926,8 +926,12 @@ static int norm_fuse_from_env() {
     const char* e = getenv("RLT_NORM_FUSE");
     return e ? atoi(e) : 0;
 }
+// merged_in: the previous block already wrote this block's merge input (Y);
+// fuse_out: end with the state hand-off fused with the next block's merge
+// input (one position per row, RLT-1/2, inside a replayed run of blocks).
 template <typename T>
-static void step_block(rlt_state* s, int n, cudaStream_t st) {
+static void step_block(rlt_state* s, int n, cudaStream_t st, bool merged_in = false,
+                       bool fuse_out = false) {
     using namespace rlt;
     rlt_model* m = s->m;
     const rlt_config& c = m->cfg;
@@ -955,7 +959,9 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
                             0.f, z, norm0, Y, eps, B, n, d, st);
     } else {
         const float* fb = c.variant == 2 ? s->Rr : s->s;
-        launch_merge_input<T>(s->e, s->T_cap, s->pos_dec, fb, m->merge_norm, Y, B, n, d, eps, st);
+        if (!merged_in)
+            launch_merge_input<T>(s->e, s->T_cap, s->pos_dec, fb, m->merge_norm, Y, B, n, d, eps,
+                                  st);
         // one GEMM for both projections: gate pre-activations in columns
         // 0..d-1 of the slabs, W_s r in columns d..2d-1
         const int nGS = gemm_p(Y, 2 * d, (const T*)m->wgs, 2 * d, 2 * d, P);
@@ -1038,8 +1044,14 @@ static void step_block(rlt_state* s, int n, cudaStream_t st) {
         else
             nres = gemm_p(Hd, fp, (const T*)L.w2, d, fp, P);
     }
-    launch_set_state(z, nres ? P : nullptr, nres, slab, s->s, c.variant == 2 ? s->Rr : nullptr,
-                     s->pos_dec, c.chunk, B, n, d, /*bump=*/true, st);
+    if (fuse_out)
+        launch_state_merge<T>(z, nres ? P : nullptr, nres, slab, s->s,
+                              c.variant == 2 ? s->Rr : nullptr, s->pos_dec, c.chunk, s->e, s->T_cap,
+                              m->merge_norm, Y, B, d, eps, st);
+    else
+        launch_set_state(z, nres ? P : nullptr, nres, slab, s->s,
+                         c.variant == 2 ? s->Rr : nullptr, s->pos_dec, c.chunk, B, n, d,
+                         /*bump=*/true, st);
 }
 
 static int run_block(rlt_state* s, int n, cudaStream_t st) {
@@ -1095,10 +1107,14 @@ static int run_graph(rlt_state* s, int n, cudaStream_t st) {
         cudaGraphExec_t ex = nullptr;
         bool ok = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
         if (ok) {
+            // consecutive one-position blocks hand the state to the next
+            // block's merge input in one kernel
+            const bool chain = n == 1 && s->m->cfg.variant != 0;
             for (int k = 0; k < kGraphBlocks; ++k) {
                 s->prof_block = k;
-                if (s->m->cfg.dtype == RLT_DTYPE_BF16) step_block<bf16>(s, n, st);
-                else step_block<float>(s, n, st);
+                const bool in = chain && k > 0, out = chain && k + 1 < kGraphBlocks;
+                if (s->m->cfg.dtype == RLT_DTYPE_BF16) step_block<bf16>(s, n, st, in, out);
+                else step_block<float>(s, n, st, in, out);
             }
             ok = cudaStreamEndCapture(st, &g) == cudaSuccess && g != nullptr;
         }
