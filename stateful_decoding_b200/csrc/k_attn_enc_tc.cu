@@ -82,26 +82,47 @@ k_attn_enc_tc(const float* __restrict__ Q, const bf16* __restrict__ cache, size_
     const bf16* kg = cache + (size_t)b * row_stride + (size_t)h * T_cap * EDH;
     const bf16* vg = kg + (size_t)heads * T_cap * EDH;
 
-    // ---- stage Q (fp32 -> bf16), K, V^T
-    for (int e = threadIdx.x; e < EQ * 8; e += ENT) {
-        const int r = e >> 3, c = e & 7;
-        uint4 w = make_uint4(0, 0, 0, 0);
-        if (r < nq) {
-            const float* src = Q + (size_t)(b * n + q0 + r) * d + h * EDH + c * 8;
-            const float4 a = *reinterpret_cast<const float4*>(src);
-            const float4 a2 = *reinterpret_cast<const float4*>(src + 4);
-            w = make_uint4(pack2(a.x, a.y), pack2(a.z, a.w), pack2(a2.x, a2.y), pack2(a2.z, a2.w));
+    // ---- stage Q (fp32 -> bf16), K, V^T: each thread issues all its loads
+    // of a phase before its first store
+    {
+        constexpr int QI = EQ * 8 / ENT;           // 16-byte bf16 chunks of Q per thread
+        float4 qa[QI], qb[QI];
+#pragma unroll
+        for (int u = 0; u < QI; ++u) {
+            const int e = threadIdx.x + u * ENT, r = e >> 3, c = e & 7;
+            qa[u] = qb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r < nq) {
+                const float* src = Q + (size_t)(b * n + q0 + r) * d + h * EDH + c * 8;
+                qa[u] = *reinterpret_cast<const float4*>(src);
+                qb[u] = *reinterpret_cast<const float4*>(src + 4);
+            }
         }
-        *reinterpret_cast<uint4*>(sQ + sw128(r, c)) = w;
+#pragma unroll
+        for (int u = 0; u < QI; ++u) {
+            const int e = threadIdx.x + u * ENT, r = e >> 3, c = e & 7;
+            *reinterpret_cast<uint4*>(sQ + sw128(r, c)) =
+                make_uint4(pack2(qa[u].x, qa[u].y), pack2(qa[u].z, qa[u].w), pack2(qb[u].x, qb[u].y),
+                           pack2(qb[u].z, qb[u].w));
+        }
     }
-    for (int e = threadIdx.x; e < NK * 8; e += ENT) {
-        const int k = e >> 3, c = e & 7;
-        uint4 w = make_uint4(0, 0, 0, 0);
-        if (k < kvalid) w = *reinterpret_cast<const uint4*>(kg + (size_t)k * EDH + c * 8);
-        *reinterpret_cast<uint4*>(sR2 + (k >> 7) * KT_BYTES + sw128(k & 127, c)) = w;
+    {
+        constexpr int KI = NK * 8 / ENT;           // 16-byte chunks of K per thread
+        uint4 kv[KI];
+#pragma unroll
+        for (int u = 0; u < KI; ++u) {
+            const int e = threadIdx.x + u * ENT, k = e >> 3, c = e & 7;
+            kv[u] = make_uint4(0, 0, 0, 0);
+            if (k < kvalid) kv[u] = *reinterpret_cast<const uint4*>(kg + (size_t)k * EDH + c * 8);
+        }
+#pragma unroll
+        for (int u = 0; u < KI; ++u) {
+            const int e = threadIdx.x + u * ENT, k = e >> 3, c = e & 7;
+            *reinterpret_cast<uint4*>(sR2 + (k >> 7) * KT_BYTES + sw128(k & 127, c)) = kv[u];
+        }
     }
     // V^T: a thread takes 8 consecutive keys of one 8-wide column chunk and
     // writes them as 8 rows (one per d_h index) of 8 keys each
+#pragma unroll
     for (int e = threadIdx.x; e < (NK / 8) * 8; e += ENT) {
         const int kgrp = e >> 3, c = e & 7;        // keys 8*kgrp .. +7, d_h 8c .. 8c+7
         uint32_t in[8][4];
