@@ -343,7 +343,8 @@ def run_ours(args, cfg):
         "dtype": "bf16" if cfg.dtype == ri.DT_BF16 else "f32", "data": "synthetic",
         "config": dict(workload_desc(cfg), global_batch=B * world,
                        parallelism=f"replicas x{world} (rows sharded, no collective)",
-                       l2="working set per step > L2: caches of all rows (see DESIGN.md)"),
+                       l2="no flush: each step writes and reads > 126 MB "
+                          "(encoder cache, memory, rings of all rows)"),
         "gpu_launches": launches,
         "e2e": {"value": job_tokens_per_s(B, T + D, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
