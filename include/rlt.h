@@ -48,6 +48,7 @@ extern "C" {
 #define RLT_E_DEVICE      -6  /* a CUDA call failed (no device, launch error, fault)      */
 #define RLT_E_TIMEOUT     -7  /* a bounded device wait gave up                            */
 #define RLT_E_UNSUPPORTED -8  /* configuration this build does not run                    */
+#define RLT_E_SNAPSHOT    -9  /* snapshot: bad magic, version or size, or other weights   */
 
 #define RLT_DTYPE_F32  0
 #define RLT_DTYPE_BF16 1
@@ -166,6 +167,55 @@ int rlt_state_positions(const rlt_state* state, int32_t* pos_enc, int32_t* pos_d
 #define RLT_PART_ENC  5
 int rlt_state_read(rlt_state* state, int part, void* dst, size_t nbytes, size_t* nbytes_out,
                    void* stream);
+
+/* Exact prefix snapshot of one row: everything the row needs to continue
+ * exactly as if it had never stopped -- the encoder cache C^E and memory M of
+ * every encoded position, s_t (and the RLT-2 register R), the window rings
+ * C^D, the encoder outputs e_t of positions not yet transitioned, pos_enc,
+ * pos_dec, and the identity of the weights and config (jiphyeonjeon review
+ * §6.5, multi-turn serving; greeksharifa App. E, App. H).  A row restored
+ * into any state of the same model -- another row, batch size, max_len,
+ * process -- continues with the same results as the row it was taken from
+ * (rows are independent, see above).  New tokens (a tool's output, a user
+ * turn) are appended with rlt_encode and consumed with rlt_prefill, as on the
+ * original row.  The sampler keeps no state: a sampled continuation repeats
+ * with the same rng_seed and rng_step.
+ *
+ * Snapshot bytes (little-endian), independent of batch and max_len:
+ *   [0,4) "RLTS"  [4,8) u32 version 1  [8,16) u64 checksum of the weight
+ *   blob's payload  [16,20) i32 pos_enc  [20,24) i32 pos_dec  [24,72) the 12
+ *   int32 fields of rlt_config in declaration order  [72,96) alpha, eps,
+ *   rope_base as f64  [96,128) zero;
+ *   then, with P = pos_enc, h heads, d_h = d/h, G' = G if L_D > 0 else 0:
+ *   s fp32 [d]; R fp32 [d]; e fp32 [P][d]; C^E [L_E][2][h][P][d_h] and
+ *   M [G'][2][h][P][d_h] in the model dtype; C^D [L_D][2][h][W-1][d_h] in
+ *   the model dtype (ring slot of position t: (t-1) mod (W-1)).
+ * Size = 128 + 8d + 4Pd + (2 h L_E + 2 h G') P d_h e + 2 h L_D (W-1) d_h e,
+ * e = 2 (bf16) or 4 (fp32).
+ *
+ * rlt_state_save: writes row `row`'s snapshot to `dst` (host or device),
+ * `nbytes` exactly its size (query with dst = NULL: *nbytes_out receives it).
+ * Ordered after the work already queued on `stream`; synchronises `stream`.
+ * RLT_E_ARG for a null state, a row outside [0, batch) or a wrong nbytes.
+ *
+ * rlt_state_load: replaces row `row` with the snapshot at `src` (host or
+ * device, `nbytes` its size); other rows are untouched.  Synchronises
+ * `stream`; `src` may be freed on return.  Errors, checked before anything is
+ * written: RLT_E_ARG (null state or src, bad row), RLT_E_SNAPSHOT (bad magic,
+ * version or reserved bytes, nbytes not the size the header implies, or a
+ * checksum or config other than the state's model), RLT_E_CAPACITY (pos_enc
+ * above the state's max_len).  RLT_E_DEVICE if a copy fails: the row's
+ * contents are then undefined until it is reset or loaded again.
+ *
+ * rlt_snapshot_info: checks a snapshot in HOST memory without a device and
+ * returns its config and positions (each output may be NULL); errors as
+ * rlt_state_load's format checks (RLT_E_ARG for a null snapshot). */
+#define RLT_SNAPSHOT_HEADER_BYTES 128
+int rlt_state_save(rlt_state* state, int row, void* dst, size_t nbytes, size_t* nbytes_out,
+                   void* stream);
+int rlt_state_load(rlt_state* state, int row, const void* src, size_t nbytes, void* stream);
+int rlt_snapshot_info(const void* snap, size_t nbytes, rlt_config* cfg, int32_t* pos_enc,
+                      int32_t* pos_dec);
 
 /* Synchronise `stream` and report the state's sticky device error word
  * (RLT_OK, RLT_E_TIMEOUT, ...), clearing it. */

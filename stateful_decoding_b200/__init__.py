@@ -26,6 +26,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 RLT_OK, RLT_E_ARG, RLT_E_OOM, RLT_E_CAPACITY, RLT_E_ORDER = 0, -1, -2, -3, -4
 RLT_E_BLOB, RLT_E_DEVICE, RLT_E_TIMEOUT, RLT_E_UNSUPPORTED = -5, -6, -7, -8
+RLT_E_SNAPSHOT = -9
+SNAPSHOT_HEADER_BYTES = 128                # RLT_SNAPSHOT_HEADER_BYTES
 PART_S, PART_R, PART_E, PART_MEM, PART_RING, PART_ENC = range(6)
 PROF_XATTN, PROF_SWA, PROF_STEP, PROF_ENC = range(4)
 READOUT_ROWS_SCRATCH_BYTES = 16 << 20      # RLT_READOUT_ROWS_SCRATCH_BYTES
@@ -55,6 +57,10 @@ _SIGS = {
     "rlt_state_positions": (_i, [_vp, _vp, _vp]),
     "rlt_state_read": (_i, [_vp, _i, _vp, _sz, ctypes.POINTER(_sz), _vp]),
     "rlt_state_check": (_i, [_vp, _vp]),
+    "rlt_state_save": (_i, [_vp, _i, _vp, _sz, ctypes.POINTER(_sz), _vp]),
+    "rlt_state_load": (_i, [_vp, _i, _vp, _sz, _vp]),
+    "rlt_snapshot_info": (_i, [_vp, _sz, ctypes.POINTER(rlt_config), ctypes.POINTER(ctypes.c_int32),
+                               ctypes.POINTER(ctypes.c_int32)]),
     "rlt_kernel_launches": (_u64, []),
     "rlt_strerror": (ctypes.c_char_p, [_i]),
     "rlt_profile_enable": (_i, [_vp, _i]),
@@ -201,6 +207,40 @@ def rlt_state_check(state, stream=None) -> int:
     return _lib.rlt_state_check(state, _stream(stream))
 
 
+def rlt_state_save(state, row: int, dst=None, nbytes: int = 0, stream=None):
+    out = _sz()
+    code = _lib.rlt_state_save(state, row, _ptr(dst), nbytes, ctypes.byref(out), _stream(stream))
+    return code, out.value
+
+
+def rlt_state_load(state, row: int, src, nbytes: int, stream=None) -> int:
+    return _lib.rlt_state_load(state, row, _ptr(src), nbytes, _stream(stream))
+
+
+def rlt_snapshot_info(snap, nbytes: int):
+    """(code, rlt_config, pos_enc, pos_dec) of a snapshot in host memory."""
+    c, pe, pd = rlt_config(), ctypes.c_int32(), ctypes.c_int32()
+    code = _lib.rlt_snapshot_info(_ptr(snap), nbytes, ctypes.byref(c), ctypes.byref(pe),
+                                  ctypes.byref(pd))
+    return code, c, pe.value, pd.value
+
+
+def _as_bytes_array(snap):
+    """A host snapshot as a contiguous numpy uint8 array (bytes are copied)."""
+    import numpy as np
+    if isinstance(snap, (bytes, bytearray, memoryview)):
+        return np.frombuffer(bytes(snap), np.uint8).copy()
+    return snap
+
+
+def snapshot_info(snap):
+    """Config and positions of a snapshot held in host memory."""
+    a = _as_bytes_array(snap)
+    code, c, pe, pd = rlt_snapshot_info(a, a.nbytes)
+    _check(code, "rlt_snapshot_info")
+    return c, pe, pd
+
+
 def rlt_profile_enable(state, on: bool) -> int:
     return _lib.rlt_profile_enable(state, int(on))
 
@@ -308,6 +348,23 @@ class State:
 
     def check(self, stream=None):
         return _check(rlt_state_check(self.handle, stream), "rlt_state_check")
+
+    def save(self, row: int, dst=None, stream=None):
+        """Snapshot of one row: into a new host numpy uint8 array, or into
+        `dst` (a host or CUDA buffer of exactly the snapshot's size)."""
+        import numpy as np
+        code, nbytes = rlt_state_save(self.handle, row)
+        _check(code, "rlt_state_save")
+        if dst is None:
+            dst = np.empty(nbytes, np.uint8)
+        _check(rlt_state_save(self.handle, row, dst, nbytes, stream)[0], "rlt_state_save")
+        return dst
+
+    def load(self, row: int, snap, stream=None):
+        """Replace one row with a snapshot (host bytes / numpy, or a CUDA tensor)."""
+        a = _as_bytes_array(snap)
+        nbytes = a.nbytes if hasattr(a, "nbytes") else a.numel() * a.element_size()
+        return _check(rlt_state_load(self.handle, row, a, nbytes, stream), "rlt_state_load")
 
     def profile(self, on: int):
         """0: off; 1: time kernel classes (graph-replayed transition blocks

@@ -119,6 +119,7 @@ float bf16_bits_to_float(uint16_t h) {
 
 struct ParsedBlob {
     rlt_config cfg;
+    uint64_t checksum = 0;              // of the payload: identifies the weights
     std::vector<const uint8_t*> data;   // per manifest entry
 };
 
@@ -173,6 +174,7 @@ int parse_blob(const void* blob, size_t nbytes, ParsedBlob* out) {
         off += bytes + ((64 - bytes % 64) % 64);
     }
     out->cfg = c;
+    out->checksum = ck;
     return RLT_OK;
 }
 
@@ -192,6 +194,7 @@ struct DecLayerW {
 
 struct rlt_model {
     rlt_config cfg;
+    uint64_t checksum = 0;          // the blob payload's checksum (the model's identity)
     int device = 0;
     int dh = 0, fpad = 0;
     size_t elt = 4;
@@ -323,6 +326,7 @@ extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model
 
     rlt_model* m = new rlt_model();
     m->cfg = c;
+    m->checksum = pb.checksum;
     m->device = device;
     m->dh = dh;
     m->fpad = (c.ffn + 63) / 64 * 64;
@@ -1356,6 +1360,225 @@ extern "C" int rlt_state_read(rlt_state* s, int part, void* dst, size_t nbytes,
     return RLT_OK;
 }
 
+// ============================================================================
+// exact prefix snapshots of one row
+// ============================================================================
+// A row resumes exactly from: the encoder cache C^E and the memory M of every
+// encoded position, the decoder state s (and the RLT-2 register R), the window
+// rings C^D, the encoder outputs e_t that transitions still have to merge,
+// both positions, and the identity of the weights and config the row was
+// built under (jiphyeonjeon review §6.5, multi-turn serving; greeksharifa
+// App. E, App. H).  The byte layout is the one include/rlt.h documents; it
+// does not depend on the state's batch or max_len.
+namespace {
+constexpr size_t kSnapHeader = RLT_SNAPSHOT_HEADER_BYTES;
+constexpr uint32_t kSnapVersion = 1;
+
+struct SnapGeom {
+    size_t d, dh, elt;
+    size_t enc_planes, mem_planes;   // [T_cap][d_h] planes of one row's C^E and M
+    size_t ring;                     // elements of one row's window rings
+};
+
+SnapGeom snap_geom(const rlt_config& c) {
+    SnapGeom g;
+    g.d = (size_t)c.d;
+    g.dh = (size_t)(c.d / c.heads);
+    g.elt = c.dtype == RLT_DTYPE_BF16 ? 2 : 4;
+    g.enc_planes = (size_t)c.n_enc * 2 * c.heads;
+    g.mem_planes = (size_t)(c.n_dec > 0 ? c.groups : 0) * 2 * c.heads;
+    g.ring = (size_t)c.n_dec * 2 * c.heads * (size_t)std::max(0, c.window - 1) * g.dh;
+    return g;
+}
+
+size_t snap_bytes(const SnapGeom& g, int pos_enc) {
+    const size_t p = (size_t)pos_enc;
+    return kSnapHeader + 2 * g.d * 4 + p * g.d * 4 +
+           (g.enc_planes + g.mem_planes) * p * g.dh * g.elt + g.ring * g.elt;
+}
+
+void snap_write_header(uint8_t* h, const rlt_config& c, uint64_t checksum, int32_t pos_enc,
+                       int32_t pos_dec) {
+    memset(h, 0, kSnapHeader);
+    memcpy(h, "RLTS", 4);
+    memcpy(h + 4, &kSnapVersion, 4);
+    memcpy(h + 8, &checksum, 8);
+    memcpy(h + 16, &pos_enc, 4);
+    memcpy(h + 20, &pos_dec, 4);
+    const int32_t f[12] = {c.vocab, c.d,     c.heads, c.n_enc,   c.n_dec, c.ffn,
+                           c.window, c.groups, c.chunk, c.variant, c.tied,  c.dtype};
+    memcpy(h + 24, f, sizeof f);
+    memcpy(h + 72, &c.alpha, 8);
+    memcpy(h + 80, &c.eps, 8);
+    memcpy(h + 88, &c.rope_base, 8);
+}
+
+// Reads and checks a header against the snapshot's total size.  The bounds
+// keep every size product below 2^63.
+int snap_read_header(const uint8_t* h, size_t nbytes, rlt_config* c, uint64_t* checksum,
+                     int32_t* pos_enc, int32_t* pos_dec) {
+    if (nbytes < kSnapHeader || memcmp(h, "RLTS", 4) != 0) return RLT_E_SNAPSHOT;
+    uint32_t ver;
+    memcpy(&ver, h + 4, 4);
+    if (ver != kSnapVersion) return RLT_E_SNAPSHOT;
+    for (size_t i = 96; i < kSnapHeader; ++i)
+        if (h[i]) return RLT_E_SNAPSHOT;
+    memcpy(checksum, h + 8, 8);
+    memcpy(pos_enc, h + 16, 4);
+    memcpy(pos_dec, h + 20, 4);
+    int32_t f[12];
+    memcpy(f, h + 24, sizeof f);
+    c->vocab = f[0]; c->d = f[1]; c->heads = f[2]; c->n_enc = f[3]; c->n_dec = f[4];
+    c->ffn = f[5]; c->window = f[6]; c->groups = f[7]; c->chunk = f[8]; c->variant = f[9];
+    c->tied = f[10]; c->dtype = f[11];
+    memcpy(&c->alpha, h + 72, 8);
+    memcpy(&c->eps, h + 80, 8);
+    memcpy(&c->rope_base, h + 88, 8);
+    if (c->d <= 0 || c->d > (1 << 16) || c->heads <= 0 || c->d % c->heads || c->n_enc < 0 ||
+        c->n_enc > 1024 || c->n_dec < 0 || c->n_dec > 1024 || c->window < 1 ||
+        c->window > (1 << 24) || c->groups < 1 || c->groups > 1024 ||
+        (c->dtype != RLT_DTYPE_F32 && c->dtype != RLT_DTYPE_BF16))
+        return RLT_E_SNAPSHOT;
+    if (*pos_enc < 0 || *pos_enc > (1 << 28) || *pos_dec < 0 || *pos_dec > *pos_enc)
+        return RLT_E_SNAPSHOT;
+    if (nbytes != snap_bytes(snap_geom(*c), *pos_enc)) return RLT_E_SNAPSHOT;
+    return RLT_OK;
+}
+
+bool same_config(const rlt_config& a, const rlt_config& b) {
+    return a.vocab == b.vocab && a.d == b.d && a.heads == b.heads && a.n_enc == b.n_enc &&
+           a.n_dec == b.n_dec && a.ffn == b.ffn && a.window == b.window &&
+           a.groups == b.groups && a.chunk == b.chunk && a.variant == b.variant &&
+           a.tied == b.tied && a.dtype == b.dtype && memcmp(&a.alpha, &b.alpha, 8) == 0 &&
+           memcmp(&a.eps, &b.eps, 8) == 0 && memcmp(&a.rope_base, &b.rope_base, 8) == 0;
+}
+
+// Copies between one row of a state and a packed snapshot: the snapshot's
+// sections in their order, each section a plain copy except C^E and M, whose
+// first pos_enc positions of every [T_cap][d_h] plane are packed.
+struct SnapCopier {
+    rlt_state* s;
+    int row, pos;
+    SnapGeom g;
+    uint8_t* snap;
+    bool to_snap;                // state -> snapshot (save) or back (load)
+    cudaMemcpyKind kind;
+    cudaStream_t st;
+    size_t off = kSnapHeader;
+    cudaError_t e = cudaSuccess;
+
+    void flat(void* state_part, size_t bytes) {
+        if (e == cudaSuccess && bytes)
+            e = to_snap ? cudaMemcpyAsync(snap + off, state_part, bytes, kind, st)
+                        : cudaMemcpyAsync(state_part, snap + off, bytes, kind, st);
+        off += bytes;
+    }
+    void planes(void* state_row, size_t n_planes) {
+        const size_t w = (size_t)pos * g.dh * g.elt, pitch = (size_t)s->T_cap * g.dh * g.elt;
+        if (e == cudaSuccess && w && n_planes)
+            e = to_snap ? cudaMemcpy2DAsync(snap + off, w, state_row, pitch, w, n_planes, kind, st)
+                        : cudaMemcpy2DAsync(state_row, pitch, snap + off, w, w, n_planes, kind, st);
+        off += w * n_planes;
+    }
+    void all() {
+        const size_t r = (size_t)row;
+        flat(s->s + r * g.d, g.d * 4);
+        flat(s->Rr + r * g.d, g.d * 4);
+        flat(s->e + r * s->T_cap * g.d, (size_t)pos * g.d * 4);
+        planes((uint8_t*)s->enc + r * s->enc_row * g.elt, g.enc_planes);
+        planes((uint8_t*)s->mem + r * s->mem_row * g.elt, g.mem_planes);
+        flat((uint8_t*)s->ring + r * s->ring_row * g.elt, g.ring * g.elt);
+    }
+};
+}  // namespace
+
+extern "C" int rlt_snapshot_info(const void* snap, size_t nbytes, rlt_config* cfg,
+                                 int32_t* pos_enc, int32_t* pos_dec) {
+    if (!snap) return RLT_E_ARG;
+    rlt_config c;
+    uint64_t ck;
+    int32_t pe, pd;
+    const int rc = snap_read_header((const uint8_t*)snap, nbytes, &c, &ck, &pe, &pd);
+    if (rc) return rc;
+    if (cfg) *cfg = c;
+    if (pos_enc) *pos_enc = pe;
+    if (pos_dec) *pos_dec = pd;
+    return RLT_OK;
+}
+
+extern "C" int rlt_state_save(rlt_state* s, int row, void* dst, size_t nbytes,
+                              size_t* nbytes_out, void* stream) {
+    if (!s || row < 0 || row >= s->B) return RLT_E_ARG;
+    const rlt_model* m = s->m;
+    const SnapGeom g = snap_geom(m->cfg);
+    const int32_t pe = s->h_pos_enc[row], pd = s->h_pos_dec[row];
+    const size_t sz = snap_bytes(g, pe);
+    if (nbytes_out) *nbytes_out = sz;
+    if (!dst) return RLT_OK;
+    if (nbytes != sz) return RLT_E_ARG;
+    if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
+    const cudaStream_t st = (cudaStream_t)stream;
+    const bool dev = is_device_ptr(dst);
+    uint8_t hdr[kSnapHeader];
+    snap_write_header(hdr, m->cfg, m->checksum, pe, pd);
+    SnapCopier cp{s, row, pe, g, (uint8_t*)dst, true,
+                  dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost, st};
+    if (dev) cp.e = cudaMemcpyAsync(dst, hdr, kSnapHeader, cudaMemcpyHostToDevice, st);
+    else memcpy(dst, hdr, kSnapHeader);
+    cp.all();
+    // the header's host copy and a host destination are done with on return
+    if (cp.e == cudaSuccess) cp.e = cudaStreamSynchronize(st);
+    if (cp.e != cudaSuccess || cp.off != sz) {
+        cudaGetLastError();
+        return RLT_E_DEVICE;
+    }
+    return RLT_OK;
+}
+
+extern "C" int rlt_state_load(rlt_state* s, int row, const void* src, size_t nbytes,
+                              void* stream) {
+    if (!s || !src || row < 0 || row >= s->B) return RLT_E_ARG;
+    const rlt_model* m = s->m;
+    if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
+    const cudaStream_t st = (cudaStream_t)stream;
+    const bool dev = is_device_ptr(src);
+    uint8_t hdr[kSnapHeader];
+    if (nbytes < kSnapHeader) return RLT_E_SNAPSHOT;
+    if (dev) {
+        if (cudaMemcpyAsync(hdr, src, kSnapHeader, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+            cudaStreamSynchronize(st) != cudaSuccess) {
+            cudaGetLastError();
+            return RLT_E_DEVICE;
+        }
+    } else {
+        memcpy(hdr, src, kSnapHeader);
+    }
+    rlt_config c;
+    uint64_t ck;
+    int32_t pe, pd;
+    int rc = snap_read_header(hdr, nbytes, &c, &ck, &pe, &pd);
+    if (rc) return rc;
+    if (ck != m->checksum || !same_config(c, m->cfg)) return RLT_E_SNAPSHOT;
+    if (pe > s->T_cap) return RLT_E_CAPACITY;
+    const SnapGeom g = snap_geom(m->cfg);
+    SnapCopier cp{s, row, pe, g, (uint8_t*)const_cast<void*>(src), false,
+                  dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, st};
+    cp.all();
+    // positions straight from the snapshot's header fields
+    const uint8_t* sp = (const uint8_t*)src;
+    if (cp.e == cudaSuccess) cp.e = cudaMemcpyAsync(s->pos_enc + row, sp + 16, 4, cp.kind, st);
+    if (cp.e == cudaSuccess) cp.e = cudaMemcpyAsync(s->pos_dec + row, sp + 20, 4, cp.kind, st);
+    // a host source may be freed on return
+    if (cp.e == cudaSuccess) cp.e = cudaStreamSynchronize(st);
+    if (cp.e != cudaSuccess || cp.off != nbytes) {
+        cudaGetLastError();
+        return RLT_E_DEVICE;
+    }
+    s->h_pos_enc[row] = pe;
+    s->h_pos_dec[row] = pd;
+    return RLT_OK;
+}
+
 extern "C" int rlt_state_check(rlt_state* s, void* stream) {
     if (!s) return RLT_E_ARG;
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
@@ -1429,6 +1652,7 @@ extern "C" const char* rlt_strerror(int code) {
         case RLT_E_DEVICE: return "CUDA error";
         case RLT_E_TIMEOUT: return "bounded device wait gave up";
         case RLT_E_UNSUPPORTED: return "unsupported configuration";
+        case RLT_E_SNAPSHOT: return "bad snapshot (magic, version, size) or taken under other weights";
         default: return "unknown error";
     }
 }

@@ -34,7 +34,7 @@ def test_exports_every_declared_function(lib):
 
 
 def test_strerror_covers_codes(lib):
-    for code in range(0, -9, -1):
+    for code in range(0, -10, -1):
         assert lib.rlt_strerror(code) != "unknown error"
     assert lib.rlt_strerror(-99) == "unknown error"
 
@@ -76,6 +76,9 @@ def test_null_arguments(lib):
     assert lib._lib.rlt_prefill(None, 1, None) == lib.RLT_E_ARG
     assert lib._lib.rlt_readout(None, None, None, None, 0, 0, 1.0, None) == lib.RLT_E_ARG
     assert lib._lib.rlt_state_check(None, None) == lib.RLT_E_ARG
+    assert lib._lib.rlt_state_save(None, 0, None, 0, None, None) == lib.RLT_E_ARG
+    assert lib._lib.rlt_state_load(None, 0, None, 0, None) == lib.RLT_E_ARG
+    assert lib._lib.rlt_snapshot_info(None, 0, None, None, None) == lib.RLT_E_ARG
     assert lib.rlt_kernel_launches() >= 0
 
 
@@ -114,3 +117,63 @@ def test_readout_rows_scratch_limit_matches_header():
             if sd.readout_rows_scratch_bytes(r, 2048, 32000, True, True)
             <= sd.READOUT_ROWS_SCRATCH_BYTES]
     assert max(fits) == 127 and "at most 127 rows" in hdr
+
+
+# ---------------------------------------------------------------- snapshots
+def _snapshot_bytes(cfg, pos_enc, pos_dec, checksum=0x0123456789ABCDEF):
+    """A snapshot laid out as include/rlt.h states it (header fields, then
+    zero-filled sections of the stated sizes), written independently of the
+    library."""
+    import struct
+    h, dh = cfg.heads, cfg.d // cfg.heads
+    e = 2 if cfg.dtype == ri.DT_BF16 else 4
+    g_ = cfg.groups if cfg.n_dec > 0 else 0
+    hdr = b"RLTS" + struct.pack("<IQii", 1, checksum, pos_enc, pos_dec)
+    hdr += struct.pack("<12i", cfg.vocab, cfg.d, cfg.heads, cfg.n_enc, cfg.n_dec, cfg.ffn,
+                       cfg.window, cfg.groups, cfg.chunk, cfg.variant, int(cfg.tied), cfg.dtype)
+    hdr += struct.pack("<3d", cfg.alpha, cfg.eps, cfg.rope_base)
+    assert len(hdr) == 96
+    hdr += bytes(128 - 96)
+    body = (8 * cfg.d + 4 * pos_enc * cfg.d + (2 * h * cfg.n_enc + 2 * h * g_) * pos_enc * dh * e
+            + 2 * h * cfg.n_dec * (cfg.window - 1) * dh * e)
+    return bytearray(hdr + bytes(body))
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "parity_bf16", "s5_bf16", "rlt2_mod5_bf16"])
+def test_snapshot_info_reads_the_documented_layout(lib, name):
+    cfg = ri.CONFIGS[name]
+    snap = _snapshot_bytes(cfg, 7, 5)
+    c, pe, pd = lib.snapshot_info(bytes(snap))
+    assert (pe, pd) == (7, 5)
+    for f in ("vocab", "d", "heads", "n_enc", "n_dec", "ffn", "window", "groups", "chunk",
+              "variant", "dtype"):
+        assert getattr(c, f) == getattr(cfg, f), f
+    assert (c.alpha, c.eps, c.rope_base) == (cfg.alpha, cfg.eps, cfg.rope_base)
+    # a fresh row (nothing encoded) has only s, R and the rings
+    c0, pe0, pd0 = lib.snapshot_info(bytes(_snapshot_bytes(cfg, 0, 0)))
+    assert (pe0, pd0) == (0, 0)
+
+
+def test_snapshot_info_rejects_malformed(lib):
+    cfg = ri.CONFIGS["parity_bf16"]
+    good = _snapshot_bytes(cfg, 6, 6)
+    info = lambda b: lib.rlt_snapshot_info(np.frombuffer(bytes(b), np.uint8).copy(), len(b))[0]  # noqa: E731
+    assert info(good) == lib.RLT_OK
+    bad = bytearray(good); bad[0:4] = b"RLTB"                      # magic
+    assert info(bad) == lib.RLT_E_SNAPSHOT
+    bad = bytearray(good); bad[4] = 2                              # version
+    assert info(bad) == lib.RLT_E_SNAPSHOT
+    bad = bytearray(good); bad[100] = 1                            # reserved bytes
+    assert info(bad) == lib.RLT_E_SNAPSHOT
+    assert info(good[:-1]) == lib.RLT_E_SNAPSHOT                   # truncated
+    assert info(good + b"\0") == lib.RLT_E_SNAPSHOT               # trailing byte
+    assert info(good[:100]) == lib.RLT_E_SNAPSHOT                  # shorter than a header
+    assert info(_snapshot_bytes(cfg, 3, 4)) == lib.RLT_E_SNAPSHOT  # pos_dec > pos_enc
+    bad = _snapshot_bytes(cfg, 0, 0); bad[16:20] = (-1).to_bytes(4, "little", signed=True)
+    assert info(bad) == lib.RLT_E_SNAPSHOT                         # negative pos_enc
+    # the size follows pos_enc: a snapshot relabelled with another pos_enc no longer fits
+    bad = bytearray(good); bad[16] = 7
+    assert info(bad) == lib.RLT_E_SNAPSHOT
+    # heads not dividing d
+    bad = bytearray(good); bad[32:36] = (7).to_bytes(4, "little")
+    assert info(bad) == lib.RLT_E_SNAPSHOT
