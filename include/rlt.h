@@ -68,7 +68,9 @@ typedef struct rlt_config {
  * named tensor records in the fixed manifest order of the config.  Errors:
  * RLT_E_BLOB (bad magic/version/manifest/checksum), RLT_E_UNSUPPORTED (head
  * size other than 16, 32, 64, 128, or width d above 2048), RLT_E_DEVICE,
- * RLT_E_OOM. */
+ * RLT_E_OOM.  One device per process: kernels' shared-memory attributes are
+ * set once per process, on the device that launches them first, so calls on
+ * models of a second device in the same process may fail with RLT_E_DEVICE. */
 int rlt_create(const void* blob, size_t nbytes, int device, rlt_model** out);
 void rlt_destroy(rlt_model* model);
 int rlt_model_config(const rlt_model* model, rlt_config* out);
