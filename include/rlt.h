@@ -127,6 +127,31 @@ int rlt_prefill(rlt_state* state, int T, void* stream);
 int rlt_readout(rlt_state* state, float* logits, int32_t* argmax, int32_t* sampled,
                 uint64_t rng_seed, uint64_t rng_step, float temperature, void* stream);
 
+/* Replay: log-probabilities of given tokens under the current weights, each
+ * read from the state that precedes it, then the token is consumed
+ * (jiphyeonjeon review §6.2, eq. 5.3-5.5: log pi(y|c) = sum_i log p(y_i | c,
+ * y_<i); greeksharifa App. D.3, F.4).  tokens: int32 [batch][n], host or
+ * device, appended to every row as by rlt_encode; then for j = 0..n-1
+ *   logprobs[b][j] = log softmax(logits_b / temperature)[tokens[b][j]],
+ * logits_b = W_out RMSNorm_out(s) of row b before token j is consumed (for
+ * a reset row and j = 0, the readout of s_star), followed by one transition.
+ * temperature = 1 is the model's own distribution; the sampler's temperature
+ * gives the distribution rlt_readout samples from (same max and summation,
+ * so exp(logprob) is the sampling probability up to rounding).  Afterwards
+ * every row has consumed the n tokens: the same state as rlt_encode +
+ * rlt_prefill(n).  A replay from the sequence start resets the rows first;
+ * the prompt's terms come out beside the response's and the caller keeps the
+ * ones it needs.  logprobs: fp32 [batch][n], host or device (host: valid on
+ * return; the call then synchronises `stream`).  One readout and one
+ * transition per position (no graph replay).  The first call allocates
+ * 8 * batch * max_len bytes of scratch in the state.  Errors: RLT_E_ARG (null
+ * pointers, n < 0, temperature <= 0, a host token outside [0, vocab)),
+ * RLT_E_ORDER (a row has encoded tokens not yet consumed), RLT_E_CAPACITY;
+ * a device token outside [0, vocab) gives NaN and RLT_E_ARG from
+ * rlt_state_check. */
+int rlt_replay_logprobs(rlt_state* state, const int32_t* tokens, int n, float* logprobs,
+                        float temperature, void* stream);
+
 /* Readout of caller-supplied state vectors that allocates nothing (no
  * counterpart in the method: a serving convenience for callers that hold a
  * model but no state, and may not allocate device memory).  s_rows: device

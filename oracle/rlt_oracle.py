@@ -26,7 +26,10 @@ What it computes, one sequence ("row") at a time, in float64:
   for prompt and response tokens -- jiphyeonjeon review §3.1 (paper eq. 2.7);
 * RLT-2 (register held inside B-token chunks counted from BOS, replaced by s
   at a complete chunk's end) and RLT-0 (u_t = e_t) -- greeksharifa §2.7, App. I;
-* the readout: RMSNorm, linear map, softmax -- greeksharifa §2.3.
+* the readout: RMSNorm, linear map, softmax -- greeksharifa §2.3;
+* the replay log-probabilities log p(y_i | c, y_<i), each read from the state
+  that precedes the token -- jiphyeonjeon review §6.2 (paper eq. 5.3-5.5),
+  greeksharifa App. D.3, F.4.
 
 Where the pages leave a step open (the block equations are missing from the
 extracted text) this follows these readings: pre-norm RMSNorm (eps 1e-6,
@@ -47,7 +50,9 @@ B=1 RLT-2 = RLT-1, encoder schedules), closed forms (one-key attention,
 W=1 window, W >= T window = full causal attention, alpha = 0 = RLT-0,
 saturated gates), independent parallel formulations (RLT-0 teacher-forced
 pass; full-history windowed decoder), parameter counts printed on the pages,
-and the random-init loss ~ ln V.  Absolute logit values have no worked
+and the random-init loss ~ ln V; the replay against closed forms of the
+log-softmax, scipy's log_softmax, and the chain rule (the probabilities of all
+continuations of a fixed length sum to one).  Absolute logit values have no worked
 example on the pages: beyond those identities they are parity unpinned.
 """
 from __future__ import annotations
@@ -397,4 +402,34 @@ def run_sequence(model: RLTOracle, tokens: Sequence[int]) -> List[np.ndarray]:
     for _ in range(len(tokens)):
         model.transition(st)
         out.append(model.readout(st))
+    return out
+
+
+# ----------------------------------------------------------------------------
+# Replay: the policy's per-token log-probabilities
+# ----------------------------------------------------------------------------
+
+
+def log_softmax_at(logits: np.ndarray, index: int, temperature: float = 1.0) -> float:
+    """log p_index with p = softmax(logits / temperature), from its definition:
+    z_index - log sum_j exp(z_j), the sum taken after subtracting max z."""
+    z = np.asarray(logits, dtype=np.float64) / temperature
+    m = z.max()
+    return float((z[index] - m) - np.log(np.sum(np.exp(z - m))))
+
+
+def replay_logprobs(model: RLTOracle, st: RowState, tokens: Sequence[int],
+                    temperature: float = 1.0) -> np.ndarray:
+    """The trainer's side of the replay contract (jiphyeonjeon review §6.2,
+    eq. 5.3-5.5; greeksharifa App. D.3, F.4): for each given token in order,
+    read log p(token | everything consumed so far) from the current state,
+    then consume the token -- encode it onto the cache and take one transition.
+    ``st`` must have consumed every token it encoded.  Returns the log-
+    probabilities; ``st`` ends having consumed all the tokens."""
+    assert st.pos_dec == st.pos_enc, "replay starts from a state with nothing pending"
+    out = np.empty(len(tokens), np.float64)
+    for j, tok in enumerate(tokens):
+        out[j] = log_softmax_at(model.readout(st), int(tok), temperature)
+        model.encode(st, [int(tok)])
+        model.transition(st)
     return out

@@ -54,6 +54,7 @@ _SIGS = {
     "rlt_prefill": (_i, [_vp, _i, _vp]),
     "rlt_readout": (_i, [_vp, _vp, _vp, _vp, _u64, _u64, ctypes.c_float, _vp]),
     "rlt_readout_rows": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _u64, _u64, ctypes.c_float, _vp]),
+    "rlt_replay_logprobs": (_i, [_vp, _vp, _i, _vp, ctypes.c_float, _vp]),
     "rlt_state_positions": (_i, [_vp, _vp, _vp]),
     "rlt_state_read": (_i, [_vp, _i, _vp, _sz, ctypes.POINTER(_sz), _vp]),
     "rlt_state_check": (_i, [_vp, _vp]),
@@ -182,6 +183,12 @@ def rlt_readout_rows(model, s_rows, rows: int, logits=None, argmax=None, sampled
                      stream=None) -> int:
     return _lib.rlt_readout_rows(model, _ptr(s_rows), rows, _ptr(logits), _ptr(argmax),
                                  _ptr(sampled), rng_seed, rng_step, temperature, _stream(stream))
+
+
+def rlt_replay_logprobs(state, tokens, n: int, logprobs, temperature: float = 1.0,
+                        stream=None) -> int:
+    return _lib.rlt_replay_logprobs(state, _ptr(tokens), n, _ptr(logprobs), temperature,
+                                    _stream(stream))
 
 
 def readout_rows_scratch_bytes(rows: int, d: int, vocab: int, bf16: bool,
@@ -329,6 +336,17 @@ class State:
                 stream=None):
         return _check(rlt_readout(self.handle, logits, argmax, sampled, seed, step, temperature,
                                   stream), "rlt_readout")
+
+    def replay_logprobs(self, tokens, logprobs=None, temperature=1.0, stream=None):
+        """log p of each given token (int32 [batch][n]) read before it is
+        consumed; returns `logprobs` (fp32 [batch][n], host numpy by default)."""
+        import numpy as np
+        n = int(tokens.shape[1])
+        if logprobs is None:
+            logprobs = np.empty((self.batch, n), np.float32)
+        _check(rlt_replay_logprobs(self.handle, tokens, n, logprobs, temperature, stream),
+               "rlt_replay_logprobs")
+        return logprobs
 
     def positions(self):
         import numpy as np

@@ -95,7 +95,61 @@ k_sample(const float* __restrict__ logits, int V, int32_t* __restrict__ argmax_o
         sampled_out[row] = pick;
     }
 }
+
+// log softmax(logits / temperature)[id] for one given id per row: the log of
+// the probability k_sample draws that id with, its max and its fp64 sum
+// formed the same way (each thread a contiguous index range, the partial sums
+// added in thread order).  This is the per-token term of the policy's
+// log-likelihood that a replay reads before consuming the token
+// (jiphyeonjeon review §6.2, eq. 5.3 and 5.5).  An id outside [0, V) gives
+// NaN and the bounds code in *err.
+__global__ void __launch_bounds__(NT)
+k_logprob(const float* __restrict__ logits, int V, const int32_t* __restrict__ ids,
+          int ids_stride, float* __restrict__ out, int out_stride, float temperature,
+          int* __restrict__ err) {
+    pdl_enter();
+    __shared__ float s_max[NT];
+    __shared__ double s_sum[NT];
+    const int row = blockIdx.x, tid = threadIdx.x;
+    const float* lg = logits + (size_t)row * V;
+    const int chunk = (V + NT - 1) / NT;
+    const int lo = min(V, tid * chunk), hi = min(V, lo + chunk);
+
+    float bv = -INFINITY;
+    for (int i = lo; i < hi; ++i) bv = fmaxf(bv, lg[i]);
+    s_max[tid] = bv;
+    __syncthreads();
+    for (int off = NT / 2; off > 0; off >>= 1) {
+        if (tid < off) s_max[tid] = fmaxf(s_max[tid], s_max[tid + off]);
+        __syncthreads();
+    }
+    const float mx = s_max[0];
+    const float inv_t = 1.0f / temperature;
+    double local = 0.0;
+    for (int i = lo; i < hi; ++i) local += (double)expf((lg[i] - mx) * inv_t);
+    s_sum[tid] = local;
+    __syncthreads();
+    if (tid == 0) {
+        double total = 0.0;
+        for (int k = 0; k < NT; ++k) total += s_sum[k];
+        const int id = ids[(size_t)row * ids_stride];
+        float lp = NAN;
+        if (id >= 0 && id < V)
+            lp = (float)((double)((lg[id] - mx) * inv_t) - log(total));
+        else if (err)
+            atomicExch(err, kDevBounds);
+        out[(size_t)row * out_stride] = lp;
+    }
+}
 }  // namespace
+
+void launch_logprob(const float* logits, int V, int B, const int32_t* ids, int ids_stride,
+                    float* out, int out_stride, float temperature, int* err, cudaStream_t st) {
+    if (B <= 0) return;
+    launch(k_logprob, B, NT, 0, st, logits, V, ids, ids_stride, out, out_stride, temperature,
+           err);
+    rlt_count_launch();
+}
 
 void launch_sample(const float* logits, int V, int B, int32_t* argmax, int32_t* sampled,
                    uint64_t seed, uint64_t step, float temperature, cudaStream_t st) {

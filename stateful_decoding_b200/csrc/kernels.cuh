@@ -125,6 +125,9 @@ void launch_attn_cross(const float* Q, const T* mem, size_t row_stride, int T_ca
 // readout sampler: one block per row over logits fp32 [B][V]
 void launch_sample(const float* logits, int V, int B, int32_t* argmax, int32_t* sampled,
                    uint64_t seed, uint64_t step, float temperature, cudaStream_t st);
+// log softmax(logits/temperature) at ids[b * ids_stride] -> out[b * out_stride]
+void launch_logprob(const float* logits, int V, int B, const int32_t* ids, int ids_stride,
+                    float* out, int out_stride, float temperature, int* err, cudaStream_t st);
 
 int read_and_clear_device_error();  // device error word of the bounded-wait kernels
 int read_and_clear_attn_error();

@@ -512,6 +512,8 @@ struct rlt_state {
     float* logits = nullptr;
     int32_t* ids = nullptr;
     int32_t* rows = nullptr;
+    float* replay_lp = nullptr;     // rlt_replay_logprobs: [B][T_cap], allocated on first use
+    int32_t* replay_tok = nullptr;
     float* P = nullptr;             // split-K partial slabs of the transition's projections
     size_t p_cols = 0;              // columns of one slab row (the widest projection)
     int p_slabs = 1;                // slabs allocated
@@ -1259,20 +1261,11 @@ extern "C" int rlt_prefill(rlt_state* s, int T, void* stream) {
 // ============================================================================
 // readout
 // ============================================================================
-extern "C" int rlt_readout(rlt_state* s, float* logits, int32_t* argmax, int32_t* sampled,
-                           uint64_t seed, uint64_t step, float temperature, void* stream) {
-    if (!s || !(temperature > 0.f)) return RLT_E_ARG;
-    rlt_model* m = s->m;
-    if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
+// logits fp32 [B][V] = W_out RMSNorm_out(s_t) of every row, into lbuf
+static void readout_logits(rlt_state* s, float* lbuf, cudaStream_t st) {
+    const rlt_model* m = s->m;
     const rlt_config& c = m->cfg;
-    cudaStream_t st = (cudaStream_t)stream;
     const int B = s->B, d = c.d, V = c.vocab;
-    const bool ld = logits && is_device_ptr(logits);
-    const bool ad = argmax && is_device_ptr(argmax);
-    const bool sd = sampled && is_device_ptr(sampled);
-    float* lbuf = ld ? logits : s->logits;
-    int32_t* abuf = argmax ? (ad ? argmax : s->ids) : nullptr;
-    int32_t* sbuf = sampled ? (sd ? sampled : s->ids + B) : nullptr;
     if (c.dtype == RLT_DTYPE_BF16) {
         rlt::launch_rmsnorm<bf16>(s->s, d, m->out_norm, (bf16*)s->Y, d, B, d, (float)c.eps, st);
         rlt::launch_gemm<bf16>((const bf16*)s->Y, d, (const bf16*)m->wout, d, lbuf, V, nullptr,
@@ -1282,6 +1275,23 @@ extern "C" int rlt_readout(rlt_state* s, float* logits, int32_t* argmax, int32_t
         rlt::launch_gemm<float>((const float*)s->Y, d, (const float*)m->wout, d, lbuf, V,
                                 nullptr, 0, B, V, d, rlt::kStoreF32, st);
     }
+}
+
+extern "C" int rlt_readout(rlt_state* s, float* logits, int32_t* argmax, int32_t* sampled,
+                           uint64_t seed, uint64_t step, float temperature, void* stream) {
+    if (!s || !(temperature > 0.f)) return RLT_E_ARG;
+    rlt_model* m = s->m;
+    if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
+    const rlt_config& c = m->cfg;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int B = s->B, V = c.vocab;
+    const bool ld = logits && is_device_ptr(logits);
+    const bool ad = argmax && is_device_ptr(argmax);
+    const bool sd = sampled && is_device_ptr(sampled);
+    float* lbuf = ld ? logits : s->logits;
+    int32_t* abuf = argmax ? (ad ? argmax : s->ids) : nullptr;
+    int32_t* sbuf = sampled ? (sd ? sampled : s->ids + B) : nullptr;
+    readout_logits(s, lbuf, st);
     rlt::launch_sample(lbuf, V, B, abuf, sbuf, seed, step, temperature, st);
     int rc = launch_status();
     if (rc) return rc;
@@ -1294,6 +1304,58 @@ extern "C" int rlt_readout(rlt_state* s, float* logits, int32_t* argmax, int32_t
     if (sampled && !sd &&
         cudaMemcpyAsync(sampled, sbuf, (size_t)B * 4, cudaMemcpyDeviceToHost, st))
         return RLT_E_DEVICE;
+    return RLT_OK;
+}
+
+// ============================================================================
+// replay: log-probabilities of given tokens, each read before it is consumed
+// ============================================================================
+// The trainer's side of the replay contract: from the rows' current states
+// (H_0 after a reset), append the tokens to the encoder in one parallel pass
+// (causal, so later tokens do not change earlier features), then per position
+// read log p(token | everything before it) from the current s and consume the
+// token with one transition (jiphyeonjeon review §6.2, eq. 5.3-5.5;
+// greeksharifa App. D.3, F.4).
+extern "C" int rlt_replay_logprobs(rlt_state* s, const int32_t* tokens, int n, float* logprobs,
+                                   float temperature, void* stream) {
+    if (!s || !tokens || !logprobs || n < 0 || !(temperature > 0.f)) return RLT_E_ARG;
+    if (n == 0) return RLT_OK;
+    for (int b = 0; b < s->B; ++b)
+        if (s->h_pos_dec[b] != s->h_pos_enc[b]) return RLT_E_ORDER;
+    if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    const cudaStream_t st = (cudaStream_t)stream;
+    const int B = s->B, V = s->m->cfg.vocab;
+    if (!s->replay_lp) {
+        int rc = salloc(s, (void**)&s->replay_lp, (size_t)B * s->T_cap * 4);
+        if (rc == RLT_OK) rc = salloc(s, (void**)&s->replay_tok, (size_t)B * s->T_cap * 4);
+        if (rc != RLT_OK) return rc;
+    }
+    const bool tdev = is_device_ptr(tokens), odev = is_device_ptr(logprobs);
+    // capacity and (host) token range are checked here, before anything runs
+    int rc = rlt_encode(s, tokens, n, stream);
+    if (rc) return rc;
+    const int32_t* ids = tokens;
+    if (!tdev) {
+        if (cudaMemcpyAsync(s->replay_tok, tokens, (size_t)B * n * 4, cudaMemcpyHostToDevice,
+                            st) != cudaSuccess)
+            return RLT_E_DEVICE;
+        ids = s->replay_tok;
+    }
+    float* out = odev ? logprobs : s->replay_lp;
+    for (int j = 0; j < n; ++j) {
+        readout_logits(s, s->logits, st);
+        rlt::launch_logprob(s->logits, V, B, ids + j, n, out + j, n, temperature, s->err, st);
+        rc = launch_status();
+        if (rc) return rc;
+        rc = s->m->fused ? run_fused(s, 1, st) : run_block(s, 1, st);
+        if (rc) return rc;
+    }
+    if (!odev) {
+        if (cudaMemcpyAsync(logprobs, out, (size_t)B * n * 4, cudaMemcpyDeviceToHost, st) !=
+                cudaSuccess ||
+            cudaStreamSynchronize(st) != cudaSuccess)
+            return RLT_E_DEVICE;
+    }
     return RLT_OK;
 }
 

@@ -16,7 +16,8 @@ import pytest
 
 import rlt_inputs as ri
 from oracle import RLTOracle, argmax_lowest, attend, rmsnorm, rope, round_bf16
-from oracle.rlt_oracle import sample_inverse_cdf, softmax
+from oracle.rlt_oracle import (log_softmax_at, replay_logprobs, run_sequence, sample_inverse_cdf,
+                               softmax)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -615,3 +616,71 @@ def test_bf16_mode_rounds_stored_keys_and_stays_close():
     for arr in st.mem_k + st.enc_k:
         np.testing.assert_array_equal(round_bf16(arr), arr)
     assert 0 < np.max(np.abs(a - b)) < 0.1
+
+
+# ----------------------------------------------------------------------------
+# replay log-probabilities (jiphyeonjeon review §6.2, eq. 5.3-5.5)
+# ----------------------------------------------------------------------------
+
+
+def test_log_softmax_at_closed_forms_and_scipy():
+    from scipy.special import log_softmax
+    # equal logits: every token has probability 1/V
+    for V in (1, 2, 7, 32000):
+        assert abs(log_softmax_at(np.full(V, 3.25), V // 2) + math.log(V)) < 1e-12
+    # two logits: the logistic, log p_0 = -log(1 + exp((l_1 - l_0) / T))
+    for l0, l1, T in ((0.3, -1.2, 1.0), (2.0, 5.0, 0.7), (-4.0, 4.0, 3.0)):
+        want = -math.log1p(math.exp((l1 - l0) / T))
+        assert abs(log_softmax_at(np.array([l0, l1]), 0, T) - want) < 1e-12
+    # any logits and temperature against scipy's log_softmax
+    rng = np.random.default_rng(11)
+    for T in (1.0, 0.6, 2.5):
+        lg = rng.normal(0, 4, 513)
+        ref = log_softmax(lg / T)
+        got = np.array([log_softmax_at(lg, i, T) for i in range(len(lg))])
+        np.testing.assert_allclose(got, ref, atol=1e-12, rtol=0)
+        # a distribution: the probabilities sum to one, the argmax is the largest
+        assert abs(np.exp(got).sum() - 1.0) < 1e-12
+        assert int(np.argmax(got)) == argmax_lowest(lg)
+
+
+@pytest.mark.parametrize("variant,chunk", [(1, 1), (2, 2), (0, 1)])
+def test_replay_probabilities_of_all_continuations_sum_to_one(variant, chunk):
+    """Eq. 5.3: pi(y | c) = prod_i p(y_i | c, y_<i).  Summed over every
+    continuation y of a fixed length the product is 1 only if each factor is
+    read from the state that has consumed exactly c and y_<i (reading it
+    after consuming y_i, or from a stale state, breaks the sum).  Brute force
+    over all V^3 continuations of a small model."""
+    cfg = small_cfg(vocab=5, variant=variant, chunk=chunk)
+    m = RLTOracle(cfg, weights(cfg))
+    prompt = toks(cfg, 4)
+    st = m.new_state()
+    replay_logprobs(m, st, prompt)
+    total = 0.0
+    for a in range(cfg.vocab):
+        for b in range(cfg.vocab):
+            for c in range(cfg.vocab):
+                total += math.exp(replay_logprobs(m, st.copy(), [a, b, c]).sum())
+    assert abs(total - 1.0) < 1e-12
+
+
+def test_replay_equals_readouts_of_the_prefilled_sequence():
+    """Replay token by token = one parallel encode and a prefill, read out
+    after every position (the logits after position t give token t+1), and it
+    ends in the same state (Prop. 3.1 applied to the replay schedule)."""
+    cfg = small_cfg(variant=2, chunk=3)
+    m = RLTOracle(cfg, weights(cfg))
+    x = toks(cfg, 10)
+    for T in (1.0, 0.8):
+        st = m.new_state()
+        got = replay_logprobs(m, st, x, T)
+        ref_st = m.new_state()
+        first = m.readout(ref_st)
+        seq = [first] + run_sequence(m, list(x))[:-1]
+        want = [log_softmax_at(seq[j], int(x[j]), T) for j in range(len(x))]
+        np.testing.assert_allclose(got, want, atol=1e-12, rtol=0)
+        full = m.new_state()
+        m.encode(full, x)
+        m.prefill(full, len(x))
+        np.testing.assert_allclose(st.s, full.s, atol=1e-12, rtol=0)
+        np.testing.assert_allclose(st.R, full.R, atol=1e-12, rtol=0)
