@@ -147,10 +147,14 @@ def run_reference(args, cfg):
         v, desc, threads = oracle_sample(cfg, budget_s=max(5.0, 60.0 / max(1, args.steps)))
         vals.append(v)
     value = statistics.median(vals)
+    # the line of the run it is compared with (same N, workload and global
+    # batch); the work itself ran on rank 0's host cores, as cpu_baseline says
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-            "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_desc(cfg),
+            "data": "synthetic",
+            "config": dict(workload_desc(cfg), global_batch=cfg.batch * args.gpus),
+            "hardware": "host CPU cores of rank 0 (the float64 oracle; no GPU work)",
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
