@@ -1,0 +1,96 @@
+"""Planted mistakes in the CPU oracle, to show that its pins catch them.
+
+Test infrastructure only.  Loaded as a pytest plugin (``-p tests.oracle_mutants``)
+with the environment variable RLT_ORACLE_MUTANT=<name>, it builds a copy of
+``oracle/rlt_oracle.py`` with that one expression replaced -- in memory; no
+file is written -- and installs it as ``oracle`` and ``oracle.rlt_oracle``
+before the pins are collected.  Each mistake is one a careful reader could
+make from the pages: an off-by-one in the window or the memory prefix, a sign
+or frequency error in RoPE, a swapped or dropped term, a wrong norm, scale or
+rounding, and in the replay a token read after it is consumed.
+"""
+import os
+import sys
+import types
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ORACLE_SRC = os.path.join(ROOT, "oracle", "rlt_oracle.py")
+
+# name -> (expression in the oracle, the mistaken expression)
+MUTANTS = {
+    # window of W positions including the current one, and what the ring keeps
+    "window_off_by_one": ("lo = t - c.window + 1", "lo = t - c.window"),
+    "ring_keeps_one_more": ("keep_from = int(pos[-1]) - c.window + 2",
+                            "keep_from = int(pos[-1]) - c.window + 1"),
+    # rotate-half RoPE: sign of the second half, frequency exponent
+    "rope_sign": ("x2 * c + x1 * s", "x2 * c - x1 * s"),
+    "rope_frequency": ("inv = base ** (-2.0 * np.arange(half, dtype=np.float64) / dh)",
+                       "inv = base ** (-1.0 * np.arange(half, dtype=np.float64) / dh)"),
+    # cross-attention reads the memory prefix 1..t, not t+1
+    "memory_prefix_leak": ("st.mem_k[g][:int(pos[i])], st.mem_v[g][:int(pos[i])]",
+                           "st.mem_k[g][:int(pos[i]) + 1], st.mem_v[g][:int(pos[i]) + 1]"),
+    # the merge gate: inverted, alpha dropped, operands of W_g swapped
+    "merge_gate_inverted": ('return e + c.alpha * g * self._lin(r, "merge.ws")',
+                            'return e + c.alpha * (1 - g) * self._lin(r, "merge.ws")'),
+    "merge_alpha_dropped": ('return e + c.alpha * g * self._lin(r, "merge.ws")',
+                            'return e + g * self._lin(r, "merge.ws")'),
+    "merge_operands_swapped": ("np.concatenate([e, r], axis=1)", "np.concatenate([r, e], axis=1)"),
+    # RLT-2 register replaced one position early
+    "register_timing": ("if c.variant == 2 and t % c.chunk == 0:",
+                        "if c.variant == 2 and (t - 1) % c.chunk == 0:"),
+    # block structure: residual, the norm in front of the cross-attention
+    "ffn_residual_scaled": ('return z + self._ffn(y, p + "w1", p + "w3", p + "w2")',
+                            'return self._ffn(y, p + "w1", p + "w3", p + "w2") + z * 0.999'),
+    "cross_uses_window_norm": ('y = rmsnorm(z, W[p + "x_norm"], c.eps)',
+                               'y = rmsnorm(z, W[p + "swa_norm"], c.eps)'),
+    # the causal encoder sees one position ahead
+    "encoder_causality_leak": ("st.enc_k[l][:p0 + i + 1], st.enc_v[l][:p0 + i + 1]",
+                               "st.enc_k[l][:p0 + i + 2], st.enc_v[l][:p0 + i + 2]"),
+    # attention scale 1/d_h instead of 1/sqrt(d_h); SiLU sign
+    "attention_scale": ("scale = 1.0 / np.sqrt(q.shape[-1])", "scale = 1.0 / q.shape[-1]"),
+    "silu_sign": ("return x / (1.0 + np.exp(-x))", "return x / (1.0 + np.exp(x))"),
+    # bf16 rounding by truncation instead of nearest-even
+    "bf16_truncates": ("b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16", "b = b >> 16"),
+    # replay: temperature dropped, normaliser dropped, token read after it is consumed
+    "logprob_temperature_dropped": (
+        "    z = np.asarray(logits, dtype=np.float64) / temperature\n    m = z.max()",
+        "    z = np.asarray(logits, dtype=np.float64)\n    m = z.max()"),
+    "logprob_unnormalised": ("return float((z[index] - m) - np.log(np.sum(np.exp(z - m))))",
+                             "return float(z[index] - m)"),
+    "replay_reads_after_consuming": (
+        "        out[j] = log_softmax_at(model.readout(st), int(tok), temperature)\n"
+        "        model.encode(st, [int(tok)])\n"
+        "        model.transition(st)\n",
+        "        model.encode(st, [int(tok)])\n"
+        "        model.transition(st)\n"
+        "        out[j] = log_softmax_at(model.readout(st), int(tok), temperature)\n"),
+}
+
+
+def mutant_module(name: str) -> types.ModuleType:
+    """A copy of the oracle module with mutant `name` planted."""
+    old, new = MUTANTS[name]
+    src = open(ORACLE_SRC).read()
+    if src.count(old) != 1:
+        raise RuntimeError(f"mutant {name}: the expression is not in the oracle exactly once")
+    mod = types.ModuleType("oracle.rlt_oracle")
+    mod.__file__ = ORACLE_SRC
+    sys.modules["oracle.rlt_oracle"] = mod        # dataclasses look their module up
+    exec(compile(src.replace(old, new), f"{ORACLE_SRC} [{name}]", "exec"), mod.__dict__)
+    return mod
+
+
+def pytest_configure(config):
+    name = os.environ.get("RLT_ORACLE_MUTANT")
+    if not name:
+        return
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    mod = mutant_module(name)
+    pkg = types.ModuleType("oracle")
+    pkg.__path__ = []
+    for k, v in vars(mod).items():
+        if not k.startswith("__"):
+            setattr(pkg, k, v)
+    pkg.rlt_oracle = mod
+    sys.modules["oracle"] = pkg

@@ -469,6 +469,38 @@ def test_merge_saturated_gate_recursion():
             s = s_want
 
 
+def test_merge_gate_reads_e_then_r():
+    """g = sigmoid(W_g [e_t; r] + b_g), u = e_t + alpha g (W_s r) (greeksharifa
+    §2.5): the first d columns of W_g take e_t, the last d take r.  With the
+    r-half zero the gate depends on e_t alone, so (u - e) : (W_s r) is one
+    vector for every previous state; with the e-half zero, u - e does not
+    change with e_t.  A swapped [r; e] fails both."""
+    cfg = small_cfg(alpha=0.3)
+    d = cfg.d
+    W = weights(cfg)
+    rng = np.random.default_rng(5)
+    e1, e2 = rng.normal(size=(2, d))
+    f1, f2 = rng.normal(size=(2, d))
+
+    def with_half_zero(cols):
+        Wz = dict(W)
+        Wz["merge.wg"] = W["merge.wg"].copy()
+        Wz["merge.wg"][:, cols] = 0
+        return RLTOracle(cfg, Wz)
+
+    ws = W["merge.ws"].astype(np.float64)
+    wsr = lambda fb: ws @ rmsnorm(fb, W["merge.norm"].astype(np.float64), cfg.eps)  # noqa: E731
+    m = with_half_zero(slice(d, 2 * d))             # gate from e_t only
+    du1, du2 = m.merge(e1, f1)[0] - e1, m.merge(e1, f2)[0] - e1
+    # du_k = alpha g(e1) * (W_s r_k): cross-multiplied, g(e1) cancels
+    np.testing.assert_allclose(du1 * wsr(f2), du2 * wsr(f1), atol=1e-12, rtol=0)
+    assert np.max(np.abs(m.merge(e2, f1)[0] - e2 - du1)) > 1e-3      # the gate does read e_t
+    m = with_half_zero(slice(0, d))                 # gate from r only
+    np.testing.assert_allclose(m.merge(e1, f1)[0] - e1, m.merge(e2, f1)[0] - e2, atol=1e-12,
+                               rtol=0)
+    assert np.max(np.abs(m.merge(e1, f1)[0] - m.merge(e1, f2)[0])) > 1e-3
+
+
 def test_rlt2_register_timing_closed_form():
     """RLT-2 with L_D = 0 and an open gate: s_t = e_t + alpha W_s RMSNorm(R) where
     R = s at the last complete chunk end before t (s_star before the first)."""
