@@ -51,6 +51,33 @@ MUTANTS = {
     "silu_sign": ("return x / (1.0 + np.exp(-x))", "return x / (1.0 + np.exp(x))"),
     # bf16 rounding by truncation instead of nearest-even
     "bf16_truncates": ("b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16", "b = b >> 16"),
+    # SwiGLU gate and up projections swapped; norms dropped; projections mixed
+    "swiglu_gate_up_swapped": ("silu(self._lin(x, w1)) * self._lin(x, w3)",
+                               "silu(self._lin(x, w3)) * self._lin(x, w1)"),
+    "memory_norm_dropped": ('nu = rmsnorm(x, W["mem_norm"], c.eps)', "nu = x"),
+    "memory_v_from_wk": ('mv = self._store(self._heads(self._lin(nu, f"mem.{g}.wv")))',
+                         'mv = self._store(self._heads(self._lin(nu, f"mem.{g}.wk")))'),
+    "readout_norm_dropped": ('y = rmsnorm(np.atleast_2d(s), self.W["out_norm"], c.eps)',
+                             "y = np.atleast_2d(s)"),
+    "rmsnorm_gain_dropped": ("x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * gain",
+                             "x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)"),
+    "encoder_ffn_uses_attn_norm": ('y = rmsnorm(x, W[f"enc.{l}.ffn_norm"], c.eps)',
+                                   'y = rmsnorm(x, W[f"enc.{l}.attn_norm"], c.eps)'),
+    "decoder_ffn_uses_window_norm": ('y = rmsnorm(z, W[p + "ffn_norm"], c.eps)',
+                                     'y = rmsnorm(z, W[p + "swa_norm"], c.eps)'),
+    "cross_output_uses_wo": ('z = z + self._lin(ax.reshape(n, c.d), p + "xo")',
+                             'z = z + self._lin(ax.reshape(n, c.d), p + "wo")'),
+    # decoder keys from the un-normalised input; cross query without RoPE
+    "window_keys_unnormalised": (
+        'k = self._store(rope(self._heads(self._lin(y, p + "wk")), pos, c.rope_base))',
+        'k = self._store(rope(self._heads(self._lin(z, p + "wk")), pos, c.rope_base))'),
+    "cross_query_unrotated": ('qx = rope(self._heads(self._lin(y, p + "xq")), pos, c.rope_base)',
+                              'qx = self._heads(self._lin(y, p + "xq"))'),
+    # per-layer memory groups collapsed to group 0; embedding scaled by sqrt(d)
+    "memory_group_ignored": ("g = l if c.groups > 1 else 0", "g = 0"),
+    "embedding_scaled": ('x = W["embed"][tok].copy()', 'x = W["embed"][tok] * np.sqrt(c.d)'),
+    # the window leaves out the current position's own key
+    "window_drops_current_key": ("+ [k[m] for m in range(i + 1)", "+ [k[m] for m in range(i)"),
     # replay: temperature dropped, normaliser dropped, token read after it is consumed
     "logprob_temperature_dropped": (
         "    z = np.asarray(logits, dtype=np.float64) / temperature\n    m = z.max()",
