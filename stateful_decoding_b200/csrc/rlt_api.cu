@@ -147,6 +147,11 @@ int parse_blob(const void* blob, size_t nbytes, ParsedBlob* out) {
     const uint8_t* pay = b + kHeader;
     if (blob_checksum(pay, nb) != ck) return RLT_E_BLOB;
     if (c.dtype != RLT_DTYPE_F32 && c.dtype != RLT_DTYPE_BF16) return RLT_E_BLOB;
+    // sizes far above any model this library runs, so that a malformed header
+    // can neither overflow the manifest's int sizes nor make it huge
+    if (c.vocab > (1 << 24) || c.d > (1 << 16) || c.ffn > (1 << 20) || c.n_enc > 4096 ||
+        c.n_dec > 4096 || c.window > (1 << 24) || c.chunk > (1 << 24))
+        return RLT_E_BLOB;
     if (c.vocab <= 0 || c.d <= 0 || c.heads <= 0 || c.d % c.heads || c.n_enc < 0 ||
         c.n_dec < 0 || c.ffn <= 0 || c.window < 1 || c.chunk < 1 || c.variant < 0 ||
         c.variant > 2 || (c.variant != 2 && c.chunk != 1) ||

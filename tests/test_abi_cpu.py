@@ -177,3 +177,90 @@ def test_snapshot_info_rejects_malformed(lib):
     # heads not dividing d
     bad = bytearray(good); bad[32:36] = (7).to_bytes(4, "little")
     assert info(bad) == lib.RLT_E_SNAPSHOT
+
+
+# ---------------------------------------------------------------- blob parser
+def _no_gpu():
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present: a valid blob would create a model")
+
+
+def test_every_config_blob_parses(lib):
+    """Each workload's blob (the large one at full width and vocabulary on a
+    2+2-layer slice; zero weights, which the parser does not look at) gets
+    past the parser: without a device the call ends at RLT_E_DEVICE."""
+    _no_gpu()
+    for name, cfg in ri.CONFIGS.items():
+        if name == "large_bf16":
+            cfg = cfg.replace(n_enc=2, n_dec=2)
+        W = {n: np.zeros(shape, np.float32) for n, shape in ri.manifest(cfg)}
+        assert lib.rlt_create(ri.write_blob(cfg, W))[0] == lib.RLT_E_DEVICE, name
+
+
+def _fix_checksum(blob: bytearray) -> bytearray:
+    import struct
+    struct.pack_into("<Q", blob, 104, ri.blob_checksum(bytes(blob[256:])))
+    return blob
+
+
+_TINY_BLOB = None
+
+
+def _tiny_blob() -> bytes:
+    global _TINY_BLOB
+    if _TINY_BLOB is None:
+        _TINY_BLOB = _blob()[1]
+    return _TINY_BLOB
+
+
+def test_malformed_headers_fail_cleanly(lib):
+    """Random header fields (with a matching payload checksum, so every check
+    of the config and the manifest is reached) are rejected with an error
+    code: no crash, no overflow, no huge manifest."""
+    import struct
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+    _no_gpu()
+    edge = st.sampled_from([-(2 ** 31), -1, 0, 1, 2, 3, 4, 8, 64, 4096, 4097, 1 << 16,
+                            (1 << 16) + 1, 1 << 20, (1 << 20) + 1, 1 << 24, (1 << 24) + 1,
+                            2 ** 31 - 1])
+    i32 = st.one_of(st.integers(-(2 ** 31), 2 ** 31 - 1), edge)
+
+    @settings(max_examples=400, deadline=None, derandomize=True,
+              suppress_health_check=list(HealthCheck))
+    @given(fields=st.lists(i32, min_size=12, max_size=12),
+           keep=st.lists(st.booleans(), min_size=12, max_size=12),
+           nt=st.one_of(st.just(None), st.integers(0, 2 ** 64 - 1)))
+    def run(fields, keep, nt):
+        blob = bytearray(_tiny_blob())
+        orig = struct.unpack_from("<12i", blob, 8)
+        struct.pack_into("<12i", blob, 8, *[o if k else f for o, k, f in zip(orig, keep, fields)])
+        if nt is not None:
+            struct.pack_into("<Q", blob, 88, nt)
+        code = lib.rlt_create(bytes(blob))[0]
+        assert code in (lib.RLT_E_BLOB, lib.RLT_E_UNSUPPORTED, lib.RLT_E_DEVICE), code
+
+    run()
+
+
+def test_malformed_records_fail_cleanly(lib):
+    """Random bytes written over the tensor records (checksum fixed up) are
+    rejected, or -- where they only hit weight values -- still parse."""
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+    _no_gpu()
+    base = _tiny_blob()
+
+    @settings(max_examples=300, deadline=None, derandomize=True,
+              suppress_health_check=list(HealthCheck))
+    @given(at=st.integers(256, min(len(base) - 1, 256 + 8192)),
+           data=st.binary(min_size=1, max_size=16))
+    def run(at, data):
+        blob = bytearray(base)
+        blob[at:at + len(data)] = data
+        blob = _fix_checksum(blob[:len(base)] if len(blob) > len(base) else blob)
+        code = lib.rlt_create(bytes(blob))[0]
+        assert code in (lib.RLT_E_BLOB, lib.RLT_E_DEVICE), code
+
+    run()
