@@ -645,6 +645,16 @@ extern "C" int rlt_state_create(rlt_model* m, int batch, int max_len, rlt_state*
     *out = nullptr;
     if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
     const rlt_config& c = m->cfg;
+    {   // every allocation below (caches, rings, scratch, split-K slabs,
+        // logits) is at most this product of the caller's sizes: refuse the
+        // sizes whose byte counts could wrap around
+        using u128 = unsigned __int128;
+        const u128 bound = (u128)batch *
+                           (u128)((size_t)max_len + (size_t)c.window + (size_t)c.chunk + 16) *
+                           (u128)(3 * (size_t)c.d + 2 * (size_t)m->fpad + (size_t)c.vocab) * 4 *
+                           (u128)(2 * ((size_t)c.n_enc + c.n_dec + c.groups) + 8);
+        if (bound > ((u128)1 << 60)) return RLT_E_OOM;
+    }
     rlt_state* s = new rlt_state();
     s->m = m;
     s->B = batch;
