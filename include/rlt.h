@@ -82,8 +82,9 @@ int rlt_model_config(const rlt_model* model, rlt_config* out);
  * eq. 3.3 (jiphyeonjeon review §4.2) -- plus scratch for one call.  The
  * state starts reset (H_0).  Library-owned.  RLT_E_ARG for batch or max_len
  * <= 0; RLT_E_OOM when an allocation fails, or before allocating when
- * batch x (max_len + W + B_c + 16) x (3d + 2f + vocab) x 4 x (2(L_E + L_D + G)
- * + 8) -- a bound on every buffer's bytes -- exceeds 2^60. */
+ * batch x (max_len + W + B_c + 16) x (3d + 2f' + vocab) x 4 x (2(L_E + L_D + G)
+ * + 8), f' = f rounded up to 64 -- a bound on every buffer's bytes -- exceeds
+ * 2^60. */
 int rlt_state_create(rlt_model* model, int batch, int max_len, rlt_state** out);
 void rlt_state_destroy(rlt_state* state);
 
