@@ -108,6 +108,28 @@ def _ptr(x) -> Optional[int]:
     raise TypeError(f"cannot take the address of {type(x)}")
 
 
+def _numel(x) -> int:
+    return int(x.numel()) if hasattr(x, "numel") else int(x.size)
+
+
+def _check_buf(x, dtype: str, what: str, numel: Optional[int] = None,
+               rows: Optional[int] = None) -> None:
+    """The owners' guard on caller buffers (numpy arrays or torch tensors):
+    element type `dtype` ('int32', 'float32' or 'uint8'), and `numel`
+    elements in all or a 2-D shape with `rows` rows, when given.  The library
+    reads raw memory: an int64 token array would be read as pairs of int32."""
+    if x is None:
+        return
+    dt = getattr(x, "dtype", None)
+    name = str(dt).replace("torch.", "") if dt is not None else None
+    if name != dtype:
+        raise TypeError(f"{what}: element type {dt}, expected {dtype}")
+    if rows is not None and (len(x.shape) != 2 or int(x.shape[0]) != rows):
+        raise ValueError(f"{what}: shape {tuple(x.shape)}, expected ({rows}, n)")
+    if numel is not None and _numel(x) != numel:
+        raise ValueError(f"{what}: {_numel(x)} elements, expected {numel}")
+
+
 def _stream(s) -> Optional[int]:
     if s is None:
         return None
@@ -273,6 +295,11 @@ class Model:
         """Readout of caller-supplied state vectors (device fp32 [rows][d])
         with no allocation: the scratch is a static device array."""
         rows = int(s_rows.shape[0])
+        c = self.config
+        _check_buf(s_rows, "float32", "s_rows", rows * c.d)
+        _check_buf(logits, "float32", "logits", rows * c.vocab)
+        _check_buf(argmax, "int32", "argmax", rows)
+        _check_buf(sampled, "int32", "sampled", rows)
         code = rlt_readout_rows(self.handle, s_rows, rows, logits, argmax, sampled, seed, step,
                                 temperature, stream)
         if code == RLT_E_ARG:
@@ -323,7 +350,9 @@ class State:
         return _check(rlt_state_reset(self.handle, r, len(r), stream), "rlt_state_reset")
 
     def encode(self, tokens, stream=None):
-        n = tokens.shape[1]
+        """Append int32 [batch][n] tokens (host numpy / torch, or CUDA)."""
+        _check_buf(tokens, "int32", "tokens", rows=self.batch)
+        n = int(tokens.shape[1])
         return _check(rlt_encode(self.handle, tokens, n, stream), "rlt_encode")
 
     def step(self, stream=None):
@@ -334,6 +363,11 @@ class State:
 
     def readout(self, logits=None, argmax=None, sampled=None, seed=0, step=0, temperature=1.0,
                 stream=None):
+        """Outputs (each optional, host or CUDA): logits fp32 [batch][vocab],
+        argmax and sampled int32 [batch]."""
+        _check_buf(logits, "float32", "logits", self.batch * self.model.config.vocab)
+        _check_buf(argmax, "int32", "argmax", self.batch)
+        _check_buf(sampled, "int32", "sampled", self.batch)
         return _check(rlt_readout(self.handle, logits, argmax, sampled, seed, step, temperature,
                                   stream), "rlt_readout")
 
@@ -341,9 +375,11 @@ class State:
         """log p of each given token (int32 [batch][n]) read before it is
         consumed; returns `logprobs` (fp32 [batch][n], host numpy by default)."""
         import numpy as np
+        _check_buf(tokens, "int32", "tokens", rows=self.batch)
         n = int(tokens.shape[1])
         if logprobs is None:
             logprobs = np.empty((self.batch, n), np.float32)
+        _check_buf(logprobs, "float32", "logprobs", self.batch * n)
         _check(rlt_replay_logprobs(self.handle, tokens, n, logprobs, temperature, stream),
                "rlt_replay_logprobs")
         return logprobs
@@ -375,13 +411,15 @@ class State:
         _check(code, "rlt_state_save")
         if dst is None:
             dst = np.empty(nbytes, np.uint8)
+        _check_buf(dst, "uint8", "snapshot buffer", nbytes)
         _check(rlt_state_save(self.handle, row, dst, nbytes, stream)[0], "rlt_state_save")
         return dst
 
     def load(self, row: int, snap, stream=None):
         """Replace one row with a snapshot (host bytes / numpy, or a CUDA tensor)."""
         a = _as_bytes_array(snap)
-        nbytes = a.nbytes if hasattr(a, "nbytes") else a.numel() * a.element_size()
+        _check_buf(a, "uint8", "snapshot")
+        nbytes = _numel(a)
         return _check(rlt_state_load(self.handle, row, a, nbytes, stream), "rlt_state_load")
 
     def profile(self, on: int):

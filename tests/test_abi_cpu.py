@@ -264,3 +264,44 @@ def test_malformed_records_fail_cleanly(lib):
         assert code in (lib.RLT_E_BLOB, lib.RLT_E_DEVICE), code
 
     run()
+
+
+# ---------------------------------------------------------------- binding guards
+def test_owner_methods_reject_wrong_buffers_before_the_library(lib):
+    """The owners check element types and sizes of caller buffers before any
+    library call (the library reads raw memory): checked here on a State
+    shell whose handle would fail any real call."""
+    cfg = ri.CONFIGS["tiny_fp32"]
+    model = lib.Model.__new__(lib.Model)
+    model.handle, model.config, model.device = None, lib.rlt_config(vocab=cfg.vocab, d=cfg.d), 0
+    st = lib.State.__new__(lib.State)
+    st.model, st.batch, st.max_len, st.handle = model, 2, 8, None
+    with pytest.raises(TypeError, match="int32"):
+        st.encode(np.zeros((2, 3), np.int64))          # numpy's default integer
+    with pytest.raises(ValueError, match="shape"):
+        st.encode(np.zeros((3, 3), np.int32))          # rows != batch
+    with pytest.raises(ValueError, match="shape"):
+        st.encode(np.zeros(6, np.int32))
+    with pytest.raises(TypeError, match="float32"):
+        st.readout(logits=np.zeros((2, cfg.vocab), np.float64))
+    with pytest.raises(ValueError, match="elements"):
+        st.readout(logits=np.zeros((2, cfg.vocab - 1), np.float32))
+    with pytest.raises(TypeError, match="int32"):
+        st.readout(argmax=np.zeros(2, np.int64))
+    with pytest.raises(ValueError, match="elements"):
+        st.readout(sampled=np.zeros(3, np.int32))
+    with pytest.raises(TypeError, match="int32"):
+        st.replay_logprobs(np.zeros((2, 4), np.int64))
+    with pytest.raises(ValueError, match="elements"):
+        st.replay_logprobs(np.zeros((2, 4), np.int32), logprobs=np.zeros((2, 3), np.float32))
+    with pytest.raises(TypeError, match="uint8"):
+        st.load(0, np.zeros(200, np.float32))
+    with pytest.raises(TypeError, match="float32"):
+        model.readout_rows(np.zeros((2, cfg.d), np.float64))
+    with pytest.raises(ValueError, match="elements"):
+        model.readout_rows(np.zeros((2, cfg.d), np.float32), logits=np.zeros(5, np.float32))
+    torch = pytest.importorskip("torch")
+    with pytest.raises(TypeError, match="int32"):
+        st.encode(torch.zeros(2, 3, dtype=torch.int64))
+    lib._check_buf(torch.zeros(2, 3, dtype=torch.int32), "int32", "t", 6, rows=2)
+    lib._check_buf(np.zeros((2, 3), np.int32), "int32", "t", 6, rows=2)
