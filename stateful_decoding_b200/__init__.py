@@ -7,7 +7,9 @@ raw handles or None (legacy default stream).  All computation runs in the
 library's CUDA kernels; there is no fallback: if librlt.so is missing or does
 not load, importing this package raises.
 
-``Model`` and ``State`` are small owners that call the same functions.
+``Model`` and ``State`` are small owners that call the same functions; they
+also check the element types and sizes of the buffers they are given (the
+library reads raw memory), which the ``rlt_*`` functions leave to the caller.
 """
 from __future__ import annotations
 
