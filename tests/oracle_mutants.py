@@ -51,6 +51,17 @@ MUTANTS = {
     "silu_sign": ("return x / (1.0 + np.exp(-x))", "return x / (1.0 + np.exp(x))"),
     # bf16 rounding by truncation instead of nearest-even
     "bf16_truncates": ("b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16", "b = b >> 16"),
+    # bf16 mode: a value cache or the product inputs left unrounded
+    "bf16_encoder_values_unrounded": (
+        'v = self._store(self._heads(self._lin(y, self._enc(l, "wv"))))',
+        'v = self._heads(self._lin(y, self._enc(l, "wv")))'),
+    "bf16_memory_values_unrounded": (
+        'mv = self._store(self._heads(self._lin(nu, f"mem.{g}.wv")))',
+        'mv = self._heads(self._lin(nu, f"mem.{g}.wv"))'),
+    "bf16_ring_values_unrounded": ('v = self._store(self._heads(self._lin(y, p + "wv")))',
+                                   'v = self._heads(self._lin(y, p + "wv"))'),
+    "bf16_product_inputs_unrounded": ("return self._store(x) @ self.W[name].T",
+                                      "return x @ self.W[name].T"),
     # SwiGLU gate and up projections swapped; norms dropped; projections mixed
     "swiglu_gate_up_swapped": ("silu(self._lin(x, w1)) * self._lin(x, w3)",
                                "silu(self._lin(x, w3)) * self._lin(x, w1)"),

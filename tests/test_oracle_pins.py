@@ -650,6 +650,27 @@ def test_bf16_mode_rounds_stored_keys_and_stays_close():
     assert 0 < np.max(np.abs(a - b)) < 0.1
 
 
+def test_bf16_mode_rounds_every_cache_and_product_input():
+    """Reading c14: in bf16 mode every stored key and value (encoder cache,
+    memory, window ring) is a bf16 value, and every matrix-product input is
+    rounded -- rounding it before the call changes nothing (rounding is
+    idempotent), while the fp64 mode's product does change."""
+    cfg = small_cfg(dtype=ri.DT_BF16, window=3)
+    W = {k: ri.bf16_bits_to_f32(ri.to_bf16_bits(v)).reshape(v.shape)
+         for k, v in weights(cfg, seed=5).items()}
+    m = RLTOracle(cfg, W, "bf16")
+    _, st = logits_token_by_token(m, toks(cfg, 8))
+    ring = [a for cache in st.swa for kv in cache.values() for a in kv]
+    assert ring
+    for arr in st.enc_k + st.enc_v + st.mem_k + st.mem_v + ring:
+        np.testing.assert_array_equal(round_bf16(arr), arr)
+    y = np.random.default_rng(3).normal(size=(3, cfg.d))
+    for name in ("dec.0.wq", "dec.1.w1", "mem.0.wk", "out"):
+        np.testing.assert_array_equal(m._lin(y, name), m._lin(round_bf16(y), name))
+    f64 = RLTOracle(cfg, W, "fp64")
+    assert not np.array_equal(f64._lin(y, "out"), f64._lin(round_bf16(y), "out"))
+
+
 # ----------------------------------------------------------------------------
 # replay log-probabilities (jiphyeonjeon review §6.2, eq. 5.3-5.5)
 # ----------------------------------------------------------------------------
