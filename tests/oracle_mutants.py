@@ -22,6 +22,9 @@ MUTANTS = {
     "window_off_by_one": ("lo = t - c.window + 1", "lo = t - c.window"),
     "ring_keeps_one_more": ("keep_from = int(pos[-1]) - c.window + 2",
                             "keep_from = int(pos[-1]) - c.window + 1"),
+    "window_too_short": ("lo = t - c.window + 1", "lo = t - c.window + 2"),
+    "ring_keeps_one_fewer": ("keep_from = int(pos[-1]) - c.window + 2",
+                             "keep_from = int(pos[-1]) - c.window + 3"),
     # rotate-half RoPE: sign of the second half, frequency exponent
     "rope_sign": ("x2 * c + x1 * s", "x2 * c - x1 * s"),
     "rope_frequency": ("inv = base ** (-2.0 * np.arange(half, dtype=np.float64) / dh)",
@@ -35,6 +38,21 @@ MUTANTS = {
     "merge_alpha_dropped": ('return e + c.alpha * g * self._lin(r, "merge.ws")',
                             'return e + g * self._lin(r, "merge.ws")'),
     "merge_operands_swapped": ("np.concatenate([e, r], axis=1)", "np.concatenate([r, e], axis=1)"),
+    "merge_gate_silu": (
+        'g = sigmoid(self._lin(np.concatenate([e, r], axis=1), "merge.wg") + W["merge.bg"])',
+        'g = silu(self._lin(np.concatenate([e, r], axis=1), "merge.wg") + W["merge.bg"])'),
+    "merge_gate_bias_dropped": (
+        'g = sigmoid(self._lin(np.concatenate([e, r], axis=1), "merge.wg") + W["merge.bg"])',
+        'g = sigmoid(self._lin(np.concatenate([e, r], axis=1), "merge.wg"))'),
+    # the merge reads a normalised encoder output instead of the raw e_t
+    "merge_input_normalised": ("st.e.extend(list(x))",
+                               'st.e.extend(list(rmsnorm(x, W["mem_norm"], c.eps)))'),
+    # tied encoder layer l borrowing decoder layer l+1
+    "tied_layer_shifted": (
+        'return f"dec.{l}.{name}" if self.cfg.tied else f"enc.{l}.{name}"',
+        'return f"dec.{(l + 1) % self.cfg.n_dec}.{name}" if self.cfg.tied else f"enc.{l}.{name}"'),
+    # attention weights not normalised by their sum
+    "attention_unnormalised": ("p = p / p.sum(axis=1, keepdims=True)", "p = p / p.shape[1]"),
     # RLT-2 register replaced one position early
     "register_timing": ("if c.variant == 2 and t % c.chunk == 0:",
                         "if c.variant == 2 and (t - 1) % c.chunk == 0:"),
@@ -89,6 +107,10 @@ MUTANTS = {
     "embedding_scaled": ('x = W["embed"][tok].copy()', 'x = W["embed"][tok] * np.sqrt(c.d)'),
     # the window leaves out the current position's own key
     "window_drops_current_key": ("+ [k[m] for m in range(i + 1)", "+ [k[m] for m in range(i)"),
+    # sampling: the temperature dropped from the sampled distribution
+    "sampler_temperature_dropped": (
+        "    z = np.asarray(logits, dtype=np.float64) / temperature\n    z = z - z.max()",
+        "    z = np.asarray(logits, dtype=np.float64)\n    z = z - z.max()"),
     # replay: temperature dropped, normaliser dropped, token read after it is consumed
     "logprob_temperature_dropped": (
         "    z = np.asarray(logits, dtype=np.float64) / temperature\n    m = z.max()",

@@ -207,6 +207,13 @@ def test_sampling_inverse_cdf_brute_force():
                                atol=0.015)
     assert argmax_lowest(np.array([1.0, 3.0, 3.0, 2.0])) == 1
     np.testing.assert_allclose(softmax(np.array([0.0, math.log(3.0)]), 1.0), [0.25, 0.75])
+    # temperature 1/2 squares the probabilities: [1, 4, 9, 16] / 30
+    edges = np.cumsum([1, 4, 9, 16]) / 30.0
+    np.testing.assert_allclose(softmax(logits, 0.5), np.array([1, 4, 9, 16]) / 30.0, rtol=1e-12)
+    for u in np.linspace(0, 0.999, 101):
+        if np.min(np.abs(edges - u)) < 1e-9:
+            continue
+        assert sample_inverse_cdf(logits, u, 0.5) == int(np.searchsorted(edges, u, side="right"))
 
 
 # ----------------------------------------------------------------------------
