@@ -29,6 +29,19 @@ MUTANTS = {
     "rope_sign": ("x2 * c + x1 * s", "x2 * c - x1 * s"),
     "rope_frequency": ("inv = base ** (-2.0 * np.arange(half, dtype=np.float64) / dh)",
                        "inv = base ** (-1.0 * np.arange(half, dtype=np.float64) / dh)"),
+    "rope_pairs_interleaved": (
+        "x1, x2 = x[..., :half], x[..., half:]\n"
+        "    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)",
+        "x1, x2 = x[..., 0::2], x[..., 1::2]\n    out = np.empty_like(x)\n"
+        "    out[..., 0::2] = x1 * c - x2 * s\n    out[..., 1::2] = x2 * c + x1 * s\n"
+        "    return out"),
+    "memory_keys_rotated_one_back": (
+        'mk = self._store(rope(self._heads(self._lin(nu, f"mem.{g}.wk")), pos, c.rope_base))',
+        'mk = self._store(rope(self._heads(self._lin(nu, f"mem.{g}.wk")), pos - 1, c.rope_base))'),
+    # heads split with the wrong layout; the state normalised before it is carried
+    "heads_layout_transposed": ("return x.reshape(x.shape[0], self.h, self.dh)",
+                                "return x.reshape(x.shape[0], self.dh, self.h).transpose(0, 2, 1)"),
+    "state_normalised": ("st.s = z[0].copy()", 'st.s = rmsnorm(z[0], self.W["out_norm"], c.eps)'),
     # cross-attention reads the memory prefix 1..t, not t+1
     "memory_prefix_leak": ("st.mem_k[g][:int(pos[i])], st.mem_v[g][:int(pos[i])]",
                            "st.mem_k[g][:int(pos[i]) + 1], st.mem_v[g][:int(pos[i]) + 1]"),
