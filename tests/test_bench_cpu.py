@@ -36,3 +36,37 @@ def test_reference_arm_line(monkeypatch):
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s",
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_clock_summary_parses_nvidia_smi_rows():
+    """The clocks record of the JSON line: median SM clock under load, the
+    max clock, and every throttle reason seen active."""
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.ClockSampler(0)
+    c.out = "\n".join([
+        "0, 1965, 1965, 650.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1950, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1965, 1965, 700.3, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ])
+    s = c.summary()
+    assert s == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                 "samples": 3}
+    c.out = ""
+    assert c.summary() is None
+
+
+def test_committed_traffic_record_matches_the_kernel_source():
+    """The dominant kernel's ncu traffic is reported only while the kernel's
+    source is the one captured; it is scaled by the algorithmic bytes."""
+    import hashlib
+    sys.path.insert(0, ROOT)
+    import bench
+    rec = json.load(open(os.path.join(ROOT, "profiles", "dominant_kernel_traffic.json")))
+    src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    assert hashlib.sha256(src).hexdigest() == rec["source_sha256"]
+    t = bench.kernel_traffic(2 * rec["alg_bytes"])
+    assert t == 2 * rec["dram_bytes"]
+    assert 1.0 <= rec["dram_bytes"] / rec["alg_bytes"] < 1.2
