@@ -19,9 +19,22 @@
 #include <set>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/rlt.h"
 #include "fused.cuh"
 #include "kernels.cuh"
+
+// An NVTX range over each public call, so that a profiler's timeline shows
+// which call the kernels and copies belong to (no-op without a profiler).
+namespace {
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+}  // namespace
 
 static std::atomic<uint64_t> g_launches{0};
 void rlt_count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
@@ -903,6 +916,7 @@ static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t s
 }
 
 extern "C" int rlt_encode(rlt_state* s, const int32_t* tokens, int n, void* stream) {
+    NvtxRange nvtx("rlt_encode");
     if (!s || !tokens || n < 0) return RLT_E_ARG;
     if (n == 0) return RLT_OK;
     rlt_model* m = s->m;
@@ -1231,6 +1245,7 @@ static int run_fused(rlt_state* s, int nsteps, cudaStream_t st) {
 }
 
 extern "C" int rlt_step(rlt_state* s, void* stream) {
+    NvtxRange nvtx("rlt_step");
     if (!s) return RLT_E_ARG;
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
     if (s->m->fused) return run_fused(s, 1, (cudaStream_t)stream);
@@ -1238,6 +1253,7 @@ extern "C" int rlt_step(rlt_state* s, void* stream) {
 }
 
 extern "C" int rlt_prefill(rlt_state* s, int T, void* stream) {
+    NvtxRange nvtx("rlt_prefill");
     if (!s || T < 0) return RLT_E_ARG;
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
     const rlt_config& c = s->m->cfg;
@@ -1294,6 +1310,7 @@ static void readout_logits(rlt_state* s, float* lbuf, cudaStream_t st) {
 
 extern "C" int rlt_readout(rlt_state* s, float* logits, int32_t* argmax, int32_t* sampled,
                            uint64_t seed, uint64_t step, float temperature, void* stream) {
+    NvtxRange nvtx("rlt_readout");
     if (!s || !(temperature > 0.f)) return RLT_E_ARG;
     rlt_model* m = s->m;
     if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
@@ -1333,6 +1350,7 @@ extern "C" int rlt_readout(rlt_state* s, float* logits, int32_t* argmax, int32_t
 // greeksharifa App. D.3, F.4).
 extern "C" int rlt_replay_logprobs(rlt_state* s, const int32_t* tokens, int n, float* logprobs,
                                    float temperature, void* stream) {
+    NvtxRange nvtx("rlt_replay_logprobs");
     if (!s || !tokens || !logprobs || n < 0 || !(temperature > 0.f)) return RLT_E_ARG;
     if (n == 0) return RLT_OK;
     for (int b = 0; b < s->B; ++b)
@@ -1378,6 +1396,7 @@ extern "C" int rlt_replay_logprobs(rlt_state* s, const int32_t* tokens, int n, f
 // reset, positions, export, errors
 // ============================================================================
 extern "C" int rlt_state_reset(rlt_state* s, const int32_t* rows, int n, void* stream) {
+    NvtxRange nvtx("rlt_state_reset");
     if (!s) return RLT_E_ARG;
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
     cudaStream_t st = (cudaStream_t)stream;
@@ -1585,6 +1604,7 @@ extern "C" int rlt_snapshot_info(const void* snap, size_t nbytes, rlt_config* cf
 
 extern "C" int rlt_state_save(rlt_state* s, int row, void* dst, size_t nbytes,
                               size_t* nbytes_out, void* stream) {
+    NvtxRange nvtx("rlt_state_save");
     if (!s || row < 0 || row >= s->B) return RLT_E_ARG;
     const rlt_model* m = s->m;
     const SnapGeom g = snap_geom(m->cfg);
@@ -1614,6 +1634,7 @@ extern "C" int rlt_state_save(rlt_state* s, int row, void* dst, size_t nbytes,
 
 extern "C" int rlt_state_load(rlt_state* s, int row, const void* src, size_t nbytes,
                               void* stream) {
+    NvtxRange nvtx("rlt_state_load");
     if (!s || !src || row < 0 || row >= s->B) return RLT_E_ARG;
     const rlt_model* m = s->m;
     if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
@@ -1769,6 +1790,7 @@ void* rows_scratch(int device) {
 extern "C" int rlt_readout_rows(const rlt_model* m, const float* s_rows, int rows, float* logits,
                                 int32_t* argmax, int32_t* sampled, uint64_t seed, uint64_t step,
                                 float temperature, void* stream) {
+    NvtxRange nvtx("rlt_readout_rows");
     if (!m || !s_rows || rows < 0 || !(temperature > 0.f)) return RLT_E_ARG;
     if (m->device < 0 || m->device >= kScratchDevices) return RLT_E_DEVICE;
     if (cudaSetDevice(m->device) != cudaSuccess) return RLT_E_DEVICE;
