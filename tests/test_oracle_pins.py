@@ -86,6 +86,44 @@ def test_splitmix64_published_outputs():
     assert [int(x) for x in ri.splitmix64_stream(g["seed"], 0, 3)] == want
 
 
+def test_token_recipes_follow_the_documented_structure():
+    """The synthetic token streams that stand in for the pages' task suites
+    have the structure the workload table documents, and a row's tokens do
+    not depend on the batch it is drawn in."""
+    C = ri.CONFIGS
+    sizes = {n: (c.batch, c.prompt, c.decode) for n, c in C.items()}
+    assert sizes == {"tiny_fp32": (2, 16, 6), "parity_bf16": (256, 256, 0),
+                     "s5_bf16": (512, 256, 0), "rlt2_mod5_bf16": (1024, 64, 0),
+                     "large_bf16": (64, 4096, 512)}
+    x = ri.make_tokens(C["parity_bf16"])                   # [BOS=2, bits, SEP=3]
+    assert x.dtype == np.int32 and x.shape == (256, 256)
+    assert (x[:, 0] == 2).all() and (x[:, -1] == 3).all()
+    bits = x[:, 1:-1]
+    assert set(np.unique(bits)) == {0, 1} and abs(bits.mean() - 0.5) < 0.01
+    x = ri.make_tokens(C["s5_bf16"])                       # [BOS=11, ops 0..10]
+    assert (x[:, 0] == 11).all() and x[:, 1:].min() == 0 and x[:, 1:].max() == 10
+    counts = np.bincount(x[:, 1:].ravel(), minlength=11)
+    assert counts.min() > 0.9 * counts.mean()
+    x = ri.make_tokens(C["rlt2_mod5_bf16"])                # BOS=9, digit, op, ..., '=', digit
+    assert (x[:, 0] == 9).all() and (x[:, -2] == 8).all()
+    digits = x[:, 1:-2:2]
+    ops = x[:, 2:-2:2]
+    assert digits.min() == 0 and digits.max() == 4 and ops.min() == 5 and ops.max() == 7
+    assert x[:, -1].max() <= 4
+    big = C["large_bf16"]
+    x = ri.make_tokens(big, 8, 4096)                       # BOS=0, then Zipf(1.1) over 1..V-1
+    assert (x[:, 0] == 0).all() and x[:, 1:].min() >= 1 and x[:, 1:].max() < big.vocab
+    f = np.bincount(x[:, 1:].ravel(), minlength=big.vocab)
+    assert f[1] > f[2] > f[3] > f[10]
+    assert abs(f[1] / f[2] - 2 ** 1.1) < 0.15               # rank-frequency slope
+    x = ri.make_tokens(C["tiny_fp32"], 4, 50)
+    assert x.min() >= 0 and x.max() < 32
+    for name in C:                                          # rows independent of the batch
+        a = ri.make_tokens(C[name], 5, 12)
+        b = ri.make_tokens(C[name], 1, 12, row0=3)
+        np.testing.assert_array_equal(a[3], b[0])
+
+
 def test_box_muller_moments():
     z = ri.normal(123, 200000, 1.0)
     assert abs(z.mean()) < 0.01 and abs(z.std() - 1.0) < 0.01
