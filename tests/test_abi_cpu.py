@@ -305,3 +305,36 @@ def test_owner_methods_reject_wrong_buffers_before_the_library(lib):
         st.encode(torch.zeros(2, 3, dtype=torch.int64))
     lib._check_buf(torch.zeros(2, 3, dtype=torch.int32), "int32", "t", 6, rows=2)
     lib._check_buf(np.zeros((2, 3), np.int32), "int32", "t", 6, rows=2)
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """include/rlt.h compiles as C99 with warnings as errors, and a C program
+    links against librlt.so and calls functions that need no device."""
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "rlt.h"
+int main(void) {
+    rlt_config c;
+    int32_t pe = -1, pd = -1;
+    unsigned char junk[RLT_SNAPSHOT_HEADER_BYTES];
+    memset(junk, 0, sizeof junk);
+    if (rlt_snapshot_info(junk, sizeof junk, &c, &pe, &pd) != RLT_E_SNAPSHOT) return 1;
+    if (rlt_snapshot_info(NULL, 0, NULL, NULL, NULL) != RLT_E_ARG) return 2;
+    if (rlt_step(NULL, NULL) != RLT_E_ARG) return 3;
+    if (strcmp(rlt_strerror(RLT_OK), "ok") != 0) return 4;
+    printf("%s|%s\n", rlt_strerror(RLT_E_SNAPSHOT), rlt_strerror(RLT_E_UNSUPPORTED));
+    return 0;
+}
+''')
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(lib.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                        "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                        "-L", libdir, "-lrlt", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert r.stdout.strip() == f"{lib.rlt_strerror(-9)}|{lib.rlt_strerror(-8)}"
