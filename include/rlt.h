@@ -28,6 +28,12 @@
  *   on other rows' tokens, bit for bit (greeksharifa App. C.1, batching
  *   independent sequences).
  * - Positions are 1-based; BOS is position 1 (greeksharifa App. I).
+ * - Threads: one model or state must not be used by two host threads at
+ *   once; different states may run on different threads and streams.  A
+ *   bounded wait that gives up inside the GEMMs or the bulk-copy attention
+ *   kernels records it in a device-wide word (other kernels use the state's
+ *   own), which the first rlt_state_check on that device to run afterwards
+ *   reports and clears.
  */
 #ifndef RLT_H
 #define RLT_H
