@@ -162,6 +162,28 @@ int rlt_readout(rlt_state* state, float* logits, int32_t* argmax, int32_t* sampl
 int rlt_replay_logprobs(rlt_state* state, const int32_t* tokens, int n, float* logprobs,
                         float temperature, void* stream);
 
+/* Packed documents: several independent documents one after another in each
+ * row.  tokens: int32 [batch][n], host or device; doc_start: uint8
+ * [batch][n], HOST memory, nonzero where a document starts.  Before token j
+ * of row b with doc_start[b][j] != 0 the row restarts from H_0 (as
+ * rlt_state_reset: s = R = s_star, positions 0, so token j is position 1 of
+ * its document): the recurrent output, window rings, encoder cache and
+ * positions are per document, and no attention crosses a document start
+ * (jiphyeonjeon review §6.1; greeksharifa App. F).  Every token is encoded
+ * and consumed (one transition each); a row without a start at column 0
+ * continues its current document.  Row b then holds the state of its last
+ * document, exactly as if that document alone had been encoded and
+ * prefilled in a fresh row.  The columns are cut where any row starts a
+ * document, and each piece is one rlt_encode + rlt_prefill for all rows, so
+ * rows sit at different positions.  Synchronises `stream` at every cut.
+ * Errors, checked before anything runs: RLT_E_ARG (null pointers, n < 0, a
+ * host token outside [0, vocab)), RLT_E_ORDER (a row has encoded tokens not
+ * yet consumed), RLT_E_CAPACITY (a document would pass max_len); later,
+ * RLT_E_DEVICE if a CUDA call fails (the rows then hold the pieces before
+ * it). */
+int rlt_prefill_packed(rlt_state* state, const int32_t* tokens, const uint8_t* doc_start, int n,
+                       void* stream);
+
 /* Readout of caller-supplied state vectors that allocates nothing (no
  * counterpart in the method: a serving convenience for callers that hold a
  * model but no state, and may not allocate device memory).  s_rows: device

@@ -29,7 +29,9 @@ What it computes, one sequence ("row") at a time, in float64:
 * the readout: RMSNorm, linear map, softmax -- greeksharifa §2.3;
 * the replay log-probabilities log p(y_i | c, y_<i), each read from the state
   that precedes the token -- jiphyeonjeon review §6.2 (paper eq. 5.3-5.5),
-  greeksharifa App. D.3, F.4.
+  greeksharifa App. D.3, F.4;
+* packed documents, each restarting from H_0 -- jiphyeonjeon review §6.1,
+  greeksharifa App. F.
 
 Where the pages leave a step open (the block equations are missing from the
 extracted text) this follows these readings: pre-norm RMSNorm (eps 1e-6,
@@ -433,3 +435,24 @@ def replay_logprobs(model: RLTOracle, st: RowState, tokens: Sequence[int],
         model.encode(st, [int(tok)])
         model.transition(st)
     return out
+
+
+# ----------------------------------------------------------------------------
+# Packed documents
+# ----------------------------------------------------------------------------
+
+
+def prefill_packed(model: RLTOracle, tokens: Sequence[int], starts: Sequence[bool],
+                   st: Optional[RowState] = None) -> RowState:
+    """One row holding independent documents one after another: where a
+    document starts the row restarts from H_0 -- recurrent output, window
+    cache, encoder cache and positions all reset -- then every token is
+    encoded and consumed in order (jiphyeonjeon review §6.1; greeksharifa
+    App. F).  Returns the state of the last document."""
+    st = model.new_state() if st is None else st
+    for tok, start in zip(tokens, starts):
+        if start:
+            st = model.new_state()
+        model.encode(st, [int(tok)])
+        model.transition(st)
+    return st

@@ -57,6 +57,7 @@ _SIGS = {
     "rlt_readout": (_i, [_vp, _vp, _vp, _vp, _u64, _u64, ctypes.c_float, _vp]),
     "rlt_readout_rows": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _u64, _u64, ctypes.c_float, _vp]),
     "rlt_replay_logprobs": (_i, [_vp, _vp, _i, _vp, ctypes.c_float, _vp]),
+    "rlt_prefill_packed": (_i, [_vp, _vp, _vp, _i, _vp]),
     "rlt_state_positions": (_i, [_vp, _vp, _vp]),
     "rlt_state_read": (_i, [_vp, _i, _vp, _sz, ctypes.POINTER(_sz), _vp]),
     "rlt_state_check": (_i, [_vp, _vp]),
@@ -213,6 +214,10 @@ def rlt_replay_logprobs(state, tokens, n: int, logprobs, temperature: float = 1.
                         stream=None) -> int:
     return _lib.rlt_replay_logprobs(state, _ptr(tokens), n, _ptr(logprobs), temperature,
                                     _stream(stream))
+
+
+def rlt_prefill_packed(state, tokens, doc_start, n: int, stream=None) -> int:
+    return _lib.rlt_prefill_packed(state, _ptr(tokens), _ptr(doc_start), n, _stream(stream))
 
 
 def readout_rows_scratch_bytes(rows: int, d: int, vocab: int, bf16: bool,
@@ -385,6 +390,18 @@ class State:
         _check(rlt_replay_logprobs(self.handle, tokens, n, logprobs, temperature, stream),
                "rlt_replay_logprobs")
         return logprobs
+
+    def prefill_packed(self, tokens, doc_start, stream=None):
+        """Encode and consume int32 [batch][n] tokens holding packed documents;
+        doc_start (host, bool or uint8 [batch][n]) marks where each starts."""
+        import numpy as np
+        _check_buf(tokens, "int32", "tokens", rows=self.batch)
+        n = int(tokens.shape[1])
+        starts = np.ascontiguousarray(doc_start, dtype=np.uint8)
+        if starts.shape != (self.batch, n):
+            raise ValueError(f"doc_start: shape {starts.shape}, expected ({self.batch}, {n})")
+        return _check(rlt_prefill_packed(self.handle, tokens, starts, n, stream),
+                      "rlt_prefill_packed")
 
     def positions(self):
         import numpy as np

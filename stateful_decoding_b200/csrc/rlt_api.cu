@@ -1339,6 +1339,16 @@ extern "C" int rlt_readout(rlt_state* s, float* logits, int32_t* argmax, int32_t
     return RLT_OK;
 }
 
+// [B][T_cap] fp32 and int32 buffers for the calls that stage per-position
+// values or pieces of the caller's tokens, allocated on first use
+static int call_scratch(rlt_state* s) {
+    if (s->replay_lp) return RLT_OK;
+    const size_t n = (size_t)s->B * s->T_cap * 4;
+    int rc = salloc(s, (void**)&s->replay_lp, n);
+    if (rc == RLT_OK) rc = salloc(s, (void**)&s->replay_tok, n);
+    return rc;
+}
+
 // ============================================================================
 // replay: log-probabilities of given tokens, each read before it is consumed
 // ============================================================================
@@ -1358,11 +1368,7 @@ extern "C" int rlt_replay_logprobs(rlt_state* s, const int32_t* tokens, int n, f
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
     const cudaStream_t st = (cudaStream_t)stream;
     const int B = s->B, V = s->m->cfg.vocab;
-    if (!s->replay_lp) {
-        int rc = salloc(s, (void**)&s->replay_lp, (size_t)B * s->T_cap * 4);
-        if (rc == RLT_OK) rc = salloc(s, (void**)&s->replay_tok, (size_t)B * s->T_cap * 4);
-        if (rc != RLT_OK) return rc;
-    }
+    if (int rc = call_scratch(s)) return rc;
     const bool tdev = is_device_ptr(tokens), odev = is_device_ptr(logprobs);
     // capacity and (host) token range are checked here, before anything runs
     int rc = rlt_encode(s, tokens, n, stream);
@@ -1388,6 +1394,76 @@ extern "C" int rlt_replay_logprobs(rlt_state* s, const int32_t* tokens, int n, f
                 cudaSuccess ||
             cudaStreamSynchronize(st) != cudaSuccess)
             return RLT_E_DEVICE;
+    }
+    return RLT_OK;
+}
+
+// ============================================================================
+// packed documents: a row restarts from H_0 where a document starts
+// ============================================================================
+// Independent documents packed one after another in a row reset the
+// recurrent output, the window rings, the encoder cache and the positions at
+// each document start, so no state and no attention crosses the boundary
+// (jiphyeonjeon review §6.1; greeksharifa App. F).  The columns are cut
+// wherever any row starts a document; each piece is encoded and consumed by
+// every row, after the rows that start a document at the piece's first column
+// are reset.  Rows then sit at different positions, which every kernel
+// handles through its row's own counters.
+extern "C" int rlt_prefill_packed(rlt_state* s, const int32_t* tokens, const uint8_t* doc_start,
+                                  int n, void* stream) {
+    NvtxRange nvtx("rlt_prefill_packed");
+    if (!s || !tokens || !doc_start || n < 0) return RLT_E_ARG;
+    if (n == 0) return RLT_OK;
+    const int B = s->B;
+    for (int b = 0; b < B; ++b)
+        if (s->h_pos_dec[b] != s->h_pos_enc[b]) return RLT_E_ORDER;
+    if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    const bool tdev = is_device_ptr(tokens);
+    // everything that could fail part-way is checked before the first piece
+    for (int b = 0; b < B; ++b) {
+        int p = s->h_pos_enc[b];
+        for (int j = 0; j < n; ++j) {
+            p = doc_start[(size_t)b * n + j] ? 1 : p + 1;
+            if (p > s->T_cap) return RLT_E_CAPACITY;
+            if (!tdev && (tokens[(size_t)b * n + j] < 0 ||
+                          tokens[(size_t)b * n + j] >= s->m->cfg.vocab))
+                return RLT_E_ARG;
+        }
+    }
+    if (tdev)
+        if (int rc = call_scratch(s)) return rc;
+    const cudaStream_t st = (cudaStream_t)stream;
+    auto starts_at = [&](int j) {
+        for (int b = 0; b < B; ++b)
+            if (doc_start[(size_t)b * n + j]) return true;
+        return false;
+    };
+    std::vector<int32_t> piece_h, rows;
+    for (int j0 = 0; j0 < n;) {
+        int j1 = j0 + 1;
+        while (j1 < n && !starts_at(j1)) ++j1;
+        const int len = j1 - j0;
+        rows.clear();
+        for (int b = 0; b < B; ++b)
+            if (doc_start[(size_t)b * n + j0]) rows.push_back(b);
+        if (!rows.empty())
+            if (int rc = rlt_state_reset(s, rows.data(), (int)rows.size(), stream)) return rc;
+        const int32_t* piece;
+        if (tdev) {
+            if (cudaMemcpy2DAsync(s->replay_tok, (size_t)len * 4, tokens + j0, (size_t)n * 4,
+                                  (size_t)len * 4, B, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+                return RLT_E_DEVICE;
+            piece = s->replay_tok;
+        } else {
+            // rlt_encode stages a pageable host piece before it returns
+            piece_h.resize((size_t)B * len);
+            for (int b = 0; b < B; ++b)
+                memcpy(&piece_h[(size_t)b * len], tokens + (size_t)b * n + j0, (size_t)len * 4);
+            piece = piece_h.data();
+        }
+        if (int rc = rlt_encode(s, piece, len, stream)) return rc;
+        if (int rc = rlt_prefill(s, len, stream)) return rc;
+        j0 = j1;
     }
     return RLT_OK;
 }

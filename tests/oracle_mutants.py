@@ -124,6 +124,9 @@ MUTANTS = {
     "sampler_temperature_dropped": (
         "    z = np.asarray(logits, dtype=np.float64) / temperature\n    z = z - z.max()",
         "    z = np.asarray(logits, dtype=np.float64)\n    z = z - z.max()"),
+    # packed documents: the reset at a document start left out
+    "packed_reset_dropped": ("        if start:\n            st = model.new_state()\n",
+                             "        if start and st is None:\n            st = model.new_state()\n"),
     # replay: temperature dropped, normaliser dropped, token read after it is consumed
     "logprob_temperature_dropped": (
         "    z = np.asarray(logits, dtype=np.float64) / temperature\n    m = z.max()",

@@ -79,6 +79,8 @@ def test_null_arguments(lib):
     assert lib._lib.rlt_state_save(None, 0, None, 0, None, None) == lib.RLT_E_ARG
     assert lib._lib.rlt_state_load(None, 0, None, 0, None) == lib.RLT_E_ARG
     assert lib._lib.rlt_snapshot_info(None, 0, None, None, None) == lib.RLT_E_ARG
+    assert lib._lib.rlt_prefill_packed(None, None, None, 1, None) == lib.RLT_E_ARG
+    assert lib._lib.rlt_replay_logprobs(None, None, 1, None, 1.0, None) == lib.RLT_E_ARG
     assert lib.rlt_kernel_launches() >= 0
 
 

@@ -16,8 +16,8 @@ import pytest
 
 import rlt_inputs as ri
 from oracle import RLTOracle, argmax_lowest, attend, rmsnorm, rope, round_bf16
-from oracle.rlt_oracle import (log_softmax_at, replay_logprobs, run_sequence, sample_inverse_cdf,
-                               softmax)
+from oracle.rlt_oracle import (log_softmax_at, prefill_packed, replay_logprobs, run_sequence,
+                               sample_inverse_cdf, softmax)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -782,3 +782,43 @@ def test_replay_equals_readouts_of_the_prefilled_sequence():
         m.prefill(full, len(x))
         np.testing.assert_allclose(st.s, full.s, atol=1e-12, rtol=0)
         np.testing.assert_allclose(st.R, full.R, atol=1e-12, rtol=0)
+
+
+# ----------------------------------------------------------------------------
+# packed documents (jiphyeonjeon review §6.1: independent documents reset the
+# recurrent output, the decoder window cache, the encoder cache and positions)
+# ----------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("variant,chunk", [(1, 1), (2, 3), (0, 1)])
+def test_packed_documents_are_independent(variant, chunk):
+    cfg = small_cfg(variant=variant, chunk=chunk)
+    m = RLTOracle(cfg, weights(cfg))
+    x = toks(cfg, 20)
+    starts = np.zeros(20, bool)
+    starts[[0, 7, 12]] = True
+    st = prefill_packed(m, x, starts)
+    # the last document alone, from a fresh state, in one encode + prefill
+    alone = m.new_state()
+    m.encode(alone, x[12:])
+    m.prefill(alone, 8)
+    assert (st.pos_enc, st.pos_dec) == (8, 8)
+    np.testing.assert_allclose(st.s, alone.s, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(m.readout(st), m.readout(alone), atol=1e-12, rtol=0)
+    # earlier documents leave no trace: change every token before the start
+    y = x.copy()
+    y[:12] = (y[:12] + 5) % cfg.vocab
+    other = prefill_packed(m, y, starts)
+    np.testing.assert_array_equal(m.readout(other), m.readout(st))
+    # one document from column 0 is the plain run
+    one = prefill_packed(m, x, np.eye(1, 20, 0, dtype=bool)[0])
+    plain = m.new_state()
+    m.encode(plain, x)
+    m.prefill(plain, 20)
+    np.testing.assert_allclose(one.s, plain.s, atol=1e-12, rtol=0)
+    # a start at every column: the last token alone
+    last = prefill_packed(m, x, np.ones(20, bool))
+    solo = m.new_state()
+    m.encode(solo, x[-1:])
+    m.prefill(solo, 1)
+    np.testing.assert_allclose(last.s, solo.s, atol=1e-12, rtol=0)
