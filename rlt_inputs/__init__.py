@@ -95,9 +95,11 @@ def substream_key(seed: int, *labels: int) -> int:
     return key
 
 
-def normal(seed: int, n: int, std: float) -> np.ndarray:
-    """n draws of N(0, std^2) by Box-Muller (cosine branch) from one SplitMix64 stream."""
-    raw = splitmix64_stream(seed, 0, 2 * n)
+def normal(seed: int, n: int, std: float, start: int = 0) -> np.ndarray:
+    """Draws start .. start+n-1 of N(0, std^2) by Box-Muller (cosine branch)
+    from one SplitMix64 stream: draw i uses stream outputs 2i+1 and 2i+2, so
+    any range of draws can be produced on its own."""
+    raw = splitmix64_stream(seed, 2 * start, 2 * n)
     u1 = (raw[0::2] >> np.uint64(11)).astype(np.float64) + 1.0
     u1 *= 1.0 / 9007199254740992.0          # (0, 1]: log never sees 0
     u2 = u53(raw[1::2])
@@ -263,27 +265,53 @@ def _init_kind(name: str) -> str:
     return "normal"
 
 
-def generate_weights(cfg: RLTConfig, seed: int = WEIGHT_SEED, std: float = 0.02
-                     ) -> Dict[str, np.ndarray]:
+_GEN_CHUNK = 1 << 22        # draws per piece when a tensor is generated in pieces
+
+
+def generate_weights(cfg: RLTConfig, seed: int = WEIGHT_SEED, std: float = 0.02,
+                     threads: int | None = None) -> Dict[str, np.ndarray]:
     """Seeded weights as float32 arrays (already bf16-valued for bf16 configs).
 
     Tensor k of the manifest draws from its own SplitMix64 substream, so any
-    tensor can be regenerated alone.
+    tensor can be regenerated alone.  Large tensors are produced in pieces of
+    consecutive draws on a thread pool (numpy releases the GIL inside its
+    array operations); the values do not depend on the number of threads.
     """
     cfg.validate()
+    import concurrent.futures as cf
+    import os
     W: Dict[str, np.ndarray] = {}
+    jobs = []
     for k, (name, shape) in enumerate(manifest(cfg)):
         n = int(np.prod(shape))
         kind = _init_kind(name)
         if kind == "ones":
-            a = np.ones(n, np.float32)
+            W[name] = np.ones(shape, np.float32)
         elif kind == "zeros":
-            a = np.zeros(n, np.float32)
+            W[name] = np.zeros(shape, np.float32)
         else:
-            a = normal(substream_key(seed, k), n, std).astype(np.float32)
+            a = np.empty(n, np.float32)
+            W[name] = a
+            key = substream_key(seed, k)
+            for i0 in range(0, n, _GEN_CHUNK):
+                jobs.append((a, key, i0, min(n, i0 + _GEN_CHUNK)))
+
+    def fill(job):
+        a, key, i0, i1 = job
+        v = normal(key, i1 - i0, std, start=i0).astype(np.float32)
         if cfg.dtype == DT_BF16:
-            a = bf16_bits_to_f32(to_bf16_bits(a))
-        W[name] = a.reshape(shape)
+            v = bf16_bits_to_f32(to_bf16_bits(v))
+        a[i0:i1] = v
+
+    nthr = threads if threads is not None else min(16, os.cpu_count() or 1)
+    if nthr <= 1 or len(jobs) <= 1:
+        for j in jobs:
+            fill(j)
+    else:
+        with cf.ThreadPoolExecutor(nthr) as ex:
+            list(ex.map(fill, jobs))
+    for name, shape in manifest(cfg):
+        W[name] = W[name].reshape(shape)
     return W
 
 

@@ -130,6 +130,30 @@ def test_box_muller_moments():
     assert abs(np.mean(z ** 4) - 3.0) < 0.05            # Gaussian kurtosis
 
 
+def test_normal_draws_by_range_and_threads():
+    """Draw i of a stream uses its outputs 2i+1, 2i+2: any range of draws
+    equals the same slice of the whole stream, and weights generated in
+    pieces on a thread pool equal the single-thread ones bit for bit."""
+    z = ri.normal(77, 1000, 0.5)
+    for i0, i1 in ((0, 1), (3, 500), (999, 1000)):
+        np.testing.assert_array_equal(ri.normal(77, i1 - i0, 0.5, start=i0), z[i0:i1])
+    # the first draw from its published definition: SplitMix64 outputs 1 and 2
+    o1, o2 = ri.splitmix64_stream_int(77, 2)
+    u1 = ((o1 >> 11) + 1) / 9007199254740992.0
+    u2 = (o2 >> 11) / 9007199254740992.0
+    assert z[0] == 0.5 * np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+    cfg = ri.CONFIGS["parity_bf16"].replace(vocab=50)
+    old = ri._GEN_CHUNK
+    try:
+        ri._GEN_CHUNK = 1000                    # many pieces per tensor
+        a = ri.generate_weights(cfg, threads=8)
+    finally:
+        ri._GEN_CHUNK = old
+    b = ri.generate_weights(cfg, threads=1)
+    for k in b:
+        np.testing.assert_array_equal(a[k], b[k])
+
+
 def test_blob_roundtrip_and_checksum():
     for name in ("tiny_fp32", "rlt2_mod5_bf16"):
         cfg = ri.CONFIGS[name].replace(d=32, heads=4, ffn=40, vocab=10)
