@@ -47,14 +47,15 @@ def peaks():
             "fallback"
 
 
-def kernel_traffic(alg_bytes_per_launch: float):
+def kernel_traffic(alg_bytes_per_launch: float, record: str | None = None):
     """DRAM bytes per launch of the dominant kernel from its committed ncu
     capture (profiles/dominant_kernel_traffic.json), scaled from the captured
     launch to the average launch by the algorithmic bytes.  None when there is
     no capture or the kernel's source changed since it was taken."""
     import hashlib
     try:
-        rec = json.load(open(os.path.join(ROOT, "profiles", "dominant_kernel_traffic.json")))
+        path = record or os.path.join(ROOT, "profiles", "dominant_kernel_traffic.json")
+        rec = json.load(open(path))
         src = open(os.path.join(ROOT, rec["source"]), "rb").read()
         if hashlib.sha256(src).hexdigest() != rec["source_sha256"]:
             return None

@@ -74,9 +74,9 @@ typedef struct rlt_config {
  * named tensor records in the fixed manifest order of the config.  Errors:
  * RLT_E_BLOB (bad magic/version/manifest/checksum), RLT_E_UNSUPPORTED (head
  * size other than 16, 32, 64, 128, or width d above 2048), RLT_E_DEVICE,
- * RLT_E_OOM.  One device per process: kernels' shared-memory attributes are
- * set once per process, on the device that launches them first, so calls on
- * models of a second device in the same process may fail with RLT_E_DEVICE. */
+ * RLT_E_OOM.  Models on several devices may share a process: every call
+ * makes its model's device current, and kernel attributes are set per
+ * device. */
 int rlt_create(const void* blob, size_t nbytes, int device, rlt_model** out);
 void rlt_destroy(rlt_model* model);
 int rlt_model_config(const rlt_model* model, rlt_config* out);
@@ -133,7 +133,9 @@ int rlt_prefill(rlt_state* state, int T, void* stream);
  * u = the SplitMix64 uniform of (rng_seed, row, rng_step):
  *   key = mix64(rng_seed ^ mix64((row+1)*G)), u = top53(mix64(key + (rng_step+1)*G))
  * with G = 0x9E3779B97F4A7C15 and mix64 the SplitMix64 finaliser.  No top-k/p
- * truncation (jiphyeonjeon review §6.2).  temperature > 0. */
+ * truncation (jiphyeonjeon review §6.2).  temperature > 0.  Each output may
+ * be device or host memory; device outputs are written in stream order, host
+ * outputs are valid on return (the call then synchronises `stream`). */
 int rlt_readout(rlt_state* state, float* logits, int32_t* argmax, int32_t* sampled,
                 uint64_t rng_seed, uint64_t rng_step, float temperature, void* stream);
 
@@ -172,12 +174,14 @@ int rlt_replay_logprobs(rlt_state* state, const int32_t* tokens, int n, float* l
  * (jiphyeonjeon review §6.1; greeksharifa App. F).  Every token is encoded
  * and consumed (one transition each); a row without a start at column 0
  * continues its current document.  Row b then holds the state of its last
- * document, exactly as if that document alone had been encoded and
- * prefilled in a fresh row.  The columns are cut where any row starts a
+ * document as if that document alone had been encoded and prefilled in a
+ * fresh row: bit for bit for RLT-1 and RLT-0; for RLT-2 within the rounding
+ * of the two schedules (a lone prefill runs each chunk's positions as one
+ * block, the packed run meets chunks cut at document starts).  The columns are cut where any row starts a
  * document, and each piece is one rlt_encode + rlt_prefill for all rows, so
  * rows sit at different positions.  Synchronises `stream` at every cut.
- * Errors, checked before anything runs: RLT_E_ARG (null pointers, n < 0, a
- * host token outside [0, vocab)), RLT_E_ORDER (a row has encoded tokens not
+ * Errors, checked before anything runs: RLT_E_ARG (null pointers, n < 0,
+ * doc_start in device memory, a host token outside [0, vocab)), RLT_E_ORDER (a row has encoded tokens not
  * yet consumed), RLT_E_CAPACITY (a document would pass max_len); later,
  * RLT_E_DEVICE if a CUDA call fails (the rows then hold the pieces before
  * it). */
@@ -190,7 +194,8 @@ int rlt_prefill_packed(rlt_state* state, const int32_t* tokens, const uint8_t* d
  * fp32 [rows][d]; row r is read out exactly as rlt_readout reads out row r of
  * a state whose s_t equals it (same logits, argmax and sampled id for the
  * same rng_seed, rng_step, temperature).  Outputs as in rlt_readout: each may
- * be NULL, device or host memory.
+ * be NULL, device or host memory; host outputs are valid on return (the call
+ * then synchronises `stream`, which also ends its use of the scratch).
  * Scratch: a file-scope device array of RLT_READOUT_ROWS_SCRATCH_BYTES (16 MiB)
  * per device.  A call needs rows*d*(2 for bf16, 4 for fp32) bytes, plus
  * rows*vocab*4 when `logits` is not a device pointer, plus rows*8, each rounded

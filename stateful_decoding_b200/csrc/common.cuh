@@ -68,6 +68,11 @@ bool pdl_enabled();
 // for every kernel of the library, so that consecutive kernels never make an
 // SM switch its L1 / shared-memory split (defined in rlt_api.cu).
 void set_carveout_once(const void* kernel);
+// The kernel's dynamic shared-memory limit, set once per (device, kernel,
+// size); false when the device refuses it.
+bool set_smem_once(const void* kernel, size_t bytes);
+// Multiprocessors of the current device (0 on error).
+int sm_count();
 
 // kernel<<<grid, block, smem, st>>>(args...) with the programmatic-serialisation
 // attribute set when PDL is enabled.

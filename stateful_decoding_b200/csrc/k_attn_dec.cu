@@ -590,14 +590,8 @@ bool launch_one(const float* Q, const bf16* base, size_t row_stride, int span, c
                 const bf16* Vc, const int32_t* pos, int W, bf16* A, int B, int n, int heads,
                 const ProjIn& pin, cudaStream_t st) {
     constexpr size_t smem = 2 * NSTG * (size_t)CH * DH * 2;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(k_attn_stream<DH, NQ, SWA, PRO, NSTG>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return false;
-        attr = true;
-    }
+    if (!set_smem_once(reinterpret_cast<const void*>(k_attn_stream<DH, NQ, SWA, PRO, NSTG>), smem))
+        return false;
     launch(k_attn_stream<DH, NQ, SWA, PRO, NSTG>, dim3(B * heads, (n + NQ - 1) / NQ), NW * 32,
            smem, st, Q, base, row_stride, span, Kc, Vc, pos, W, A, n, heads, pin);
     rlt_count_launch();

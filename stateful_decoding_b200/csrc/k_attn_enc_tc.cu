@@ -266,13 +266,7 @@ bool launch_nk(const float* Q, const bf16* cache, size_t row_stride, int T_cap, 
     constexpr size_t smem = (size_t)NK / 64 * 64 * 128 + (NK / 128) * EQ * 128 + EQ * 128 + 1024;
     constexpr size_t smem_p = (size_t)NK / 64 * 64 * 128 + (size_t)NK / 64 * EQ * 128 + 1024;
     constexpr size_t bytes = smem > smem_p ? smem : smem_p;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(k_attn_enc_tc<NK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)bytes) != cudaSuccess)
-            return false;
-        attr = true;
-    }
+    if (!set_smem_once(reinterpret_cast<const void*>(k_attn_enc_tc<NK>), bytes)) return false;
     launch(k_attn_enc_tc<NK>, dim3(B * heads, (n + EQ - 1) / EQ), ENT, bytes, st, Q, cache,
            row_stride, T_cap, pos, A, n, heads, err);
     rlt_count_launch();

@@ -831,13 +831,8 @@ k_dec_fused(const __grid_constant__ FusedParams P) {
 
 // Launch nsteps fused transitions for all rows; false if the launch failed.
 bool launch_dec_fused(const fz::FusedParams& p, cudaStream_t st) {
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(fz::k_dec_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 fz::SMEM_DYN) != cudaSuccess)
-            return false;
-        attr = true;
-    }
+    if (!set_smem_once(reinterpret_cast<const void*>(fz::k_dec_fused), fz::SMEM_DYN))
+        return false;
     const int nclusters = (p.B + fz::RB - 1) / fz::RB;
     fz::k_dec_fused<<<nclusters * fz::CL, fz::NT, fz::SMEM_DYN, st>>>(p);
     rlt_count_launch();

@@ -206,13 +206,8 @@ bool launch_bn(const bf16* A, int lda, const bf16* W, int ldw, float* Z, const f
     CUtensorMap ta, tb;
     if (!make_tma_2d_bf16(&ta, A, M, K, lda, BM) || !make_tma_2d_bf16(&tb, W, N, K, ldw, BN))
         return false;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(k_gemm_norm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem_bytes<BN>()) != cudaSuccess)
-            return false;
-        attr = true;
-    }
+    if (!set_smem_once(reinterpret_cast<const void*>(k_gemm_norm<BN>), smem_bytes<BN>()))
+        return false;
     set_carveout_once(reinterpret_cast<const void*>(k_gemm_norm<BN>));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(N / BN, (M + BM - 1) / BM, 1);

@@ -205,16 +205,9 @@ bool launch_mode(const bf16* A, int lda, const bf16* W, int ldw, float* C, int l
     CUtensorMap ta, tb;
     if (!make_tma_2d_bf16(&ta, A, M, K, lda, BM) || !make_tma_2d_bf16(&tb, W, N, K, ldw, BN))
         return false;
-    static int sms = 0;
-    if (!sms) {
-        if (cudaFuncSetAttribute(k_gemm_persist<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)SMEM) != cudaSuccess)
-            return false;
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return false;
-    }
+    if (!set_smem_once(reinterpret_cast<const void*>(k_gemm_persist<MODE>), SMEM)) return false;
+    const int sms = sm_count();
+    if (sms <= 0) return false;
     const int tiles = ((M + BM - 1) / BM) * (N / BN);
     launch(k_gemm_persist<MODE>, std::min(tiles, sms), NTHREADS, SMEM, st, ta, tb, C, ldc, Ct,
            ldct, M, N, K);

@@ -337,13 +337,8 @@ bool launch_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc
                int ldct, int M, int N, int K, int splits, size_t slab, cudaStream_t st) {
     CUtensorMap ta, tb;
     if (!make_map(&ta, A, M, K, lda, BM) || !make_map(&tb, W, N, K, ldw, BN)) return false;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem_bytes<BN>()) != cudaSuccess)
-            return false;
-        attr = true;
-    }
+    if (!set_smem_once(reinterpret_cast<const void*>(k_gemm_tc<BN, MODE>), smem_bytes<BN>()))
+        return false;
     const int nk = K / BK, cps = (nk + splits - 1) / splits;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, (nk + cps - 1) / cps);
     launch(k_gemm_tc<BN, MODE>, grid, NTHREADS, smem_bytes<BN>(), st, ta, tb, C, ldc, Ct, ldct, M, N,

@@ -17,6 +17,7 @@
 #include <map>
 #include <mutex>
 #include <set>
+#include <tuple>
 #include <vector>
 
 #include <nvtx3/nvToolsExt.h>
@@ -49,14 +50,46 @@ bool pdl_enabled() {
     }();
     return on;
 }
+// Function attributes are per device: each is set once per (device, kernel).
+namespace {
+std::mutex g_attr_mu;
+std::set<std::tuple<int, const void*, int>> g_attr_done;   // (device, kernel, what)
+int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    return dev;
+}
+}  // namespace
 void set_carveout_once(const void* kernel) {
-    static std::mutex mu;
-    static std::set<const void*> done;
-    std::lock_guard<std::mutex> lk(mu);
-    if (!done.insert(kernel).second) return;
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    if (!g_attr_done.insert({current_device(), kernel, -1}).second) return;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         cudaGetLastError();        // a preference only: launching works without it
+}
+bool set_smem_once(const void* kernel, size_t bytes) {
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    const auto key = std::make_tuple(current_device(), kernel, (int)bytes);
+    if (g_attr_done.count(key)) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    g_attr_done.insert(key);
+    return true;
+}
+int sm_count() {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, current_device()) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
 }
 template <typename T>
 void launch_gemm(const T* A, int lda, const T* W, int ldw, float* C, int ldc, T* Ct, int ldct,
@@ -1336,6 +1369,10 @@ extern "C" int rlt_readout(rlt_state* s, float* logits, int32_t* argmax, int32_t
     if (sampled && !sd &&
         cudaMemcpyAsync(sampled, sbuf, (size_t)B * 4, cudaMemcpyDeviceToHost, st))
         return RLT_E_DEVICE;
+    // host outputs are valid on return (pinned memory would otherwise fill later)
+    if (((logits && !ld) || (argmax && !ad) || (sampled && !sd)) &&
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return RLT_E_DEVICE;
     return RLT_OK;
 }
 
@@ -1418,6 +1455,7 @@ extern "C" int rlt_prefill_packed(rlt_state* s, const int32_t* tokens, const uin
     for (int b = 0; b < B; ++b)
         if (s->h_pos_dec[b] != s->h_pos_enc[b]) return RLT_E_ORDER;
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    if (is_device_ptr(doc_start)) return RLT_E_ARG;     // read on the host below
     const bool tdev = is_device_ptr(tokens);
     // everything that could fail part-way is checked before the first piece
     for (int b = 0; b < B; ++b) {
@@ -1915,6 +1953,11 @@ extern "C" int rlt_readout_rows(const rlt_model* m, const float* s_rows, int row
         return RLT_E_DEVICE;
     if (sampled && !sd &&
         cudaMemcpyAsync(sampled, sbuf, (size_t)rows * 4, cudaMemcpyDeviceToHost, st))
+        return RLT_E_DEVICE;
+    // host outputs are valid on return, and the copies out of the shared
+    // array have finished before the next call can overwrite it
+    if (((logits && !ld) || (argmax && !ad) || (sampled && !sd)) &&
+        cudaStreamSynchronize(st) != cudaSuccess)
         return RLT_E_DEVICE;
     return RLT_OK;
 }

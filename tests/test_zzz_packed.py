@@ -39,6 +39,7 @@ def _logits(st, cfg):
 
 
 STARTS = {0: [0, 9], 1: [0, 4, 17], 2: [0]}      # row -> columns where documents start
+RLT2_SCHEDULE_GAP = TOL_BF16 / 3
 
 
 @pytest.mark.parametrize("name", ["tiny_fp32", "parity_bf16", "rlt2_mod5_bf16"])
@@ -68,8 +69,12 @@ def test_packed_rows_equal_their_last_document_alone(sd, name):
         alone.prefill(n - j)
         la = _logits(alone, cfg)[0]
         # RLT-2: the lone prefill runs whole chunks together, the packed one
-        # steps token by token (rows at different positions)
-        np.testing.assert_allclose(lg[b], la, atol=0 if cfg.variant == 1 else TOL_BF16, rtol=0)
+        # meets chunks cut at document starts (rows at different positions);
+        # the two schedules differ by rounding only, well inside the bf16
+        # tolerance (the bound is a third of it)
+        gap = float(np.max(np.abs(lg[b] - la)))
+        print(f"{name} row {b}: packed vs alone max|dlogit| {gap:.3e}")
+        assert gap <= (0 if cfg.variant != 2 else RLT2_SCHEDULE_GAP)
         ref = prefill_packed(orc, toks[b], starts[b].astype(bool))
         assert np.max(np.abs(lg[b] - orc.readout(ref))) <= tol
         alone.close()
@@ -107,6 +112,10 @@ def test_packed_continues_and_rejects(sd):
     assert e.value.code == sd.RLT_E_CAPACITY
     bad = np.full((B, 3), cfg.vocab, np.int32)
     assert sd.rlt_prefill_packed(short.handle, bad, np.zeros((B, 3), np.uint8), 3) == sd.RLT_E_ARG
+    import torch
+    dev_starts = torch.zeros((B, 3), dtype=torch.uint8, device="cuda")   # must be host memory
+    assert sd.rlt_prefill_packed(short.handle, np.ascontiguousarray(toks[:, :3]), dev_starts,
+                                 3) == sd.RLT_E_ARG
     short.encode(np.ascontiguousarray(toks[:, :1]))
     with pytest.raises(sd.RLTError) as e:
         short.prefill_packed(np.ascontiguousarray(toks[:, :2]), np.zeros((B, 2), np.uint8))

@@ -1,7 +1,19 @@
-"""rlt_readout_rows: the readout of caller-supplied state vectors whose scratch
-is a static device array (no allocation in the call), against rlt_readout on
-the same s_t.  Named to be collected last: it must pass alone and after every
-other test of the session has used the device.
+"""rlt_readout_rows: reading out state vectors the caller supplies, with no
+device allocation inside the call.
+
+Who needs it: a serving process that scores exported or candidate state
+vectors while its memory pool already holds the rest of the device (a
+cudaMalloc there fails or forces an eviction), or while other streams run
+(cudaMalloc and cudaFree can synchronise the device and stall them).  The
+call therefore works out of a fixed file-scope device array instead of
+allocating.
+
+Checked here against rlt_readout on the same s_t, two calls in a row (they
+share the one array), with device and host outputs, for both dtypes; the
+device's free memory is the same before and after a call; oversize requests
+and bad arguments are rejected.  The file name sorts last, so a run that
+stops at the first failure has run every other test before this one; it
+also passes alone in a fresh process.
 """
 import numpy as np
 import pytest
@@ -42,24 +54,39 @@ def test_readout_rows_matches_readout(sd, name, B, T):
     s_rows = torch.from_numpy(st.read(sd.PART_S).view(np.float32).reshape(B, cfg.d).copy()).cuda()
 
     stream = torch.cuda.Stream()
+    # every buffer exists before the calls, so that only the library could
+    # change the device's free memory during one
+    lg_d = torch.empty((B, cfg.vocab), device="cuda")
+    am_d = torch.empty((B,), dtype=torch.int32, device="cuda")
+    sp_d = torch.empty((B,), dtype=torch.int32, device="cuda")
+    lg_h = np.empty((B, cfg.vocab), np.float32)
+    am_h = np.empty(B, np.int32)
+    sp_h = np.empty(B, np.int32)
     for call in range(2):          # two calls in a row reuse the one scratch
         # device outputs
-        lg_d = torch.full((B, cfg.vocab), float("nan"), device="cuda")
-        am_d = torch.full((B,), -1, dtype=torch.int32, device="cuda")
-        sp_d = torch.full((B,), -1, dtype=torch.int32, device="cuda")
+        lg_d.fill_(float("nan"))
+        am_d.fill_(-1)
+        sp_d.fill_(-1)
+        torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
         model.readout_rows(s_rows, lg_d, am_d, sp_d, seed=seed, step=step, temperature=temp,
                            stream=stream)
         stream.synchronize()
+        free1 = torch.cuda.mem_get_info()[0]
+        if call == 1:               # the first call may load the module on this device
+            assert free1 == free0, f"device free memory moved by {free0 - free1} bytes"
         np.testing.assert_allclose(lg_d.cpu().numpy(), lg, atol=TOL, rtol=0)
         np.testing.assert_array_equal(am_d.cpu().numpy(), am)
         np.testing.assert_array_equal(sp_d.cpu().numpy(), sp)
-        # host outputs: logits and ids pass through the scratch
-        lg_h = np.full((B, cfg.vocab), np.nan, np.float32)
-        am_h = np.full(B, -1, np.int32)
-        sp_h = np.full(B, -1, np.int32)
+        # host outputs: logits and ids pass through the scratch, valid on return
+        lg_h.fill(np.nan)
+        am_h.fill(-1)
+        sp_h.fill(-1)
+        free0 = torch.cuda.mem_get_info()[0]
         model.readout_rows(s_rows, lg_h, am_h, sp_h, seed=seed, step=step, temperature=temp,
                            stream=stream)
-        stream.synchronize()
+        free1 = torch.cuda.mem_get_info()[0]
+        assert free1 == free0, f"device free memory moved by {free0 - free1} bytes"
         np.testing.assert_allclose(lg_h, lg, atol=TOL, rtol=0)
         np.testing.assert_array_equal(am_h, am)
         np.testing.assert_array_equal(sp_h, sp)
