@@ -15,7 +15,8 @@ per-GPU batch: weak scaling); there is no collective on the data path, only
 the barrier and the max-over-ranks reduction of the timing.
 
 --impl reference times the CPU oracle (test infrastructure, float64 numpy)
-on the host cores on a bounded sample of the same workload.
+on all host cores, one process per core over rows, on a bounded sample of
+the same workload.
 """
 from __future__ import annotations
 
@@ -64,6 +65,19 @@ def kernel_traffic(alg_bytes_per_launch: float, record: str | None = None):
         return None
 
 
+def encoder_flops(cfg, rows: int, T: int) -> float:
+    """Algorithmic FLOPs of encoding T positions of `rows` rows from empty
+    caches: per position and encoder layer 2 (4 d^2 + 3 d f) for the
+    projections and the SwiGLU FFN, per layer the causal attention
+    2 * 2 d * t summed over t = 1..T, and 2 * 2 d^2 per memory group."""
+    d, f = cfg.d, cfg.ffn
+    per_pos = cfg.n_enc * 2 * (4 * d * d + 3 * d * f)
+    if cfg.n_dec > 0:
+        per_pos += cfg.groups * 2 * 2 * d * d
+    attn = cfg.n_enc * 2 * d * T * (T + 1)
+    return float(rows) * (per_pos * T + attn)
+
+
 def workload_desc(cfg) -> dict:
     kind = {0: "RLT-0", 1: "RLT-1", 2: f"RLT-2 (feedback chunk {cfg.chunk})"}[cfg.variant]
     dt = "bf16" if cfg.dtype == ri.DT_BF16 else "fp32"
@@ -78,37 +92,71 @@ def workload_desc(cfg) -> dict:
 # ----------------------------------------------------------------------------
 # CPU oracle leg
 # ----------------------------------------------------------------------------
-def oracle_sample(cfg, budget_s: float = 15.0):
-    """Time the oracle (float64, as it stands) on rows of the workload until the
-    budget is spent; returns (tokens/s, description, threads)."""
-    from oracle import RLTOracle
+def _oracle_worker(job):
+    """One host process of the CPU baseline: run the oracle (float64, as it
+    stands, one BLAS thread) on whole rows of the workload until the budget
+    is spent; returns (transitions, rows, seconds)."""
+    fields, row0, stride, T, budget_s = job
     try:
         import threadpoolctl
-        threads = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()) \
-            if threadpoolctl.threadpool_info() else 1
+        threadpoolctl.threadpool_limits(1)
     except Exception:
-        threads = os.cpu_count() or 1
-    W = ri.generate_weights(cfg)
-    orc = RLTOracle(cfg, W, "fp64")
-    T = min(cfg.prompt, 256)
-    done_tok, rows, t0 = 0, 0, time.perf_counter()
-    while True:
-        toks = ri.make_tokens(cfg, 1, T, row0=rows)[0]
+        pass
+    from oracle import RLTOracle
+    cfg = ri.RLTConfig(**fields)
+    orc = RLTOracle(cfg, ri.generate_weights(cfg, threads=1), "fp64")
+    done, rows, row = 0, 0, row0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
         st = orc.new_state()
-        orc.encode(st, toks)
+        orc.encode(st, ri.make_tokens(cfg, 1, T, row0=row)[0])
         for _ in range(T):
             orc.transition(st)
-            done_tok += 1
+            done += 1
             if time.perf_counter() - t0 > budget_s:
                 break
         orc.readout(st)
         rows += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
-    desc = (f"{rows} row(s) of the same workload, prompt {T}: encode + {done_tok} transitions "
-            f"+ readout, float64 numpy oracle, {dt:.1f} s")
-    return done_tok / dt, desc, threads
+        row += stride
+    return done, rows, time.perf_counter() - t0
+
+
+def oracle_processes(cfg) -> int:
+    """Host processes for the CPU baseline: one per core, fewer when the
+    oracle's float64 copy of the weights would not fit in host memory."""
+    cores = os.cpu_count() or 1
+    wbytes = 8.0 * ri.param_count(cfg) * 2.2          # float64 copy + generation buffers
+    try:
+        avail = os.sysconf("SC_AVPHYS_PAGES") * os.sysconf("SC_PAGE_SIZE")
+        cores = max(1, min(cores, int(0.6 * avail // wbytes)))
+    except (ValueError, OSError, AttributeError):
+        pass
+    return cores
+
+
+def oracle_sample(cfg, budget_s: float = 15.0):
+    """The CPU baseline: the oracle as it stands (float64 numpy, one row at a
+    time) on all host cores, one process per core over independent rows of
+    the workload (spawned, so no process inherits a CUDA context).  Returns
+    (tokens/s, description, processes)."""
+    import multiprocessing as mp
+    procs = oracle_processes(cfg)
+    T = min(cfg.prompt, 256)
+    import dataclasses
+    fields = dataclasses.asdict(cfg)
+    jobs = [(fields, p, procs, T, budget_s) for p in range(procs)]
+    t0 = time.perf_counter()
+    with mp.get_context("spawn").Pool(procs) as pool:
+        res = pool.map(_oracle_worker, jobs)
+    wall = time.perf_counter() - t0
+    done = sum(r[0] for r in res)
+    rows = sum(r[1] for r in res)
+    busy = max(r[2] for r in res)
+    desc = (f"{rows} row(s) of the same workload, prompt {T} (encode + transitions + readout; "
+            f"the last row of each process cut at the budget), float64 numpy oracle, one "
+            f"process per core with one BLAS thread each: {done} transitions in {busy:.1f} s "
+            f"({wall:.1f} s with process start-up and weight generation)")
+    return done / busy, desc, procs
 
 
 # ----------------------------------------------------------------------------
@@ -142,8 +190,10 @@ def run_reference(args, cfg):
     if rank != 0:
         return
     vals = []
+    # every sample starts its own processes; their start-up and weight
+    # generation stay outside the timed part
     for _ in range(args.warmup):
-        oracle_sample(cfg, budget_s=2.0)
+        oracle_sample(cfg, budget_s=1.0)
     for _ in range(args.steps):
         v, desc, threads = oracle_sample(cfg, budget_s=max(5.0, 60.0 / max(1, args.steps)))
         vals.append(v)
@@ -155,7 +205,8 @@ def run_reference(args, cfg):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": dict(workload_desc(cfg), global_batch=cfg.batch * args.gpus),
-            "hardware": "host CPU cores of rank 0 (the float64 oracle; no GPU work)",
+            "hardware": "host CPU cores of rank 0 (the float64 oracle, one process per core; "
+                        "no GPU work)",
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -331,6 +382,9 @@ def run_ours(args, cfg):
     pk, pk_kind = peaks()
     n_s, ms_s, by_s = prof["step"]
     step_gbs = (by_s / ms_s * 1e3 / 1e9) if ms_s else 0.0
+    enc_ms = prof["enc"][1] / args.steps
+    enc_tf = encoder_flops(cfg, B, T) / (enc_ms / 1e3) / 1e12 if enc_ms else 0.0
+    tc_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
     n, ms, by = kprof["xattn"]
     kname = "decoder cross-attention (k_attn_dec1: one warp per (row, head), q from the projection slabs)"
     xattn_timed = bool(n)
@@ -361,6 +415,17 @@ def run_ours(args, cfg):
                      "peak_kind": f"{pk_kind} hbm_gbs", "launches": n,
                      "avg_launch_us": (ms / n * 1e3) if n else None,
                      "alg_bytes_per_launch": (by / n) if n else None},
+        # the whole decoder step (every kernel of the transition blocks)
+        # against its HBM roofline, and the encoder against the tensor peak
+        "roofline_decoder_step": {
+            "bound": "hbm", "achieved": step_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": step_gbs / pk["hbm_gbs"], "peak_kind": f"{pk_kind} hbm_gbs",
+            "alg_bytes_per_step": by_s / args.steps, "ms_per_step": ms_s / args.steps},
+        "roofline_encoder": {
+            "bound": "tensor", "achieved": enc_tf, "peak": tc_peak, "unit": "TFLOP/s",
+            "frac": enc_tf / tc_peak if tc_peak else None,
+            "peak_kind": f"{pk_kind} bf16_tflops_sustained",
+            "flops_per_step": encoder_flops(cfg, B, T), "ms_per_step": enc_ms},
         "breakdown": {
             "decoder_step": {"launches": n_s, "avg_us": (ms_s / n_s * 1e3) if n_s else None,
                              "alg_GBps": step_gbs, "frac_hbm": step_gbs / pk["hbm_gbs"]},
@@ -399,10 +464,21 @@ def main():
                     help="override the rows per GPU (small profiling cases only)")
     ap.add_argument("--prompt", type=int, default=None,
                     help="override the prompt length (small profiling cases only)")
+    ap.add_argument("--variant", type=int, default=None, choices=[0, 1, 2],
+                    help="run the workload's model as RLT-0, RLT-1 or RLT-2 (feedback variants)")
+    ap.add_argument("--chunk", type=int, default=None,
+                    help="RLT-2 feedback chunk B_c (with --variant 2)")
     args = ap.parse_args()
     cfg = ri.CONFIGS[args.config]
     if args.batch or args.prompt:
         cfg = cfg.replace(batch=args.batch or cfg.batch, prompt=args.prompt or cfg.prompt)
+    if args.variant is not None:
+        v = args.variant
+        chunk = (args.chunk or cfg.chunk) if v == 2 else 1
+        cfg = cfg.replace(name=f"{cfg.name} as RLT-{v}" + (f" B_c={chunk}" if v == 2 else ""),
+                          variant=v, chunk=chunk)
+    elif args.chunk is not None:
+        ap.error("--chunk needs --variant 2")
     if args.impl == "reference":
         run_reference(args, cfg)
     else:

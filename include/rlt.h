@@ -285,6 +285,20 @@ int rlt_snapshot_info(const void* snap, size_t nbytes, rlt_config* cfg, int32_t*
  * (RLT_OK, RLT_E_TIMEOUT, ...), clearing it. */
 int rlt_state_check(rlt_state* state, void* stream);
 
+/* Failure-detection self-test (no counterpart in the method).  Enqueues on
+ * `stream` one small kernel whose single wait nothing will ever satisfy --
+ * kind 0: an mbarrier in shared memory that no thread arrives on; kind 1: a
+ * word in global memory that no thread sets -- bounded by `polls` polls
+ * through the same helpers as the library's own waits.  When the wait gives
+ * up the kernel records a timeout in the state's error word and returns, so
+ * the next rlt_state_check reports RLT_E_TIMEOUT (and clears it) and the
+ * context stays usable; the state's contents are not touched.  No copy is in
+ * flight and no tensor memory is held when it gives up.  A poll of kind 0
+ * lasts as long as the hardware's try-wait suspends (a system-dependent
+ * limit); a poll of kind 1 sleeps about 256 ns.  RLT_E_ARG for a null state,
+ * another kind, or polls outside [1, 2^24]. */
+int rlt_selftest_wait(rlt_state* state, int kind, uint32_t polls, void* stream);
+
 /* Number of kernels this library has launched in this process. */
 uint64_t rlt_kernel_launches(void);
 

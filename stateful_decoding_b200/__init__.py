@@ -61,6 +61,7 @@ _SIGS = {
     "rlt_state_positions": (_i, [_vp, _vp, _vp]),
     "rlt_state_read": (_i, [_vp, _i, _vp, _sz, ctypes.POINTER(_sz), _vp]),
     "rlt_state_check": (_i, [_vp, _vp]),
+    "rlt_selftest_wait": (_i, [_vp, _i, ctypes.c_uint32, _vp]),
     "rlt_state_save": (_i, [_vp, _i, _vp, _sz, ctypes.POINTER(_sz), _vp]),
     "rlt_state_load": (_i, [_vp, _i, _vp, _sz, _vp]),
     "rlt_snapshot_info": (_i, [_vp, _sz, ctypes.POINTER(rlt_config), ctypes.POINTER(ctypes.c_int32),
@@ -241,6 +242,10 @@ def rlt_state_read(state, part: int, dst=None, nbytes: int = 0, stream=None):
 
 def rlt_state_check(state, stream=None) -> int:
     return _lib.rlt_state_check(state, _stream(stream))
+
+
+def rlt_selftest_wait(state, kind: int, polls: int, stream=None) -> int:
+    return _lib.rlt_selftest_wait(state, kind, polls, _stream(stream))
 
 
 def rlt_state_save(state, row: int, dst=None, nbytes: int = 0, stream=None):

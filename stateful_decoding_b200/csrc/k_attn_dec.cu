@@ -575,6 +575,151 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
     }
 }
 
+// One-position cross-attention with the keys of one (row, head) split over
+// the XS warps of a CTA (flash-decoding style), for long memory prefixes with
+// few (row, head) items: warp w streams the w-th contiguous part of keys
+// 1..t exactly as k_attn_dec1 streams a whole run (two batches in flight),
+// then the warps' partial maxima, sums and outputs are merged in warp order.
+// The split depends on t alone, so a row's result does not depend on its
+// batch.
+constexpr int XS = 4;
+
+template <int DH>
+__global__ void __launch_bounds__(XS * 32)
+k_attn_xsplit(const bf16* __restrict__ base, size_t row_stride, int span,
+              const int32_t* __restrict__ pos, bf16* __restrict__ A, int heads, ProjIn pin) {
+    constexpr int LPK = DH / 8, KPR = 32 / LPK, HALF = DH / 2;
+    constexpr int BATCH = DRB * KPR;             // keys per batch
+    __shared__ __align__(16) float s_q[DH];
+    __shared__ float s_m[XS], s_l[XS];
+    __shared__ __align__(16) float s_o[XS][DH];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.x / heads, h = blockIdx.x % heads;
+    const int d = heads * DH, seg = lane % LPK, grp = lane / LPK;
+    const int t = __ldcg(pos + b) + 1;
+    // warp w: keys [jlo, jhi) of the run 0..t-1, parts rounded to whole batches
+    const int part = ((t + XS - 1) / XS + BATCH - 1) / BATCH * BATCH;
+    const int jlo = min(t, warp * part), jhi = min(t, jlo + part);
+    const bf16* kg = base + (size_t)b * row_stride + (size_t)h * span * DH + seg * 8;
+    const bf16* vg = kg + (size_t)heads * span * DH;
+    const uint64_t l2pol = l2_evict_last_policy();
+    uint4 kb0[DRB], vb0[DRB], kb1[DRB], vb1[DRB];
+    auto load_batch = [&](int j0, uint4 (&kb)[DRB], uint4 (&vb)[DRB]) {
+#pragma unroll
+        for (int r = 0; r < DRB; ++r) {
+            const int j = j0 + r * KPR + grp;
+            if (j < jhi) {
+                kb[r] = ld_kv<true>(kg + (size_t)j * DH, l2pol);
+                vb[r] = ld_kv<true>(vg + (size_t)j * DH, l2pol);
+            }
+        }
+    };
+    if (jlo < jhi) load_batch(jlo, kb0, vb0);
+    if (jlo + BATCH < jhi) load_batch(jlo + BATCH, kb1, vb1);
+    pdl_enter();
+
+    // q: formed once by warp 0 (rotate-half pairs at position t, slab sums in
+    // slab order), shared by the four warps
+    if (warp == 0) {
+        const size_t rb = (size_t)b * pin.ldp + h * DH;
+        const float* cs = pin.rope.cs + (size_t)t * HALF;
+        const float* sn = pin.rope.sn + (size_t)t * HALF;
+        for (int j = lane; j < HALF; j += 32) {
+            float y1, y2;
+            rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + j),
+                     slab_sum8(pin.P, pin.S, pin.slab, rb + j + HALF), cs[j], sn[j], y1, y2);
+            s_q[j] = y1;
+            s_q[j + HALF] = y2;
+        }
+    }
+    __syncthreads();
+    const float sc = 1.0f / sqrtf((float)DH);
+    float q[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) q[x] = s_q[seg * 8 + x] * sc;
+
+    float m = -INFINITY, l = 0.f, acc[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+    auto fold = [&](int j0, const uint4 (&kb)[DRB], const uint4 (&vb)[DRB]) {
+        float s[DRB];
+#pragma unroll
+        for (int r = 0; r < DRB; ++r) {
+            const bool v = j0 + r * KPR + grp < jhi;
+            float kf[8] = {};
+            if (v) unpack8(kb[r], kf);
+            float dot = 0.f;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) dot = fmaf(q[x], kf[x], dot);
+#pragma unroll
+            for (int o = LPK / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            s[r] = v ? dot : -INFINITY;
+        }
+        float bm = s[0];
+#pragma unroll
+        for (int r = 1; r < DRB; ++r) bm = fmaxf(bm, s[r]);
+#pragma unroll
+        for (int o = 16; o >= LPK; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+        const float mn = fmaxf(m, bm);          // finite: the batch holds a key
+        const float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
+        float ps = 0.f;
+#pragma unroll
+        for (int r = 0; r < DRB; ++r) {
+            s[r] = (s[r] == -INFINITY) ? 0.f : __expf(s[r] - mn);
+            ps += s[r];
+        }
+#pragma unroll
+        for (int o = 16; o >= LPK; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        l = l * corr + ps;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc[x] *= corr;
+        m = mn;
+#pragma unroll
+        for (int r = 0; r < DRB; ++r) {
+            if (!(j0 + r * KPR + grp < jhi)) continue;
+            float vf[8];
+            unpack8(vb[r], vf);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) acc[x] = fmaf(s[r], vf[x], acc[x]);
+        }
+    };
+    for (int j0 = jlo; j0 < jhi; j0 += 2 * BATCH) {
+        fold(j0, kb0, vb0);
+        if (j0 + 2 * BATCH < jhi) load_batch(j0 + 2 * BATCH, kb0, vb0);
+        if (j0 + BATCH >= jhi) break;
+        fold(j0 + BATCH, kb1, vb1);
+        if (j0 + 3 * BATCH < jhi) load_batch(j0 + 3 * BATCH, kb1, vb1);
+    }
+#pragma unroll
+    for (int x = 0; x < 8; ++x)
+#pragma unroll
+        for (int o = 16; o >= LPK; o >>= 1) acc[x] += __shfl_xor_sync(0xffffffffu, acc[x], o);
+    if (grp == 0) {
+#pragma unroll
+        for (int x = 0; x < 8; ++x) s_o[warp][seg * 8 + x] = acc[x];
+        if (lane == 0) {
+            s_m[warp] = m;
+            s_l[warp] = l;
+        }
+    }
+    __syncthreads();
+    // merge the parts in warp order (part 0 always holds key 1)
+    for (int x = threadIdx.x; x < DH; x += XS * 32) {
+        float M = s_m[0];
+#pragma unroll
+        for (int w = 1; w < XS; ++w) M = fmaxf(M, s_m[w]);
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int w = 0; w < XS; ++w) {
+            if (s_m[w] == -INFINITY) continue;
+            const float f = __expf(s_m[w] - M);
+            L += s_l[w] * f;
+            O += s_o[w][x] * f;
+        }
+        A[(size_t)b * d + h * DH + x] = __float2bfloat16_rn(O / L);
+    }
+}
+
 template <int DH, bool SWA>
 bool launch_dec1(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W, bf16* A,
                  int B, int heads, const ProjIn& pin, cudaStream_t st) {
@@ -679,6 +824,14 @@ bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_strid
                             cudaStream_t st) {
     if (!fast_attn_enabled() || (dh != 64 && dh != 128)) return false;
     if (B * n <= 0) return true;
+    if (n == 1 && pin.S <= 8 && dh == 128) {
+        // the wide heads come with long memory prefixes and few items per
+        // launch: split each item's keys over four warps
+        launch(k_attn_xsplit<128>, B * heads, XS * 32, 0, st, mem, row_stride, T_cap, pos, A,
+               heads, pin);
+        rlt_count_launch();
+        return true;
+    }
     if (n == 1 && pin.S <= 8)
         return dh == 64 ? launch_dec1<64, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st)
                         : launch_dec1<128, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st);

@@ -278,7 +278,10 @@ bool launch_nk(const float* Q, const bf16* cache, size_t row_stride, int T_cap, 
 bool launch_attn_enc_tc(const float* Q, const bf16* cache, size_t row_stride, int T_cap,
                         const int32_t* pos, bf16* A, int B, int n, int heads, int dh, int max_keys,
                         int* err, cudaStream_t st) {
-    if (dh != EDH || max_keys > 256 || B * n <= 0) return false;
+    if (B * n <= 0) return false;
+    // longer prefixes and d_h = 128: key tiles with a running softmax
+    if (dh != EDH || max_keys > 256)
+        return launch_attn_enc_fa(Q, cache, row_stride, T_cap, pos, A, B, n, heads, dh, err, st);
     if (max_keys <= 128)
         return launch_nk<128>(Q, cache, row_stride, T_cap, pos, A, B, n, heads, err, st);
     return launch_nk<256>(Q, cache, row_stride, T_cap, pos, A, B, n, heads, err, st);

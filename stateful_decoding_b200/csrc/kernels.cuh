@@ -151,12 +151,26 @@ bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_strid
                             const int32_t* pos_dec, bf16* A, int B, int n, int heads, int dh,
                             cudaStream_t st);
 bool fast_attn_enabled();           // false when RLT_ATTN=warp
-// Encoder causal attention on the tensor cores (k_attn_enc_tc.cu) for d_h = 64
-// and at most 256 keys per row (max_keys = max over rows of pos_enc + n);
-// false (nothing launched) otherwise.  err: the state's device error word.
+// Encoder causal attention on the tensor cores: k_attn_enc_tc.cu (exact
+// two-pass softmax) for d_h = 64 and at most 256 keys per row (max_keys =
+// max over rows of pos_enc + n), k_attn_enc_fa.cu for longer prefixes and
+// d_h = 128; false (nothing launched) for other head sizes.  err: the
+// state's device error word.
 bool launch_attn_enc_tc(const float* Q, const bf16* cache, size_t row_stride, int T_cap,
                         const int32_t* pos, bf16* A, int B, int n, int heads, int dh, int max_keys,
                         int* err, cudaStream_t st);
+// The same over prefixes of any length for d_h = 64 or 128 (k_attn_enc_fa.cu:
+// key tiles of 128, running softmax, O accumulated in tensor memory); false
+// (nothing launched) for other head sizes.
+bool launch_attn_enc_fa(const float* Q, const bf16* cache, size_t row_stride, int T_cap,
+                        const int32_t* pos, bf16* A, int B, int n, int heads, int dh, int* err,
+                        cudaStream_t st);
     // same, for the streaming attention kernels
+
+// Failure-detection self-test (k_selftest.cu): one CTA whose single wait is
+// never satisfied (kind 0: an mbarrier nobody arrives on; kind 1: a global
+// word nobody sets), bounded by `polls` polls; on giving up it writes
+// kDevTimeout to *err.
+void launch_selftest_wait(int kind, uint32_t polls, int* err, cudaStream_t st);
 
 }  // namespace rlt

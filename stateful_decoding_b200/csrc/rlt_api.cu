@@ -1791,6 +1791,14 @@ extern "C" int rlt_state_load(rlt_state* s, int row, const void* src, size_t nby
     return RLT_OK;
 }
 
+extern "C" int rlt_selftest_wait(rlt_state* s, int kind, uint32_t polls, void* stream) {
+    NvtxRange nvtx("rlt_selftest_wait");
+    if (!s || (kind != 0 && kind != 1) || polls == 0 || polls > (1u << 24)) return RLT_E_ARG;
+    if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    rlt::launch_selftest_wait(kind, polls, s->err, (cudaStream_t)stream);
+    return launch_status();
+}
+
 extern "C" int rlt_state_check(rlt_state* s, void* stream) {
     if (!s) return RLT_E_ARG;
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;

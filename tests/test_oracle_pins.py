@@ -199,6 +199,34 @@ def test_layer_split_parameter_deltas():
         assert abs(ours - paper) <= 2 * g["rounding"] + 1e-9, (a, b, ours, paper)
 
 
+def _no_vocab_count(cfg):
+    """Parameters outside the vocabulary matrices (embedding and readout)."""
+    return ri.param_count(cfg) - 2 * cfg.vocab * cfg.d
+
+
+def test_printed_totals_share_one_constant():
+    """Every total the pages print -- RLT-0 4+4 exactly, the five RLT-1 splits
+    and the GPT Layer 8 baseline to 0.01M -- equals our count of the layers,
+    memory and merge plus one constant C shared by all of them (the
+    vocabulary matrices and whatever else the pages' model carries outside
+    the layers).  GPT Layer 8 has the shape of RLT-0 8+0 in our manifest
+    (eight causal self-attention + FFN blocks, no memory, no merge), so its
+    printed count checks the decoder's cross-attention and memory terms
+    against a model without them."""
+    g = json.load(open(os.path.join(GOLDEN, "pages_numbers.json")))
+    C = g["rlt0_params_4p4"]["value"] - _no_vocab_count(_paper_cfg(4, 4, 0))
+    r1 = g["rlt1_params_8layer_M"]
+    for split, want in r1["value"].items():
+        ours = (_no_vocab_count(_paper_cfg(int(split[0]), int(split[2]))) + C) / 1e6
+        assert abs(ours - want) <= r1["rounding"] + 1e-9, (split, ours, want)
+    gpt = g["gpt8_params_M"]
+    ours = (_no_vocab_count(_paper_cfg(8, 0, 0)) + C) / 1e6
+    assert abs(ours - gpt["value"]) <= gpt["rounding"] + 1e-9, ours
+    # the constant is not a whole number of untied (or tied) vocabulary rows
+    # of width 512: 1024 * 141 + 128 -- the departure the readings record
+    assert C == 144512 and C % 512 == 128
+
+
 # ----------------------------------------------------------------------------
 # helpers: closed forms and library routines
 # ----------------------------------------------------------------------------

@@ -198,30 +198,6 @@ def test_fused_projection_norm_kernel(sd, monkeypatch, level):
         assert np.max(np.abs(lg[b] - orc.readout(r))) <= 3e-2
 
 
-def test_full_size_bench_config_sampled_rows(sd):
-    """parity_bf16 at its full size (256 rows x 256) in the bench's launch
-    configuration (one encode call, one prefill call); rows 0, 131 and 255
-    are recomputed by the oracle."""
-    cfg = ri.CONFIGS["parity_bf16"]
-    B, T = cfg.batch, cfg.prompt
-    W, model, st = make(sd, cfg, B, T)
-    toks = ri.make_tokens(cfg)
-    st.encode(toks)
-    st.prefill(T)
-    lg, am, _ = readout_host(st, cfg)
-    s_gpu = state_vec(st, sd.PART_S, B, cfg.d)
-    orc = RLTOracle(cfg, W, "bf16")
-    tally = Tally()
-    for b in (0, 131, 255):
-        r = orc.new_state()
-        orc.encode(r, toks[b])
-        orc.prefill(r, T)
-        ol = orc.readout(r)
-        assert np.max(np.abs(lg[b] - ol)) <= 3e-2
-        np.testing.assert_allclose(s_gpu[b], r.s, atol=0.1, rtol=0)
-        check_argmax(int(am[b]), ol, 3e-2, tally)
-
-
 # ----------------------------------------------------------------------------
 # identities the pages state, on the GPU path itself (bit-exact)
 # ----------------------------------------------------------------------------
