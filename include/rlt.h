@@ -299,6 +299,26 @@ int rlt_state_check(rlt_state* state, void* stream);
  * another kind, or polls outside [1, 2^24]. */
 int rlt_selftest_wait(rlt_state* state, int kind, uint32_t polls, void* stream);
 
+/* Build flags of the loaded library.  RLT_BUILD_DEBUG: built with RLT_DEBUG=1
+ * (librlt_debug.so): the kernels validate every row's position counters
+ * before each encoder and transition block (0 <= pos_dec, pos_dec + n <=
+ * pos_enc <= max_len; pos_enc + n <= max_len when encoding), check ring
+ * slots and key indices where the decode attention forms them, and token
+ * ids as every build does; a violation is recorded in the state's error
+ * word -- rlt_state_check then returns RLT_E_ORDER, RLT_E_CAPACITY or
+ * RLT_E_ARG -- and the access it guards is skipped.  Nothing traps. */
+#define RLT_BUILD_DEBUG 1u
+uint32_t rlt_build_flags(void);
+
+/* Debug builds only: overwrite the DEVICE position counters of one row,
+ * leaving the host's copy unchanged -- a stand-in for a corrupted or stale
+ * device state, for testing the checks above.  Synchronises `stream`.
+ * Returns RLT_E_UNSUPPORTED in other builds; RLT_E_ARG for a null state or a
+ * row outside [0, batch).  A counter past max_len makes the next encode write
+ * past the row's buffers: only a transition or a readout may follow. */
+int rlt_debug_set_positions(rlt_state* state, int row, int32_t pos_enc, int32_t pos_dec,
+                            void* stream);
+
 /* Number of kernels this library has launched in this process. */
 uint64_t rlt_kernel_launches(void);
 

@@ -19,16 +19,21 @@ import re
 from typing import Optional, Sequence
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "librlt.so")
+# RLT_LIB=debug loads the bounds-checking build (librlt_debug.so) instead
+LIB_PATH = os.path.join(_HERE, "librlt_debug.so" if os.environ.get("RLT_LIB") == "debug"
+                        else "librlt.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "rlt.h")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"librlt.so not built at {LIB_PATH}; run `python -m stateful_decoding_b200.build`")
+    raise ImportError(f"{os.path.basename(LIB_PATH)} not built at {LIB_PATH}; run "
+                      f"`python stateful_decoding_b200/build.py`"
+                      f"{' --debug' if LIB_PATH.endswith('_debug.so') else ''}")
 _lib = ctypes.CDLL(LIB_PATH)
 
 RLT_OK, RLT_E_ARG, RLT_E_OOM, RLT_E_CAPACITY, RLT_E_ORDER = 0, -1, -2, -3, -4
 RLT_E_BLOB, RLT_E_DEVICE, RLT_E_TIMEOUT, RLT_E_UNSUPPORTED = -5, -6, -7, -8
 RLT_E_SNAPSHOT = -9
+RLT_BUILD_DEBUG = 1
 SNAPSHOT_HEADER_BYTES = 128                # RLT_SNAPSHOT_HEADER_BYTES
 PART_S, PART_R, PART_E, PART_MEM, PART_RING, PART_ENC = range(6)
 PROF_XATTN, PROF_SWA, PROF_STEP, PROF_ENC = range(4)
@@ -67,6 +72,8 @@ _SIGS = {
     "rlt_snapshot_info": (_i, [_vp, _sz, ctypes.POINTER(rlt_config), ctypes.POINTER(ctypes.c_int32),
                                ctypes.POINTER(ctypes.c_int32)]),
     "rlt_kernel_launches": (_u64, []),
+    "rlt_build_flags": (ctypes.c_uint32, []),
+    "rlt_debug_set_positions": (_i, [_vp, _i, ctypes.c_int32, ctypes.c_int32, _vp]),
     "rlt_strerror": (ctypes.c_char_p, [_i]),
     "rlt_profile_enable": (_i, [_vp, _i]),
     "rlt_profile_query": (_i, [_vp, _i, ctypes.POINTER(_u64), ctypes.POINTER(ctypes.c_double),
@@ -242,6 +249,14 @@ def rlt_state_read(state, part: int, dst=None, nbytes: int = 0, stream=None):
 
 def rlt_state_check(state, stream=None) -> int:
     return _lib.rlt_state_check(state, _stream(stream))
+
+
+def rlt_build_flags() -> int:
+    return _lib.rlt_build_flags()
+
+
+def rlt_debug_set_positions(state, row: int, pos_enc: int, pos_dec: int, stream=None) -> int:
+    return _lib.rlt_debug_set_positions(state, row, pos_enc, pos_dec, _stream(stream))
 
 
 def rlt_selftest_wait(state, kind: int, polls: int, stream=None) -> int:

@@ -1,6 +1,6 @@
 """Build librlt.so (sm_100a) in-tree with nvcc.
 
-    python stateful_decoding_b200/build.py [--force] [--jobs N] [--ptxas-v]
+    python stateful_decoding_b200/build.py [--force] [--jobs N] [--ptxas-v] [--debug]
 
 (Run it by path, or load it with ``load_builder()``: importing the package
 itself loads the library it builds.)
@@ -22,6 +22,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "librlt.so")
+# the bounds-checking variant (RLT_DEBUG=1): same sources, own objects
+DEBUG_BUILD = os.path.join(BUILD, "debug")
+DEBUG_LIB = os.path.join(HERE, "librlt_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -38,8 +41,8 @@ def _headers():
         [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))]
 
 
-def _compile(src: str, force: bool, extra) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, force: bool, extra, outdir: str = BUILD) -> str:
+    obj = os.path.join(outdir, os.path.basename(src)[:-3] + ".o")
     newest = max([os.path.getmtime(src)] + [os.path.getmtime(h) for h in _headers()])
     if not force and os.path.exists(obj) and os.path.getmtime(obj) >= newest:
         return obj
@@ -61,20 +64,24 @@ def load_builder():
     return mod
 
 
-def build(force: bool = False, jobs: int | None = None, extra=()) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, jobs: int | None = None, extra=(), debug: bool = False) -> str:
+    """Build librlt.so, or with debug=True librlt_debug.so (RLT_DEBUG=1: the
+    kernels' bounds checks compiled in)."""
+    outdir, lib = (DEBUG_BUILD, DEBUG_LIB) if debug else (BUILD, LIB)
+    extra = list(extra) + (["-DRLT_DEBUG=1"] if debug else [])
+    os.makedirs(outdir, exist_ok=True)
     srcs = _sources()
     jobs = jobs or min(8, os.cpu_count() or 4)
     with cf.ThreadPoolExecutor(jobs) as ex:
-        objs = list(ex.map(lambda s: _compile(s, force, extra), srcs))
-    if not force and os.path.exists(LIB) and \
-            os.path.getmtime(LIB) >= max(os.path.getmtime(o) for o in objs):
-        return LIB
-    cmd = [NVCC] + ARCH + ["-shared", "-o", LIB] + objs + ["-lcudart", "-lcuda"]
+        objs = list(ex.map(lambda s: _compile(s, force, extra, outdir), srcs))
+    if not force and os.path.exists(lib) and \
+            os.path.getmtime(lib) >= max(os.path.getmtime(o) for o in objs):
+        return lib
+    cmd = [NVCC] + ARCH + ["-shared", "-o", lib] + objs + ["-lcudart", "-lcuda"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
@@ -82,6 +89,8 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--jobs", type=int, default=None)
     ap.add_argument("--ptxas-v", action="store_true", help="print register/smem usage")
+    ap.add_argument("--debug", action="store_true",
+                    help="build librlt_debug.so (RLT_DEBUG=1 bounds checks)")
     a = ap.parse_args()
     extra = ["-Xptxas", "-v"] if a.ptxas_v else []
-    print(build(force=a.force or a.ptxas_v, jobs=a.jobs, extra=extra))
+    print(build(force=a.force or a.ptxas_v, jobs=a.jobs, extra=extra, debug=a.debug))

@@ -40,7 +40,31 @@ __host__ __device__ __forceinline__ uint64_t mix64(uint64_t z) {
 static constexpr uint64_t kGolden = 0x9E3779B97F4A7C15ull;
 
 // Sticky per-state error codes written by device code (0 = none).
-enum DevError : int { kDevOk = 0, kDevTimeout = 1, kDevBounds = 2 };
+enum DevError : int {
+    kDevOk = 0,
+    kDevTimeout = 1,     // a bounded wait gave up
+    kDevBounds = 2,      // a token id outside [0, vocab)
+    kDevOrder = 3,       // debug builds: a block would consume positions not yet encoded
+    kDevCapacity = 4,    // debug builds: a position or ring slot outside its buffer
+};
+
+// RLT_DEBUG=1 (the librlt_debug.so build) compiles in bounds checks of
+// positions, ring slots and key indices; a failed check records its code in
+// the error word (the first code wins) and the access it guards is skipped.
+// Nothing traps.
+#ifndef RLT_DEBUG
+#define RLT_DEBUG 0
+#endif
+__device__ __forceinline__ bool dcheck(bool ok, int* err, int code) {
+#if RLT_DEBUG
+    if (!ok) atomicCAS(err, 0, code);
+    return ok;
+#else
+    (void)err;
+    (void)code;
+    return true;
+#endif
+}
 
 }  // namespace rlt
 

@@ -415,10 +415,15 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
     __shared__ __align__(16) bf16 s_v[DWARPS][DH];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int it = blockIdx.x * DWARPS + warp;
-    const bool live = it < B * heads;
-    const int b = live ? it / heads : 0, h = live ? it % heads : 0;
+    const bool in_range = it < B * heads;
+    const int b = in_range ? it / heads : 0, h = in_range ? it % heads : 0;
     const int d = heads * DH, seg = lane % LPK, grp = lane / LPK;
-    const int pd = live ? __ldcg(pos + b) : 0, t = pd + 1;
+    const int pd = in_range ? __ldcg(pos + b) : 0, t = pd + 1;
+    // debug builds: the position must have rows in the RoPE tables and (for
+    // the memory) keys 1..t inside the buffer; the ring slot pd mod (W-1) is
+    // then inside the ring.  A failed check skips the item.
+    const bool live = in_range && dcheck(pd >= 0 && t <= pin.rope.max_pos && (SWA || t <= span),
+                                         &g_attn_error, kDevCapacity);
     const int nreg = !live ? 0 : (SWA ? (W > 1 ? min(pd, span) : 0) : t);
     const bf16* kg = base + (size_t)b * row_stride + (size_t)h * span * DH + seg * 8;
     const bf16* vg = kg + (size_t)heads * span * DH;
@@ -596,7 +601,11 @@ k_attn_xsplit(const bf16* __restrict__ base, size_t row_stride, int span,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x / heads, h = blockIdx.x % heads;
     const int d = heads * DH, seg = lane % LPK, grp = lane / LPK;
-    const int t = __ldcg(pos + b) + 1;
+    const int t0 = __ldcg(pos + b) + 1;
+    // debug builds: keys 1..t and the RoPE row of t must exist (else no keys)
+    const bool live = dcheck(t0 >= 1 && t0 <= span && t0 <= pin.rope.max_pos, &g_attn_error,
+                             kDevCapacity);
+    const int t = live ? t0 : 0;
     // warp w: keys [jlo, jhi) of the run 0..t-1, parts rounded to whole batches
     const int part = ((t + XS - 1) / XS + BATCH - 1) / BATCH * BATCH;
     const int jlo = min(t, warp * part), jhi = min(t, jlo + part);
@@ -704,7 +713,7 @@ k_attn_xsplit(const bf16* __restrict__ base, size_t row_stride, int span,
     }
     __syncthreads();
     // merge the parts in warp order (part 0 always holds key 1)
-    for (int x = threadIdx.x; x < DH; x += XS * 32) {
+    for (int x = threadIdx.x; live && x < DH; x += XS * 32) {
         float M = s_m[0];
 #pragma unroll
         for (int w = 1; w < XS; ++w) M = fmaxf(M, s_m[w]);

@@ -23,6 +23,7 @@ struct RopeTab {          // cos/sin of p * base^(-2i/dh), p = 0..max_pos, i < d
     const float* cs;      // [max_pos+1][dh/2] cos
     const float* sn;      // [max_pos+1][dh/2] sin
     int half;
+    int max_pos;          // last position with a row in the tables
 };
 
 template <typename T>
@@ -172,5 +173,11 @@ bool launch_attn_enc_fa(const float* Q, const bf16* cache, size_t row_stride, in
 // word nobody sets), bounded by `polls` polls; on giving up it writes
 // kDevTimeout to *err.
 void launch_selftest_wait(int kind, uint32_t polls, int* err, cudaStream_t st);
+
+// Debug builds (RLT_DEBUG=1): validate the rows' position counters before a
+// transition block (encoding = false) or an encoder block of n positions
+// (k_debug.cu); a no-op in other builds.
+void launch_check_positions(const int32_t* pos_enc, const int32_t* pos_dec, int B, int n,
+                            int T_cap, bool encoding, int* err, cudaStream_t st);
 
 }  // namespace rlt

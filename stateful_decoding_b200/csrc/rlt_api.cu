@@ -810,7 +810,7 @@ static int launch_status() {
 }
 
 static rlt::RopeTab rope_of(rlt_state* s) {
-    return rlt::RopeTab{s->rope_cs, s->rope_sn, s->m->dh / 2};
+    return rlt::RopeTab{s->rope_cs, s->rope_sn, s->m->dh / 2, s->T_cap};
 }
 
 // ============================================================================
@@ -904,6 +904,7 @@ static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t s
     T* Hd = (T*)s->Hd;
     T* enc = (T*)s->enc;
     const size_t layer_enc = (size_t)2 * h * s->T_cap * dh;
+    launch_check_positions(s->pos_enc, s->pos_dec, B, n, s->T_cap, true, s->err, st);
     launch_embed<T>((const T*)m->embed, tok, s->X, R, d, c.vocab, s->err, st);
     int max_keys = 0;                        // longest cache prefix any row attends to
     for (int b = 0; b < B; ++b) max_keys = std::max(max_keys, s->h_pos_enc[b] + n);
@@ -1022,6 +1023,7 @@ static void step_block(rlt_state* s, int n, cudaStream_t st, bool merged_in = fa
     };
     // the merge kernel also applies the first decoder block's input RMSNorm
     const float* norm0 = c.n_dec > 0 ? m->dec[0].swa_norm : nullptr;
+    launch_check_positions(s->pos_enc, s->pos_dec, B, n, s->T_cap, false, s->err, st);
     if (c.variant == 0) {
         launch_merge_out<T>(s->e, s->T_cap, s->pos_dec, nullptr, 0, 0, nullptr, nullptr, 0, 0, d,
                             0.f, z, norm0, Y, eps, B, n, d, st);
@@ -1799,6 +1801,21 @@ extern "C" int rlt_selftest_wait(rlt_state* s, int kind, uint32_t polls, void* s
     return launch_status();
 }
 
+extern "C" uint32_t rlt_build_flags(void) { return RLT_DEBUG ? RLT_BUILD_DEBUG : 0u; }
+
+extern "C" int rlt_debug_set_positions(rlt_state* s, int row, int32_t pos_enc, int32_t pos_dec,
+                                       void* stream) {
+    if (!RLT_DEBUG) return RLT_E_UNSUPPORTED;
+    if (!s || row < 0 || row >= s->B) return RLT_E_ARG;
+    if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(s->pos_enc + row, &pos_enc, 4, cudaMemcpyHostToDevice, st) ||
+        cudaMemcpyAsync(s->pos_dec + row, &pos_dec, 4, cudaMemcpyHostToDevice, st) ||
+        cudaStreamSynchronize(st))
+        return RLT_E_DEVICE;
+    return RLT_OK;
+}
+
 extern "C" int rlt_state_check(rlt_state* s, void* stream) {
     if (!s) return RLT_E_ARG;
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
@@ -1813,6 +1830,8 @@ extern "C" int rlt_state_check(rlt_state* s, void* stream) {
     if (w == 0) w = g ? g : (ga ? ga : gp);
     if (w == rlt::kDevTimeout) return RLT_E_TIMEOUT;
     if (w == rlt::kDevBounds) return RLT_E_ARG;
+    if (w == rlt::kDevOrder) return RLT_E_ORDER;
+    if (w == rlt::kDevCapacity) return RLT_E_CAPACITY;
     return w ? RLT_E_DEVICE : RLT_OK;
 }
 
