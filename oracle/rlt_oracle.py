@@ -42,9 +42,14 @@ final encoder norm; the merge reads the raw encoder output e_t; untied readout.
 
 Precision modes.  ``mode="fp64"`` computes everything in float64 on the
 stored weights.  ``mode="bf16"`` rounds, in addition, at exactly the points
-where the bf16 CUDA path stores bf16: every matrix-product input activation,
-and every stored key/value (encoder cache, memory, window cache; the current
-position's key/value are used rounded too).  Everything else stays float64.
+where the bf16 CUDA path stores bf16: every matrix-product input activation
+-- the projections' inputs, and in the encoder's causal attention the query
+and the probabilities, which enter the products q K^T and P V (the
+normaliser then sums the rounded probabilities) -- and every stored
+key/value (encoder cache, memory, window cache; the current position's
+key/value are used rounded too).  The decoder's attention is a matrix-vector
+computation on the CUDA path and keeps q and p unrounded.  Everything else
+stays float64.
 
 Pinning: every function here is checked by ``tests/test_oracle_pins.py``
 against identities the pages state (serving-split invariance, causality,
@@ -100,12 +105,20 @@ def rope(x: np.ndarray, pos: np.ndarray, base: float) -> np.ndarray:
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
 
 
-def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
-    """Per-head softmax attention of one query q[h,dh] over keys K[m,h,dh]."""
+def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, rounded: bool = False) -> np.ndarray:
+    """Per-head softmax attention of one query q[h,dh] over keys K[m,h,dh].
+
+    With ``rounded`` the query and the probabilities exp(s - max s) are bf16
+    values -- they are the inputs of the two matrix products q K^T and P V --
+    and the normaliser is the sum of the rounded probabilities."""
     scale = 1.0 / np.sqrt(q.shape[-1])
+    if rounded:
+        q = round_bf16(q)
     s = np.einsum("hd,mhd->hm", q, K) * scale
     s = s - s.max(axis=1, keepdims=True)
     p = np.exp(s)
+    if rounded:
+        p = round_bf16(p)
     p = p / p.sum(axis=1, keepdims=True)
     return np.einsum("hm,mhd->hd", p, V)
 
@@ -222,7 +235,8 @@ class RLTOracle:
             v = self._store(self._heads(self._lin(y, self._enc(l, "wv"))))
             st.enc_k[l] = np.concatenate([st.enc_k[l], k])
             st.enc_v[l] = np.concatenate([st.enc_v[l], v])
-            a = np.stack([attend(q[i], st.enc_k[l][:p0 + i + 1], st.enc_v[l][:p0 + i + 1])
+            a = np.stack([attend(q[i], st.enc_k[l][:p0 + i + 1], st.enc_v[l][:p0 + i + 1],
+                                 rounded=self.mode == "bf16")
                           for i in range(n)])
             x = x + self._lin(a.reshape(n, c.d), self._enc(l, "wo"))
             y = rmsnorm(x, W[f"enc.{l}.ffn_norm"], c.eps)

@@ -3,8 +3,8 @@
 // the encoder runs in parallel over the known tokens; greeksharifa
 // "Recurrent Looped Transformer 요약 설명" §2.2).  For one (row, head) and a
 // tile of 128 query positions the keys 1..t are visited in tiles of 128:
-// S = Q K^T into tensor memory, a running softmax per query row, P in bf16
-// in shared memory, and O += P V accumulated in tensor memory across tiles.
+// S = Q K^T into tensor memory, P in bf16 in shared memory, and O += P V
+// accumulated in tensor memory across tiles.
 //
 // d_h = 64 or 128.  One CTA of 4 warps; thread r owns query row r (TMEM
 // lane r).  Operands are staged by the threads in the K-major
@@ -12,16 +12,14 @@
 // K copied, V transposed (rows = d_h, keys along K).  Keys past the CTA's
 // last query are staged as zeros and masked by position.
 //
-// Running softmax: each row keeps the maximum m it exponentiates against and
-// the sum l of its rounded probabilities.  A tile only moves m (and rescales
-// the row of O in tensor memory and l by exp(m_old - m_new)) when its maximum
-// exceeds m by more than kRescale; otherwise its probabilities are
-// exp(s - m) <= e^kRescale, well inside fp32 and bf16 range.  The result
-// O / l is the softmax-weighted sum whichever m was used; as in the short
-// kernel, q and the probabilities enter the MMAs rounded to bf16 and l sums
-// the rounded probabilities.  Waits are bounded; a timeout sets the state's
-// error word, ends the key loop for the whole CTA, and the CTA still frees
-// its tensor memory.
+// Exact softmax in two passes over the key tiles: the first forms S tile by
+// tile for each row's maximum m only; the second forms S again, the
+// probabilities exp(s - m) rounded to bf16 (their sum l taken over the
+// rounded values), and O += P V in tensor memory.  The rounding is therefore
+// the short kernel's (k_attn_enc_tc.cu): q and the probabilities enter the
+// MMAs as bf16, everything else stays fp32.  Waits are bounded; a timeout
+// sets the state's error word, ends the key loops for the whole CTA, and the
+// CTA still frees its tensor memory.
 #include <math.h>
 
 #include "kernels.cuh"
@@ -33,7 +31,6 @@ namespace {
 constexpr int FQ = 128;              // query rows per CTA
 constexpr int FK = 128;              // keys per tile
 constexpr int FNT = 128;             // threads
-constexpr float kRescale = 8.0f;     // move the row maximum only past this margin
 
 __device__ __forceinline__ uint32_t sw128(int r, int c) {
     return (uint32_t)r * 128u + (uint32_t)((c ^ (r & 7)) << 4);
@@ -45,26 +42,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 __device__ __forceinline__ void proxy_fence() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// 32 lanes x 32 consecutive 32-bit columns: thread i writes lane (base + i).
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
-        "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
-        "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
-        "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-        "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
-        "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
-        "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
-        "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-        : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
 template <int DH>
 struct FaLayout {
     static constexpr int CH = DH / 64;                          // 64-wide chunks of d_h
@@ -148,13 +125,11 @@ k_attn_enc_fa(const float* __restrict__ Q, const bf16* __restrict__ cache, size_
     const int qpos = p0 + 1 + q0 + r;               // keys 0 .. qpos-1 are visible
     const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
     const float sc = 1.0f / sqrtf((float)DH);
-    float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    uint32_t s_uses = 0;                            // completed phases of bar_s
 
-#pragma unroll 1
-    for (int j = 0; j < ntile; ++j) {
-        const int kb = j * FK;
-        // ---- K tile: eight 16-byte chunks per thread per pass
+    // K tile of keys kb..kb+127: eight 16-byte chunks per thread per pass
+    auto stage_k = [&](int kb) {
 #pragma unroll 1
         for (int e0 = 0; e0 < FK * QC; e0 += FNT * 8) {
             uint4 kv[8];
@@ -171,8 +146,10 @@ k_attn_enc_fa(const float* __restrict__ Q, const bf16* __restrict__ cache, size_
                 *reinterpret_cast<uint4*>(sK + (c >> 3) * L::QK_CHUNK + sw128(k, c & 7)) = kv[u];
             }
         }
-        // ---- V^T tile: a thread takes 8 consecutive keys of one 8-wide
-        // column chunk and writes them as 8 rows (one per d_h index)
+    };
+    // V^T tile: a thread takes 8 consecutive keys of one 8-wide column chunk
+    // and writes them as 8 rows (one per d_h index)
+    auto stage_vt = [&](int kb) {
 #pragma unroll 1
         for (int e = threadIdx.x; e < (FK / 8) * QC; e += FNT) {
             const int kgrp = e / QC, c = e % QC;
@@ -202,13 +179,15 @@ k_attn_enc_fa(const float* __restrict__ Q, const bf16* __restrict__ cache, size_
                     make_uint4(o[0], o[1], o[2], o[3]);
             }
         }
+    };
+    // staged operands -> S = Q K^T (N = 128 keys) in TMEM columns 0..127;
+    // false when the CTA gave up
+    auto scores = [&]() -> bool {
         proxy_fence();
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
-        if (s_abort) break;
-
-        // ---- S = Q K^T (N = 128 keys) into TMEM columns 0..127
+        if (s_abort) return false;
         if (threadIdx.x == 0) {
             constexpr uint32_t idS = idesc_bf16(FQ, FK);
 #pragma unroll
@@ -219,13 +198,21 @@ k_attn_enc_fa(const float* __restrict__ Q, const bf16* __restrict__ cache, size_
             }
             mma_commit(&bar_s);
         }
-        if (!mbar_wait(&bar_s, (uint32_t)j & 1u)) ok = false;
+        if (!mbar_wait(&bar_s, s_uses & 1u)) ok = false;
+        ++s_uses;
         ok = __all_sync(0xffffffffu, ok);
         fence_after_sync();
+        return true;
+    };
 
-        // ---- running softmax of row r over this tile
+    // ---- pass 1: each row's maximum scaled score over its visible keys
+    float m = -INFINITY;
+#pragma unroll 1
+    for (int j = 0; j < ntile; ++j) {
+        const int kb = j * FK;
+        stage_k(kb);
+        if (!scores()) break;
         const int nvis = r < nq ? min(max(qpos - kb, 0), FK) : 0;
-        float mt = -INFINITY;
         if (ok) {
 #pragma unroll 1
             for (int c = 0; c < FK; c += 64) {
@@ -233,32 +220,22 @@ k_attn_enc_fa(const float* __restrict__ Q, const bf16* __restrict__ cache, size_
                 tmem_ld64(trow + (uint32_t)c, v);
 #pragma unroll
                 for (int jj = 0; jj < 64; ++jj)
-                    if (c + jj < nvis) mt = fmaxf(mt, v[jj] * sc);
+                    if (c + jj < nvis) m = fmaxf(m, v[jj] * sc);
             }
         }
-        float corr = 1.f;
-        bool resc = false;
-        if (mt != -INFINITY) {
-            if (m_used == -INFINITY) {
-                m_used = mt;                  // this row's O is still zero
-            } else if (mt > m_used + kRescale) {
-                corr = __expf(m_used - mt);
-                m_used = mt;
-                resc = true;
-            }
-        }
-        l *= corr;
-        if (ok && __any_sync(0xffffffffu, resc)) {
-            // the warp's rows of O scaled in place (warp-collective accesses)
+        if (!ok) s_abort = 1;
+        fence_before_sync();       // the TMEM reads finish before S is overwritten
+    }
+
+    // ---- pass 2: P = bf16(exp(s - m)), l = sum of P, O += P V
+    float l = 0.f;
 #pragma unroll 1
-            for (int c = 0; c < DH; c += 32) {
-                float o[32];
-                tmem_ld32(trow + 128u + (uint32_t)c, o);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) o[i] *= corr;
-                tmem_st32(trow + 128u + (uint32_t)c, o);
-            }
-        }
+    for (int j = 0; j < ntile && !s_abort; ++j) {
+        const int kb = j * FK;
+        stage_k(kb);
+        stage_vt(kb);
+        if (!scores()) break;
+        const int nvis = r < nq ? min(max(qpos - kb, 0), FK) : 0;
         float sum = 0.f;
         if (ok) {
 #pragma unroll 1
@@ -272,8 +249,8 @@ k_attn_enc_fa(const float* __restrict__ Q, const bf16* __restrict__ cache, size_
 #pragma unroll
                     for (int jj = 0; jj < 8; jj += 2) {
                         const int k = 8 * ch + jj;
-                        const float e0 = (c + k < nvis) ? __expf(v[k] * sc - m_used) : 0.f;
-                        const float e1 = (c + k + 1 < nvis) ? __expf(v[k + 1] * sc - m_used) : 0.f;
+                        const float e0 = (c + k < nvis) ? __expf(v[k] * sc - m) : 0.f;
+                        const float e1 = (c + k + 1 < nvis) ? __expf(v[k + 1] * sc - m) : 0.f;
                         __nv_bfloat162 p2 = __floats2bfloat162_rn(e0, e1);
                         sum += __low2float(p2) + __high2float(p2);
                         w[jj / 2] = *reinterpret_cast<uint32_t*>(&p2);

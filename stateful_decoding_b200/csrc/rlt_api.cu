@@ -978,8 +978,10 @@ extern "C" int rlt_encode(rlt_state* s, const int32_t* tokens, int n, void* stre
         }
         int rc = launch_status();
         if (rc) return rc;
+        // the next block's launch shapes (its longest key prefix) read the
+        // host copy of the positions: advance it block by block
+        for (int b = 0; b < s->B; ++b) s->h_pos_enc[b] += nb;
     }
-    for (int b = 0; b < s->B; ++b) s->h_pos_enc[b] += n;
     return RLT_OK;
 }
 

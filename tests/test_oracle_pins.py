@@ -766,6 +766,32 @@ def test_bf16_mode_rounds_every_cache_and_product_input():
         np.testing.assert_array_equal(m._lin(y, name), m._lin(round_bf16(y), name))
     f64 = RLTOracle(cfg, W, "fp64")
     assert not np.array_equal(f64._lin(y, "out"), f64._lin(round_bf16(y), "out"))
+    # the encoder attention's products take a bf16 query and bf16
+    # probabilities: rounding q first changes nothing, the unrounded
+    # attention differs, and one key still returns its value exactly
+    rng = np.random.default_rng(4)
+    q, K, V = rng.normal(size=(2, 8)), rng.normal(size=(5, 2, 8)), rng.normal(size=(5, 2, 8))
+    np.testing.assert_array_equal(attend(q, K, V, rounded=True),
+                                  attend(round_bf16(q), K, V, rounded=True))
+    assert not np.array_equal(attend(q, K, V, rounded=True), attend(q, K, V))
+    np.testing.assert_allclose(attend(q, K[:1], V[:1], rounded=True), V[0], rtol=1e-15)
+    # and encode() uses it in bf16 mode only
+    import oracle.rlt_oracle as ro
+    seen = []
+    real = ro.attend
+
+    def spy(q_, K_, V_, rounded=False):
+        seen.append(rounded)
+        return real(q_, K_, V_, rounded)
+    ro.attend = spy
+    try:
+        m.encode(m.new_state(), toks(cfg, 3))
+        assert seen and all(seen)
+        seen.clear()
+        f64.encode(f64.new_state(), toks(cfg, 3))
+        assert seen and not any(seen)
+    finally:
+        ro.attend = real
 
 
 # ----------------------------------------------------------------------------

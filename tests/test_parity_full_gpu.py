@@ -98,10 +98,50 @@ def test_full_size_bench_launch_sampled_rows(sd, name):
     model.close()
 
 
+def test_encode_split_into_blocks(sd, monkeypatch):
+    """One rlt_encode call split into several encoder blocks (RLT_MAX_ROWS
+    bounds the rows of one block: 4 rows x 200 positions become blocks of 64
+    positions), so later blocks attend over cache prefixes written by earlier
+    blocks of the same call: equal, bit for bit, to the same call as one
+    block, and to the oracle."""
+    cfg = ri.CONFIGS["parity_bf16"]
+    B, T = 4, 200
+    W = ri.generate_weights(cfg)
+    model = sd.Model(ri.write_blob(cfg, W))
+    toks = ri.make_tokens(cfg, B, T)
+    one = sd.State(model, B, T)
+    monkeypatch.setenv("RLT_MAX_ROWS", "256")          # read when a state is created
+    blocks = sd.State(model, B, T)
+    monkeypatch.delenv("RLT_MAX_ROWS")
+    for st in (one, blocks):
+        st.encode(toks)
+        st.prefill(T)
+    l1, _, _ = readout_host(one, cfg)
+    lb, _, _ = readout_host(blocks, cfg)
+    np.testing.assert_array_equal(lb, l1)
+    orc = RLTOracle(cfg, W, "bf16")
+    for b in (0, B - 1):
+        r = orc.new_state()
+        orc.encode(r, toks[b])
+        orc.prefill(r, T)
+        assert np.max(np.abs(lb[b] - orc.readout(r))) <= tol_for(cfg)
+    for st in (one, blocks):
+        st.check()
+        st.close()
+    model.close()
+
+
 def test_large_full_depth_prompt_and_sampled_generation(sd):
     """large_bf16 at full depth on 2 rows: a 256-token prompt encoded and
     prefilled in one call each, then 32 tokens sampled one at a time and fed
-    back (the oracle follows the GPU's ids); every readout compared."""
+    back (the oracle follows the GPU's ids); every readout compared.
+
+    Through 48 bf16 layers the mirrored oracle is itself chaotic at the level
+    of single rounding flips: a second mirror whose embeddings are nudged by a
+    relative 1e-6 (a perturbation the size of fp32 summation-order noise)
+    moves its logits by a floor of ~2-3e-2, the size of the 3e-2 bar.  So
+    each readout must agree within max(3e-2, 2 x that floor), measured at the
+    same readout; the worst gap and the floors are printed."""
     import torch
     cfg = ri.CONFIGS["large_bf16"]
     B, T, G = 2, 256, 32
@@ -109,40 +149,50 @@ def test_large_full_depth_prompt_and_sampled_generation(sd):
     toks = ri.make_tokens(cfg, B, T)
     st.encode(toks)
     st.prefill(T)
-    orc = RLTOracle(cfg, W, "bf16")
-    rows = []
+    Wn = dict(W)
+    Wn["embed"] = W["embed"].astype(np.float64) * (1.0 + 1e-6)
+    orc, nud = RLTOracle(cfg, W, "bf16"), RLTOracle(cfg, Wn, "bf16")
+    rows, rows_n = [], []
     for b in range(B):
-        r = orc.new_state()
-        orc.encode(r, toks[b])
-        orc.prefill(r, T)
-        rows.append(r)
+        for o, lst in ((orc, rows), (nud, rows_n)):
+            r = o.new_state()
+            o.encode(r, toks[b])
+            o.prefill(r, T)
+            lst.append(r)
     tally = Tally()
     tol = tol_for(cfg)
-    errs = []
+    gaps, floors = [], []
     temp = 1.0
     for k in range(G + 1):
         lg, am, sp = readout_host(st, cfg, seed=ri.SAMPLE_SEED, step=k, temperature=temp)
         for b in range(B):
             ol = orc.readout(rows[b])
+            floor = float(np.max(np.abs(nud.readout(rows_n[b]) - ol)))
             err = float(np.max(np.abs(lg[b] - ol)))
-            errs.append(err)
-            assert err <= tol, f"row {b} t={T + k}: |dlogit| {err}"
-            check_argmax(int(am[b]), ol, tol, tally, f"row {b} t={T + k}")
-            check_sample(int(sp[b]), ol, ri.sample_uniform(ri.SAMPLE_SEED, b, k), temp, tol,
+            gaps.append(err)
+            floors.append(floor)
+            bound = max(tol, 2.0 * floor)
+            assert err <= bound, f"row {b} t={T + k}: |dlogit| {err} > {bound} (floor {floor})"
+            check_argmax(int(am[b]), ol, bound, tally, f"row {b} t={T + k}")
+            check_sample(int(sp[b]), ol, ri.sample_uniform(ri.SAMPLE_SEED, b, k), temp, bound,
                          tally, f"row {b} t={T + k}")
         if k == G:
             break
         st.encode(torch.from_numpy(sp.reshape(B, 1)).cuda())
         st.step()
         for b in range(B):
-            orc.encode(rows[b], [int(sp[b])])
-            orc.transition(rows[b])
+            for o, lst in ((orc, rows), (nud, rows_n)):
+                o.encode(lst[b], [int(sp[b])])
+                o.transition(lst[b])
     s_gpu = state_vec(st, sd.PART_S, B, cfg.d)
     rel = max(check_state(s_gpu[b], rows[b].s, f"row {b} s", tol) for b in range(B))
     st.check()
-    print(f"large_bf16 24+24, 2 x (256 + 32): max|dlogit| {max(errs):.3e} (first readout "
-          f"{max(errs[:2]):.3e}, last {max(errs[-2:]):.3e}), |ds|/|s| {rel:.3e}, "
-          f"argmax ties {tally.argmax_ties}, sample ties {tally.sample_ties}")
+    g, f = np.array(gaps), np.array(floors)
+    print(f"large_bf16 24+24, 2 x (256 + 32): GPU vs mirror max|dlogit| {g.max():.3e} "
+          f"(median {np.median(g):.3e}, {int((g > tol).sum())} of {g.size} readouts above "
+          f"{tol}); mirror floor max {f.max():.3e} median {np.median(f):.3e}; worst gap/floor "
+          f"{(g / np.maximum(f, 1e-12)).max():.2f}; |ds|/|s| {rel:.3e}; argmax ties "
+          f"{tally.argmax_ties}, sample ties {tally.sample_ties}")
     st.close()
     model.close()
 
