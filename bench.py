@@ -377,6 +377,14 @@ def run_ours(args, cfg):
     step(toks, logits, ids, am)
     kprof = {name: st.profile_query(cls, stream) for name, cls in
              (("xattn", sd.PROF_XATTN), ("swa", sd.PROF_SWA))}
+    per_layer = {}
+    for name, cls in (("xattn", sd.PROF_XATTN), ("swa", sd.PROF_SWA)):
+        rows = []
+        for lyr in range(cfg.n_dec):
+            n_l, ms_l, by_l = st.profile_query(cls + sd.PROF_NCLS * (lyr + 1), stream)
+            rows.append({"layer": lyr, "avg_us": ms_l / n_l * 1e3 if n_l else None,
+                         "alg_GBps": by_l / ms_l * 1e3 / 1e9 if ms_l else None})
+        per_layer[name] = rows
     st.profile(0)
 
     pk, pk_kind = peaks()
@@ -431,6 +439,7 @@ def run_ours(args, cfg):
                              "alg_GBps": step_gbs, "frac_hbm": step_gbs / pk["hbm_gbs"]},
             "swa": {"launches": n_w, "avg_us": (ms_w / n_w * 1e3) if n_w else None,
                     "alg_GBps": swa_gbs, "frac_hbm": swa_gbs / pk["hbm_gbs"]},
+            "attention_by_layer": per_layer,
             "encoder_ms_per_step": prof["enc"][1] / args.steps,
             "decoder_ms_per_step": ms_s / args.steps,
         },

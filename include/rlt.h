@@ -338,6 +338,8 @@ uint64_t rlt_kernel_launches(void);
 #define RLT_PROF_STEP  2  /* one whole transition block (merge .. s_t)   */
 #define RLT_PROF_ENC   3  /* one whole encoder block (embed .. memory)   */
 #define RLT_PROF_NCLS  4
+/* cls + RLT_PROF_NCLS * (l + 1) queries the window or cross-attention
+ * launches of decoder layer l alone (0 <= l < L_D). */
 int rlt_profile_enable(rlt_state* state, int on);
 int rlt_profile_query(rlt_state* state, int cls, uint64_t* launches, double* total_ms,
                       double* bytes, void* stream);

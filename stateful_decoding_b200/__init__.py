@@ -37,6 +37,7 @@ RLT_BUILD_DEBUG = 1
 SNAPSHOT_HEADER_BYTES = 128                # RLT_SNAPSHOT_HEADER_BYTES
 PART_S, PART_R, PART_E, PART_MEM, PART_RING, PART_ENC = range(6)
 PROF_XATTN, PROF_SWA, PROF_STEP, PROF_ENC = range(4)
+PROF_NCLS = 4          # cls + PROF_NCLS * (layer + 1): one decoder layer's launches
 READOUT_ROWS_SCRATCH_BYTES = 16 << 20      # RLT_READOUT_ROWS_SCRATCH_BYTES
 
 

@@ -12,6 +12,8 @@ namespace rlt {
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
                     int ldct, int M, int N, int K, int mode, int splits, size_t slab,
                     cudaStream_t st);
+bool launch_gemm_tc_runs(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc,
+                         int M, int N, int K, int splits, cudaStream_t st);
 
 static bool tc_enabled() {
     static int v = -1;
@@ -39,7 +41,10 @@ void launch_gemm<bf16>(const bf16* A, int lda, const bf16* W, int ldw, float* C,
 // Split-K partial sums: with `splits` > 1, slab z = C + z*slab holds the sum
 // over the z-th run of K-chunks; the consumer adds the slabs in order.  The
 // split count must depend on N and K only, never on M, so that a row's result
-// does not depend on its batch.  Returns the number of slabs written.
+// does not depend on its batch.  From kRunsRows rows on, one slab holds the
+// runs' sum already (the same additions in the same order, made in the GEMM's
+// epilogue).  Returns the number of slabs written.
+static constexpr int kRunsRows = 1024;
 template <>
 int launch_gemm_split<float>(const float* A, int lda, const float* W, int ldw, float* C, int ldc,
                              int M, int N, int K, int splits, size_t slab, cudaStream_t st) {
@@ -54,6 +59,10 @@ int launch_gemm_split<bf16>(const bf16* A, int lda, const bf16* W, int ldw, floa
                             int M, int N, int K, int splits, size_t slab, cudaStream_t st) {
     if (tc_enabled() && splits > 1 && K % 64 == 0) {
         const int nk = K / 64, cps = (nk + splits - 1) / splits, s = (nk + cps - 1) / cps;
+        // enough rows to fill the machine without splitting CTAs: the runs
+        // stay in tensor memory and one slab holds their ordered sum
+        if (M >= kRunsRows && launch_gemm_tc_runs(A, lda, W, ldw, C, ldc, M, N, K, s, st))
+            return 1;
         if (launch_gemm_tc(A, lda, W, ldw, C, ldc, nullptr, 0, M, N, K, kStoreF32, s, slab, st))
             return s;
     }

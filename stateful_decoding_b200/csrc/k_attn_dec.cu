@@ -581,15 +581,13 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
 }
 
 // One-position cross-attention with the keys of one (row, head) split over
-// the XS warps of a CTA (flash-decoding style), for long memory prefixes with
-// few (row, head) items: warp w streams the w-th contiguous part of keys
-// 1..t exactly as k_attn_dec1 streams a whole run (two batches in flight),
-// then the warps' partial maxima, sums and outputs are merged in warp order.
-// The split depends on t alone, so a row's result does not depend on its
-// batch.
-constexpr int XS = 4;
-
-template <int DH>
+// the XS warps of a CTA (flash-decoding style): warp w streams the w-th
+// contiguous part of keys 1..t exactly as k_attn_dec1 streams a whole run
+// (two batches in flight), then the warps' partial maxima, sums and outputs
+// are merged in warp order.  Each warp's chain of dependent loads is XS
+// times shorter.  The split depends on t and the head size alone, so a row's
+// result does not depend on its batch.
+template <int DH, int XS>
 __global__ void __launch_bounds__(XS * 32)
 k_attn_xsplit(const bf16* __restrict__ base, size_t row_stride, int span,
               const int32_t* __restrict__ pos, bf16* __restrict__ A, int heads, ProjIn pin) {
@@ -828,6 +826,17 @@ bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int 
                                           W, A, B, n, heads, pin, st);
 }
 
+// RLT_XSPLIT=2 or 4: the one-position cross-attention at d_h = 64 splits
+// each (row, head) over that many warps (read once per process).
+static int xsplit64() {
+    static const int v = [] {
+        const char* e = getenv("RLT_XSPLIT");
+        const int x = e ? atoi(e) : 0;
+        return (x == 2 || x == 4) ? x : 0;
+    }();
+    return v;
+}
+
 bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_stride, int T_cap,
                             const int32_t* pos, bf16* A, int B, int n, int heads, int dh,
                             cudaStream_t st) {
@@ -836,8 +845,18 @@ bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_strid
     if (n == 1 && pin.S <= 8 && dh == 128) {
         // the wide heads come with long memory prefixes and few items per
         // launch: split each item's keys over four warps
-        launch(k_attn_xsplit<128>, B * heads, XS * 32, 0, st, mem, row_stride, T_cap, pos, A,
+        launch(k_attn_xsplit<128, 4>, B * heads, 4 * 32, 0, st, mem, row_stride, T_cap, pos, A,
                heads, pin);
+        rlt_count_launch();
+        return true;
+    }
+    if (n == 1 && pin.S <= 8 && dh == 64 && xsplit64() > 1) {
+        if (xsplit64() == 2)
+            launch(k_attn_xsplit<64, 2>, B * heads, 2 * 32, 0, st, mem, row_stride, T_cap, pos,
+                   A, heads, pin);
+        else
+            launch(k_attn_xsplit<64, 4>, B * heads, 4 * 32, 0, st, mem, row_stride, T_cap, pos,
+                   A, heads, pin);
         rlt_count_launch();
         return true;
     }

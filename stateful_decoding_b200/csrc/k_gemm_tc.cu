@@ -39,6 +39,10 @@ constexpr int BM = 128, BK = 64, STAGES = 4, NTHREADS = 192;
 
 template <int BN>
 constexpr uint32_t stage_bytes() { return (uint32_t)(BM * BK * 2 + BN * BK * 2); }
+// TMEM allocations are powers of two of at least 32 columns
+__host__ __device__ constexpr uint32_t tmem_cols(int n) {
+    return n <= 32 ? 32u : n <= 64 ? 64u : n <= 128 ? 128u : n <= 256 ? 256u : 512u;
+}
 template <int BN>
 constexpr size_t smem_bytes() { return (size_t)STAGES * stage_bytes<BN>() + 1024; }
 
@@ -46,7 +50,7 @@ template <int BN, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
           float* __restrict__ C, int ldc, bf16* __restrict__ Ct, int ldct, int M, int N, int K,
-          int cps, size_t slab) {
+          int cps, size_t slab, int tsplit) {
     using namespace tc;
     constexpr uint32_t A_BYTES = BM * BK * 2, STAGE = stage_bytes<BN>();
     extern __shared__ uint8_t smem_raw[];
@@ -58,10 +62,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
     // split-K: this CTA sums K-chunks [kbeg, kbeg+nk) and, with several
-    // splits, writes its partial sums to slab blockIdx.z of C
-    const int kbeg = blockIdx.z * cps;
-    const int nk = min(K / BK - kbeg, cps);
+    // splits, writes its partial sums to slab blockIdx.z of C.  With tsplit
+    // > 1 the CTA takes every K-chunk instead, sums each run of cps chunks in
+    // its own TMEM accumulator, and its epilogue adds the runs in run order
+    // -- the sum a consumer of tsplit slabs forms -- into one slab.
+    const int kbeg = tsplit > 1 ? 0 : blockIdx.z * cps;
+    const int nk = tsplit > 1 ? K / BK : min(K / BK - kbeg, cps);
     C += (size_t)blockIdx.z * slab;
+    const uint32_t tcols = tmem_cols(BN * tsplit);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -76,7 +84,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
         prefetch_map(&ta);
         prefetch_map(&tb);
     }
-    if (warp == 1) tmem_alloc(&tmem_base, BN);
+    if (warp == 1) tmem_alloc(&tmem_base, tcols);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -122,10 +130,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                     break;
                 }
                 const uint32_t a = smem_u32(smem + s * STAGE), b = a + A_BYTES;
+                // run of this chunk (tsplit > 1): its own accumulator, restarted
+                // at the run's first chunk
+                const int run = tsplit > 1 ? kt / cps : 0;
+                const int kin = kt - run * cps;
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
-                    mma_bf16(tmem, sdesc_k_sw128(a + kk * 32), sdesc_k_sw128(b + kk * 32), idesc,
-                             (kt | kk) != 0);
+                    mma_bf16(tmem + (uint32_t)(run * BN), sdesc_k_sw128(a + kk * 32),
+                             sdesc_k_sw128(b + kk * 32), idesc, (kin | kk) != 0);
                 // release the stage only if the producer will refill it
                 if (kt + STAGES < nk) mma_commit(&empty[s]);
             }
@@ -195,6 +207,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                     for (int c = 0; c < BN; c += 64) {
                         float v[64];
                         tmem_ld64(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c, v);
+                        // later runs added in run order (v = ((P0 + P1) + P2) ...)
+                        for (int run = 1; run < tsplit; ++run) {
+                            float w[64];
+                            tmem_ld64(tmem + ((uint32_t)(32 * q) << 16) +
+                                          (uint32_t)(run * BN + c), w);
+#pragma unroll
+                            for (int i = 0; i < 64; ++i) v[i] += w[i];
+                        }
                         float4* d4 = reinterpret_cast<float4*>(stg + (size_t)r * SP + c);
 #pragma unroll
                         for (int u = 0; u < 16; ++u)
@@ -291,7 +311,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
 epilogue_done:
     fence_before_sync();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tmem, BN);
+    if (warp == 1) tmem_dealloc(tmem, tcols);
     if (threadIdx.x == 0 && abort_flag) atomicExch(&g_dev_error, kDevTimeout);
 }
 
@@ -332,17 +352,20 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int ld, in
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// in_tmem: the split runs stay in one CTA's tensor memory (see the kernel)
 template <int BN, int MODE>
 bool launch_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
-               int ldct, int M, int N, int K, int splits, size_t slab, cudaStream_t st) {
+               int ldct, int M, int N, int K, int splits, size_t slab, cudaStream_t st,
+               bool in_tmem = false) {
     CUtensorMap ta, tb;
     if (!make_map(&ta, A, M, K, lda, BM) || !make_map(&tb, W, N, K, ldw, BN)) return false;
     if (!set_smem_once(reinterpret_cast<const void*>(k_gemm_tc<BN, MODE>), smem_bytes<BN>()))
         return false;
-    const int nk = K / BK, cps = (nk + splits - 1) / splits;
-    dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, (nk + cps - 1) / cps);
+    const int nk = K / BK, cps = (nk + splits - 1) / splits, runs = (nk + cps - 1) / cps;
+    if (in_tmem && BN * runs > 512) return false;
+    dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, in_tmem ? 1 : runs);
     launch(k_gemm_tc<BN, MODE>, grid, NTHREADS, smem_bytes<BN>(), st, ta, tb, C, ldc, Ct, ldct, M, N,
-                                                                 K, cps, slab);
+           K, cps, slab, in_tmem ? runs : 1);
     rlt_count_launch();
     return true;
 }
@@ -379,6 +402,19 @@ static bool persist_enabled() {
         return !(e && strcmp(e, "0") == 0);
     }();
     return on;
+}
+
+// A split product of many rows in one slab: 64-wide tiles, every CTA over
+// the whole K range with the split runs in separate TMEM accumulators, added
+// in run order in the epilogue -- bit for bit the sum a consumer of the
+// split's slabs forms, without the slabs.  False when it does not apply.
+bool launch_gemm_tc_runs(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc,
+                         int M, int N, int K, int splits, cudaStream_t st) {
+    if (M <= 0 || N < 16 || K < BK || K % BK || splits < 2) return false;
+    if (lda % 8 || ldw % 8 || ((uintptr_t)A & 15) || ((uintptr_t)W & 15)) return false;
+    if ((ldc & 3) || ((uintptr_t)C & 15) || N % 64) return false;
+    return launch_tc<64, kStoreF32>(A, lda, W, ldw, C, ldc, nullptr, 0, M, N, K, splits, 0, st,
+                                    true);
 }
 
 // Returns false (and launches nothing) when the shape or alignment does not

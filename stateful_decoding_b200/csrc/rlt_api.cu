@@ -576,12 +576,12 @@ struct rlt_state {
     int prof_level = 0;               // 2: also time each attention launch inside the graphs
     // a record holds its events until queried, or (events owned by a graph)
     // the elapsed time read right after the replay
-    struct ProfRec { int cls; cudaEvent_t a, b; double bytes; float ms; };
+    struct ProfRec { int cls; cudaEvent_t a, b; double bytes; float ms; int layer; };
     std::vector<ProfRec> prof_recs;
     std::vector<cudaEvent_t> prof_pool;
     // event pairs captured into a graph (cudaEventRecordExternal nodes), with
     // the index of the block they bracket
-    struct CapRec { int cls; cudaEvent_t a, b; int block; };
+    struct CapRec { int cls; cudaEvent_t a, b; int block; int layer; };
     bool prof_capture = false;
     int prof_block = 0;
     std::vector<CapRec> cap_recs;
@@ -608,9 +608,11 @@ struct ProfScope {
     int cls;
     cudaStream_t st;
     double bytes;
+    int layer;
     cudaEvent_t a = nullptr;
     bool cap = false;
-    ProfScope(rlt_state* s_, int c, cudaStream_t st_, double b) : s(s_), cls(c), st(st_), bytes(b) {
+    ProfScope(rlt_state* s_, int c, cudaStream_t st_, double b, int l = -1)
+        : s(s_), cls(c), st(st_), bytes(b), layer(l) {
         if (s->prof_capture) {          // becomes an event node of the graph being captured
             if (cudaEventCreate(&a) != cudaSuccess) {
                 cudaGetLastError();
@@ -633,13 +635,13 @@ struct ProfScope {
                 return;
             }
             cudaEventRecordWithFlags(b, st, cudaEventRecordExternal);
-            s->cap_recs.push_back({cls, a, b, s->prof_block});
+            s->cap_recs.push_back({cls, a, b, s->prof_block, layer});
             return;
         }
         cudaEvent_t b = prof_event(s);
         if (!b) return;
         cudaEventRecord(b, st);
-        s->prof_recs.push_back({cls, a, b, bytes, -1.f});
+        s->prof_recs.push_back({cls, a, b, bytes, -1.f, layer});
     }
 };
 
@@ -1062,7 +1064,7 @@ static void step_block(rlt_state* s, int n, cudaStream_t st, bool merged_in = fa
         {
             // bf16: the attention kernel forms q, k, v from the slabs and
             // updates the ring itself; otherwise scatter, attend, write
-            ProfScope ps(s, RLT_PROF_SWA, st, s->prof ? swa_bytes(s, n) : 0.0);
+            ProfScope ps(s, RLT_PROF_SWA, st, s->prof ? swa_bytes(s, n) : 0.0, l);
             bool done = false;
             if constexpr (std::is_same<T, bf16>::value)
                 done = launch_attn_swa_proj(ProjIn{P, np, slab, 3 * d, rope_of(s)}, ring,
@@ -1083,7 +1085,7 @@ static void step_block(rlt_state* s, int n, cudaStream_t st, bool merged_in = fa
         np = gemm_p(Y, d, (const T*)L.xq, d, d, P);
         const T* mem = (const T*)s->mem + (c.groups > 1 ? l : 0) * layer_mem;
         {
-            ProfScope ps(s, RLT_PROF_XATTN, st, s->prof ? xattn_bytes(s, n) : 0.0);
+            ProfScope ps(s, RLT_PROF_XATTN, st, s->prof ? xattn_bytes(s, n) : 0.0, l);
             bool done = false;
             if constexpr (std::is_same<T, bf16>::value)
                 done = launch_attn_cross_proj(ProjIn{P, np, slab, d, rope_of(s)}, mem, s->mem_row,
@@ -1236,7 +1238,7 @@ static int run_graph(rlt_state* s, int n, cudaStream_t st) {
             for (int b = 0; b < s->B; ++b) s->h_pos_dec[b] = saved[b] + c.block * n;
             const double cb = c.cls == RLT_PROF_XATTN ? xattn_bytes(s, n)
                               : c.cls == RLT_PROF_SWA ? swa_bytes(s, n) : 0.0;
-            s->prof_recs.push_back({c.cls, nullptr, nullptr, cb, t});
+            s->prof_recs.push_back({c.cls, nullptr, nullptr, cb, t, c.layer});
         }
         s->h_pos_dec = saved;
     }
@@ -1855,13 +1857,16 @@ extern "C" int rlt_profile_enable(rlt_state* s, int on) {
 
 extern "C" int rlt_profile_query(rlt_state* s, int cls, uint64_t* launches, double* total_ms,
                                  double* bytes, void* stream) {
-    if (!s || cls < 0 || cls >= RLT_PROF_NCLS) return RLT_E_ARG;
+    // cls + RLT_PROF_NCLS * (l + 1): the class's launches in decoder layer l only
+    if (!s || cls < 0 || cls >= RLT_PROF_NCLS * (1 + std::max(0, s->m->cfg.n_dec)))
+        return RLT_E_ARG;
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RLT_E_DEVICE;
+    const int base = cls % RLT_PROF_NCLS, want_layer = cls / RLT_PROF_NCLS - 1;
     uint64_t n = 0;
     double ms = 0, by = 0;
     for (auto& r : s->prof_recs) {
-        if (r.cls != cls) continue;
+        if (r.cls != base || (want_layer >= 0 && r.layer != want_layer)) continue;
         float t = r.ms;
         if (!r.a) {                      // resolved right after its graph replay
             ++n;

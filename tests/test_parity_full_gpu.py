@@ -131,6 +131,31 @@ def test_encode_split_into_blocks(sd, monkeypatch):
     model.close()
 
 
+@pytest.mark.parametrize("name,B,T", [("rlt2_mod5_bf16", 300, 12), ("parity_bf16", 1030, 3)])
+def test_many_row_products_match_rows_alone(sd, name, B, T):
+    """From 1024 rows on, a split product keeps its split runs in one CTA's
+    tensor memory and adds them in run order in its epilogue; below, the runs
+    are separate CTAs whose slabs the consumer adds.  The two must agree bit
+    for bit: rows of a big batch (RLT-2 chunks of 4 -> 1200 rows per product;
+    RLT-1, 1030 rows) against the same rows run alone."""
+    cfg = ri.CONFIGS[name]
+    W, model, big = make(sd, cfg, B, T)
+    toks = ri.make_tokens(cfg, B, T)
+    big.encode(toks)
+    big.prefill(T)
+    lbig, _, _ = readout_host(big, cfg)
+    for r in (0, B - 1):
+        one = sd.State(model, 1, T)
+        one.encode(np.ascontiguousarray(toks[r:r + 1]))
+        one.prefill(T)
+        l1, _, _ = readout_host(one, cfg)
+        np.testing.assert_array_equal(l1[0], lbig[r])
+        one.close()
+    big.check()
+    big.close()
+    model.close()
+
+
 def test_large_full_depth_prompt_and_sampled_generation(sd):
     """large_bf16 at full depth on 2 rows: a 256-token prompt encoded and
     prefilled in one call each, then 32 tokens sampled one at a time and fed
