@@ -43,9 +43,10 @@ final encoder norm; the merge reads the raw encoder output e_t; untied readout.
 Precision modes.  ``mode="fp64"`` computes everything in float64 on the
 stored weights.  ``mode="bf16"`` rounds, in addition, at exactly the points
 where the bf16 CUDA path stores bf16: every matrix-product input activation
--- the projections' inputs, and in the encoder's causal attention the query
-and the probabilities, which enter the products q K^T and P V (the
-normaliser then sums the rounded probabilities) -- and every stored
+-- the projections' inputs, and in the encoder's causal attention of a call
+of at least ENC_TC_MIN_POSITIONS tokens the query and the probabilities,
+which enter the products q K^T and P V (the normaliser then sums the
+rounded probabilities) -- and every stored
 key/value (encoder cache, memory, window cache; the current position's
 key/value are used rounded too).  The decoder's attention is a matrix-vector
 computation on the CUDA path and keeps q and p unrounded.  Everything else
@@ -69,6 +70,10 @@ from typing import Dict, List, Optional, Sequence
 
 import numpy as np
 
+
+# Encode calls of at least this many tokens form the encoder attention's
+# products from bf16 q and probabilities in mode "bf16" (see RLTOracle.encode).
+ENC_TC_MIN_POSITIONS = 16
 
 # ----------------------------------------------------------------------------
 # Scalar helpers (float64)
@@ -227,6 +232,11 @@ class RLTOracle:
             return np.zeros((0, c.d))
         p0 = st.pos_enc
         pos = p0 + 1 + np.arange(n)
+        # bf16 mode: calls of at least ENC_TC_MIN_POSITIONS tokens (prompts)
+        # take q and the attention probabilities as bf16 values, where the
+        # bf16 path multiplies them on the tensor cores; shorter calls keep
+        # them unrounded, as its key-streaming kernel does
+        rounded_attn = self.mode == "bf16" and n >= ENC_TC_MIN_POSITIONS
         x = W["embed"][tok].copy()
         for l in range(c.n_enc):
             y = rmsnorm(x, W[f"enc.{l}.attn_norm"], c.eps)
@@ -236,7 +246,7 @@ class RLTOracle:
             st.enc_k[l] = np.concatenate([st.enc_k[l], k])
             st.enc_v[l] = np.concatenate([st.enc_v[l], v])
             a = np.stack([attend(q[i], st.enc_k[l][:p0 + i + 1], st.enc_v[l][:p0 + i + 1],
-                                 rounded=self.mode == "bf16")
+                                 rounded=rounded_attn)
                           for i in range(n)])
             x = x + self._lin(a.reshape(n, c.d), self._enc(l, "wo"))
             y = rmsnorm(x, W[f"enc.{l}.ffn_norm"], c.eps)

@@ -580,6 +580,262 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
     }
 }
 
+// Blocks of NQ = 2..4 positions per row (RLT-2 chunks): one warp per (row,
+// head) as in k_attn_dec1, every key scored against all NQ queries of the
+// block, an online softmax per query.  The window attention takes the ring's
+// keys (query i at t_i = pd+1+i sees positions t_i-W+1 .. t_i, so the oldest
+// slots fall out of the later queries' windows), then the block's own
+// positions e <= i, formed from the projection slabs after the key loop, and
+// finally moves the block's positions into their ring slots -- after every
+// read of the ring (the warp owns its (row, head) ring).  The
+// cross-attention takes memory keys 1..t_i for query i.  Key order and every
+// reduction order depend on positions only.
+constexpr int DRBN = 2;        // rounds per batch for multi-query blocks (registers)
+
+template <int DH, bool SWA, int NQ>
+__global__ void __launch_bounds__(DWARPS * 32)
+k_attn_decn(const bf16* __restrict__ base, size_t row_stride, int span,
+            const int32_t* __restrict__ pos, int W, bf16* __restrict__ A, int B, int heads,
+            ProjIn pin) {
+    constexpr int LPK = DH / 8, KPR = 32 / LPK, HALF = DH / 2;
+    constexpr int BATCH = DRBN * KPR;
+    __shared__ __align__(16) float s_q[DWARPS][NQ][DH];
+    __shared__ __align__(16) bf16 s_k[DWARPS][SWA ? NQ : 1][DH];
+    __shared__ __align__(16) bf16 s_v[DWARPS][SWA ? NQ : 1][DH];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int it = blockIdx.x * DWARPS + warp;
+    const bool in_range = it < B * heads;
+    const int b = in_range ? it / heads : 0, h = in_range ? it % heads : 0;
+    const int d = heads * DH, seg = lane % LPK, grp = lane / LPK;
+    const int pd = in_range ? __ldcg(pos + b) : 0;
+    const bool live = in_range && dcheck(pd >= 0 && pd + NQ <= pin.rope.max_pos &&
+                                             (SWA || pd + NQ <= span),
+                                         &g_attn_error, kDevCapacity);
+    const int nreg = !live ? 0 : (SWA ? (W > 1 ? min(pd, span) : 0) : pd + NQ);
+    const bf16* kg = base + (size_t)b * row_stride + (size_t)h * span * DH + seg * 8;
+    const bf16* vg = kg + (size_t)heads * span * DH;
+    const uint64_t l2pol = SWA ? 0 : l2_evict_last_policy();
+    uint4 kb0[DRBN], vb0[DRBN], kb1[DRBN], vb1[DRBN];
+    auto load_batch = [&](int j0, uint4 (&kb)[DRBN], uint4 (&vb)[DRBN]) {
+#pragma unroll
+        for (int r = 0; r < DRBN; ++r) {
+            const int j = j0 + r * KPR + grp;
+            if (j < nreg) {
+                kb[r] = ld_kv<!SWA>(kg + (size_t)j * DH, l2pol);
+                vb[r] = ld_kv<!SWA>(vg + (size_t)j * DH, l2pol);
+            }
+        }
+    };
+    load_batch(0, kb0, vb0);
+    if (BATCH < nreg) load_batch(BATCH, kb1, vb1);
+    pdl_enter();
+
+    // the block's queries: rows b*NQ + i of the slabs, RoPE at t_i
+    if (live) {
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+            const size_t rb = (size_t)(b * NQ + i) * pin.ldp + h * DH;
+            const float* cs = pin.rope.cs + (size_t)(pd + 1 + i) * HALF;
+            const float* sn = pin.rope.sn + (size_t)(pd + 1 + i) * HALF;
+            for (int j = lane; j < HALF; j += 32) {
+                float y1, y2;
+                rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + j),
+                         slab_sum8(pin.P, pin.S, pin.slab, rb + j + HALF), cs[j], sn[j], y1, y2);
+                s_q[warp][i][j] = y1;
+                s_q[warp][i][j + HALF] = y2;
+            }
+        }
+    }
+    __syncwarp();
+    const float sc = 1.0f / sqrtf((float)DH);
+    float q[NQ][8];
+#pragma unroll
+    for (int i = 0; i < NQ; ++i)
+#pragma unroll
+        for (int x = 0; x < 8; ++x) q[i][x] = s_q[warp][i][seg * 8 + x] * sc;
+    float m[NQ], l[NQ], acc[NQ][8];
+    int lo[NQ];                      // first visible position of query i
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) {
+        m[i] = -INFINITY;
+        l[i] = 0.f;
+        lo[i] = SWA ? max(1, pd + 1 + i - W + 1) : 1;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc[i][x] = 0.f;
+    }
+    // position of run key j: ring slot j holds the newest position <= pd of
+    // its residue; memory key j is position j + 1
+    auto pos_of = [&](int j) -> int { return SWA ? pd - ((pd - 1 - j) % span) : j + 1; };
+    // fold `cnt` keys (their scores per query in s, masked by -inf) into the
+    // per-query state; vf: the keys' values
+    auto fold = [&](float (&s)[NQ][DRBN], const float (&vf)[DRBN][8], int cnt) {
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+            float bm = s[i][0];
+#pragma unroll
+            for (int r = 1; r < DRBN; ++r)
+                if (r < cnt) bm = fmaxf(bm, s[i][r]);
+#pragma unroll
+            for (int o = 16; o >= LPK; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+            const float mn = fmaxf(m[i], bm);
+            if (mn == -INFINITY) continue;            // no visible key yet (warp-uniform)
+            const float corr = (m[i] == -INFINITY) ? 0.f : __expf(m[i] - mn);
+            float ps = 0.f;
+#pragma unroll
+            for (int r = 0; r < DRBN; ++r) {
+                s[i][r] = (r >= cnt || s[i][r] == -INFINITY) ? 0.f : __expf(s[i][r] - mn);
+                ps += s[i][r];
+            }
+#pragma unroll
+            for (int o = 16; o >= LPK; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+            l[i] = l[i] * corr + ps;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                float a = acc[i][x] * corr;
+#pragma unroll
+                for (int r = 0; r < DRBN; ++r) a = fmaf(s[i][r], vf[r][x], a);
+                acc[i][x] = a;
+            }
+            m[i] = mn;
+        }
+    };
+    auto fold_batch = [&](int j0, const uint4 (&kb)[DRBN], const uint4 (&vb)[DRBN]) {
+        float s[NQ][DRBN], vf[DRBN][8];
+#pragma unroll
+        for (int r = 0; r < DRBN; ++r) {
+            const int j = j0 + r * KPR + grp;
+            const bool v = j < nreg;
+            const int p = v ? pos_of(j) : 0;
+            float kf[8] = {};
+            if (v) {
+                unpack8(kb[r], kf);
+                unpack8(vb[r], vf[r]);
+            } else {
+#pragma unroll
+                for (int x = 0; x < 8; ++x) vf[r][x] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) {
+                float dot = 0.f;
+#pragma unroll
+                for (int x = 0; x < 8; ++x) dot = fmaf(q[i][x], kf[x], dot);
+#pragma unroll
+                for (int o = LPK / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                s[i][r] = (v && p >= lo[i] && p <= pd + 1 + i) ? dot : -INFINITY;
+            }
+        }
+        fold(s, vf, DRBN);
+    };
+    for (int j0 = 0; j0 < nreg; j0 += 2 * BATCH) {
+        fold_batch(j0, kb0, vb0);
+        if (j0 + 2 * BATCH < nreg) load_batch(j0 + 2 * BATCH, kb0, vb0);
+        if (j0 + BATCH >= nreg) break;
+        fold_batch(j0 + BATCH, kb1, vb1);
+        if (j0 + 3 * BATCH < nreg) load_batch(j0 + 3 * BATCH, kb1, vb1);
+    }
+    if (SWA && live) {
+        // the block's own keys and values, rounded like the stored ones
+#pragma unroll
+        for (int e = 0; e < NQ; ++e) {
+            const size_t rb = (size_t)(b * NQ + e) * pin.ldp + h * DH;
+            const float* cs = pin.rope.cs + (size_t)(pd + 1 + e) * HALF;
+            const float* sn = pin.rope.sn + (size_t)(pd + 1 + e) * HALF;
+            for (int j = lane; j < HALF; j += 32) {
+                float y1, y2;
+                rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + d + j),
+                         slab_sum8(pin.P, pin.S, pin.slab, rb + d + j + HALF), cs[j], sn[j], y1,
+                         y2);
+                s_k[warp][e][j] = __float2bfloat16_rn(y1);
+                s_k[warp][e][j + HALF] = __float2bfloat16_rn(y2);
+                s_v[warp][e][j] = __float2bfloat16_rn(slab_sum8(pin.P, pin.S, pin.slab, rb + 2 * d + j));
+                s_v[warp][e][j + HALF] =
+                    __float2bfloat16_rn(slab_sum8(pin.P, pin.S, pin.slab, rb + 2 * d + j + HALF));
+            }
+        }
+        __syncwarp();
+        // own position e (t_e = pd+1+e): every lane group scores it, group 0
+        // carries its value (the others add zeros)
+#pragma unroll
+        for (int e = 0; e < NQ; ++e) {
+            float kf[8], s[NQ][DRBN], vf[DRBN][8];
+            unpack8(*reinterpret_cast<const uint4*>(&s_k[warp][e][seg * 8]), kf);
+            unpack8(*reinterpret_cast<const uint4*>(&s_v[warp][e][seg * 8]), vf[0]);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                if (grp != 0) vf[0][x] = 0.f;
+#pragma unroll
+                for (int r = 1; r < DRBN; ++r) vf[r][x] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) {
+                float dot = 0.f;
+#pragma unroll
+                for (int x = 0; x < 8; ++x) dot = fmaf(q[i][x], kf[x], dot);
+#pragma unroll
+                for (int o = LPK / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                // one key per lane group would be counted KPR times: only
+                // group 0 contributes the score to the block max and the sum
+                const bool vis = e <= i && pd + 1 + e >= lo[i];
+                s[i][0] = (vis && grp == 0) ? dot : -INFINITY;
+#pragma unroll
+                for (int r = 1; r < DRBN; ++r) s[i][r] = -INFINITY;
+            }
+            fold(s, vf, 1);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NQ; ++i)
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+#pragma unroll
+            for (int o = 16; o >= LPK; o >>= 1) acc[i][x] += __shfl_xor_sync(0xffffffffu, acc[i][x], o);
+    if (live && grp == 0) {
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+            const float inv = 1.0f / l[i];
+            uint4 w;
+            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                __nv_bfloat162 p2 =
+                    __floats2bfloat162_rn(acc[i][2 * x] * inv, acc[i][2 * x + 1] * inv);
+                wp[x] = *reinterpret_cast<uint32_t*>(&p2);
+            }
+            *reinterpret_cast<uint4*>(A + (size_t)(b * NQ + i) * d + h * DH + seg * 8) = w;
+        }
+        if (SWA && W > 1) {
+            // every read of this head's ring is done: the block's positions
+            // enter slots (pd + e) mod (W-1), the last min(NQ, W-1) of them
+#pragma unroll
+            for (int e = 0; e < NQ; ++e) {
+                if (NQ - e > span) continue;
+                const size_t slot = (size_t)((pd + e) % span) * DH;
+                *reinterpret_cast<uint4*>(const_cast<bf16*>(kg) + slot) =
+                    *reinterpret_cast<const uint4*>(&s_k[warp][e][seg * 8]);
+                *reinterpret_cast<uint4*>(const_cast<bf16*>(vg) + slot) =
+                    *reinterpret_cast<const uint4*>(&s_v[warp][e][seg * 8]);
+            }
+        }
+    }
+}
+
+template <bool SWA>
+bool launch_decn64(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W,
+                   bf16* A, int B, int n, int heads, const ProjIn& pin, cudaStream_t st) {
+    const int grid = (B * heads + DWARPS - 1) / DWARPS;
+    if (n == 2)
+        launch(k_attn_decn<64, SWA, 2>, grid, DWARPS * 32, 0, st, base, row_stride, span, pos, W,
+               A, B, heads, pin);
+    else if (n == 3)
+        launch(k_attn_decn<64, SWA, 3>, grid, DWARPS * 32, 0, st, base, row_stride, span, pos, W,
+               A, B, heads, pin);
+    else
+        launch(k_attn_decn<64, SWA, 4>, grid, DWARPS * 32, 0, st, base, row_stride, span, pos, W,
+               A, B, heads, pin);
+    rlt_count_launch();
+    return true;
+}
+
 // One-position cross-attention with the keys of one (row, head) split over
 // the XS warps of a CTA (flash-decoding style): warp w streams the w-th
 // contiguous part of keys 1..t exactly as k_attn_dec1 streams a whole run
@@ -808,22 +1064,14 @@ bool launch_attn_swa_fast(const float* Q, const bf16* Kc, const bf16* Vc, const 
     return false;
 }
 
-bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int W,
-                          const int32_t* pos, bf16* A, int B, int n, int heads, int dh,
-                          cudaStream_t st) {
-    // one query group per (sequence, head): the kernel then owns every read
-    // and write of that head's ring for the block
-    if (!fast_attn_enabled() || n > 4 || (dh != 64 && dh != 128)) return false;
-    if (B * n <= 0) return true;
-    const int slots = W > 1 ? W - 1 : 1;
-    if (n == 1 && pin.S <= 8)
-        return dh == 64 ? launch_dec1<64, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st)
-                        : launch_dec1<128, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st);
-    if (dh == 64)
-        return launch_stream<64, true, true>(nullptr, ring, row_stride, slots, nullptr, nullptr,
-                                             pos, W, A, B, n, heads, pin, st);
-    return launch_stream<128, true, true>(nullptr, ring, row_stride, slots, nullptr, nullptr, pos,
-                                          W, A, B, n, heads, pin, st);
+// Blocks of 2..4 positions (RLT-2 chunks) on one warp per (row, head);
+// RLT_DECN=0 keeps them on the shared-memory pipeline kernel (read once).
+static bool multi_query_warp() {
+    static const bool on = [] {
+        const char* e = getenv("RLT_DECN");
+        return !(e && strcmp(e, "0") == 0);
+    }();
+    return on;
 }
 
 // RLT_XSPLIT=2 or 4: the one-position cross-attention at d_h = 64 splits
@@ -835,6 +1083,26 @@ static int xsplit64() {
         return (x == 2 || x == 4) ? x : 0;
     }();
     return v;
+}
+
+bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int W,
+                          const int32_t* pos, bf16* A, int B, int n, int heads, int dh,
+                          cudaStream_t st) {
+    // one query group per (sequence, head): the kernel then owns every read
+    // and write of that head's ring for the block
+    if (!fast_attn_enabled() || n > 4 || (dh != 64 && dh != 128)) return false;
+    if (B * n <= 0) return true;
+    const int slots = W > 1 ? W - 1 : 1;
+    if (n == 1 && pin.S <= 8)
+        return dh == 64 ? launch_dec1<64, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st)
+                        : launch_dec1<128, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st);
+    if (dh == 64 && pin.S <= 8 && W > 4 && multi_query_warp())
+        return launch_decn64<true>(ring, row_stride, slots, pos, W, A, B, n, heads, pin, st);
+    if (dh == 64)
+        return launch_stream<64, true, true>(nullptr, ring, row_stride, slots, nullptr, nullptr,
+                                             pos, W, A, B, n, heads, pin, st);
+    return launch_stream<128, true, true>(nullptr, ring, row_stride, slots, nullptr, nullptr, pos,
+                                          W, A, B, n, heads, pin, st);
 }
 
 bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_stride, int T_cap,
@@ -863,6 +1131,8 @@ bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_strid
     if (n == 1 && pin.S <= 8)
         return dh == 64 ? launch_dec1<64, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st)
                         : launch_dec1<128, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st);
+    if (dh == 64 && pin.S <= 8 && n <= 4 && multi_query_warp())
+        return launch_decn64<false>(mem, row_stride, T_cap, pos, 0, A, B, n, heads, pin, st);
     if (dh == 64)
         return launch_stream<64, false, true>(nullptr, mem, row_stride, T_cap, nullptr, nullptr,
                                               pos, 0, A, B, n, heads, pin, st);

@@ -894,8 +894,16 @@ static int max_dec_splits(const rlt_config& c, int fp) {
 // ============================================================================
 // encoder
 // ============================================================================
+// Encode calls of at least this many new positions per row (prompts) run the
+// causal attention on the tensor cores, where q and the probabilities enter
+// the MMAs as bf16; shorter calls (generation steps) stream the keys on the
+// CUDA cores with q and p in fp32 (a 128-row query tile would be mostly
+// empty).
+static constexpr int kEncTcMinPositions = 16;
+
 template <typename T>
-static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t st) {
+static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t st,
+                         bool tc_attn) {
     using namespace rlt;
     rlt_model* m = s->m;
     const rlt_config& c = m->cfg;
@@ -919,7 +927,7 @@ static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t s
                           s->T_cap, B, n, h, dh, st);
         bool attn_done = false;
         if constexpr (std::is_same<T, bf16>::value)
-            attn_done = fast_attn_enabled() &&
+            attn_done = tc_attn && fast_attn_enabled() &&
                         launch_attn_enc_tc(s->Q, enc + l * layer_enc, s->enc_row, s->T_cap,
                                            s->pos_enc, A, B, n, h, dh, max_keys, s->err, st);
         if (!attn_done)
@@ -975,8 +983,9 @@ extern "C" int rlt_encode(rlt_state* s, const int32_t* tokens, int n, void* stre
         if (e != cudaSuccess) return RLT_E_DEVICE;
         {
             ProfScope ps(s, RLT_PROF_ENC, st, s->prof ? enc_bytes(s, nb) : 0.0);
-            if (m->cfg.dtype == RLT_DTYPE_BF16) encode_block<bf16>(s, s->tok, nb, st);
-            else encode_block<float>(s, s->tok, nb, st);
+            const bool tc = n >= kEncTcMinPositions;      // by the call, not the block
+            if (m->cfg.dtype == RLT_DTYPE_BF16) encode_block<bf16>(s, s->tok, nb, st, tc);
+            else encode_block<float>(s, s->tok, nb, st, tc);
         }
         int rc = launch_status();
         if (rc) return rc;

@@ -775,7 +775,8 @@ def test_bf16_mode_rounds_every_cache_and_product_input():
                                   attend(round_bf16(q), K, V, rounded=True))
     assert not np.array_equal(attend(q, K, V, rounded=True), attend(q, K, V))
     np.testing.assert_allclose(attend(q, K[:1], V[:1], rounded=True), V[0], rtol=1e-15)
-    # and encode() uses it in bf16 mode only
+    # and encode() uses it in bf16 mode for calls of at least
+    # ENC_TC_MIN_POSITIONS tokens only
     import oracle.rlt_oracle as ro
     seen = []
     real = ro.attend
@@ -785,10 +786,15 @@ def test_bf16_mode_rounds_every_cache_and_product_input():
         return real(q_, K_, V_, rounded)
     ro.attend = spy
     try:
-        m.encode(m.new_state(), toks(cfg, 3))
+        n_tc = ro.ENC_TC_MIN_POSITIONS
+        st_ = m.new_state()
+        m.encode(st_, toks(cfg, n_tc))
         assert seen and all(seen)
         seen.clear()
-        f64.encode(f64.new_state(), toks(cfg, 3))
+        m.encode(st_, toks(cfg, n_tc - 1))
+        assert seen and not any(seen)
+        seen.clear()
+        f64.encode(f64.new_state(), toks(cfg, n_tc))
         assert seen and not any(seen)
     finally:
         ro.attend = real

@@ -290,8 +290,11 @@ def test_snapshot_continuation_matches_oracle(sd, name):
     orc = RLTOracle(cfg, W, oracle_mode(cfg))
     rows = []
     for i in range(B):
+        # the same encode calls as the GPU's (the bf16 mirror's attention
+        # rounding follows the call size), uninterrupted by any snapshot
         r = orc.new_state()
-        orc.encode(r, toks[src[i]])
+        orc.encode(r, toks[src[i], :P])
+        orc.encode(r, toks[src[i], P:])
         orc.prefill(r, T, chunked=True)
         rows.append(r)
     tally = Tally()
