@@ -43,10 +43,11 @@ final encoder norm; the merge reads the raw encoder output e_t; untied readout.
 Precision modes.  ``mode="fp64"`` computes everything in float64 on the
 stored weights.  ``mode="bf16"`` rounds, in addition, at exactly the points
 where the bf16 CUDA path stores bf16: every matrix-product input activation
--- the projections' inputs, and in the encoder's causal attention of a call
-of at least ENC_TC_MIN_POSITIONS tokens the query and the probabilities,
-which enter the products q K^T and P V (the normaliser then sums the
-rounded probabilities) -- and every stored
+-- the projections' inputs, and in the encoder's causal attention the query
+and the probabilities, which enter the products q K^T and P V (the
+normaliser then sums the rounded probabilities): at head size 64 with
+prefixes of at most 256 keys always, otherwise in calls of at least
+ENC_TC_MIN_POSITIONS tokens -- and every stored
 key/value (encoder cache, memory, window cache; the current position's
 key/value are used rounded too).  The decoder's attention is a matrix-vector
 computation on the CUDA path and keeps q and p unrounded.  Everything else
@@ -72,7 +73,8 @@ import numpy as np
 
 
 # Encode calls of at least this many tokens form the encoder attention's
-# products from bf16 q and probabilities in mode "bf16" (see RLTOracle.encode).
+# products from bf16 q and probabilities in mode "bf16" at any head size and
+# prefix length (see RLTOracle.encode).
 ENC_TC_MIN_POSITIONS = 16
 
 # ----------------------------------------------------------------------------
@@ -232,11 +234,13 @@ class RLTOracle:
             return np.zeros((0, c.d))
         p0 = st.pos_enc
         pos = p0 + 1 + np.arange(n)
-        # bf16 mode: calls of at least ENC_TC_MIN_POSITIONS tokens (prompts)
-        # take q and the attention probabilities as bf16 values, where the
-        # bf16 path multiplies them on the tensor cores; shorter calls keep
-        # them unrounded, as its key-streaming kernel does
-        rounded_attn = self.mode == "bf16" and n >= ENC_TC_MIN_POSITIONS
+        # bf16 mode: q and the attention probabilities are bf16 values where
+        # the bf16 path multiplies them on the tensor cores -- every call at
+        # head size 64 with prefixes of at most 256 keys, and calls of at
+        # least ENC_TC_MIN_POSITIONS tokens otherwise; elsewhere they stay
+        # unrounded, as its key-streaming kernel keeps them
+        rounded_attn = self.mode == "bf16" and (
+            n >= ENC_TC_MIN_POSITIONS or (self.dh == 64 and p0 + n <= 256))
         x = W["embed"][tok].copy()
         for l in range(c.n_enc):
             y = rmsnorm(x, W[f"enc.{l}.attn_norm"], c.eps)

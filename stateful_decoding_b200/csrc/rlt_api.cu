@@ -894,11 +894,13 @@ static int max_dec_splits(const rlt_config& c, int fp) {
 // ============================================================================
 // encoder
 // ============================================================================
-// Encode calls of at least this many new positions per row (prompts) run the
-// causal attention on the tensor cores, where q and the probabilities enter
-// the MMAs as bf16; shorter calls (generation steps) stream the keys on the
-// CUDA cores with q and p in fp32 (a 128-row query tile would be mostly
-// empty).
+// The encoder's causal attention runs on the tensor cores (q and the
+// probabilities enter the MMAs as bf16) with the short kernel whenever
+// d_h = 64 and no row's prefix passes 256 keys, and with the key-tiled
+// kernel (d_h = 128, longer prefixes) for encode calls of at least this many
+// new positions per row (prompts); shorter calls there (generation steps)
+// stream the keys on the CUDA cores with q and p in fp32: the key-tiled
+// kernel would walk every key tile twice for a mostly empty query tile.
 static constexpr int kEncTcMinPositions = 16;
 
 template <typename T>
@@ -927,7 +929,7 @@ static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t s
                           s->T_cap, B, n, h, dh, st);
         bool attn_done = false;
         if constexpr (std::is_same<T, bf16>::value)
-            attn_done = tc_attn && fast_attn_enabled() &&
+            attn_done = (tc_attn || (dh == 64 && max_keys <= 256)) && fast_attn_enabled() &&
                         launch_attn_enc_tc(s->Q, enc + l * layer_enc, s->enc_row, s->T_cap,
                                            s->pos_enc, A, B, n, h, dh, max_keys, s->err, st);
         if (!attn_done)

@@ -775,8 +775,9 @@ def test_bf16_mode_rounds_every_cache_and_product_input():
                                   attend(round_bf16(q), K, V, rounded=True))
     assert not np.array_equal(attend(q, K, V, rounded=True), attend(q, K, V))
     np.testing.assert_allclose(attend(q, K[:1], V[:1], rounded=True), V[0], rtol=1e-15)
-    # and encode() uses it in bf16 mode for calls of at least
-    # ENC_TC_MIN_POSITIONS tokens only
+    # and encode() uses it in bf16 mode: at head size 64 with short prefixes
+    # for any call, otherwise for calls of at least ENC_TC_MIN_POSITIONS
+    # tokens (the pin model's head size is 8, so the call size decides)
     import oracle.rlt_oracle as ro
     seen = []
     real = ro.attend
