@@ -8,7 +8,10 @@
 // in all) and commits it; warps 2-5 drain accumulator j % 2 and apply the
 // epilogue while the MMAs of tile j+1 already run into the other one.  The
 // epilogues are those of k_gemm_tc (fp32 store, fp32 accumulate, SwiGLU over
-// interleaved W1/W3 columns).  Each output element sums its K products in the
+// interleaved W1/W3 columns); each epilogue warp stages 32 rows x 32 columns
+// at a time in shared memory and writes them row segment by row segment
+// (128-byte coalesced stores; the accumulate mode reads z the same way).
+// Each output element sums its K products in the
 // same order as k_gemm_tc, whatever the tile's position.  Waits are bounded:
 // a wait that gives up records a timeout in the device error word, the roles
 // stop, and the CTA still frees its tensor memory.
@@ -23,7 +26,11 @@ namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, NTHREADS = 192;
 constexpr uint32_t A_BYTES = BM * BK * 2, STAGE = BM * BK * 2 + BN * BK * 2;
-constexpr size_t SMEM = (size_t)STAGES * STAGE + 1024;
+// epilogue staging: each epilogue warp passes 32 rows x 32 columns of fp32
+// through shared memory so that global stores cover whole row segments
+constexpr int SPITCH = 36;                       // floats per staged row
+constexpr uint32_t STG_WARP = 32 * SPITCH * 4;   // bytes per epilogue warp
+constexpr size_t SMEM = (size_t)STAGES * STAGE + 4 * STG_WARP + 1024;
 
 __device__ int g_persist_error;
 
@@ -133,8 +140,10 @@ k_gemm_persist(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
             }
             fence_after_sync();
             const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
-            const int row = m0 + 32 * q + lane;
             const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
+            // this warp's staging area: 32 rows x SPITCH floats
+            float* stg = reinterpret_cast<float*>(smem + STAGES * STAGE + q * STG_WARP);
+            const int rbase = m0 + 32 * q;             // first row of this warp
             if (MODE == kSwiGLU) {
 #pragma unroll 1
                 for (int g0 = 0; g0 < BN; g0 += 128) {
@@ -143,25 +152,34 @@ k_gemm_persist(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
                         float a[32], u[32];
                         tmem_ld32(tq + (uint32_t)(g0 + c), a);
                         tmem_ld32(tq + (uint32_t)(g0 + 64 + c), u);
-                        if (row < M) {
-                            uint4* dst = reinterpret_cast<uint4*>(
-                                Ct + (size_t)row * ldct + (n0 + g0) / 2 + c);
+                        // 32 bf16 outputs of this row = 16 words, staged
+                        uint32_t* srow = reinterpret_cast<uint32_t*>(stg) + lane * SPITCH;
 #pragma unroll
-                            for (int h = 0; h < 4; ++h) {
-                                uint4 w;
-                                uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+                        for (int h = 0; h < 4; ++h) {
+                            uint4 w;
+                            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-                                for (int k = 0; k < 4; ++k) {
-                                    const int e = 8 * h + 2 * k;
-                                    const float y0 = a[e] / (1.0f + expf(-a[e])) * u[e];
-                                    const float y1 =
-                                        a[e + 1] / (1.0f + expf(-a[e + 1])) * u[e + 1];
-                                    __nv_bfloat162 p2 = __floats2bfloat162_rn(y0, y1);
-                                    wp[k] = *reinterpret_cast<uint32_t*>(&p2);
-                                }
-                                dst[h] = w;
+                            for (int k = 0; k < 4; ++k) {
+                                const int e = 8 * h + 2 * k;
+                                const float y0 = a[e] / (1.0f + expf(-a[e])) * u[e];
+                                const float y1 = a[e + 1] / (1.0f + expf(-a[e + 1])) * u[e + 1];
+                                __nv_bfloat162 p2 = __floats2bfloat162_rn(y0, y1);
+                                wp[k] = *reinterpret_cast<uint32_t*>(&p2);
                             }
+                            *reinterpret_cast<uint4*>(srow + 4 * h) = w;
                         }
+                        __syncwarp();
+                        // 4 lanes per row (16 bytes each): 8 rows per store
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int rr = 8 * k + (lane >> 2), c4 = lane & 3;
+                            if (rbase + rr < M)
+                                *reinterpret_cast<uint4*>(Ct + (size_t)(rbase + rr) * ldct +
+                                                          (n0 + g0) / 2 + c + 8 * c4) =
+                                    *reinterpret_cast<const uint4*>(
+                                        reinterpret_cast<uint32_t*>(stg) + rr * SPITCH + 4 * c4);
+                        }
+                        __syncwarp();
                     }
                 }
             } else {
@@ -169,21 +187,33 @@ k_gemm_persist(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
                 for (int c = 0; c < BN; c += 64) {
                     float v[64];
                     tmem_ld64(tq + (uint32_t)c, v);
-                    if (row < M) {
-                        float4* dst = reinterpret_cast<float4*>(C + (size_t)row * ldc + n0 + c);
 #pragma unroll
-                        for (int u = 0; u < 16; ++u) {
-                            float4 w = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2],
-                                                   v[4 * u + 3]);
+                    for (int hf = 0; hf < 2; ++hf) {
+                        float* srow = stg + lane * SPITCH;
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            *reinterpret_cast<float4*>(srow + 4 * u) =
+                                make_float4(v[32 * hf + 4 * u], v[32 * hf + 4 * u + 1],
+                                            v[32 * hf + 4 * u + 2], v[32 * hf + 4 * u + 3]);
+                        __syncwarp();
+                        // 8 lanes per row (16 bytes each): 4 rows per store
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const int rr = 4 * k + (lane >> 3), c4 = lane & 7;
+                            if (rbase + rr >= M) continue;
+                            float4 w = *reinterpret_cast<const float4*>(stg + rr * SPITCH + 4 * c4);
+                            float4* dst = reinterpret_cast<float4*>(
+                                C + (size_t)(rbase + rr) * ldc + n0 + c + 32 * hf + 4 * c4);
                             if (MODE == kAddF32) {
-                                const float4 o = dst[u];
+                                const float4 o = *dst;
                                 w.x += o.x;
                                 w.y += o.y;
                                 w.z += o.z;
                                 w.w += o.w;
                             }
-                            dst[u] = w;
+                            *dst = w;
                         }
+                        __syncwarp();
                     }
                 }
             }
