@@ -72,7 +72,7 @@ int launch_gemm_split<bf16>(const bf16* A, int lda, const bf16* W, int ldw, floa
 
 bool launch_gemm_swiglu(const bf16* A, int lda, const bf16* W13, int ldw, bf16* Hd, int ldh, int M,
                         int N, int K, cudaStream_t st) {
-    if (!tc_enabled() || N % 128) return false;
+    if (!tc_enabled() || N % (2 * kW13Block)) return false;
     return launch_gemm_tc(A, lda, W13, ldw, nullptr, 0, Hd, ldh, M, N, K, kSwiGLU, 1, 0, st);
 }
 

@@ -382,10 +382,10 @@ __global__ void __launch_bounds__(256) k_swiglu(const float* __restrict__ H, int
     const int r = blockIdx.x;
     const int j = 4 * (blockIdx.y * blockDim.x + threadIdx.x);
     if (j >= fpad) return;
-    // interleaved W1;W3 (w13_gate_col): 4 consecutive units share a 64-block
+    // interleaved W1;W3 (w13_gate_col): 4 consecutive units share a block
     const size_t base = (size_t)r * 2 * fpad + w13_gate_col(j);
     const float4 a = slab_sum4(H, S, slab, base);
-    const float4 u = slab_sum4(H, S, slab, base + 64);
+    const float4 u = slab_sum4(H, S, slab, base + kW13Block);
     float4 y;
     y.x = a.x / (1.0f + expf(-a.x)) * u.x;
     y.y = a.y / (1.0f + expf(-a.y)) * u.y;

@@ -17,7 +17,6 @@
 // stop, and the CTA still frees its tensor memory.
 #include <cuda.h>
 
-#include "fused.cuh"
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -145,13 +144,14 @@ k_gemm_persist(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
             float* stg = reinterpret_cast<float*>(smem + STAGES * STAGE + q * STG_WARP);
             const int rbase = m0 + 32 * q;             // first row of this warp
             if (MODE == kSwiGLU) {
+                // 64-wide groups (kW13Block = 32): 32 gates, then their 32 ups
 #pragma unroll 1
-                for (int g0 = 0; g0 < BN; g0 += 128) {
-#pragma unroll 1
-                    for (int c = 0; c < 64; c += 32) {
+                for (int g0 = 0; g0 < BN; g0 += 2 * kW13Block) {
+                    {
+                        const int c = 0;
                         float a[32], u[32];
-                        tmem_ld32(tq + (uint32_t)(g0 + c), a);
-                        tmem_ld32(tq + (uint32_t)(g0 + 64 + c), u);
+                        tmem_ld32(tq + (uint32_t)g0, a);
+                        tmem_ld32(tq + (uint32_t)(g0 + kW13Block), u);
                         // 32 bf16 outputs of this row = 16 words, staged
                         uint32_t* srow = reinterpret_cast<uint32_t*>(stg) + lane * SPITCH;
 #pragma unroll

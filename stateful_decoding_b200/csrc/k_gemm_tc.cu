@@ -145,22 +145,22 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
         }
     } else {
         if (MODE == kSwiGLU) {
-            // columns come in 128-wide groups: 64 gates, then the 64 matching
-            // up projections; unit u of group g0 goes to Ct column (n0+g0)/2+u
+            // columns come in 64-wide groups (kW13Block = 32): 32 gates, then
+            // the 32 matching up projections; unit u of group g0 goes to Ct
+            // column (n0+g0)/2+u
             if (mbar_wait(&accum, 0)) {
                 fence_after_sync();
                 const int q = warp & 3;
                 const int row = m0 + 32 * q + lane;
                 const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
-                for (int g0 = 0; g0 < BN; g0 += 128) {
-                    // the group's 64 gates, then its 64 up projections: 16 at a time
-#pragma unroll 1
-                    for (int c = 0; c < 64; c += 32) {
+                for (int g0 = 0; g0 < BN; g0 += 2 * kW13Block) {
+                    {
+                        const int c = 0;
                         float a[32], u[32];
-                        tmem_ld32(tq + (uint32_t)(g0 + c), a);
-                        tmem_ld32(tq + (uint32_t)(g0 + 64 + c), u);
-                        if (row < M && n0 + g0 + 128 <= N) {
+                        tmem_ld32(tq + (uint32_t)g0, a);
+                        tmem_ld32(tq + (uint32_t)(g0 + kW13Block), u);
+                        if (row < M && n0 + g0 + 2 * kW13Block <= N) {
                             uint4* dst = reinterpret_cast<uint4*>(
                                 Ct + (size_t)row * ldct + (n0 + g0) / 2 + c);
 #pragma unroll
@@ -378,7 +378,7 @@ bool launch_tc_mode(const bf16* A, int lda, const bf16* W, int ldw, float* C, in
         return launch_tc<BN, kStoreF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, splits, slab, st);
     if (splits != 1) return false;          // partial sums only go to fp32 slabs
     if (mode == kSwiGLU) {
-        if constexpr (BN % 128 == 0)
+        if constexpr (BN % (2 * kW13Block) == 0)
             return launch_tc<BN, kSwiGLU>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, 1, 0, st);
         return false;
     }
@@ -423,7 +423,8 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, in
                     int ldct, int M, int N, int K, int mode, int splits, size_t slab,
                     cudaStream_t st) {
     if (M <= 0 || N < 16 || K < BK || K % BK || splits < 1) return false;
-    if (mode == kSwiGLU && (N % 128 || (ldct % 8) || ((uintptr_t)Ct & 15))) return false;
+    if (mode == kSwiGLU && (N % (2 * kW13Block) || (ldct % 8) || ((uintptr_t)Ct & 15)))
+        return false;
     if (lda % 8 || ldw % 8 || ((uintptr_t)A & 15) || ((uintptr_t)W & 15)) return false;
     // many rows: the persistent kernel with two accumulators (epilogue of one
     // tile under the MMAs of the next); RLT_GEMM_PERSIST=0 turns it off
@@ -434,10 +435,8 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, in
     // otherwise; the SwiGLU epilogue needs whole 128-column gate/up groups
     if (M >= 2048)
         return launch_tc_mode<256>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, splits, slab, st);
-    if (mode == kSwiGLU) {
-        if (N % 128 || (ldct % 8) || ((uintptr_t)Ct & 15)) return false;
-        return launch_tc_mode<128>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, 1, 0, st);
-    }
+    if (mode == kSwiGLU)        // 64-wide tiles: 32 gates and their 32 ups each
+        return launch_tc_mode<64>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, 1, 0, st);
     return launch_tc_mode<64>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, splits, slab, st);
 }
 

@@ -8,6 +8,8 @@
 // pos[b] + 1 + i).
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace rlt {
@@ -15,9 +17,13 @@ namespace rlt {
 // GEMM epilogues: C (fp32) = acc | C += acc | Ct (storage type) = acc
 enum GemmMode { kStoreF32 = 0, kAddF32 = 1, kStoreT = 2, kSwiGLU = 3 };
 // The fused FFN input projection stores W1 and W3 interleaved in blocks of
-// 64 rows: packed rows [128k, 128k+64) are W1 rows [64k, 64k+64) (gates),
-// rows [128k+64, 128k+128) the W3 rows of the same units.
-__host__ __device__ __forceinline__ int w13_gate_col(int j) { return (j / 64) * 128 + j % 64; }
+// kW13Block rows: packed rows [64k, 64k+32) are W1 rows [32k, 32k+32)
+// (gates), rows [64k+32, 64k+64) the W3 rows of the same units, so any
+// 64-column output tile holds 32 gates and their 32 up projections.
+constexpr int kW13Block = 32;
+__host__ __device__ __forceinline__ int w13_gate_col(int j) {
+    return (j / kW13Block) * 2 * kW13Block + j % kW13Block;
+}
 
 struct RopeTab {          // cos/sin of p * base^(-2i/dh), p = 0..max_pos, i < dh/2
     const float* cs;      // [max_pos+1][dh/2] cos
@@ -36,11 +42,10 @@ void launch_rmsnorm(const float* X, int ldx, const float* gain, T* Y, int ldy, i
 template <typename T>
 void launch_gemm(const T* A, int lda, const T* W, int ldw, float* C, int ldc, T* Ct, int ldct,
                  int M, int N, int K, int mode, cudaStream_t st);
-// z[M, N] += A . W^T and Y = RMSNorm(z) * gain in one kernel (k_gemm_norm.cu;
-// N = d, a cluster of CTAs spans each row block); false (nothing launched)
-// for shapes it does not handle.  err: the state's device error word.
-bool launch_gemm_norm(const bf16* A, int lda, const bf16* W, int ldw, float* Z, const float* gain,
-                      bf16* Y, int M, int N, int K, float eps, int* err, cudaStream_t st);
+// 2-D bf16 TMA map over a row-major [rows][cols] matrix of row pitch ld:
+// boxes of 64 columns (128 bytes, swizzled) x box_rows rows (k_gemm_tc.cu).
+bool make_tma_2d_bf16(CUtensorMap* map, const void* base, int rows, int cols, int ld,
+                      int box_rows);
 // Hd[M, N/2] = SwiGLU of A . W13^T (interleaved W13, N = 2 f_pad) in the
 // tensor-core GEMM's epilogue; false (nothing launched) where unsupported.
 bool launch_gemm_swiglu(const bf16* A, int lda, const bf16* W13, int ldw, bf16* Hd, int ldh, int M,

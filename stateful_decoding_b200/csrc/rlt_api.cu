@@ -23,7 +23,6 @@
 #include <nvtx3/nvToolsExt.h>
 
 #include "../../include/rlt.h"
-#include "fused.cuh"
 #include "kernels.cuh"
 
 // An NVTX range over each public call, so that a profiler's timeline shows
@@ -257,67 +256,11 @@ struct rlt_model {
     float* mem_norm = nullptr;
     std::vector<void*> wmem;        // per group [2d][d]: K rows then V rows
     float *merge_norm = nullptr, *bg = nullptr;
-    void *wg = nullptr, *ws = nullptr, *wgs = nullptr;
+    void* wgs = nullptr;
     std::vector<DecLayerW> dec;
     float* out_norm = nullptr;
     void* wout = nullptr;
-    // fused transition kernel: usable for this model, and its weight maps
-    bool fused = false;
-    rlt::fz::FusedParams fp{};
 };
-
-// The fused transition kernel runs bf16 RLT-1 models of width 512 with 8
-// heads and a 1365/1408-wide FFN (the d=512 workloads).  It is opt-in
-// (RLT_FUSED=1): at 16 sequences per cluster its tensor-core MMAs have
-// N = 16, where a K chunk costs ~0.4 us of issue time, and the per-kernel
-// path with graph replay is faster on the measured workloads.
-static void setup_fused(rlt_model* m) {
-    const rlt_config& c = m->cfg;
-    const char* env = getenv("RLT_FUSED");
-    if (!env || strcmp(env, "1") != 0) return;
-    namespace fz = rlt::fz;
-    if (c.dtype != RLT_DTYPE_BF16 || c.d != fz::D || c.heads != fz::H || m->fpad != fz::FP ||
-        c.variant != 1 || c.n_dec < 1 || c.window < 1)
-        return;
-    const size_t elt = 2, d = c.d, fp = m->fpad;
-    // every decoder kind must be one contiguous [L * rows][cols] matrix
-    for (int l = 1; l < c.n_dec; ++l) {
-        auto at = [&](void* p0, size_t per) { return (uint8_t*)p0 + l * per; };
-        if (m->dec[l].wqkv != at(m->dec[0].wqkv, 3 * d * d * elt) ||
-            m->dec[l].wo != at(m->dec[0].wo, d * d * elt) ||
-            m->dec[l].xq != at(m->dec[0].xq, d * d * elt) ||
-            m->dec[l].xo != at(m->dec[0].xo, d * d * elt) ||
-            m->dec[l].w13 != at(m->dec[0].w13, 2 * fp * d * elt) ||
-            m->dec[l].w2 != at(m->dec[0].w2, d * fp * elt) ||
-            m->dec[l].swa_norm != m->dec[0].swa_norm + l * d ||
-            m->dec[l].x_norm != m->dec[0].x_norm + l * d ||
-            m->dec[l].ffn_norm != m->dec[0].ffn_norm + l * d)
-            return;
-    }
-    fz::FusedParams& p = m->fp;
-    const int L = c.n_dec;
-    bool ok = rlt::make_tma_2d_bf16(&p.m_qkv, m->dec[0].wqkv, L * 3 * fz::D, fz::D, fz::D, 64) &&
-              rlt::make_tma_2d_bf16(&p.m_o, m->dec[0].wo, L * fz::D, fz::D, fz::D, 64) &&
-              rlt::make_tma_2d_bf16(&p.m_xq, m->dec[0].xq, L * fz::D, fz::D, fz::D, 64) &&
-              rlt::make_tma_2d_bf16(&p.m_xo, m->dec[0].xo, L * fz::D, fz::D, fz::D, 64) &&
-              rlt::make_tma_2d_bf16(&p.m_13, m->dec[0].w13, L * 2 * fz::FP, fz::D, fz::D, 64) &&
-              rlt::make_tma_2d_bf16(&p.m_2, m->dec[0].w2, L * fz::D, fz::FP, fz::FP, 64) &&
-              rlt::make_tma_2d_bf16(&p.m_g, m->wg, fz::D, 2 * fz::D, 2 * fz::D, 64) &&
-              rlt::make_tma_2d_bf16(&p.m_s, m->ws, fz::D, fz::D, fz::D, 64);
-    if (!ok) return;
-    p.g_swa = m->dec[0].swa_norm;
-    p.g_x = m->dec[0].x_norm;
-    p.g_ffn = m->dec[0].ffn_norm;
-    p.g_merge = m->merge_norm;
-    p.bg = m->bg;
-    p.L = L;
-    p.W = c.window;
-    p.G = c.groups;
-    p.variant = c.variant;
-    p.alpha = (float)c.alpha;
-    p.eps = (float)c.eps;
-    m->fused = true;
-}
 
 namespace {
 
@@ -420,7 +363,7 @@ extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model
         for (int r = 0; r < c.ffn; ++r) {
             const int gr = rlt::w13_gate_col(r);
             put_mat(ar, o13, elt, w1 + (size_t)r * d * elt, 1, d, d, gr);
-            put_mat(ar, o13, elt, w3 + (size_t)r * d * elt, 1, d, d, gr + 64);
+            put_mat(ar, o13, elt, w3 + (size_t)r * d * elt, 1, d, d, gr + rlt::kW13Block);
         }
     };
     auto ffn = [&](const std::string& p, void** w13, void** w2) {
@@ -436,9 +379,8 @@ extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model
     m->dec.resize(c.n_dec);
     mat_plain("embed", c.vocab, d, &m->embed);
     if (c.variant != 0) vecf("s_star", &m->s_star);
-    // decoder weights kind by kind, so that each kind is one [L_D * rows][cols]
-    // matrix (every per-layer size is a multiple of the 256-byte arena step):
-    // the fused transition kernel addresses all layers through one tensor map
+    // decoder weights kind by kind: each kind is one [L_D * rows][cols] matrix
+    // (every per-layer size is a multiple of the 256-byte arena step)
     auto dec_p = [&](int l) { return "dec." + std::to_string(l) + "."; };
     for (int l = 0; l < c.n_dec; ++l) vecf(dec_p(l) + "swa_norm", &m->dec[l].swa_norm);
     for (int l = 0; l < c.n_dec; ++l) vecf(dec_p(l) + "x_norm", &m->dec[l].x_norm);
@@ -485,8 +427,6 @@ extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model
     if (c.variant != 0) {
         vecf("merge.norm", &m->merge_norm);
         vecf("merge.bg", &m->bg);
-        mat_plain("merge.wg", d, 2 * d, &m->wg);
-        mat_plain("merge.ws", d, d, &m->ws);
         // both merge projections as one [2d][2d] matrix over [e_t; r]: rows
         // 0..d-1 are W_g, rows d..2d-1 are [0 | W_s] (one GEMM launch)
         size_t og = a.take((size_t)4 * d * d * elt);
@@ -524,7 +464,6 @@ extern "C" int rlt_create(const void* blob, size_t nbytes, int device, rlt_model
             m->enc[l].w2 = m->dec[l].w2;
         }
     }
-    setup_fused(m);
     *out = m;
     return RLT_OK;
 }
@@ -571,7 +510,6 @@ struct rlt_state {
     std::vector<void*> allocs;
     size_t bytes = 0;
     // live timing (rlt_profile_*)
-    int norm_fuse = 0;                // see norm_fuse_from_env
     bool prof = false;
     int prof_level = 0;               // 2: also time each attention launch inside the graphs
     // a record holds its events until queried, or (events owned by a graph)
@@ -680,7 +618,6 @@ extern "C" void rlt_state_destroy(rlt_state* s) {
 }
 
 static int max_dec_splits(const rlt_config& c, int fp);
-static int norm_fuse_from_env();
 
 static size_t max_rows_per_call() {
     const char* v = getenv("RLT_MAX_ROWS");
@@ -707,7 +644,6 @@ extern "C" int rlt_state_create(rlt_model* m, int batch, int max_len, rlt_state*
     s->m = m;
     s->B = batch;
     s->T_cap = max_len;
-    s->norm_fuse = norm_fuse_from_env();
     const size_t elt = m->elt, d = c.d, dh = m->dh, h = c.heads, B = batch, T = max_len;
     const size_t slots = (size_t)std::max(0, c.window - 1);
     size_t maxr = max_rows_per_call();
@@ -1001,15 +937,6 @@ extern "C" int rlt_encode(rlt_state* s, const int32_t* tokens, int n, void* stre
 // ============================================================================
 // transition
 // ============================================================================
-// RLT_NORM_FUSE (read when a state is created): 0 (default) = split-K GEMM
-// and a row kernel for each residual projection and the RMSNorm after it;
-// 1 = one clustered kernel (k_gemm_norm.cu) for the attention output
-// projections; 2 = also for W_2.  Measured on B200 at 256 rows the clustered
-// kernel is slower (16 CTAs each running the whole K range), so it is opt-in.
-static int norm_fuse_from_env() {
-    const char* e = getenv("RLT_NORM_FUSE");
-    return e ? atoi(e) : 0;
-}
 // merged_in: the previous block already wrote this block's merge input (Y);
 // fuse_out: end with the state hand-off fused with the next block's merge
 // input (one position per row, RLT-1/2, inside a replayed run of blocks).
@@ -1055,22 +982,12 @@ static void step_block(rlt_state* s, int n, cudaStream_t st, bool merged_in = fa
     }
     const size_t layer_ring = (size_t)2 * h * std::max(0, c.window - 1) * dh;
     const size_t layer_mem = (size_t)2 * h * s->T_cap * dh;
-    // residual projection + the RMSNorm after it in one clustered kernel
-    // (level 1: attention output projections; level 2: also W_2)
-    const int fuse = s->norm_fuse;
-    auto proj_norm = [&](const T* Ain, int lda, const T* Wt, int K, const float* gain) -> bool {
-        if constexpr (std::is_same<T, bf16>::value)
-            return launch_gemm_norm(Ain, lda, Wt, K, z, gain, Y, R, d, K, eps, s->err, st);
-        return false;
-    };
     int nres = 0;                       // pending residual partial slabs in P
-    bool normed = false;                // Y already holds this block's input norm
     for (int l = 0; l < c.n_dec; ++l) {
         const DecLayerW& L = m->dec[l];
         T* ring = (T*)s->ring + l * layer_ring;
-        if (l > 0 && !normed)
+        if (l > 0)
             launch_add_rmsnorm<T>(z, nres ? P : nullptr, nres, slab, L.swa_norm, Y, R, d, eps, st);
-        normed = false;
         int np = gemm_p(Y, d, (const T*)L.wqkv, 3 * d, d, P);
         {
             // bf16: the attention kernel forms q, k, v from the slabs and
@@ -1089,10 +1006,8 @@ static void step_block(rlt_state* s, int n, cudaStream_t st, bool merged_in = fa
                                      st);
             }
         }
-        if (!(fuse >= 1 && proj_norm(A, d, (const T*)L.wo, d, L.x_norm))) {
-            nres = gemm_p(A, d, (const T*)L.wo, d, d, P);
-            launch_add_rmsnorm<T>(z, P, nres, slab, L.x_norm, Y, R, d, eps, st);
-        }
+        nres = gemm_p(A, d, (const T*)L.wo, d, d, P);
+        launch_add_rmsnorm<T>(z, P, nres, slab, L.x_norm, Y, R, d, eps, st);
         np = gemm_p(Y, d, (const T*)L.xq, d, d, P);
         const T* mem = (const T*)s->mem + (c.groups > 1 ? l : 0) * layer_mem;
         {
@@ -1107,27 +1022,20 @@ static void step_block(rlt_state* s, int n, cudaStream_t st, bool merged_in = fa
                                      st);
             }
         }
-        if (!(fuse >= 1 && proj_norm(A, d, (const T*)L.xo, d, L.ffn_norm))) {
-            nres = gemm_p(A, d, (const T*)L.xo, d, d, P);
-            launch_add_rmsnorm<T>(z, P, nres, slab, L.ffn_norm, Y, R, d, eps, st);
-        }
-        // SwiGLU in the GEMM epilogue only when the rows alone fill the
-        // machine: at a few hundred rows the split-K GEMM plus a row kernel
-        // is faster (measured on B200)
+        nres = gemm_p(A, d, (const T*)L.xo, d, d, P);
+        launch_add_rmsnorm<T>(z, P, nres, slab, L.ffn_norm, Y, R, d, eps, st);
+        // SwiGLU in the GEMM epilogue whenever W1;W3 is not split (64-wide
+        // tiles hold 32 gates and their ups); a split product goes through
+        // its slabs and the row kernel
         bool ffn_done = false;
         if constexpr (std::is_same<T, bf16>::value)
-            ffn_done = R >= 2048 &&
+            ffn_done = (R >= 2048 || dec_splits(s, 2 * fp, d) == 1) &&
                        launch_gemm_swiglu(Y, d, (const bf16*)L.w13, d, Hd, fp, R, 2 * fp, d, st);
         if (!ffn_done) {
             np = gemm_p(Y, d, (const T*)L.w13, 2 * fp, d, P);
             launch_swiglu<T>(P, np, slab, fp, Hd, R, st);
         }
-        nres = 0;
-        if (fuse >= 2 && l + 1 < c.n_dec &&
-            proj_norm(Hd, fp, (const T*)L.w2, fp, m->dec[l + 1].swa_norm))
-            normed = true;              // the next block's input norm is done
-        else
-            nres = gemm_p(Hd, fp, (const T*)L.w2, d, fp, P);
+        nres = gemm_p(Hd, fp, (const T*)L.w2, d, fp, P);
     }
     if (fuse_out)
         launch_state_merge<T>(z, nres ? P : nullptr, nres, slab, s->s,
@@ -1257,48 +1165,10 @@ static int run_graph(rlt_state* s, int n, cudaStream_t st) {
     return RLT_OK;
 }
 
-// nsteps transitions of every row through the fused kernel (one launch).
-static int run_fused(rlt_state* s, int nsteps, cudaStream_t st) {
-    for (int b = 0; b < s->B; ++b) {
-        if (s->h_pos_dec[b] + nsteps > s->h_pos_enc[b]) return RLT_E_ORDER;
-        if (s->h_pos_dec[b] + nsteps > s->T_cap) return RLT_E_CAPACITY;
-    }
-    rlt::fz::FusedParams p = s->m->fp;
-    p.e = s->e;
-    p.s = s->s;
-    p.pos_dec = s->pos_dec;
-    p.err = s->err;
-    p.mem = (const bf16*)s->mem;
-    p.ring = (bf16*)s->ring;
-    p.rope_cs = s->rope_cs;
-    p.rope_sn = s->rope_sn;
-    p.mem_row = s->mem_row;
-    p.ring_row = s->ring_row;
-    p.B = s->B;
-    p.T_cap = s->T_cap;
-    p.nsteps = nsteps;
-    double by = 0;
-    if (s->prof) {
-        std::vector<int32_t> saved = s->h_pos_dec;
-        for (int k = 0; k < nsteps; ++k) {
-            by += step_bytes(s, 1);
-            for (int b = 0; b < s->B; ++b) s->h_pos_dec[b] += 1;
-        }
-        s->h_pos_dec = saved;
-    }
-    {
-        ProfScope ps(s, RLT_PROF_STEP, st, by);
-        if (!rlt::launch_dec_fused(p, st)) return RLT_E_DEVICE;
-    }
-    for (int b = 0; b < s->B; ++b) s->h_pos_dec[b] += nsteps;
-    return RLT_OK;
-}
-
 extern "C" int rlt_step(rlt_state* s, void* stream) {
     NvtxRange nvtx("rlt_step");
     if (!s) return RLT_E_ARG;
     if (cudaSetDevice(s->m->device) != cudaSuccess) return RLT_E_DEVICE;
-    if (s->m->fused) return run_fused(s, 1, (cudaStream_t)stream);
     return run_block(s, 1, (cudaStream_t)stream);
 }
 
@@ -1312,7 +1182,6 @@ extern "C" int rlt_prefill(rlt_state* s, int T, void* stream) {
         if (s->h_pos_dec[b] + T > s->T_cap) return RLT_E_CAPACITY;
     }
     const cudaStream_t st = (cudaStream_t)stream;
-    if (s->m->fused) return T > 0 ? run_fused(s, T, st) : RLT_OK;
     int done = 0;
     while (done < T) {
         const int pd = s->h_pos_dec[0];
@@ -1440,7 +1309,7 @@ extern "C" int rlt_replay_logprobs(rlt_state* s, const int32_t* tokens, int n, f
         rlt::launch_logprob(s->logits, V, B, ids + j, n, out + j, n, temperature, s->err, st);
         rc = launch_status();
         if (rc) return rc;
-        rc = s->m->fused ? run_fused(s, 1, st) : run_block(s, 1, st);
+        rc = run_block(s, 1, st);
         if (rc) return rc;
     }
     if (!odev) {

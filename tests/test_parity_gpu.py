@@ -154,50 +154,6 @@ def test_large_config_slice(sd):
     run_stepwise_and_compare(sd, cfg, 2, 12, n_decode=2)
 
 
-def test_fused_transition_kernel(sd, monkeypatch):
-    """The opt-in fused cluster kernel (RLT_FUSED=1) against the oracle on a
-    ragged batch (20 rows: one full and one partial 16-row cluster), stepwise
-    and through one prefill launch."""
-    monkeypatch.setenv("RLT_FUSED", "1")
-    cfg = ri.CONFIGS["parity_bf16"]
-    run_stepwise_and_compare(sd, cfg, 20, 21, n_decode=1)
-    B, T = 20, 33
-    W, model, st = make(sd, cfg, B, T)
-    toks = ri.make_tokens(cfg, B, T)
-    st.encode(toks)
-    st.prefill(T)
-    lg, _, _ = readout_host(st, cfg)
-    orc = RLTOracle(cfg, W, "bf16")
-    for b in (0, 17, 19):
-        r = orc.new_state()
-        orc.encode(r, toks[b])
-        orc.prefill(r, T)
-        assert np.max(np.abs(lg[b] - orc.readout(r))) <= 3e-2
-
-
-@pytest.mark.parametrize("level", [1, 2])
-def test_fused_projection_norm_kernel(sd, monkeypatch, level):
-    """The opt-in clustered projection + RMSNorm kernel (RLT_NORM_FUSE=1: the
-    attention output projections; 2: also W_2) against the oracle, stepwise
-    on a ragged batch (two 128-row tiles, the second partial) and through
-    one prefill."""
-    monkeypatch.setenv("RLT_NORM_FUSE", str(level))
-    cfg = ri.CONFIGS["parity_bf16"]
-    run_stepwise_and_compare(sd, cfg, 3, 13, n_decode=1)
-    B, T = 130, 9
-    W, model, st = make(sd, cfg, B, T)
-    toks = ri.make_tokens(cfg, B, T)
-    st.encode(toks)
-    st.prefill(T)
-    lg, _, _ = readout_host(st, cfg)
-    orc = RLTOracle(cfg, W, "bf16")
-    for b in (0, 129):
-        r = orc.new_state()
-        orc.encode(r, toks[b])
-        orc.prefill(r, T)
-        assert np.max(np.abs(lg[b] - orc.readout(r))) <= 3e-2
-
-
 # ----------------------------------------------------------------------------
 # identities the pages state, on the GPU path itself (bit-exact)
 # ----------------------------------------------------------------------------
