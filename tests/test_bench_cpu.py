@@ -1,5 +1,6 @@
-"""The bench's reference arm on CPU: the float64 oracle timed on the host
-cores, printed as one JSON line of the bench contract."""
+"""The bench's reference arm on CPU: the float64 oracle timed on all host
+cores (one spawned process per core over rows), printed as one JSON line of
+the bench contract."""
 import contextlib
 import io
 import json
@@ -34,6 +35,10 @@ def test_reference_arm_line(monkeypatch):
     assert line["config"]["workload"].startswith("tiny_fp32")
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    # the core count is the number of oracle processes that ran (one per host
+    # core unless host memory bounds them), each on one BLAS thread
+    assert cb["cores"] == bench.oracle_processes(cfg) <= (os.cpu_count() or 1)
+    assert "one process per core" in cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s",
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
