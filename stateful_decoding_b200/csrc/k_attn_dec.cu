@@ -847,7 +847,10 @@ bool launch_decn64(const bf16* base, size_t row_stride, int span, const int32_t*
 // are merged in warp order.  Each warp's chain of dependent loads is XS
 // times shorter.  The split depends on t and the head size alone, so a row's
 // result does not depend on its batch.
-template <int DH, int XS>
+// QIN: the query is read ready-rotated from an fp32 [B][d] buffer (pin.P,
+// row pitch pin.ldp) -- the encoder's generation steps -- instead of being
+// formed from projection slabs.
+template <int DH, int XS, bool QIN = false>
 __global__ void __launch_bounds__(XS * 32)
 k_attn_xsplit(const bf16* __restrict__ base, size_t row_stride, int span,
               const int32_t* __restrict__ pos, bf16* __restrict__ A, int heads, ProjIn pin) {
@@ -887,7 +890,10 @@ k_attn_xsplit(const bf16* __restrict__ base, size_t row_stride, int span,
 
     // q: formed once by warp 0 (rotate-half pairs at position t, slab sums in
     // slab order), shared by the four warps
-    if (warp == 0) {
+    if (QIN) {
+        for (int j = threadIdx.x; j < DH; j += XS * 32)
+            s_q[j] = pin.P[(size_t)b * pin.ldp + h * DH + j];
+    } else if (warp == 0) {
         const size_t rb = (size_t)b * pin.ldp + h * DH;
         const float* cs = pin.rope.cs + (size_t)t * HALF;
         const float* sn = pin.rope.sn + (size_t)t * HALF;
@@ -1107,6 +1113,29 @@ bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int 
                                              pos, W, A, B, n, heads, pin, st);
     return launch_stream<128, true, true>(nullptr, ring, row_stride, slots, nullptr, nullptr, pos,
                                           W, A, B, n, heads, pin, st);
+}
+
+bool launch_attn_enc_step(const float* Q, const bf16* cache, size_t row_stride, int T_cap,
+                          const int32_t* pos_enc, bf16* A, int B, int heads, int dh,
+                          cudaStream_t st) {
+    // one new position per row over a long cache prefix, d_h = 128: the
+    // split-key kernel, the query already rotated in Q (RLT_ENC_STEP=stream
+    // keeps these on the shared-memory pipeline kernel; read once)
+    static const bool on = [] {
+        const char* e = getenv("RLT_ENC_STEP");
+        return !(e && strcmp(e, "stream") == 0);
+    }();
+    if (!on || !fast_attn_enabled() || dh != 128) return false;
+    if (B <= 0) return true;
+    ProjIn pin{};
+    pin.P = Q;
+    pin.S = 1;
+    pin.ldp = heads * dh;
+    pin.rope.max_pos = T_cap;
+    launch(k_attn_xsplit<128, 4, true>, B * heads, 4 * 32, 0, st, cache, row_stride, T_cap,
+           pos_enc, A, heads, pin);
+    rlt_count_launch();
+    return true;
 }
 
 bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_stride, int T_cap,

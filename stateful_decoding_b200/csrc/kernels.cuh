@@ -171,6 +171,12 @@ bool launch_attn_enc_tc(const float* Q, const bf16* cache, size_t row_stride, in
 bool launch_attn_enc_fa(const float* Q, const bf16* cache, size_t row_stride, int T_cap,
                         const int32_t* pos, bf16* A, int B, int n, int heads, int dh, int* err,
                         cudaStream_t st);
+// The encoder's attention for one new position per row at d_h = 128 (the
+// large model's generation steps): keys split over 4 warps per (row, head),
+// q read rotated from Q; false (nothing launched) for other head sizes.
+bool launch_attn_enc_step(const float* Q, const bf16* cache, size_t row_stride, int T_cap,
+                          const int32_t* pos_enc, bf16* A, int B, int heads, int dh,
+                          cudaStream_t st);
     // same, for the streaming attention kernels
 
 // Failure-detection self-test (k_selftest.cu): one CTA whose single wait is

@@ -868,6 +868,10 @@ static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t s
             attn_done = (tc_attn || (dh == 64 && max_keys <= 256)) && fast_attn_enabled() &&
                         launch_attn_enc_tc(s->Q, enc + l * layer_enc, s->enc_row, s->T_cap,
                                            s->pos_enc, A, B, n, h, dh, max_keys, s->err, st);
+        if constexpr (std::is_same<T, bf16>::value)
+            if (!attn_done && n == 1)
+                attn_done = launch_attn_enc_step(s->Q, enc + l * layer_enc, s->enc_row, s->T_cap,
+                                                 s->pos_enc, A, B, h, dh, st);
         if (!attn_done)
             launch_attn_enc<T>(s->Q, enc + l * layer_enc, s->enc_row, s->T_cap, s->pos_enc, A, B,
                                n, h, dh, st);
