@@ -344,7 +344,7 @@ def run_ours(args, cfg):
     launches = sd.rlt_kernel_launches() - launches0
     prof = {name: st.profile_query(cls, stream) for name, cls in
             (("xattn", sd.PROF_XATTN), ("swa", sd.PROF_SWA), ("step", sd.PROF_STEP),
-             ("enc", sd.PROF_ENC))}
+             ("enc", sd.PROF_ENC), ("enc1", sd.PROF_ENC1))}
     st.profile(False)
     ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / args.steps
@@ -392,6 +392,10 @@ def run_ours(args, cfg):
     step_gbs = (by_s / ms_s * 1e3 / 1e9) if ms_s else 0.0
     enc_ms = prof["enc"][1] / args.steps
     enc_tf = encoder_flops(cfg, B, T) / (enc_ms / 1e3) / 1e12 if enc_ms else 0.0
+    # the one-position encoder calls of the generation loop: HBM-bound reads
+    # of the cached keys and values (weights not counted)
+    n_e1, ms_e1, by_e1 = prof["enc1"]
+    enc1_gbs = (by_e1 / ms_e1 * 1e3 / 1e9) if ms_e1 else 0.0
     tc_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
     n, ms, by = kprof["xattn"]
     kname = "decoder cross-attention (k_attn_dec1: one warp per (row, head), q from the projection slabs)"
@@ -440,10 +444,18 @@ def run_ours(args, cfg):
             "swa": {"launches": n_w, "avg_us": (ms_w / n_w * 1e3) if n_w else None,
                     "alg_GBps": swa_gbs, "frac_hbm": swa_gbs / pk["hbm_gbs"]},
             "attention_by_layer": per_layer,
-            "encoder_ms_per_step": prof["enc"][1] / args.steps,
+            "encoder_ms_per_step": (prof["enc"][1] + ms_e1) / args.steps,
+            "encoder_prompt_ms_per_step": enc_ms,
+            "encoder_generation_ms_per_step": ms_e1 / args.steps,
             "decoder_ms_per_step": ms_s / args.steps,
         },
     }
+    if n_e1:
+        line["roofline_encoder_generation"] = {
+            "bound": "hbm", "achieved": enc1_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": enc1_gbs / pk["hbm_gbs"], "peak_kind": f"{pk_kind} hbm_gbs",
+            "blocks": n_e1, "alg_bytes_per_step": by_e1 / args.steps,
+            "ms_per_step": ms_e1 / args.steps}
     clk_s = clk.summary()
     if clk_s:
         line["clocks"] = clk_s

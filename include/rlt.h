@@ -337,7 +337,9 @@ uint64_t rlt_kernel_launches(void);
 #define RLT_PROF_SWA   1  /* decoder window attention over C^D           */
 #define RLT_PROF_STEP  2  /* one whole transition block (merge .. s_t)   */
 #define RLT_PROF_ENC   3  /* one whole encoder block (embed .. memory)   */
-#define RLT_PROF_NCLS  4
+#define RLT_PROF_ENC1  4  /* the same, for a one-position call (a new   */
+                          /* token during generation)                   */
+#define RLT_PROF_NCLS  5
 /* cls + RLT_PROF_NCLS * (l + 1) queries the window or cross-attention
  * launches of decoder layer l alone (0 <= l < L_D). */
 int rlt_profile_enable(rlt_state* state, int on);

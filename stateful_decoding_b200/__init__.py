@@ -36,8 +36,8 @@ RLT_E_SNAPSHOT = -9
 RLT_BUILD_DEBUG = 1
 SNAPSHOT_HEADER_BYTES = 128                # RLT_SNAPSHOT_HEADER_BYTES
 PART_S, PART_R, PART_E, PART_MEM, PART_RING, PART_ENC = range(6)
-PROF_XATTN, PROF_SWA, PROF_STEP, PROF_ENC = range(4)
-PROF_NCLS = 4          # cls + PROF_NCLS * (layer + 1): one decoder layer's launches
+PROF_XATTN, PROF_SWA, PROF_STEP, PROF_ENC, PROF_ENC1 = range(5)
+PROF_NCLS = 5          # cls + PROF_NCLS * (layer + 1): one decoder layer's launches
 READOUT_ROWS_SCRATCH_BYTES = 16 << 20      # RLT_READOUT_ROWS_SCRATCH_BYTES
 
 

@@ -185,6 +185,22 @@ k_gemm_persist(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
             } else {
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 64) {
+                    // accumulate: this chunk's z values, all 16 loads in flight
+                    // before the accumulator is read (8 lanes per row segment)
+                    float4 o[2][8];
+                    if (MODE == kAddF32) {
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                const int rr = 4 * k + (lane >> 3), c4 = lane & 7;
+                                o[hf][k] = rbase + rr < M
+                                               ? *reinterpret_cast<const float4*>(
+                                                     C + (size_t)(rbase + rr) * ldc + n0 + c +
+                                                     32 * hf + 4 * c4)
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                            }
+                    }
                     float v[64];
                     tmem_ld64(tq + (uint32_t)c, v);
 #pragma unroll
@@ -205,11 +221,10 @@ k_gemm_persist(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
                             float4* dst = reinterpret_cast<float4*>(
                                 C + (size_t)(rbase + rr) * ldc + n0 + c + 32 * hf + 4 * c4);
                             if (MODE == kAddF32) {
-                                const float4 o = *dst;
-                                w.x += o.x;
-                                w.y += o.y;
-                                w.z += o.z;
-                                w.w += o.w;
+                                w.x += o[hf][k].x;
+                                w.y += o[hf][k].y;
+                                w.z += o[hf][k].z;
+                                w.w += o[hf][k].w;
                             }
                             *dst = w;
                         }

@@ -226,28 +226,46 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                 if (abort_flag) goto epilogue_done;
                 constexpr int C4 = BN / 4;
                 const int et = threadIdx.x - 64;
-#pragma unroll 4
-                for (int i = et; i < BM * C4; i += 128) {
-                    const int rr = i / C4, c4 = i % C4, grow = m0 + rr;
-                    if (grow >= M) continue;
-                    float4 w = *reinterpret_cast<const float4*>(stg + (size_t)rr * SP + 4 * c4);
-                    if (MODE == kStoreT) {
-                        __nv_bfloat162 a = __floats2bfloat162_rn(w.x, w.y);
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(w.z, w.w);
-                        uint2 u2;
-                        u2.x = *reinterpret_cast<uint32_t*>(&a);
-                        u2.y = *reinterpret_cast<uint32_t*>(&b2);
-                        *reinterpret_cast<uint2*>(Ct + (size_t)grow * ldct + n0 + 4 * c4) = u2;
-                    } else {
-                        float4* dst = reinterpret_cast<float4*>(C + (size_t)grow * ldc + n0 + 4 * c4);
-                        if (MODE == kAddF32) {
-                            const float4 o = *dst;
-                            w.x += o.x;
-                            w.y += o.y;
-                            w.z += o.z;
-                            w.w += o.w;
+                // RA pieces per thread and pass; to accumulate, their 8 pieces
+                // of C are read ahead of the stores (a store could alias a
+                // later load, so loads and stores would not overlap otherwise)
+                constexpr int RA = MODE == kAddF32 ? 8 : 4;
+#pragma unroll 1
+                for (int i0 = et; i0 < BM * C4; i0 += RA * 128) {
+                    float4 o[RA];
+                    if (MODE == kAddF32) {
+#pragma unroll
+                        for (int u = 0; u < RA; ++u) {
+                            const int i = i0 + u * 128, grow = m0 + i / C4;
+                            o[u] = (i < BM * C4 && grow < M)
+                                       ? *reinterpret_cast<const float4*>(
+                                             C + (size_t)grow * ldc + n0 + 4 * (i % C4))
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
                         }
-                        *dst = w;
+                    }
+#pragma unroll
+                    for (int u = 0; u < RA; ++u) {
+                        const int i = i0 + u * 128;
+                        const int rr = i / C4, c4 = i % C4, grow = m0 + rr;
+                        if (i >= BM * C4 || grow >= M) continue;
+                        float4 w = *reinterpret_cast<const float4*>(stg + (size_t)rr * SP + 4 * c4);
+                        if (MODE == kStoreT) {
+                            __nv_bfloat162 a = __floats2bfloat162_rn(w.x, w.y);
+                            __nv_bfloat162 b2 = __floats2bfloat162_rn(w.z, w.w);
+                            uint2 u2;
+                            u2.x = *reinterpret_cast<uint32_t*>(&a);
+                            u2.y = *reinterpret_cast<uint32_t*>(&b2);
+                            *reinterpret_cast<uint2*>(Ct + (size_t)grow * ldct + n0 + 4 * c4) = u2;
+                        } else {
+                            float4* dst = reinterpret_cast<float4*>(C + (size_t)grow * ldc + n0 + 4 * c4);
+                            if (MODE == kAddF32) {
+                                w.x += o[u].x;
+                                w.y += o[u].y;
+                                w.z += o[u].z;
+                                w.w += o[u].w;
+                            }
+                            *dst = w;
+                        }
                     }
                 }
             } else if (__all_sync(0xffffffffu, got))

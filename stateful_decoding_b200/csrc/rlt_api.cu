@@ -924,7 +924,8 @@ extern "C" int rlt_encode(rlt_state* s, const int32_t* tokens, int n, void* stre
                                           st);
         if (e != cudaSuccess) return RLT_E_DEVICE;
         {
-            ProfScope ps(s, RLT_PROF_ENC, st, s->prof ? enc_bytes(s, nb) : 0.0);
+            ProfScope ps(s, n == 1 ? RLT_PROF_ENC1 : RLT_PROF_ENC, st,
+                         s->prof ? enc_bytes(s, nb) : 0.0);
             const bool tc = n >= kEncTcMinPositions;      // by the call, not the block
             if (m->cfg.dtype == RLT_DTYPE_BF16) encode_block<bf16>(s, s->tok, nb, st, tc);
             else encode_block<float>(s, s->tok, nb, st, tc);
