@@ -590,7 +590,7 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
 // read of the ring (the warp owns its (row, head) ring).  The
 // cross-attention takes memory keys 1..t_i for query i.  Key order and every
 // reduction order depend on positions only.
-constexpr int DRBN = 4;        // rounds per batch for multi-query blocks (two batches in flight)
+constexpr int DRBN = 2;        // rounds per batch for multi-query blocks (registers)
 
 template <int DH, bool SWA, int NQ>
 __global__ void __launch_bounds__(DWARPS * 32)
@@ -667,9 +667,8 @@ k_attn_decn(const bf16* __restrict__ base, size_t row_stride, int span,
     // its residue; memory key j is position j + 1
     auto pos_of = [&](int j) -> int { return SWA ? pd - ((pd - 1 - j) % span) : j + 1; };
     // fold `cnt` keys (their scores per query in s, masked by -inf) into the
-    // per-query state; vb: the keys' values (key r counts only where `vmask`
-    // has bit r: other lanes' or missing keys add nothing)
-    auto fold = [&](float (&s)[NQ][DRBN], const uint4 (&vb)[DRBN], int cnt, unsigned vmask) {
+    // per-query state; vf: the keys' values
+    auto fold = [&](float (&s)[NQ][DRBN], const float (&vf)[DRBN][8], int cnt) {
 #pragma unroll
         for (int i = 0; i < NQ; ++i) {
             float bm = s[i][0];
@@ -679,40 +678,29 @@ k_attn_decn(const bf16* __restrict__ base, size_t row_stride, int span,
 #pragma unroll
             for (int o = 16; o >= LPK; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
             const float mn = fmaxf(m[i], bm);
-            float corr = 1.f, ps = 0.f;
-            if (mn != -INFINITY) {                    // warp-uniform
-                corr = (m[i] == -INFINITY) ? 0.f : __expf(m[i] - mn);
+            if (mn == -INFINITY) continue;            // no visible key yet (warp-uniform)
+            const float corr = (m[i] == -INFINITY) ? 0.f : __expf(m[i] - mn);
+            float ps = 0.f;
 #pragma unroll
-                for (int r = 0; r < DRBN; ++r) {
-                    s[i][r] = (r >= cnt || s[i][r] == -INFINITY) ? 0.f : __expf(s[i][r] - mn);
-                    ps += s[i][r];
-                }
-                m[i] = mn;
-            } else {
-#pragma unroll
-                for (int r = 0; r < DRBN; ++r) s[i][r] = 0.f;
+            for (int r = 0; r < DRBN; ++r) {
+                s[i][r] = (r >= cnt || s[i][r] == -INFINITY) ? 0.f : __expf(s[i][r] - mn);
+                ps += s[i][r];
             }
 #pragma unroll
             for (int o = 16; o >= LPK; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
             l[i] = l[i] * corr + ps;
 #pragma unroll
-            for (int x = 0; x < 8; ++x) acc[i][x] *= corr;
-        }
-        // values one key at a time (8 live registers), added to every query
+            for (int x = 0; x < 8; ++x) {
+                float a = acc[i][x] * corr;
 #pragma unroll
-        for (int r = 0; r < DRBN; ++r) {
-            if (r >= cnt || !((vmask >> r) & 1u)) continue;
-            float vf[8];
-            unpack8(vb[r], vf);
-#pragma unroll
-            for (int i = 0; i < NQ; ++i)
-#pragma unroll
-                for (int x = 0; x < 8; ++x) acc[i][x] = fmaf(s[i][r], vf[x], acc[i][x]);
+                for (int r = 0; r < DRBN; ++r) a = fmaf(s[i][r], vf[r][x], a);
+                acc[i][x] = a;
+            }
+            m[i] = mn;
         }
     };
     auto fold_batch = [&](int j0, const uint4 (&kb)[DRBN], const uint4 (&vb)[DRBN]) {
-        float s[NQ][DRBN];
-        unsigned vmask = 0;
+        float s[NQ][DRBN], vf[DRBN][8];
 #pragma unroll
         for (int r = 0; r < DRBN; ++r) {
             const int j = j0 + r * KPR + grp;
@@ -721,7 +709,10 @@ k_attn_decn(const bf16* __restrict__ base, size_t row_stride, int span,
             float kf[8] = {};
             if (v) {
                 unpack8(kb[r], kf);
-                vmask |= 1u << r;
+                unpack8(vb[r], vf[r]);
+            } else {
+#pragma unroll
+                for (int x = 0; x < 8; ++x) vf[r][x] = 0.f;
             }
 #pragma unroll
             for (int i = 0; i < NQ; ++i) {
@@ -733,7 +724,7 @@ k_attn_decn(const bf16* __restrict__ base, size_t row_stride, int span,
                 s[i][r] = (v && p >= lo[i] && p <= pd + 1 + i) ? dot : -INFINITY;
             }
         }
-        fold(s, vb, DRBN, vmask);
+        fold(s, vf, DRBN);
     };
     for (int j0 = 0; j0 < nreg; j0 += 2 * BATCH) {
         fold_batch(j0, kb0, vb0);
@@ -763,13 +754,18 @@ k_attn_decn(const bf16* __restrict__ base, size_t row_stride, int span,
         }
         __syncwarp();
         // own position e (t_e = pd+1+e): every lane group scores it, group 0
-        // carries its value (the others add nothing)
+        // carries its value (the others add zeros)
 #pragma unroll
         for (int e = 0; e < NQ; ++e) {
-            float kf[8], s[NQ][DRBN];
-            uint4 vb1[DRBN];
+            float kf[8], s[NQ][DRBN], vf[DRBN][8];
             unpack8(*reinterpret_cast<const uint4*>(&s_k[warp][e][seg * 8]), kf);
-            vb1[0] = *reinterpret_cast<const uint4*>(&s_v[warp][e][seg * 8]);
+            unpack8(*reinterpret_cast<const uint4*>(&s_v[warp][e][seg * 8]), vf[0]);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                if (grp != 0) vf[0][x] = 0.f;
+#pragma unroll
+                for (int r = 1; r < DRBN; ++r) vf[r][x] = 0.f;
+            }
 #pragma unroll
             for (int i = 0; i < NQ; ++i) {
                 float dot = 0.f;
@@ -784,7 +780,7 @@ k_attn_decn(const bf16* __restrict__ base, size_t row_stride, int span,
 #pragma unroll
                 for (int r = 1; r < DRBN; ++r) s[i][r] = -INFINITY;
             }
-            fold(s, vb1, 1, grp == 0 ? 1u : 0u);
+            fold(s, vf, 1);
         }
     }
 #pragma unroll

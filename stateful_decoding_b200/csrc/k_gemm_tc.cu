@@ -431,11 +431,6 @@ bool launch_gemm_tc_runs(const bf16* A, int lda, const bf16* W, int ldw, float* 
     if (M <= 0 || N < 16 || K < BK || K % BK || splits < 2) return false;
     if (lda % 8 || ldw % 8 || ((uintptr_t)A & 15) || ((uintptr_t)W & 15)) return false;
     if ((ldc & 3) || ((uintptr_t)C & 15) || N % 64) return false;
-    // 128-wide tiles (half the A re-reads) when the runs fit TMEM beside them
-    const int nk = K / BK, cps = (nk + splits - 1) / splits, runs = (nk + cps - 1) / cps;
-    if (N % 128 == 0 && 128 * runs <= 512)
-        return launch_tc<128, kStoreF32>(A, lda, W, ldw, C, ldc, nullptr, 0, M, N, K, splits, 0,
-                                         st, true);
     return launch_tc<64, kStoreF32>(A, lda, W, ldw, C, ldc, nullptr, 0, M, N, K, splits, 0, st,
                                     true);
 }
