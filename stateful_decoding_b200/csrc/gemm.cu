@@ -15,7 +15,7 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, in
 bool launch_gemm_tc_runs(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc,
                          int M, int N, int K, int splits, cudaStream_t st);
 
-static bool tc_enabled() {
+bool tc_gemm_enabled() {
     static int v = -1;
     if (v < 0) {
         const char* e = getenv("RLT_GEMM");
@@ -33,7 +33,7 @@ void launch_gemm<float>(const float* A, int lda, const float* W, int ldw, float*
 template <>
 void launch_gemm<bf16>(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc,
                        bf16* Ct, int ldct, int M, int N, int K, int mode, cudaStream_t st) {
-    if (tc_enabled() && launch_gemm_tc(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, 1, 0, st))
+    if (tc_gemm_enabled() && launch_gemm_tc(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, 1, 0, st))
         return;
     launch_gemm_simt<bf16>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, st);
 }
@@ -57,7 +57,7 @@ int launch_gemm_split<float>(const float* A, int lda, const float* W, int ldw, f
 template <>
 int launch_gemm_split<bf16>(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc,
                             int M, int N, int K, int splits, size_t slab, cudaStream_t st) {
-    if (tc_enabled() && splits > 1 && K % 64 == 0) {
+    if (tc_gemm_enabled() && splits > 1 && K % 64 == 0) {
         const int nk = K / 64, cps = (nk + splits - 1) / splits, s = (nk + cps - 1) / cps;
         // enough rows to fill the machine without splitting CTAs: the runs
         // stay in tensor memory and one slab holds their ordered sum
@@ -72,7 +72,7 @@ int launch_gemm_split<bf16>(const bf16* A, int lda, const bf16* W, int ldw, floa
 
 bool launch_gemm_swiglu(const bf16* A, int lda, const bf16* W13, int ldw, bf16* Hd, int ldh, int M,
                         int N, int K, cudaStream_t st) {
-    if (!tc_enabled() || N % (2 * kW13Block)) return false;
+    if (!tc_gemm_enabled() || N % (2 * kW13Block)) return false;
     return launch_gemm_tc(A, lda, W13, ldw, nullptr, 0, Hd, ldh, M, N, K, kSwiGLU, 1, 0, st);
 }
 

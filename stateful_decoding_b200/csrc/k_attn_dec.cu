@@ -75,12 +75,6 @@ __device__ __forceinline__ float slab_sum8(const float* __restrict__ P, int S, s
         if (z < S) v += t[z];
     return v;
 }
-// rotate-half RoPE of one pair (j, j + d_h/2)
-__device__ __forceinline__ void rope_rot(float x1, float x2, float c, float s, float& y1,
-                                         float& y2) {
-    y1 = x1 * c - x2 * s;
-    y2 = x2 * c + x1 * s;
-}
 
 template <int DH, int NQ>
 struct Online {             // per-warp online softmax state of NQ queries
@@ -232,7 +226,7 @@ k_attn_stream(const float* __restrict__ Q, const bf16* __restrict__ base, size_t
                 const float c = pin.rope.cs[(size_t)t * HALF + j];
                 const float sn = pin.rope.sn[(size_t)t * HALF + j];
                 float y1, y2;
-                rope_rot(slab_sum8(pin.P, pin.S, pin.slab, o),
+                rope_pair(slab_sum8(pin.P, pin.S, pin.slab, o),
                          slab_sum8(pin.P, pin.S, pin.slab, o + HALF), c, sn, y1, y2);
                 if (r < HALF) {
                     s_q[i][j] = y1;
@@ -457,7 +451,7 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
     if (live) {
         for (int j = lane; j < HALF; j += 32) {
             float y1, y2;
-            rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + j),
+            rope_pair(slab_sum8(pin.P, pin.S, pin.slab, rb + j),
                      slab_sum8(pin.P, pin.S, pin.slab, rb + j + HALF), cs[j], sn[j], y1, y2);
             s_q[warp][j] = y1;
             s_q[warp][j + HALF] = y2;
@@ -527,7 +521,7 @@ k_attn_dec1(const bf16* __restrict__ base, size_t row_stride, int span,
         // batch registers are free), rounded like the stored ones
         for (int j = lane; j < HALF; j += 32) {
             float y1, y2;
-            rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + d + j),
+            rope_pair(slab_sum8(pin.P, pin.S, pin.slab, rb + d + j),
                      slab_sum8(pin.P, pin.S, pin.slab, rb + d + j + HALF), cs[j], sn[j], y1, y2);
             s_k[warp][j] = __float2bfloat16_rn(y1);
             s_k[warp][j + HALF] = __float2bfloat16_rn(y2);
@@ -639,7 +633,7 @@ k_attn_decn(const bf16* __restrict__ base, size_t row_stride, int span,
             const float* sn = pin.rope.sn + (size_t)(pd + 1 + i) * HALF;
             for (int j = lane; j < HALF; j += 32) {
                 float y1, y2;
-                rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + j),
+                rope_pair(slab_sum8(pin.P, pin.S, pin.slab, rb + j),
                          slab_sum8(pin.P, pin.S, pin.slab, rb + j + HALF), cs[j], sn[j], y1, y2);
                 s_q[warp][i][j] = y1;
                 s_q[warp][i][j + HALF] = y2;
@@ -742,7 +736,7 @@ k_attn_decn(const bf16* __restrict__ base, size_t row_stride, int span,
             const float* sn = pin.rope.sn + (size_t)(pd + 1 + e) * HALF;
             for (int j = lane; j < HALF; j += 32) {
                 float y1, y2;
-                rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + d + j),
+                rope_pair(slab_sum8(pin.P, pin.S, pin.slab, rb + d + j),
                          slab_sum8(pin.P, pin.S, pin.slab, rb + d + j + HALF), cs[j], sn[j], y1,
                          y2);
                 s_k[warp][e][j] = __float2bfloat16_rn(y1);
@@ -880,9 +874,13 @@ k_attn_xsplit(const bf16* __restrict__ base, size_t row_stride, int span,
             }
         }
     };
+    // the memory was written two or more kernels back: its first keys are
+    // requested before the wait for the previous kernel; the encoder cache
+    // (QIN) holds the new position's key, written by the kernel just before
+    if (QIN) pdl_enter();
     if (jlo < jhi) load_batch(jlo, kb0, vb0);
     if (jlo + BATCH < jhi) load_batch(jlo + BATCH, kb1, vb1);
-    pdl_enter();
+    if (!QIN) pdl_enter();
 
     // q: formed once by warp 0 (rotate-half pairs at position t, slab sums in
     // slab order), shared by the four warps
@@ -895,7 +893,7 @@ k_attn_xsplit(const bf16* __restrict__ base, size_t row_stride, int span,
         const float* sn = pin.rope.sn + (size_t)t * HALF;
         for (int j = lane; j < HALF; j += 32) {
             float y1, y2;
-            rope_rot(slab_sum8(pin.P, pin.S, pin.slab, rb + j),
+            rope_pair(slab_sum8(pin.P, pin.S, pin.slab, rb + j),
                      slab_sum8(pin.P, pin.S, pin.slab, rb + j + HALF), cs[j], sn[j], y1, y2);
             s_q[j] = y1;
             s_q[j + HALF] = y2;

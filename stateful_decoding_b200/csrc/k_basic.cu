@@ -240,11 +240,7 @@ void launch_merge_out(const float* e, int T_cap, const int32_t* pos_dec, const f
 }
 
 // ---------------------------------------------------------------- RoPE scatters
-// rotate-half: pair (j, j+half) turns by p * base^(-2j/dh)
-__device__ __forceinline__ void rot(float x1, float x2, float c, float s, float& y1, float& y2) {
-    y1 = x1 * c - x2 * s;
-    y2 = x2 * c + x1 * s;
-}
+// rotate-half: pair (j, j+half) turns by p * base^(-2j/dh) (rope_pair)
 
 template <typename T>
 __global__ void k_qkv_dec(const float* __restrict__ QKV, int S, size_t slab,
@@ -261,10 +257,10 @@ __global__ void k_qkv_dec(const float* __restrict__ QKV, int S, size_t slab,
         float c = rope.cs[(size_t)t * half + j], s = rope.sn[(size_t)t * half + j];
         int o1 = h * dh + j, o2 = o1 + half;
         float y1, y2;
-        rot(slab_sum(QKV, S, slab, base + o1), slab_sum(QKV, S, slab, base + o2), c, s, y1, y2);
+        rope_pair(slab_sum(QKV, S, slab, base + o1), slab_sum(QKV, S, slab, base + o2), c, s, y1, y2);
         Q[(size_t)r * d + o1] = y1;
         Q[(size_t)r * d + o2] = y2;
-        rot(slab_sum(QKV, S, slab, base + d + o1), slab_sum(QKV, S, slab, base + d + o2), c, s, y1,
+        rope_pair(slab_sum(QKV, S, slab, base + d + o1), slab_sum(QKV, S, slab, base + d + o2), c, s, y1,
             y2);
         Kc[(size_t)r * d + o1] = from_f<T>(y1);
         Kc[(size_t)r * d + o2] = from_f<T>(y2);
@@ -297,10 +293,10 @@ __global__ void k_qkv_enc(const float* __restrict__ QKV, const int32_t* __restri
         int o1 = h * dh + j, o2 = o1 + half;
         size_t dst = ((size_t)h * T_cap + (p - 1)) * dh + j;
         float y1, y2;
-        rot(src[o1], src[o2], c, s, y1, y2);
+        rope_pair(src[o1], src[o2], c, s, y1, y2);
         Q[(size_t)r * d + o1] = y1;
         Q[(size_t)r * d + o2] = y2;
-        rot(src[d + o1], src[d + o2], c, s, y1, y2);
+        rope_pair(src[d + o1], src[d + o2], c, s, y1, y2);
         kc[dst] = from_f<T>(y1);
         kc[dst + half] = from_f<T>(y2);
         vc[dst] = from_f<T>(src[2 * d + o1]);
@@ -333,7 +329,7 @@ __global__ void k_mem_scatter(const float* __restrict__ KV, const int32_t* __res
         int o1 = h * dh + j, o2 = o1 + half;
         size_t dst = ((size_t)h * T_cap + (p - 1)) * dh + j;
         float y1, y2;
-        rot(src[o1], src[o2], c, s, y1, y2);
+        rope_pair(src[o1], src[o2], c, s, y1, y2);
         mk[dst] = from_f<T>(y1);
         mk[dst + half] = from_f<T>(y2);
         mv[dst] = from_f<T>(src[d + o1]);
@@ -361,7 +357,7 @@ __global__ void k_rope_q(const float* __restrict__ P, int S, size_t slab,
         float c = rope.cs[(size_t)t * half + j], s = rope.sn[(size_t)t * half + j];
         int o1 = h * dh + j, o2 = o1 + half;
         float y1, y2;
-        rot(slab_sum(P, S, slab, (size_t)r * d + o1), slab_sum(P, S, slab, (size_t)r * d + o2), c,
+        rope_pair(slab_sum(P, S, slab, (size_t)r * d + o1), slab_sum(P, S, slab, (size_t)r * d + o2), c,
             s, y1, y2);
         Q[(size_t)r * d + o1] = y1;
         Q[(size_t)r * d + o2] = y2;
@@ -387,10 +383,10 @@ __global__ void __launch_bounds__(256) k_swiglu(const float* __restrict__ H, int
     const float4 a = slab_sum4(H, S, slab, base);
     const float4 u = slab_sum4(H, S, slab, base + kW13Block);
     float4 y;
-    y.x = a.x / (1.0f + expf(-a.x)) * u.x;
-    y.y = a.y / (1.0f + expf(-a.y)) * u.y;
-    y.z = a.z / (1.0f + expf(-a.z)) * u.z;
-    y.w = a.w / (1.0f + expf(-a.w)) * u.w;
+    y.x = silu_mul(a.x, u.x);
+    y.y = silu_mul(a.y, u.y);
+    y.z = silu_mul(a.z, u.z);
+    y.w = silu_mul(a.w, u.w);
     store4<T>(Hd + (size_t)r * fpad + j, y);
 }
 template <typename T>

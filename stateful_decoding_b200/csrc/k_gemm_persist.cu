@@ -37,7 +37,7 @@ template <int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
 k_gemm_persist(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
                float* __restrict__ C, int ldc, bf16* __restrict__ Ct, int ldct, int M, int N,
-               int K) {
+               int K, const RopeScatter rs) {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -161,8 +161,8 @@ k_gemm_persist(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
 #pragma unroll
                             for (int k = 0; k < 4; ++k) {
                                 const int e = 8 * h + 2 * k;
-                                const float y0 = a[e] / (1.0f + expf(-a[e])) * u[e];
-                                const float y1 = a[e + 1] / (1.0f + expf(-a[e + 1])) * u[e + 1];
+                                const float y0 = silu_mul(a[e], u[e]);
+                                const float y1 = silu_mul(a[e + 1], u[e + 1]);
                                 __nv_bfloat162 p2 = __floats2bfloat162_rn(y0, y1);
                                 wp[k] = *reinterpret_cast<uint32_t*>(&p2);
                             }
@@ -178,6 +178,94 @@ k_gemm_persist(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
                                                           (n0 + g0) / 2 + c + 8 * c4) =
                                     *reinterpret_cast<const uint4*>(
                                         reinterpret_cast<uint32_t*>(stg) + rr * SPITCH + 4 * c4);
+                        }
+                        __syncwarp();
+                    }
+                }
+            } else if (MODE == kRopeScatter) {
+                // the tile's 256 columns lie in one section: q, k or v
+                const int sec = rs.sec0 + n0 / rs.d, c0 = n0 % rs.d;
+                const int half = rs.dh >> 1, heads = rs.d / rs.dh;
+                // the row of this lane's accumulator lane: its sequence and position
+                const int row = rbase + lane;
+                int rb = 0, rp = 1;
+                if (row < M) {
+                    rb = row / rs.n;
+                    rp = __ldcg(rs.pos + rb) + 1 + row % rs.n;
+                }
+                uint32_t* stw = reinterpret_cast<uint32_t*>(stg);
+                // q: 32 rotated values of this lane's row, staged, then written
+                // as 128-byte row segments of Q (8 lanes per row)
+                auto put_q = [&](const float (&x)[32], int col) {
+                    float* srow = stg + lane * SPITCH;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        *reinterpret_cast<float4*>(srow + 4 * u) =
+                            make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+                    __syncwarp();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int rr = 4 * k + (lane >> 3), c4 = lane & 7;
+                        if (rbase + rr < M)
+                            *reinterpret_cast<float4*>(rs.Q + (size_t)(rbase + rr) * rs.d + col +
+                                                       4 * c4) =
+                                *reinterpret_cast<const float4*>(stg + rr * SPITCH + 4 * c4);
+                    }
+                    __syncwarp();
+                };
+#pragma unroll 1
+                for (int hc = 0; hc < BN; hc += rs.dh) {
+                    const int h = (c0 + hc) / rs.dh;
+#pragma unroll 1
+                    for (int j0 = 0; j0 < half; j0 += 32) {
+                        // the pairs (j, j + d_h/2) for j = j0 .. j0+31 of head h
+                        float x1[32], x2[32];
+                        tmem_ld32(tq + (uint32_t)(hc + j0), x1);
+                        tmem_ld32(tq + (uint32_t)(hc + half + j0), x2);
+                        if (sec < 2 && row < M) {
+                            const float* cs = rs.rope.cs + (size_t)rp * half + j0;
+                            const float* sn = rs.rope.sn + (size_t)rp * half + j0;
+#pragma unroll
+                            for (int u = 0; u < 32; u += 4) {
+                                const float4 c4 = __ldg(reinterpret_cast<const float4*>(cs + u));
+                                const float4 s4 = __ldg(reinterpret_cast<const float4*>(sn + u));
+                                rope_pair(x1[u], x2[u], c4.x, s4.x, x1[u], x2[u]);
+                                rope_pair(x1[u + 1], x2[u + 1], c4.y, s4.y, x1[u + 1], x2[u + 1]);
+                                rope_pair(x1[u + 2], x2[u + 2], c4.z, s4.z, x1[u + 2], x2[u + 2]);
+                                rope_pair(x1[u + 3], x2[u + 3], c4.w, s4.w, x1[u + 3], x2[u + 3]);
+                            }
+                        }
+                        if (sec == 0) {
+                            put_q(x1, h * rs.dh + j0);
+                            put_q(x2, h * rs.dh + half + j0);
+                            continue;
+                        }
+                        // k or v, rounded to bf16: the row's two 64-byte pieces
+                        // staged side by side, then 4 lanes per piece and row
+                        {
+                            uint32_t* srow = stw + lane * SPITCH;
+#pragma unroll
+                            for (int u = 0; u < 16; ++u) {
+                                __nv_bfloat162 a2 = __floats2bfloat162_rn(x1[2 * u], x1[2 * u + 1]);
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(x2[2 * u], x2[2 * u + 1]);
+                                srow[u] = *reinterpret_cast<uint32_t*>(&a2);
+                                srow[16 + u] = *reinterpret_cast<uint32_t*>(&b2);
+                            }
+                        }
+                        __syncwarp();
+                        const size_t vofs = sec == 2 ? (size_t)heads * rs.T_cap * rs.dh : 0;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int rr = 8 * k + (lane >> 2), c4 = lane & 3;
+                            const int br = __shfl_sync(0xffffffffu, rb, rr);
+                            const int pr = __shfl_sync(0xffffffffu, rp, rr);
+                            if (rbase + rr >= M) continue;
+                            bf16* dst = rs.cache + (size_t)br * rs.row_stride + vofs +
+                                        ((size_t)h * rs.T_cap + (pr - 1)) * rs.dh + j0 + 8 * c4;
+                            *reinterpret_cast<uint4*>(dst) =
+                                *reinterpret_cast<const uint4*>(stw + rr * SPITCH + 4 * c4);
+                            *reinterpret_cast<uint4*>(dst + half) =
+                                *reinterpret_cast<const uint4*>(stw + rr * SPITCH + 16 + 4 * c4);
                         }
                         __syncwarp();
                     }
@@ -246,7 +334,7 @@ k_gemm_persist(const __grid_constant__ CUtensorMap ta, const __grid_constant__ C
 
 template <int MODE>
 bool launch_mode(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc, bf16* Ct,
-                 int ldct, int M, int N, int K, cudaStream_t st) {
+                 int ldct, int M, int N, int K, cudaStream_t st, const RopeScatter& rs = {}) {
     CUtensorMap ta, tb;
     if (!make_tma_2d_bf16(&ta, A, M, K, lda, BM) || !make_tma_2d_bf16(&tb, W, N, K, ldw, BN))
         return false;
@@ -255,7 +343,7 @@ bool launch_mode(const bf16* A, int lda, const bf16* W, int ldw, float* C, int l
     if (sms <= 0) return false;
     const int tiles = ((M + BM - 1) / BM) * (N / BN);
     launch(k_gemm_persist<MODE>, std::min(tiles, sms), NTHREADS, SMEM, st, ta, tb, C, ldc, Ct,
-           ldct, M, N, K);
+           ldct, M, N, K, rs);
     rlt_count_launch();
     return true;
 }
@@ -287,6 +375,23 @@ bool launch_gemm_persist(const bf16* A, int lda, const bf16* W, int ldw, float* 
     if (mode == kAddF32)
         return launch_mode<kAddF32>(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, st);
     return false;
+}
+
+bool tc_gemm_enabled();
+bool persist_gemm_enabled();
+
+bool launch_gemm_rope_scatter(const bf16* A, int lda, const bf16* W, int ldw, int M, int N,
+                              int K, const RopeScatter& rs, cudaStream_t st) {
+    if (!tc_gemm_enabled() || !persist_gemm_enabled()) return false;
+    if (M < 2048 || N % BN || K < BK || K % BK) return false;
+    if (rs.d <= 0 || rs.d % BN || rs.n <= 0 || (rs.dh != 64 && rs.dh != 128)) return false;
+    if (rs.sec0 < 0 || rs.sec0 > 1 || N != (3 - rs.sec0) * rs.d) return false;
+    if (lda % 8 || ldw % 8 || ((uintptr_t)A & 15) || ((uintptr_t)W & 15)) return false;
+    if (((uintptr_t)rs.cache & 15) || rs.row_stride % 8 || !rs.pos ||
+        ((uintptr_t)rs.rope.cs & 15) || ((uintptr_t)rs.rope.sn & 15) || rs.rope.half != rs.dh / 2)
+        return false;
+    if (rs.sec0 == 0 && ((uintptr_t)rs.Q & 15)) return false;
+    return launch_mode<kRopeScatter>(A, lda, W, ldw, nullptr, 0, nullptr, 0, M, N, K, st, rs);
 }
 
 }  // namespace rlt

@@ -170,9 +170,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
 #pragma unroll
                                 for (int k = 0; k < 4; ++k) {
                                     const int e = 8 * h + 2 * k;
-                                    const float y0 = a[e] / (1.0f + expf(-a[e])) * u[e];
-                                    const float y1 =
-                                        a[e + 1] / (1.0f + expf(-a[e + 1])) * u[e + 1];
+                                    const float y0 = silu_mul(a[e], u[e]);
+                                    const float y1 = silu_mul(a[e + 1], u[e + 1]);
                                     __nv_bfloat162 p2 = __floats2bfloat162_rn(y0, y1);
                                     wp[k] = *reinterpret_cast<uint32_t*>(&p2);
                                 }
@@ -414,7 +413,7 @@ bool make_tma_2d_bf16(CUtensorMap* map, const void* base, int rows, int cols, in
 
 bool launch_gemm_persist(const bf16* A, int lda, const bf16* W, int ldw, float* C, int ldc,
                          bf16* Ct, int ldct, int M, int N, int K, int mode, cudaStream_t st);
-static bool persist_enabled() {
+bool persist_gemm_enabled() {
     static const bool on = [] {
         const char* e = getenv("RLT_GEMM_PERSIST");
         return !(e && strcmp(e, "0") == 0);
@@ -446,7 +445,7 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* W, int ldw, float* C, in
     if (lda % 8 || ldw % 8 || ((uintptr_t)A & 15) || ((uintptr_t)W & 15)) return false;
     // many rows: the persistent kernel with two accumulators (epilogue of one
     // tile under the MMAs of the next); RLT_GEMM_PERSIST=0 turns it off
-    if (M >= 2048 && splits == 1 && persist_enabled() &&
+    if (M >= 2048 && splits == 1 && persist_gemm_enabled() &&
         launch_gemm_persist(A, lda, W, ldw, C, ldc, Ct, ldct, M, N, K, mode, st))
         return true;
     // wide tiles when M alone fills the machine, narrow ones (more CTAs)

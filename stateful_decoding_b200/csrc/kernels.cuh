@@ -14,8 +14,9 @@
 
 namespace rlt {
 
-// GEMM epilogues: C (fp32) = acc | C += acc | Ct (storage type) = acc
-enum GemmMode { kStoreF32 = 0, kAddF32 = 1, kStoreT = 2, kSwiGLU = 3 };
+// GEMM epilogues: C (fp32) = acc | C += acc | Ct (storage type) = acc |
+// SwiGLU of interleaved W1;W3 columns | RoPE and cache scatter (RopeScatter)
+enum GemmMode { kStoreF32 = 0, kAddF32 = 1, kStoreT = 2, kSwiGLU = 3, kRopeScatter = 4 };
 // The fused FFN input projection stores W1 and W3 interleaved in blocks of
 // kW13Block rows: packed rows [64k, 64k+32) are W1 rows [32k, 32k+32)
 // (gates), rows [64k+32, 64k+64) the W3 rows of the same units, so any
@@ -31,6 +32,45 @@ struct RopeTab {          // cos/sin of p * base^(-2i/dh), p = 0..max_pos, i < d
     int half;
     int max_pos;          // last position with a row in the tables
 };
+
+// Rotate-half RoPE of one pair (j, j + d_h/2) by the angle whose cosine and
+// sine are c and s.  Written with explicit fused multiply-adds so that every
+// kernel that rotates (the scatters, the attention kernels that form q and k
+// themselves, the GEMM epilogue below) rounds alike.
+__device__ __forceinline__ void rope_pair(float x1, float x2, float c, float s, float& y1,
+                                          float& y2) {
+    y1 = fmaf(x1, c, -(x2 * s));
+    y2 = fmaf(x2, c, x1 * s);
+}
+
+// SwiGLU of one unit: SiLU(a) * u, a the gate pre-activation and u the up
+// projection, with the fast exponential and division (a few ulp in fp32; the
+// result is stored in bf16, or carries the fp32 models' 1e-4 tolerance).
+// Every kernel that applies SwiGLU uses this one form.
+__device__ __forceinline__ float silu_mul(float a, float u) {
+    return __fdividef(a, 1.0f + __expf(-a)) * u;
+}
+
+// Destination of an encoder product whose GEMM epilogue applies RoPE and
+// scatters the result (kRopeScatter): the columns are the q|k|v blocks
+// (sec0 = 0) or the memory's k|v blocks (sec0 = 1), d columns each.  Row
+// r = b*n + i is position pos[b] + 1 + i of sequence b: q goes rotated to
+// Q[r][d] (fp32), k rotated and v as they are to the cache of row b
+// (cache + b*row_stride: K [heads][T_cap][dh], then V), in bf16.
+struct RopeScatter {
+    float* Q;
+    bf16* cache;
+    size_t row_stride;
+    int T_cap;
+    const int32_t* pos;
+    RopeTab rope;
+    int n, dh, d, sec0;
+};
+// C = A . W^T with the kRopeScatter epilogue on the persistent tensor-core
+// GEMM; false (nothing launched) where it does not apply (fewer than 2048
+// rows, d not a multiple of 256, d_h not 64 or 128).
+bool launch_gemm_rope_scatter(const bf16* A, int lda, const bf16* W, int ldw, int M, int N,
+                              int K, const RopeScatter& rs, cudaStream_t st);
 
 template <typename T>
 void launch_embed(const T* E, const int32_t* tok, float* X, int R, int d, int vocab, int* err,

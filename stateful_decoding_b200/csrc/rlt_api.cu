@@ -859,10 +859,20 @@ static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t s
     for (int l = 0; l < c.n_enc; ++l) {
         const EncLayerW& L = m->enc[l];
         launch_rmsnorm<T>(s->X, d, L.attn_norm, Y, d, R, d, eps, st);
-        launch_gemm<T>(Y, d, (const T*)L.wqkv, d, s->QKV, 3 * d, nullptr, 0, R, 3 * d, d,
-                       kStoreF32, st);
-        launch_qkv_enc<T>(s->QKV, s->pos_enc, rope_of(s), s->Q, enc + l * layer_enc, s->enc_row,
-                          s->T_cap, B, n, h, dh, st);
+        // many rows: RoPE and the cache scatter in the q|k|v GEMM's epilogue
+        bool qkv_done = false;
+        if constexpr (std::is_same<T, bf16>::value)
+            qkv_done = launch_gemm_rope_scatter(
+                Y, d, (const bf16*)L.wqkv, d, R, 3 * d, d,
+                RopeScatter{s->Q, enc + l * layer_enc, s->enc_row, s->T_cap, s->pos_enc,
+                            rope_of(s), n, dh, d, 0},
+                st);
+        if (!qkv_done) {
+            launch_gemm<T>(Y, d, (const T*)L.wqkv, d, s->QKV, 3 * d, nullptr, 0, R, 3 * d, d,
+                           kStoreF32, st);
+            launch_qkv_enc<T>(s->QKV, s->pos_enc, rope_of(s), s->Q, enc + l * layer_enc,
+                              s->enc_row, s->T_cap, B, n, h, dh, st);
+        }
         bool attn_done = false;
         if constexpr (std::is_same<T, bf16>::value)
             attn_done = (tc_attn || (dh == 64 && max_keys <= 256)) && fast_attn_enabled() &&
@@ -892,10 +902,20 @@ static void encode_block(rlt_state* s, const int32_t* tok, int n, cudaStream_t s
         launch_rmsnorm<T>(s->X, d, m->mem_norm, Y, d, R, d, eps, st);
         const size_t layer_mem = (size_t)2 * h * s->T_cap * dh;
         for (int g = 0; g < c.groups; ++g) {
-            launch_gemm<T>(Y, d, (const T*)m->wmem[g], d, s->QKV, 2 * d, nullptr, 0, R, 2 * d, d,
-                           kStoreF32, st);
-            launch_mem_scatter<T>(s->QKV, s->pos_enc, rope_of(s), (T*)s->mem + g * layer_mem,
-                                  s->mem_row, s->T_cap, B, n, h, dh, st);
+            T* mem_g = (T*)s->mem + g * layer_mem;
+            bool kv_done = false;
+            if constexpr (std::is_same<T, bf16>::value)
+                kv_done = launch_gemm_rope_scatter(
+                    Y, d, (const bf16*)m->wmem[g], d, R, 2 * d, d,
+                    RopeScatter{nullptr, mem_g, s->mem_row, s->T_cap, s->pos_enc, rope_of(s), n,
+                                dh, d, 1},
+                    st);
+            if (!kv_done) {
+                launch_gemm<T>(Y, d, (const T*)m->wmem[g], d, s->QKV, 2 * d, nullptr, 0, R,
+                               2 * d, d, kStoreF32, st);
+                launch_mem_scatter<T>(s->QKV, s->pos_enc, rope_of(s), mem_g, s->mem_row,
+                                      s->T_cap, B, n, h, dh, st);
+            }
         }
     }
     launch_pos_add(s->pos_enc, B, n, st);

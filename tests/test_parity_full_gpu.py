@@ -156,6 +156,37 @@ def test_many_row_products_match_rows_alone(sd, name, B, T):
     model.close()
 
 
+def test_rope_scatter_epilogue_wide_heads(sd):
+    """From 2048 rows on, the encoder's q|k|v and memory products apply RoPE
+    and scatter into the caches in the GEMM epilogue; below, a row kernel
+    does it from the stored product.  At d_h 128 (the large model's width on
+    a 2 + 1 layer slice, 8 rows x 256 positions = 2048 rows per product) the
+    two must agree bit for bit, and the big batch must match the oracle."""
+    cfg = ri.CONFIGS["large_bf16"].replace(n_enc=2, n_dec=1)
+    B, T = 8, 256
+    W, model, big = make(sd, cfg, B, T)
+    toks = ri.make_tokens(cfg, B, T)
+    big.encode(toks)
+    big.prefill(T)
+    lbig, _, _ = readout_host(big, cfg)
+    for r in (0, B - 1):
+        one = sd.State(model, 1, T)
+        one.encode(np.ascontiguousarray(toks[r:r + 1]))
+        one.prefill(T)
+        l1, _, _ = readout_host(one, cfg)
+        np.testing.assert_array_equal(l1[0], lbig[r])
+        one.close()
+    orc = RLTOracle(cfg, W, oracle_mode(cfg))
+    r = orc.new_state()
+    orc.encode(r, toks[3])
+    orc.prefill(r, T)
+    err = float(np.max(np.abs(lbig[3] - orc.readout(r))))
+    assert err <= tol_for(cfg), f"row 3: |dlogit| {err}"
+    big.check()
+    big.close()
+    model.close()
+
+
 def test_large_full_depth_prompt_and_sampled_generation(sd):
     """large_bf16 at full depth on 2 rows: a 256-token prompt encoded and
     prefilled in one call each, then 32 tokens sampled one at a time and fed
