@@ -519,14 +519,17 @@ struct rlt_state {
     std::vector<cudaEvent_t> prof_pool;
     // event pairs captured into a graph (cudaEventRecordExternal nodes), with
     // the index of the block they bracket
-    struct CapRec { int cls; cudaEvent_t a, b; int block; int layer; };
+    struct CapRec { int cls; cudaEvent_t a, b; int block; int layer; int b0, nb; };
     bool prof_capture = false;
     int prof_block = 0;
+    int prof_b0 = 0, prof_nb = 0;     // rows of the transition block being issued
     std::vector<CapRec> cap_recs;
     // replayable transition blocks, per positions-per-block n; graphs_prof
     // carries event nodes around the attention launches (profiling level 2)
     struct Graph { cudaGraphExec_t exec; uint64_t launches; std::vector<CapRec> caps; };
     std::map<int, Graph> graphs, graphs_prof;
+    // streams of the row groups after the first inside a captured graph
+    std::vector<cudaStream_t> aux;
 };
 
 static cudaEvent_t prof_event(rlt_state* s) {
@@ -573,7 +576,7 @@ struct ProfScope {
                 return;
             }
             cudaEventRecordWithFlags(b, st, cudaEventRecordExternal);
-            s->cap_recs.push_back({cls, a, b, s->prof_block, layer});
+            s->cap_recs.push_back({cls, a, b, s->prof_block, layer, s->prof_b0, s->prof_nb});
             return;
         }
         cudaEvent_t b = prof_event(s);
@@ -613,6 +616,7 @@ extern "C" void rlt_state_destroy(rlt_state* s) {
                 cudaEventDestroy(c.b);
             }
         }
+    for (cudaStream_t a : s->aux) cudaStreamDestroy(a);
     for (void* p : s->allocs) cudaFree(p);
     delete s;
 }
@@ -757,18 +761,19 @@ static rlt::RopeTab rope_of(rlt_state* s) {
 // ============================================================================
 static double kv_bytes(const rlt_state* s) { return 2.0 * s->m->cfg.d * (double)s->m->elt; }
 
-static double xattn_bytes(const rlt_state* s, int n) {   // one cross-attention launch
+// (rows b0 .. b0+nb-1; all rows by default)
+static double xattn_bytes(const rlt_state* s, int n, int b0 = 0, int nb = -1) {
     const double d = s->m->cfg.d, elt = (double)s->m->elt;
     double by = 0;
-    for (int b = 0; b < s->B; ++b)
+    for (int b = b0; b < (nb < 0 ? s->B : b0 + nb); ++b)
         by += (s->h_pos_dec[b] + n) * kv_bytes(s) + n * (d * 4 + d * elt);
     return by;
 }
-static double swa_bytes(const rlt_state* s, int n) {     // one window-attention launch
+static double swa_bytes(const rlt_state* s, int n, int b0 = 0, int nb = -1) {
     const double d = s->m->cfg.d, elt = (double)s->m->elt;
     const int slots = std::max(0, s->m->cfg.window - 1);
     double by = 0;
-    for (int b = 0; b < s->B; ++b)
+    for (int b = b0; b < (nb < 0 ? s->B : b0 + nb); ++b)
         by += std::min(s->h_pos_dec[b], slots) * kv_bytes(s) + n * (kv_bytes(s) + d * 4 + d * elt);
     return by;
 }
@@ -965,86 +970,96 @@ extern "C" int rlt_encode(rlt_state* s, const int32_t* tokens, int n, void* stre
 // merged_in: the previous block already wrote this block's merge input (Y);
 // fuse_out: end with the state hand-off fused with the next block's merge
 // input (one position per row, RLT-1/2, inside a replayed run of blocks).
+// b0, nb: the block runs rows b0 .. b0+nb-1 only (all rows by default).  A
+// row range keeps its own part of every scratch buffer (rows b0*n.. at each
+// buffer's widest pitch), so the ranges of one block can run concurrently.
 template <typename T>
 static void step_block(rlt_state* s, int n, cudaStream_t st, bool merged_in = false,
-                       bool fuse_out = false) {
+                       bool fuse_out = false, int b0 = 0, int nb = -1) {
     using namespace rlt;
     rlt_model* m = s->m;
     const rlt_config& c = m->cfg;
-    const int B = s->B, d = c.d, h = c.heads, dh = m->dh, fp = m->fpad, R = B * n;
+    const int B = nb < 0 ? s->B : nb, d = c.d, h = c.heads, dh = m->dh, fp = m->fpad,
+              R = B * n;
     const float eps = (float)c.eps;
-    T* Y = (T*)s->Y;
-    T* A = (T*)s->A;
-    T* Hd = (T*)s->Hd;
-    T* Kc = (T*)s->Kc;
-    T* Vc = (T*)s->Vc;
-    float* z = s->X;
+    const size_t row0 = (size_t)b0 * n;
+    T* Y = (T*)s->Y + row0 * std::max(2 * d, fp);
+    T* A = (T*)s->A + row0 * d;
+    T* Hd = (T*)s->Hd + row0 * fp;
+    T* Kc = (T*)s->Kc + row0 * d;
+    T* Vc = (T*)s->Vc + row0 * d;
+    float* z = s->X + row0 * d;
+    float* Q = s->Q + row0 * d;
+    int32_t* pos_dec = s->pos_dec + b0;
+    const float* e = s->e + (size_t)b0 * s->T_cap * d;
+    float* s_vec = s->s + (size_t)b0 * d;
+    float* r_reg = s->Rr + (size_t)b0 * d;
+    s->prof_b0 = b0;
+    s->prof_nb = B;
     // Split-K partial slabs of each projection land in s->P; the kernel that
     // consumes the projection adds them in slab order (residual projections:
     // the next RMSNorm, or the state hand-off).
-    float* P = s->P;
-    const size_t slab = (size_t)R * s->p_cols;
+    float* P = s->P + row0 * s->p_cols;
+    const size_t slab = (size_t)s->B * n * s->p_cols;
     auto gemm_p = [&](const T* Ain, int lda, const T* Wt, int N, int K, float* dst) {
         return launch_gemm_split<T>(Ain, lda, Wt, K, dst, N, R, N, K, dec_splits(s, N, K), slab,
                                     st);
     };
     // the merge kernel also applies the first decoder block's input RMSNorm
     const float* norm0 = c.n_dec > 0 ? m->dec[0].swa_norm : nullptr;
-    launch_check_positions(s->pos_enc, s->pos_dec, B, n, s->T_cap, false, s->err, st);
+    launch_check_positions(s->pos_enc + b0, pos_dec, B, n, s->T_cap, false, s->err, st);
     if (c.variant == 0) {
-        launch_merge_out<T>(s->e, s->T_cap, s->pos_dec, nullptr, 0, 0, nullptr, nullptr, 0, 0, d,
-                            0.f, z, norm0, Y, eps, B, n, d, st);
+        launch_merge_out<T>(e, s->T_cap, pos_dec, nullptr, 0, 0, nullptr, nullptr, 0, 0, d, 0.f,
+                            z, norm0, Y, eps, B, n, d, st);
     } else {
-        const float* fb = c.variant == 2 ? s->Rr : s->s;
+        const float* fb = c.variant == 2 ? r_reg : s_vec;
         if (!merged_in)
-            launch_merge_input<T>(s->e, s->T_cap, s->pos_dec, fb, m->merge_norm, Y, B, n, d, eps,
-                                  st);
+            launch_merge_input<T>(e, s->T_cap, pos_dec, fb, m->merge_norm, Y, B, n, d, eps, st);
         // one GEMM for both projections: gate pre-activations in columns
         // 0..d-1 of the slabs, W_s r in columns d..2d-1
         const int nGS = gemm_p(Y, 2 * d, (const T*)m->wgs, 2 * d, 2 * d, P);
-        launch_merge_out<T>(s->e, s->T_cap, s->pos_dec, P, nGS, slab, m->bg, P + d, nGS, slab,
-                            2 * d, (float)c.alpha, z, norm0, Y, eps, B, n, d, st);
+        launch_merge_out<T>(e, s->T_cap, pos_dec, P, nGS, slab, m->bg, P + d, nGS, slab, 2 * d,
+                            (float)c.alpha, z, norm0, Y, eps, B, n, d, st);
     }
     const size_t layer_ring = (size_t)2 * h * std::max(0, c.window - 1) * dh;
     const size_t layer_mem = (size_t)2 * h * s->T_cap * dh;
     int nres = 0;                       // pending residual partial slabs in P
     for (int l = 0; l < c.n_dec; ++l) {
         const DecLayerW& L = m->dec[l];
-        T* ring = (T*)s->ring + l * layer_ring;
+        T* ring = (T*)s->ring + (size_t)b0 * s->ring_row + l * layer_ring;
         if (l > 0)
             launch_add_rmsnorm<T>(z, nres ? P : nullptr, nres, slab, L.swa_norm, Y, R, d, eps, st);
         int np = gemm_p(Y, d, (const T*)L.wqkv, 3 * d, d, P);
         {
             // bf16: the attention kernel forms q, k, v from the slabs and
             // updates the ring itself; otherwise scatter, attend, write
-            ProfScope ps(s, RLT_PROF_SWA, st, s->prof ? swa_bytes(s, n) : 0.0, l);
+            ProfScope ps(s, RLT_PROF_SWA, st, s->prof ? swa_bytes(s, n, b0, B) : 0.0, l);
             bool done = false;
             if constexpr (std::is_same<T, bf16>::value)
                 done = launch_attn_swa_proj(ProjIn{P, np, slab, 3 * d, rope_of(s)}, ring,
-                                            s->ring_row, c.window, s->pos_dec, A, B, n, h, dh, st);
+                                            s->ring_row, c.window, pos_dec, A, B, n, h, dh, st);
             if (!done) {
-                launch_qkv_dec<T>(P, np, slab, s->pos_dec, rope_of(s), s->Q, Kc, Vc, B, n, h, dh,
-                                  st);
-                launch_attn_swa<T>(s->Q, Kc, Vc, ring, s->ring_row, c.window, s->pos_dec, A, B, n,
-                                   h, dh, st);
-                launch_ring_write<T>(Kc, Vc, s->pos_dec, ring, s->ring_row, c.window, B, n, h, dh,
+                launch_qkv_dec<T>(P, np, slab, pos_dec, rope_of(s), Q, Kc, Vc, B, n, h, dh, st);
+                launch_attn_swa<T>(Q, Kc, Vc, ring, s->ring_row, c.window, pos_dec, A, B, n, h,
+                                   dh, st);
+                launch_ring_write<T>(Kc, Vc, pos_dec, ring, s->ring_row, c.window, B, n, h, dh,
                                      st);
             }
         }
         nres = gemm_p(A, d, (const T*)L.wo, d, d, P);
         launch_add_rmsnorm<T>(z, P, nres, slab, L.x_norm, Y, R, d, eps, st);
         np = gemm_p(Y, d, (const T*)L.xq, d, d, P);
-        const T* mem = (const T*)s->mem + (c.groups > 1 ? l : 0) * layer_mem;
+        const T* mem =
+            (const T*)s->mem + (size_t)b0 * s->mem_row + (c.groups > 1 ? l : 0) * layer_mem;
         {
-            ProfScope ps(s, RLT_PROF_XATTN, st, s->prof ? xattn_bytes(s, n) : 0.0, l);
+            ProfScope ps(s, RLT_PROF_XATTN, st, s->prof ? xattn_bytes(s, n, b0, B) : 0.0, l);
             bool done = false;
             if constexpr (std::is_same<T, bf16>::value)
                 done = launch_attn_cross_proj(ProjIn{P, np, slab, d, rope_of(s)}, mem, s->mem_row,
-                                              s->T_cap, s->pos_dec, A, B, n, h, dh, st);
+                                              s->T_cap, pos_dec, A, B, n, h, dh, st);
             if (!done) {
-                launch_rope_q(P, np, slab, s->Q, s->pos_dec, rope_of(s), B, n, h, dh, st);
-                launch_attn_cross<T>(s->Q, mem, s->mem_row, s->T_cap, s->pos_dec, A, B, n, h, dh,
-                                     st);
+                launch_rope_q(P, np, slab, Q, pos_dec, rope_of(s), B, n, h, dh, st);
+                launch_attn_cross<T>(Q, mem, s->mem_row, s->T_cap, pos_dec, A, B, n, h, dh, st);
             }
         }
         nres = gemm_p(A, d, (const T*)L.xo, d, d, P);
@@ -1063,12 +1078,12 @@ static void step_block(rlt_state* s, int n, cudaStream_t st, bool merged_in = fa
         nres = gemm_p(Hd, fp, (const T*)L.w2, d, fp, P);
     }
     if (fuse_out)
-        launch_state_merge<T>(z, nres ? P : nullptr, nres, slab, s->s,
-                              c.variant == 2 ? s->Rr : nullptr, s->pos_dec, c.chunk, s->e, s->T_cap,
+        launch_state_merge<T>(z, nres ? P : nullptr, nres, slab, s_vec,
+                              c.variant == 2 ? r_reg : nullptr, pos_dec, c.chunk, e, s->T_cap,
                               m->merge_norm, Y, B, d, eps, st);
     else
-        launch_set_state(z, nres ? P : nullptr, nres, slab, s->s,
-                         c.variant == 2 ? s->Rr : nullptr, s->pos_dec, c.chunk, B, n, d,
+        launch_set_state(z, nres ? P : nullptr, nres, slab, s_vec,
+                         c.variant == 2 ? r_reg : nullptr, pos_dec, c.chunk, B, n, d,
                          /*bump=*/true, st);
 }
 
@@ -1104,6 +1119,18 @@ static bool graphs_enabled(cudaStream_t st) {
     return v == 1 && st != nullptr && st != cudaStreamLegacy && st != cudaStreamPerThread;
 }
 
+// RLT_ROW_GROUPS=g: a captured run splits the rows into g contiguous groups
+// whose chains of kernels run as concurrent branches of the graph (rows never
+// interact; every kernel's result for a row is the same in any group).
+// Read once; default 1.
+static int row_groups(int B) {
+    static const int v = [] {
+        const char* e = getenv("RLT_ROW_GROUPS");
+        return e ? std::max(1, std::min(atoi(e), 8)) : 1;
+    }();
+    return std::max(1, std::min(v, B));
+}
+
 static int run_graph(rlt_state* s, int n, cudaStream_t st) {
     const int span = kGraphBlocks * n;
     for (int b = 0; b < s->B; ++b) {
@@ -1123,19 +1150,54 @@ static int run_graph(rlt_state* s, int n, cudaStream_t st) {
         const uint64_t l0 = rlt_kernel_launches();
         cudaGraph_t g = nullptr;
         cudaGraphExec_t ex = nullptr;
-        bool ok = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+        // row groups: branches forked from and joined back into st (the
+        // profiling twin issues them one after another on st, so that each
+        // timed launch runs alone)
+        int G = row_groups(s->B);
+        while ((int)s->aux.size() < G - 1) {
+            cudaStream_t a = nullptr;
+            if (cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking) != cudaSuccess) {
+                cudaGetLastError();
+                break;
+            }
+            s->aux.push_back(a);
+        }
+        G = std::min(G, 1 + (int)s->aux.size());
+        const bool branch = G > 1 && !timed;
+        std::vector<cudaEvent_t> evs(branch ? G : 0, nullptr);
+        bool ok = true;
+        for (auto& ev : evs)
+            ok = ok && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess;
+        ok = ok && cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
         if (ok) {
+            if (branch) {
+                cudaEventRecord(evs[0], st);
+                for (int k = 1; k < G; ++k) cudaStreamWaitEvent(s->aux[k - 1], evs[0], 0);
+            }
             // consecutive one-position blocks hand the state to the next
             // block's merge input in one kernel
             const bool chain = n == 1 && s->m->cfg.variant != 0;
-            for (int k = 0; k < kGraphBlocks; ++k) {
-                s->prof_block = k;
-                const bool in = chain && k > 0, out = chain && k + 1 < kGraphBlocks;
-                if (s->m->cfg.dtype == RLT_DTYPE_BF16) step_block<bf16>(s, n, st, in, out);
-                else step_block<float>(s, n, st, in, out);
+            for (int gi = 0; gi < G; ++gi) {
+                const int b0 = (int)((long)gi * s->B / G), b1 = (int)((long)(gi + 1) * s->B / G);
+                cudaStream_t sg = branch && gi > 0 ? s->aux[gi - 1] : st;
+                for (int k = 0; k < kGraphBlocks; ++k) {
+                    s->prof_block = k;
+                    const bool in = chain && k > 0, out = chain && k + 1 < kGraphBlocks;
+                    if (s->m->cfg.dtype == RLT_DTYPE_BF16)
+                        step_block<bf16>(s, n, sg, in, out, b0, b1 - b0);
+                    else
+                        step_block<float>(s, n, sg, in, out, b0, b1 - b0);
+                }
             }
+            if (branch)
+                for (int k = 1; k < G; ++k) {
+                    cudaEventRecord(evs[k], s->aux[k - 1]);
+                    cudaStreamWaitEvent(st, evs[k], 0);
+                }
             ok = cudaStreamEndCapture(st, &g) == cudaSuccess && g != nullptr;
         }
+        for (auto& ev : evs)
+            if (ev) cudaEventDestroy(ev);
         ok = ok && cudaGraphInstantiate(&ex, g, 0) == cudaSuccess;
         if (g) cudaGraphDestroy(g);
         const uint64_t captured = rlt_kernel_launches() - l0;
@@ -1180,8 +1242,8 @@ static int run_graph(rlt_state* s, int n, cudaStream_t st) {
                 continue;
             }
             for (int b = 0; b < s->B; ++b) s->h_pos_dec[b] = saved[b] + c.block * n;
-            const double cb = c.cls == RLT_PROF_XATTN ? xattn_bytes(s, n)
-                              : c.cls == RLT_PROF_SWA ? swa_bytes(s, n) : 0.0;
+            const double cb = c.cls == RLT_PROF_XATTN ? xattn_bytes(s, n, c.b0, c.nb)
+                              : c.cls == RLT_PROF_SWA ? swa_bytes(s, n, c.b0, c.nb) : 0.0;
             s->prof_recs.push_back({c.cls, nullptr, nullptr, cb, t, c.layer});
         }
         s->h_pos_dec = saved;

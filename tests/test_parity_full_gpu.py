@@ -65,13 +65,18 @@ SAMPLED_ROWS = {
 @pytest.mark.parametrize("name", ["parity_bf16", "s5_bf16", "rlt2_mod5_bf16"])
 def test_full_size_bench_launch_sampled_rows(sd, name):
     """The workload at its full batch and length, one encode call and one
-    prefill call as the bench runs it; sampled rows against the oracle."""
+    prefill call on a stream of its own as the bench runs it (the prefill
+    replays captured graphs of 16 transition blocks); sampled rows against
+    the oracle."""
+    import torch
     cfg = ri.CONFIGS[name]
     B, T = cfg.batch, cfg.prompt
     W, model, st = make(sd, cfg, B, T)
     toks = ri.make_tokens(cfg)
-    st.encode(toks)
-    st.prefill(T)
+    stream = torch.cuda.Stream()
+    st.encode(toks, stream=stream)
+    st.prefill(T, stream=stream)
+    stream.synchronize()
     lg, am, _ = readout_host(st, cfg)
     s_gpu = state_vec(st, sd.PART_S, B, cfg.d)
     R_gpu = state_vec(st, sd.PART_R, B, cfg.d)
