@@ -49,9 +49,13 @@ normaliser then sums the rounded probabilities): at head size 64 with
 prefixes of at most 256 keys always, otherwise in calls of at least
 ENC_TC_MIN_POSITIONS tokens -- and every stored
 key/value (encoder cache, memory, window cache; the current position's
-key/value are used rounded too).  The decoder's attention is a matrix-vector
-computation on the CUDA path and keeps q and p unrounded.  Everything else
-stays float64.
+key/value are used rounded too).  The decoder's attention of one position
+is a matrix-vector computation on the CUDA path and keeps q and p
+unrounded; a decoder block of DEC_MQ_MIN_POSITIONS .. DEC_MQ_MAX_POSITIONS
+positions at head size 64 (an RLT-2 chunk, a short RLT-0 block) scores its
+queries against each key tile as one small matrix product, so there q and p
+are bf16 values as in the encoder (the window's only when W exceeds the
+block).  Everything else stays float64.
 
 Pinning: every function here is checked by ``tests/test_oracle_pins.py``
 against identities the pages state (serving-split invariance, causality,
@@ -76,6 +80,10 @@ import numpy as np
 # products from bf16 q and probabilities in mode "bf16" at any head size and
 # prefix length (see RLTOracle.encode).
 ENC_TC_MIN_POSITIONS = 16
+# decoder blocks of this many positions (head size 64, bf16) multiply q and
+# the probabilities as bf16 values (the multi-query tile products)
+DEC_MQ_MIN_POSITIONS = 2
+DEC_MQ_MAX_POSITIONS = 8
 
 # ----------------------------------------------------------------------------
 # Scalar helpers (float64)
@@ -298,6 +306,10 @@ class RLTOracle:
         k = self._store(rope(self._heads(self._lin(y, p + "wk")), pos, c.rope_base))
         v = self._store(self._heads(self._lin(y, p + "wv")))
         cache = st.swa[l]
+        # bf16 mode: a block of several positions at head size 64 enters the
+        # attention products with bf16 q and probabilities
+        mq = (self.mode == "bf16" and self.dh == 64
+              and DEC_MQ_MIN_POSITIONS <= n <= DEC_MQ_MAX_POSITIONS)
         a = np.zeros((n, self.h, self.dh))
         for i in range(n):
             t = int(pos[i])
@@ -306,7 +318,7 @@ class RLTOracle:
                                                                      if pos[m] >= lo]
             vs = [cache[j][1] for j in sorted(cache) if j >= lo] + [v[m] for m in range(i + 1)
                                                                      if pos[m] >= lo]
-            a[i] = attend(q[i], np.stack(ks), np.stack(vs))
+            a[i] = attend(q[i], np.stack(ks), np.stack(vs), rounded=mq and c.window > n)
         z = z + self._lin(a.reshape(n, c.d), p + "wo")
         for m in range(n):
             cache[int(pos[m])] = (k[m], v[m])
@@ -316,8 +328,8 @@ class RLTOracle:
         y = rmsnorm(z, W[p + "x_norm"], c.eps)
         qx = rope(self._heads(self._lin(y, p + "xq")), pos, c.rope_base)
         g = l if c.groups > 1 else 0
-        ax = np.stack([attend(qx[i], st.mem_k[g][:int(pos[i])], st.mem_v[g][:int(pos[i])])
-                       for i in range(n)])
+        ax = np.stack([attend(qx[i], st.mem_k[g][:int(pos[i])], st.mem_v[g][:int(pos[i])],
+                              rounded=mq) for i in range(n)])
         z = z + self._lin(ax.reshape(n, c.d), p + "xo")
         y = rmsnorm(z, W[p + "ffn_norm"], c.eps)
         return z + self._ffn(y, p + "w1", p + "w3", p + "w2")

@@ -1094,9 +1094,13 @@ bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int 
                           cudaStream_t st) {
     // one query group per (sequence, head): the kernel then owns every read
     // and write of that head's ring for the block
-    if (!fast_attn_enabled() || n > 4 || (dh != 64 && dh != 128)) return false;
+    if (!fast_attn_enabled() || (dh != 64 && dh != 128)) return false;
     if (B * n <= 0) return true;
     const int slots = W > 1 ? W - 1 : 1;
+    if (n >= 2 && W > n &&
+        launch_attn_mq<true>(ring, row_stride, slots, pos, W, A, B, n, heads, dh, pin, st))
+        return true;
+    if (n > 4) return false;
     if (n == 1 && pin.S <= 8)
         return dh == 64 ? launch_dec1<64, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st)
                         : launch_dec1<128, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st);
@@ -1158,6 +1162,8 @@ bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_strid
     if (n == 1 && pin.S <= 8)
         return dh == 64 ? launch_dec1<64, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st)
                         : launch_dec1<128, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st);
+    if (n >= 2 && launch_attn_mq<false>(mem, row_stride, T_cap, pos, 0, A, B, n, heads, dh, pin, st))
+        return true;
     if (dh == 64 && pin.S <= 8 && n <= 4 && multi_query_warp())
         return launch_decn64<false>(mem, row_stride, T_cap, pos, 0, A, B, n, heads, pin, st);
     if (dh == 64)

@@ -178,6 +178,7 @@ void launch_logprob(const float* logits, int V, int B, const int32_t* ids, int i
 int read_and_clear_device_error();  // device error word of the bounded-wait kernels
 int read_and_clear_attn_error();
 int read_and_clear_persist_error();  // same, for the persistent GEMM
+int read_and_clear_mq_error();       // same, for the multi-query block attention
 // Partial-sum slabs of a projection, consumed directly by an attention kernel.
 struct ProjIn {
     const float* P;   // slab 0 of the fp32 partial sums, [R][ldp]
@@ -197,6 +198,14 @@ bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_strid
                             const int32_t* pos_dec, bf16* A, int B, int n, int heads, int dh,
                             cudaStream_t st);
 bool fast_attn_enabled();           // false when RLT_ATTN=warp
+// Blocks of 2..8 positions per row at d_h = 64 (k_attn_mq.cu): one warp per
+// (row, head) scores the block's queries against 16-key tiles with the
+// warp-level tensor-core MMA; the window form (SWA) also takes the block's
+// own keys from the slabs and writes them into the ring.  false (nothing
+// launched) for other shapes or when RLT_MQ=0.
+template <bool SWA>
+bool launch_attn_mq(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W,
+                    bf16* A, int B, int n, int heads, int dh, const ProjIn& pin, cudaStream_t st);
 // Encoder causal attention on the tensor cores: k_attn_enc_tc.cu (exact
 // two-pass softmax) for d_h = 64 and at most 256 keys per row (max_keys =
 // max over rows of pos_enc + n), k_attn_enc_fa.cu for longer prefixes and

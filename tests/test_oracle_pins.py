@@ -801,6 +801,45 @@ def test_bf16_mode_rounds_every_cache_and_product_input():
         ro.attend = real
 
 
+def test_decoder_blocks_round_attention_inputs_like_the_tile_products():
+    """bf16 mode, head size 64: a decoder block of 2..8 positions (an RLT-2
+    chunk) passes rounded q and probabilities to both attentions (the window
+    only when W exceeds the block); a one-position transition does not; the
+    fp64 mode never does."""
+    import oracle.rlt_oracle as ro
+    cfg = ri.CONFIGS["rlt2_mod5_bf16"].replace(name="pin_mq", n_enc=1, n_dec=1, vocab=64)
+    W = ri.generate_weights(cfg)
+    seen = []
+    real = ro.attend
+
+    def spy(q_, K_, V_, rounded=False):
+        seen.append(rounded)
+        return real(q_, K_, V_, rounded)
+    ro.attend = spy
+    try:
+        tok = (np.arange(12) % 60 + 1).astype(np.int64)
+        for mode, want_block in (("bf16", True), ("fp64", False)):
+            m = RLTOracle(cfg, W, mode)
+            st_ = m.new_state()
+            m.encode(st_, tok)
+            seen.clear()
+            m.transition_chunk(st_, cfg.chunk)          # positions 1..4: one block
+            assert len(seen) == 2 * cfg.chunk and all(x == want_block for x in seen)
+            seen.clear()
+            m.transition(st_)                           # position 5 alone
+            assert len(seen) == 2 and not any(seen)
+        # a window no longer than the block keeps the window's inputs unrounded
+        narrow = cfg.replace(name="pin_mq_w", window=cfg.chunk)
+        m = RLTOracle(narrow, W, "bf16")
+        st_ = m.new_state()
+        m.encode(st_, tok)
+        seen.clear()
+        m.transition_chunk(st_, narrow.chunk)
+        assert seen[:narrow.chunk] == [False] * narrow.chunk and all(seen[narrow.chunk:])
+    finally:
+        ro.attend = real
+
+
 # ----------------------------------------------------------------------------
 # replay log-probabilities (jiphyeonjeon review §6.2, eq. 5.3-5.5)
 # ----------------------------------------------------------------------------

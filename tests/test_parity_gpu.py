@@ -147,6 +147,38 @@ def test_prefill_matches_oracle(sd, name, B, T):
             np.testing.assert_allclose(R_gpu, r.R, atol=max(10 * tol, 1e-3), rtol=0)
 
 
+@pytest.mark.parametrize("chunk", [2, 3, 8])
+def test_rlt2_chunk_blocks_match_oracle(sd, chunk):
+    """RLT-2 at other chunk sizes B_c (greeksharifa App. J.10): rlt_prefill
+    runs each chunk as one block of B_c positions -- the multi-query tile
+    products at d_h 64 -- against the oracle's chunked run of the same
+    blocks; logits, argmax and the held register R."""
+    cfg = ri.CONFIGS["rlt2_mod5_bf16"].replace(name=f"rlt2_chunk{chunk}", chunk=chunk)
+    B, T = 3, 40
+    tol = tol_for(cfg)
+    W, model, st = make(sd, cfg, B, T)
+    toks = ri.make_tokens(cfg, B, T)
+    st.encode(toks)
+    st.prefill(T)
+    lg, am, _ = readout_host(st, cfg)
+    R_gpu = state_vec(st, sd.PART_R, B, cfg.d)
+    orc = RLTOracle(cfg, W, oracle_mode(cfg))
+    tally = Tally()
+    for b in range(B):
+        r = orc.new_state()
+        orc.encode(r, toks[b])
+        orc.prefill(r, T, chunked=True)
+        ol = orc.readout(r)
+        err = float(np.max(np.abs(lg[b] - ol)))
+        assert err <= tol, f"chunk {chunk} row {b}: |dlogit| {err}"
+        check_argmax(int(am[b]), ol, tol, tally, f"row {b}")
+        rel = float(np.linalg.norm(R_gpu[b] - r.R) / np.linalg.norm(r.R))
+        assert rel <= tol, f"chunk {chunk} row {b}: |dR|/|R| {rel}"
+    st.check()
+    st.close()
+    model.close()
+
+
 def test_large_config_slice(sd):
     """The large tied workload at full width (d=2048, 16 heads x 128, vocab
     32000, W=256) on a 2+2-layer slice, 2 rows x 12 tokens + 2 sampled."""
