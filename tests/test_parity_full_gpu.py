@@ -165,9 +165,9 @@ def test_rope_scatter_epilogue_wide_heads(sd):
     """From 2048 rows on, the encoder's q|k|v and memory products apply RoPE
     and scatter into the caches in the GEMM epilogue; below, a row kernel
     does it from the stored product.  At d_h 128 (the large model's width on
-    a 2 + 1 layer slice, 8 rows x 256 positions = 2048 rows per product) the
+    a 2 + 2 layer slice, 8 rows x 256 positions = 2048 rows per product) the
     two must agree bit for bit, and the big batch must match the oracle."""
-    cfg = ri.CONFIGS["large_bf16"].replace(n_enc=2, n_dec=1)
+    cfg = ri.CONFIGS["large_bf16"].replace(n_enc=2, n_dec=2)
     B, T = 8, 256
     W, model, big = make(sd, cfg, B, T)
     toks = ri.make_tokens(cfg, B, T)
