@@ -840,37 +840,47 @@ bool launch_decn64(const bf16* base, size_t row_stride, int span, const int32_t*
 // QIN: the query is read ready-rotated from an fp32 [B][d] buffer (pin.P,
 // row pitch pin.ldp) -- the encoder's generation steps -- instead of being
 // formed from projection slabs.
-template <int DH, int XS, bool QIN = false>
+// SWA: the window attention over the ring's occupied slots 0 .. min(pd, W-1)-1
+// (split over the warps the same way), then the position's own key, formed
+// from the slabs by warp 0 and folded into its part; after the merge the
+// position enters its ring slot (every warp has finished reading the ring).
+template <int DH, int XS, bool QIN = false, bool SWA = false>
 __global__ void __launch_bounds__(XS * 32)
 k_attn_xsplit(const bf16* __restrict__ base, size_t row_stride, int span,
-              const int32_t* __restrict__ pos, bf16* __restrict__ A, int heads, ProjIn pin) {
+              const int32_t* __restrict__ pos, bf16* __restrict__ A, int heads, ProjIn pin,
+              int W) {
     constexpr int LPK = DH / 8, KPR = 32 / LPK, HALF = DH / 2;
     constexpr int BATCH = DRB * KPR;             // keys per batch
     __shared__ __align__(16) float s_q[DH];
     __shared__ float s_m[XS], s_l[XS];
     __shared__ __align__(16) float s_o[XS][DH];
+    __shared__ __align__(16) bf16 s_k[SWA ? DH : 8], s_v[SWA ? DH : 8];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x / heads, h = blockIdx.x % heads;
     const int d = heads * DH, seg = lane % LPK, grp = lane / LPK;
     const int t0 = __ldcg(pos + b) + 1;
-    // debug builds: keys 1..t and the RoPE row of t must exist (else no keys)
-    const bool live = dcheck(t0 >= 1 && t0 <= span && t0 <= pin.rope.max_pos, &g_attn_error,
-                             kDevCapacity);
+    // debug builds: keys 1..t (memory) and the RoPE row of t must exist
+    // (else no keys)
+    const bool live = dcheck(t0 >= 1 && (SWA || t0 <= span) && t0 <= pin.rope.max_pos,
+                             &g_attn_error, kDevCapacity);
     const int t = live ? t0 : 0;
-    // warp w: keys [jlo, jhi) of the run 0..t-1, parts rounded to whole batches
-    const int part = ((t + XS - 1) / XS + BATCH - 1) / BATCH * BATCH;
-    const int jlo = min(t, warp * part), jhi = min(t, jlo + part);
+    // the run: memory keys 0..t-1, or the ring's occupied slots
+    const int nrun = SWA ? (live && W > 1 ? min(t0 - 1, span) : 0) : t;
+    // warp w: keys [jlo, jhi) of the run, parts rounded to whole batches
+    const int part = ((nrun + XS - 1) / XS + BATCH - 1) / BATCH * BATCH;
+    const int jlo = min(nrun, warp * part), jhi = min(nrun, jlo + part);
     const bf16* kg = base + (size_t)b * row_stride + (size_t)h * span * DH + seg * 8;
     const bf16* vg = kg + (size_t)heads * span * DH;
-    const uint64_t l2pol = l2_evict_last_policy();
+    // memory lines stay in L2 for the next blocks; the ring streams
+    const uint64_t l2pol = SWA ? 0 : l2_evict_last_policy();
     uint4 kb0[DRB], vb0[DRB], kb1[DRB], vb1[DRB];
     auto load_batch = [&](int j0, uint4 (&kb)[DRB], uint4 (&vb)[DRB]) {
 #pragma unroll
         for (int r = 0; r < DRB; ++r) {
             const int j = j0 + r * KPR + grp;
             if (j < jhi) {
-                kb[r] = ld_kv<true>(kg + (size_t)j * DH, l2pol);
-                vb[r] = ld_kv<true>(vg + (size_t)j * DH, l2pol);
+                kb[r] = ld_kv<!SWA>(kg + (size_t)j * DH, l2pol);
+                vb[r] = ld_kv<!SWA>(vg + (size_t)j * DH, l2pol);
             }
         }
     };
@@ -957,6 +967,38 @@ k_attn_xsplit(const bf16* __restrict__ base, size_t row_stride, int span,
         fold(j0 + BATCH, kb1, vb1);
         if (j0 + 3 * BATCH < jhi) load_batch(j0 + 3 * BATCH, kb1, vb1);
     }
+    if (SWA && warp == 0 && live) {
+        // the position's own k and v, rounded like the stored ones; every
+        // lane group scores the key, group 0 carries its value
+        const size_t rb = (size_t)b * pin.ldp + h * DH;
+        const float* cs = pin.rope.cs + (size_t)t * HALF;
+        const float* sn = pin.rope.sn + (size_t)t * HALF;
+        for (int j = lane; j < HALF; j += 32) {
+            float y1, y2;
+            rope_pair(slab_sum8(pin.P, pin.S, pin.slab, rb + d + j),
+                      slab_sum8(pin.P, pin.S, pin.slab, rb + d + j + HALF), cs[j], sn[j], y1, y2);
+            s_k[j] = __float2bfloat16_rn(y1);
+            s_k[j + HALF] = __float2bfloat16_rn(y2);
+            s_v[j] = __float2bfloat16_rn(slab_sum8(pin.P, pin.S, pin.slab, rb + 2 * d + j));
+            s_v[j + HALF] = __float2bfloat16_rn(slab_sum8(pin.P, pin.S, pin.slab, rb + 2 * d + j + HALF));
+        }
+        __syncwarp();
+        float kf[8], vf[8];
+        unpack8(*reinterpret_cast<const uint4*>(&s_k[seg * 8]), kf);
+        unpack8(*reinterpret_cast<const uint4*>(&s_v[seg * 8]), vf);
+        float dot = 0.f;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) dot = fmaf(q[x], kf[x], dot);
+#pragma unroll
+        for (int o = LPK / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        const float mn = fmaxf(m, dot);
+        const float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
+        const float p = __expf(dot - mn);
+        l = l * corr + p;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc[x] = acc[x] * corr + (grp == 0 ? p * vf[x] : 0.f);
+        m = mn;
+    }
 #pragma unroll
     for (int x = 0; x < 8; ++x)
 #pragma unroll
@@ -984,6 +1026,17 @@ k_attn_xsplit(const bf16* __restrict__ base, size_t row_stride, int span,
             O += s_o[w][x] * f;
         }
         A[(size_t)b * d + h * DH + x] = __float2bfloat16_rn(O / L);
+    }
+    if (SWA && live && W > 1) {
+        // every warp has read its part of the ring (the barrier above): the
+        // position enters slot pd mod (W-1)
+        bf16* rk = const_cast<bf16*>(base) + (size_t)b * row_stride + (size_t)h * span * DH +
+                   (size_t)((t0 - 1) % span) * DH;
+        bf16* rv = rk + (size_t)heads * span * DH;
+        for (int x = threadIdx.x; x < DH; x += XS * 32) {
+            rk[x] = s_k[x];
+            rv[x] = s_v[x];
+        }
     }
 }
 
@@ -1101,9 +1154,16 @@ bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int 
         launch_attn_mq<true>(ring, row_stride, slots, pos, W, A, B, n, heads, dh, pin, st))
         return true;
     if (n > 4) return false;
+    if (n == 1 && pin.S <= 8 && dh == 128) {
+        // the wide heads' long windows with few items per launch: split each
+        // item's ring over four warps
+        launch(k_attn_xsplit<128, 4, false, true>, B * heads, 4 * 32, 0, st, ring, row_stride,
+               slots, pos, A, heads, pin, W);
+        rlt_count_launch();
+        return true;
+    }
     if (n == 1 && pin.S <= 8)
-        return dh == 64 ? launch_dec1<64, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st)
-                        : launch_dec1<128, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st);
+        return launch_dec1<64, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st);
     if (dh == 64 && pin.S <= 8 && W > 4 && multi_query_warp())
         return launch_decn64<true>(ring, row_stride, slots, pos, W, A, B, n, heads, pin, st);
     if (dh == 64)
@@ -1131,7 +1191,7 @@ bool launch_attn_enc_step(const float* Q, const bf16* cache, size_t row_stride, 
     pin.ldp = heads * dh;
     pin.rope.max_pos = T_cap;
     launch(k_attn_xsplit<128, 4, true>, B * heads, 4 * 32, 0, st, cache, row_stride, T_cap,
-           pos_enc, A, heads, pin);
+           pos_enc, A, heads, pin, 0);
     rlt_count_launch();
     return true;
 }
@@ -1145,17 +1205,17 @@ bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_strid
         // the wide heads come with long memory prefixes and few items per
         // launch: split each item's keys over four warps
         launch(k_attn_xsplit<128, 4>, B * heads, 4 * 32, 0, st, mem, row_stride, T_cap, pos, A,
-               heads, pin);
+               heads, pin, 0);
         rlt_count_launch();
         return true;
     }
     if (n == 1 && pin.S <= 8 && dh == 64 && xsplit64() > 1) {
         if (xsplit64() == 2)
             launch(k_attn_xsplit<64, 2>, B * heads, 2 * 32, 0, st, mem, row_stride, T_cap, pos,
-                   A, heads, pin);
+                   A, heads, pin, 0);
         else
             launch(k_attn_xsplit<64, 4>, B * heads, 4 * 32, 0, st, mem, row_stride, T_cap, pos,
-                   A, heads, pin);
+                   A, heads, pin, 0);
         rlt_count_launch();
         return true;
     }

@@ -810,12 +810,17 @@ static double enc_bytes(const rlt_state* s, int n) {     // one encoder block
 // Split-K factor of a transition projection (N outputs, K inputs): as many
 // CTAs as fit one wave on the machine when M = 256 rows (a second wave costs
 // more than the longer K run), a function of N and K only (never of the
-// batch), at least two 64-wide K-chunks per split.  1 for fp32 models.
+// batch), at least two 64-wide K-chunks per split.  Products of 4 MB of
+// weights or more (the d = 2048 model, whose batches are tens of rows) stream
+// their weights: two CTAs per SM over one 128-row tile keep enough weight
+// bytes in flight.  1 for fp32 models.
 static int dec_splits_for(const rlt_config& c, int N, int K) {
     if (c.dtype != RLT_DTYPE_BF16 || K % 64) return 1;
-    const int tiles = 2 * ((N + 63) / 64);            // output tiles at M = 256
+    const int ntile = (N + 63) / 64;
+    const int tiles = 2 * ntile;                      // output tiles at M = 256
     const int nk = K / 64;
-    int want = std::max(1, 148 / tiles);
+    const bool heavy = 2.0 * N * K >= 4e6;
+    int want = heavy ? std::max(1, 2 * 148 / ntile) : std::max(1, 148 / tiles);
     want = std::min({want, std::max(1, nk / 2), 8});      // consumers sum at most 8 slabs
     const int cps = (nk + want - 1) / want;
     return (nk + cps - 1) / cps;
