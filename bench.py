@@ -485,14 +485,17 @@ def main():
                     help="override the rows per GPU (small profiling cases only)")
     ap.add_argument("--prompt", type=int, default=None,
                     help="override the prompt length (small profiling cases only)")
+    ap.add_argument("--decode", type=int, default=None,
+                    help="override the sampled tokens per row (small profiling cases only)")
     ap.add_argument("--variant", type=int, default=None, choices=[0, 1, 2],
                     help="run the workload's model as RLT-0, RLT-1 or RLT-2 (feedback variants)")
     ap.add_argument("--chunk", type=int, default=None,
                     help="RLT-2 feedback chunk B_c (with --variant 2)")
     args = ap.parse_args()
     cfg = ri.CONFIGS[args.config]
-    if args.batch or args.prompt:
-        cfg = cfg.replace(batch=args.batch or cfg.batch, prompt=args.prompt or cfg.prompt)
+    if args.batch or args.prompt or args.decode is not None:
+        cfg = cfg.replace(batch=args.batch or cfg.batch, prompt=args.prompt or cfg.prompt,
+                          decode=cfg.decode if args.decode is None else args.decode)
     if args.variant is not None:
         v = args.variant
         chunk = (args.chunk or cfg.chunk) if v == 2 else 1
