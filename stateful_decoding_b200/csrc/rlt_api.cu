@@ -1127,13 +1127,16 @@ static bool graphs_enabled(cudaStream_t st) {
 // RLT_ROW_GROUPS=g: a captured run splits the rows into g contiguous groups
 // whose chains of kernels run as concurrent branches of the graph (rows never
 // interact; every kernel's result for a row is the same in any group).
-// Read once; default 1.
+// Read once.  Default: two groups from 512 rows on (each branch then has the
+// shape of a 256-row batch, whose chain leaves the machine idle between
+// dependent kernels), one below.
 static int row_groups(int B) {
     static const int v = [] {
         const char* e = getenv("RLT_ROW_GROUPS");
-        return e ? std::max(1, std::min(atoi(e), 8)) : 1;
+        return e ? std::max(1, std::min(atoi(e), 8)) : 0;
     }();
-    return std::max(1, std::min(v, B));
+    const int g = v ? v : (B >= 512 ? 2 : 1);
+    return std::max(1, std::min(g, B));
 }
 
 static int run_graph(rlt_state* s, int n, cudaStream_t st) {
