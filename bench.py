@@ -398,7 +398,9 @@ def run_ours(args, cfg):
     enc1_gbs = (by_e1 / ms_e1 * 1e3 / 1e9) if ms_e1 else 0.0
     tc_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
     n, ms, by = kprof["xattn"]
-    kname = "decoder cross-attention (k_attn_dec1: one warp per (row, head), q from the projection slabs)"
+    kname = ("decoder cross-attention (one warp per (row, head), q from the projection slabs: "
+             + ("k_attn_sq, keys staged in shared memory by cp.async" if cfg.d // cfg.heads == 64
+                else "k_attn_xsplit, keys split over four warps") + ")")
     xattn_timed = bool(n)
     if not n:       # no per-launch records: fall back to whole transition blocks
         n, ms, by = prof["step"]

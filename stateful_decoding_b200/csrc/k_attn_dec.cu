@@ -1162,6 +1162,8 @@ bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int 
         rlt_count_launch();
         return true;
     }
+    if (n == 1 && launch_attn_sq<true>(ring, row_stride, slots, pos, W, A, B, heads, dh, pin, st))
+        return true;
     if (n == 1 && pin.S <= 8)
         return launch_dec1<64, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st);
     if (dh == 64 && pin.S <= 8 && W > 4 && multi_query_warp())
@@ -1219,6 +1221,8 @@ bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_strid
         rlt_count_launch();
         return true;
     }
+    if (n == 1 && launch_attn_sq<false>(mem, row_stride, T_cap, pos, 0, A, B, heads, dh, pin, st))
+        return true;
     if (n == 1 && pin.S <= 8)
         return dh == 64 ? launch_dec1<64, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st)
                         : launch_dec1<128, false>(mem, row_stride, T_cap, pos, 0, A, B, heads, pin, st);

@@ -324,6 +324,212 @@ k_attn_mq(const bf16* __restrict__ base, size_t row_stride, int span,
     }
 }
 
+// ---------------------------------------------------------------- one position
+// One position per row (n = 1, the decode shape) at d_h = 64, on the CUDA
+// cores: one warp per (row, head), 16-key tiles of K and V staged by
+// cp.async (three in flight, the same swizzled rows), so the bytes in flight
+// cost no registers.  Scores: two lanes per key, 32 dims each, one shuffle;
+// an online softmax per tile (one warp maximum); values: lane group g takes
+// keys 4i+g of the tile, 8 dims per lane, and the groups' partial outputs
+// are added at the end.  q and p stay fp32.  The window form folds the
+// position's own key (formed from the slabs) after the ring's tiles and then
+// writes it into the ring.
+constexpr int SQ_WARPS = 4;
+constexpr int SQ_NST = 3;
+constexpr int SQ_WARP_SMEM = SQ_NST * 2 * MQ_TB + 512;   // tiles, q (fp32), own k and v
+constexpr int SQ_SMEM = SQ_WARPS * SQ_WARP_SMEM;
+
+template <bool SWA>
+__global__ void __launch_bounds__(SQ_WARPS * 32)
+k_attn_sq(const bf16* __restrict__ base, size_t row_stride, int span,
+          const int32_t* __restrict__ pos, int W, bf16* __restrict__ A, int B, int heads,
+          ProjIn pin) {
+    constexpr int DH = 64, HALF = 32;
+    extern __shared__ __align__(1024) uint8_t sq_smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int it = blockIdx.x * SQ_WARPS + warp;
+    const bool in_range = it < B * heads;
+    const int b = in_range ? it / heads : 0, h = in_range ? it % heads : 0;
+    const int d = heads * DH;
+    const int pd = in_range ? __ldcg(pos + b) : 0, t = pd + 1;
+    const bool live = in_range && dcheck(pd >= 0 && t <= pin.rope.max_pos && (SWA || t <= span),
+                                         &g_mq_error, kDevCapacity);
+    // the run: ring slots 0 .. min(pd, W-1)-1, or memory keys 1 .. t
+    const int nrun = !live ? 0 : (SWA ? (W > 1 ? min(pd, span) : 0) : t);
+    const int ntile = (nrun + MQ_TILE - 1) / MQ_TILE;
+    const bf16* kg = base + (size_t)b * row_stride + (size_t)h * span * DH;
+    const bf16* vg = kg + (size_t)heads * span * DH;
+    uint8_t* wsm = sq_smem + warp * SQ_WARP_SMEM;
+    const uint32_t sKV = tc::smem_u32(wsm);
+    float* s_q = reinterpret_cast<float*>(wsm + SQ_NST * 2 * MQ_TB);    // 64 floats
+    bf16* s_k = reinterpret_cast<bf16*>(s_q + DH);                      // own k, v
+    bf16* s_v = s_k + DH;
+
+    auto issue = [&](int k) {
+        if (k < ntile) {
+            const uint32_t stK = sKV + (uint32_t)(2 * (k % SQ_NST)) * MQ_TB, stV = stK + MQ_TB;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int ch = lane + 32 * u, r = ch >> 3, c = ch & 7, j = k * MQ_TILE + r;
+                const bool ok = j < nrun;
+                const size_t off = (size_t)(ok ? j : 0) * DH + c * 8;
+                cp16(stK + swz(r, c), kg + off, ok);
+                cp16(stV + swz(r, c), vg + off, ok);
+            }
+        }
+        cp_commit();
+    };
+    // ring and memory were written two or more kernels back
+#pragma unroll
+    for (int k = 0; k < SQ_NST; ++k) issue(k);
+    pdl_enter();
+
+    // q (rotated, scaled) and, for the window, the position's own k and v
+    const float sc = 0.125f;                         // 1 / sqrt(64)
+    if (live) {
+        const size_t rb = (size_t)b * pin.ldp + h * DH;
+        const float* cs = pin.rope.cs + (size_t)t * HALF;
+        const float* sn = pin.rope.sn + (size_t)t * HALF;
+        const int j = lane;
+        float y1, y2;
+        rope_pair(slab_sum(pin.P, pin.S, pin.slab, rb + j),
+                  slab_sum(pin.P, pin.S, pin.slab, rb + j + HALF), cs[j], sn[j], y1, y2);
+        s_q[j] = y1 * sc;
+        s_q[j + HALF] = y2 * sc;
+        if (SWA) {
+            rope_pair(slab_sum(pin.P, pin.S, pin.slab, rb + d + j),
+                      slab_sum(pin.P, pin.S, pin.slab, rb + d + j + HALF), cs[j], sn[j], y1, y2);
+            s_k[j] = __float2bfloat16_rn(y1);
+            s_k[j + HALF] = __float2bfloat16_rn(y2);
+            s_v[j] = __float2bfloat16_rn(slab_sum(pin.P, pin.S, pin.slab, rb + 2 * d + j));
+            s_v[j + HALF] = __float2bfloat16_rn(slab_sum(pin.P, pin.S, pin.slab, rb + 2 * d + j + HALF));
+        }
+    }
+    __syncwarp();
+    // scores: lane 2r+hf holds dims 32hf .. 32hf+31 of key r of the tile
+    const int kr = lane >> 1, hf = lane & 1;
+    float q[32];
+#pragma unroll
+    for (int x = 0; x < 32; x += 4) {
+        const float4 v4 = *reinterpret_cast<const float4*>(s_q + 32 * hf + x);
+        q[x] = v4.x;
+        q[x + 1] = v4.y;
+        q[x + 2] = v4.z;
+        q[x + 3] = v4.w;
+    }
+    // values: lane group g (lane / 8) takes keys 4i+g, dims 8*seg .. 8*seg+7
+    const int grp = lane >> 3, seg = lane & 7;
+    float m = -INFINITY, lpart = 0.f, acc[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+
+    for (int k = 0; k < ntile; ++k) {
+        cp_wait<SQ_NST - 1>();
+        __syncwarp();
+        const uint32_t off = (uint32_t)(2 * (k % SQ_NST)) * MQ_TB;
+        const uint8_t* tK = wsm + off;
+        const uint8_t* tV = tK + MQ_TB;
+        // score of key kr: chunks 4hf .. 4hf+3 of its row
+        float dot = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint4 w = *reinterpret_cast<const uint4*>(tK + swz(kr, 4 * hf + u));
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const float2 f = __bfloat1622float2(h2[x]);
+                dot = fmaf(q[8 * u + 2 * x], f.x, dot);
+                dot = fmaf(q[8 * u + 2 * x + 1], f.y, dot);
+            }
+        }
+        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+        const bool vis = k * MQ_TILE + kr < nrun;
+        const float s = vis ? dot : -INFINITY;
+        float tm = s;
+#pragma unroll
+        for (int o = 2; o < 32; o <<= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, o));
+        const float mn = fmaxf(m, tm);               // finite: the tile holds a key
+        const float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
+        const float p = vis ? __expf(s - mn) : 0.f;
+        lpart = lpart * corr + (hf == 0 ? p : 0.f);
+        m = mn;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc[x] *= corr;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int j = 4 * i + grp;
+            const float pj = __shfl_sync(0xffffffffu, p, 2 * j);
+            const uint4 w = *reinterpret_cast<const uint4*>(tV + swz(j, seg));
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const float2 f = __bfloat1622float2(h2[x]);
+                acc[2 * x] = fmaf(pj, f.x, acc[2 * x]);
+                acc[2 * x + 1] = fmaf(pj, f.y, acc[2 * x + 1]);
+            }
+        }
+        __syncwarp();
+        issue(k + SQ_NST);
+    }
+    cp_wait<0>();
+    if (SWA && live) {
+        // the position itself: every lane pair scores it, lane 0 counts it,
+        // group 0 carries its value
+        float dot = 0.f;
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+            const float2 f = __bfloat1622float2(
+                *reinterpret_cast<const __nv_bfloat162*>(s_k + 32 * hf + x));
+            dot = fmaf(q[x], f.x, dot);
+            dot = fmaf(q[x + 1], f.y, dot);
+        }
+        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+        const float mn = fmaxf(m, dot);
+        const float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
+        const float p = __expf(dot - mn);
+        lpart = lpart * corr + (lane == 0 ? p : 0.f);
+        m = mn;
+        float vf[8];
+        const uint4 w = *reinterpret_cast<const uint4*>(s_v + 8 * seg);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const float2 f = __bfloat1622float2(h2[x]);
+            vf[2 * x] = f.x;
+            vf[2 * x + 1] = f.y;
+        }
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc[x] = acc[x] * corr + (grp == 0 ? p * vf[x] : 0.f);
+    }
+    // the normaliser and the output: sums over the lanes and over the groups
+    float l = lpart;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+        acc[x] += __shfl_xor_sync(0xffffffffu, acc[x], 8);
+        acc[x] += __shfl_xor_sync(0xffffffffu, acc[x], 16);
+    }
+    if (live && grp == 0) {
+        const float inv = 1.0f / l;
+        uint4 w;
+        w.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+        w.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+        w.z = pack_bf16(acc[4] * inv, acc[5] * inv);
+        w.w = pack_bf16(acc[6] * inv, acc[7] * inv);
+        *reinterpret_cast<uint4*>(A + (size_t)b * d + h * DH + 8 * seg) = w;
+        if (SWA && W > 1) {
+            // every read of this head's ring is done: the position enters
+            // slot pd mod (W-1)
+            const size_t slot = (size_t)(pd % span) * DH + 8 * seg;
+            *reinterpret_cast<uint4*>(const_cast<bf16*>(kg) + slot) =
+                *reinterpret_cast<const uint4*>(s_k + 8 * seg);
+            *reinterpret_cast<uint4*>(const_cast<bf16*>(vg) + slot) =
+                *reinterpret_cast<const uint4*>(s_v + 8 * seg);
+        }
+    }
+}
+
 template <bool SWA, int NQ>
 void launch_nq(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W, bf16* A,
                int B, int heads, const ProjIn& pin, cudaStream_t st) {
@@ -347,6 +553,31 @@ int read_and_clear_mq_error() {
     }
     return v;
 }
+
+// RLT_SQ=0 keeps one-position blocks on the register-batch kernel (read once).
+static bool sq_enabled() {
+    static const bool on = [] {
+        const char* e = getenv("RLT_SQ");
+        return !(e && e[0] == '0' && e[1] == 0);
+    }();
+    return on;
+}
+
+template <bool SWA>
+bool launch_attn_sq(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W,
+                    bf16* A, int B, int heads, int dh, const ProjIn& pin, cudaStream_t st) {
+    if (!sq_enabled() || dh != 64 || pin.S > 8) return false;
+    if (B <= 0) return true;
+    if (!set_smem_once(reinterpret_cast<const void*>(k_attn_sq<SWA>), SQ_SMEM)) return false;
+    launch(k_attn_sq<SWA>, (B * heads + SQ_WARPS - 1) / SQ_WARPS, SQ_WARPS * 32, SQ_SMEM, st,
+           base, row_stride, span, pos, W, A, B, heads, pin);
+    rlt_count_launch();
+    return true;
+}
+template bool launch_attn_sq<true>(const bf16*, size_t, int, const int32_t*, int, bf16*, int, int,
+                                   int, const ProjIn&, cudaStream_t);
+template bool launch_attn_sq<false>(const bf16*, size_t, int, const int32_t*, int, bf16*, int,
+                                    int, int, const ProjIn&, cudaStream_t);
 
 // RLT_MQ=0 keeps blocks of 2..8 positions on the earlier kernels (read once).
 static bool mq_enabled() {

@@ -203,6 +203,12 @@ bool fast_attn_enabled();           // false when RLT_ATTN=warp
 // warp-level tensor-core MMA; the window form (SWA) also takes the block's
 // own keys from the slabs and writes them into the ring.  false (nothing
 // launched) for other shapes or when RLT_MQ=0.
+// One position per row at d_h = 64 (k_attn_mq.cu): one warp per (row, head)
+// streams 16-key tiles through shared memory by cp.async and scores them on
+// the CUDA cores (q and p fp32); false when RLT_SQ=0 or for other shapes.
+template <bool SWA>
+bool launch_attn_sq(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W,
+                    bf16* A, int B, int heads, int dh, const ProjIn& pin, cudaStream_t st);
 template <bool SWA>
 bool launch_attn_mq(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W,
                     bf16* A, int B, int n, int heads, int dh, const ProjIn& pin, cudaStream_t st);
