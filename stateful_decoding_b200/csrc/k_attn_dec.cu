@@ -1154,7 +1154,11 @@ bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int 
         launch_attn_mq<true>(ring, row_stride, slots, pos, W, A, B, n, heads, dh, pin, st))
         return true;
     if (n > 4) return false;
-    if (n == 1 && pin.S <= 8 && dh == 128) {
+    static const bool xswa = [] {      // RLT_XSPLIT_SWA=0: one warp per item (read once)
+        const char* e = getenv("RLT_XSPLIT_SWA");
+        return !(e && strcmp(e, "0") == 0);
+    }();
+    if (n == 1 && pin.S <= 8 && dh == 128 && xswa) {
         // the wide heads' long windows with few items per launch: split each
         // item's ring over four warps
         launch(k_attn_xsplit<128, 4, false, true>, B * heads, 4 * 32, 0, st, ring, row_stride,
@@ -1165,7 +1169,8 @@ bool launch_attn_swa_proj(const ProjIn& pin, bf16* ring, size_t row_stride, int 
     if (n == 1 && launch_attn_sq<true>(ring, row_stride, slots, pos, W, A, B, heads, dh, pin, st))
         return true;
     if (n == 1 && pin.S <= 8)
-        return launch_dec1<64, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st);
+        return dh == 64 ? launch_dec1<64, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st)
+                        : launch_dec1<128, true>(ring, row_stride, slots, pos, W, A, B, heads, pin, st);
     if (dh == 64 && pin.S <= 8 && W > 4 && multi_query_warp())
         return launch_decn64<true>(ring, row_stride, slots, pos, W, A, B, n, heads, pin, st);
     if (dh == 64)

@@ -1139,6 +1139,16 @@ static int row_groups(int B) {
     return std::max(1, std::min(g, B));
 }
 
+// RLT_GRAPH_CHAIN=0: inside a captured run, hand the state over and build the
+// next merge input with the two kernels the uncaptured blocks use (read once).
+static bool graph_chain_enabled() {
+    static const bool on = [] {
+        const char* e = getenv("RLT_GRAPH_CHAIN");
+        return !(e && strcmp(e, "0") == 0);
+    }();
+    return on;
+}
+
 static int run_graph(rlt_state* s, int n, cudaStream_t st) {
     const int span = kGraphBlocks * n;
     for (int b = 0; b < s->B; ++b) {
@@ -1184,7 +1194,7 @@ static int run_graph(rlt_state* s, int n, cudaStream_t st) {
             }
             // consecutive one-position blocks hand the state to the next
             // block's merge input in one kernel
-            const bool chain = n == 1 && s->m->cfg.variant != 0;
+            const bool chain = n == 1 && s->m->cfg.variant != 0 && graph_chain_enabled();
             for (int gi = 0; gi < G; ++gi) {
                 const int b0 = (int)((long)gi * s->B / G), b1 = (int)((long)(gi + 1) * s->B / G);
                 cudaStream_t sg = branch && gi > 0 ? s->aux[gi - 1] : st;

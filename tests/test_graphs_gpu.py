@@ -87,7 +87,9 @@ np.savez({out!r}, lg=lg, **parts)
 def test_graph_replay_matches_launch_by_launch(sd, name, B, T):
     lg_d, parts_d = run_case(sd, name, B, T, use_stream=False)
     lg_g, parts_g = run_case(sd, name, B, T, use_stream=True)
-    np.testing.assert_array_equal(lg_g, lg_d)
+    bad = [int(b) for b in np.nonzero(np.any(lg_g != lg_d, axis=1))[0]]
+    assert not bad, (f"rows {bad} differ, max |dlogit| per row "
+                     f"{np.abs(lg_g - lg_d).max(axis=1)[bad]}")
     for k in parts_d:
         np.testing.assert_array_equal(parts_g[k], parts_d[k])
 
