@@ -25,6 +25,8 @@
 // reduction order depend on positions only, never on the batch.
 #include <math.h>
 
+#include <cstring>
+
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -326,18 +328,43 @@ k_attn_mq(const bf16* __restrict__ base, size_t row_stride, int span,
 
 // ---------------------------------------------------------------- one position
 // One position per row (n = 1, the decode shape) at d_h = 64, on the CUDA
-// cores: one warp per (row, head), 16-key tiles of K and V staged by
-// cp.async (three in flight, the same swizzled rows), so the bytes in flight
-// cost no registers.  Scores: two lanes per key, 32 dims each, one shuffle;
-// an online softmax per tile (one warp maximum); values: lane group g takes
-// keys 4i+g of the tile, 8 dims per lane, and the groups' partial outputs
-// are added at the end.  q and p stay fp32.  The window form folds the
-// position's own key (formed from the slabs) after the ring's tiles and then
-// writes it into the ring.
+// cores: one warp per (row, head).  The keys of a (row, head) are one
+// contiguous run per K and V, so a 16-key tile is one 2 KB bulk copy of each
+// (lane 0 issues them, completion counted on a per-stage mbarrier, three
+// tiles in flight): the bytes in flight hold no registers and issuing a tile
+// costs two instructions.  Scores: two lanes per key, 32 dims each, read in
+// a per-key rotated chunk order (so that the 8 lanes of a shared-memory
+// phase hit 8 different banks groups without a swizzle), packed fp32x2
+// FMAs, one shuffle; an online softmax per tile (one warp maximum); values:
+// lane group g takes keys 4i+g, 8 dims per lane, packed FMAs, the groups'
+// partial outputs added at the end.  q and p stay fp32.  The window form
+// folds the position's own key (formed from the slabs) after the ring's
+// tiles and then writes it into the ring.  Waits are bounded: a wait that
+// gives up records a timeout, the warp stops, and it waits (bounded) for the
+// copies it has in flight before it exits.
 constexpr int SQ_WARPS = 4;
 constexpr int SQ_NST = 3;
 constexpr int SQ_WARP_SMEM = SQ_NST * 2 * MQ_TB + 512;   // tiles, q (fp32), own k and v
 constexpr int SQ_SMEM = SQ_WARPS * SQ_WARP_SMEM;
+
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+        : "memory");
+}
+// d = a * b + c on a pair of fp32 values (one packed instruction)
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    unsigned long long ua, ub, uc, ud;
+    memcpy(&ua, &a, 8);
+    memcpy(&ub, &b, 8);
+    memcpy(&uc, &c, 8);
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(ud) : "l"(ua), "l"(ub), "l"(uc));
+    float2 d;
+    memcpy(&d, &ud, 8);
+    return d;
+}
 
 template <bool SWA>
 __global__ void __launch_bounds__(SQ_WARPS * 32)
@@ -346,6 +373,7 @@ k_attn_sq(const bf16* __restrict__ base, size_t row_stride, int span,
           ProjIn pin) {
     constexpr int DH = 64, HALF = 32;
     extern __shared__ __align__(1024) uint8_t sq_smem[];
+    __shared__ uint64_t bars[SQ_WARPS][SQ_NST];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int it = blockIdx.x * SQ_WARPS + warp;
     const bool in_range = it < B * heads;
@@ -364,20 +392,23 @@ k_attn_sq(const bf16* __restrict__ base, size_t row_stride, int span,
     float* s_q = reinterpret_cast<float*>(wsm + SQ_NST * 2 * MQ_TB);    // 64 floats
     bf16* s_k = reinterpret_cast<bf16*>(s_q + DH);                      // own k, v
     bf16* s_v = s_k + DH;
+    uint64_t* bar = bars[warp];
+    if (lane == 0) {
+        for (int s = 0; s < SQ_NST; ++s) tc::mbar_init(&bar[s], 1);
+        tc::fence_mbar_init();
+    }
+    __syncwarp();
 
+    // tile k of the run (its first min(16, nrun - 16k) keys) into stage k % NST
     auto issue = [&](int k) {
-        if (k < ntile) {
-            const uint32_t stK = sKV + (uint32_t)(2 * (k % SQ_NST)) * MQ_TB, stV = stK + MQ_TB;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int ch = lane + 32 * u, r = ch >> 3, c = ch & 7, j = k * MQ_TILE + r;
-                const bool ok = j < nrun;
-                const size_t off = (size_t)(ok ? j : 0) * DH + c * 8;
-                cp16(stK + swz(r, c), kg + off, ok);
-                cp16(stV + swz(r, c), vg + off, ok);
-            }
+        if (lane == 0 && k < ntile) {
+            const int s = k % SQ_NST, nv = min(MQ_TILE, nrun - k * MQ_TILE);
+            const uint32_t bytes = (uint32_t)nv * DH * 2;
+            tc::mbar_expect_tx(&bar[s], 2 * bytes);
+            const uint32_t stK = sKV + (uint32_t)(2 * s) * MQ_TB;
+            bulk_copy(stK, kg + (size_t)k * MQ_TILE * DH, bytes, &bar[s]);
+            bulk_copy(stK + MQ_TB, vg + (size_t)k * MQ_TILE * DH, bytes, &bar[s]);
         }
-        cp_commit();
     };
     // ring and memory were written two or more kernels back
 #pragma unroll
@@ -406,117 +437,127 @@ k_attn_sq(const bf16* __restrict__ base, size_t row_stride, int span,
         }
     }
     __syncwarp();
-    // scores: lane 2r+hf holds dims 32hf .. 32hf+31 of key r of the tile
+    // scores: lane 2r+hf takes dims 32hf .. 32hf+31 of key r of a tile, in
+    // the chunk order 4hf + (u + r) mod 4, u = 0..3; its q in that order
     const int kr = lane >> 1, hf = lane & 1;
-    float q[32];
+    float2 q2[16];
 #pragma unroll
-    for (int x = 0; x < 32; x += 4) {
-        const float4 v4 = *reinterpret_cast<const float4*>(s_q + 32 * hf + x);
-        q[x] = v4.x;
-        q[x + 1] = v4.y;
-        q[x + 2] = v4.z;
-        q[x + 3] = v4.w;
+    for (int u = 0; u < 4; ++u) {
+        const float* src = s_q + 32 * hf + 8 * ((u + kr) & 3);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) q2[4 * u + x] = make_float2(src[2 * x], src[2 * x + 1]);
     }
     // values: lane group g (lane / 8) takes keys 4i+g, dims 8*seg .. 8*seg+7
     const int grp = lane >> 3, seg = lane & 7;
-    float m = -INFINITY, lpart = 0.f, acc[8];
+    float m = -INFINITY, lpart = 0.f;
+    float2 acc[4];
 #pragma unroll
-    for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+    for (int x = 0; x < 4; ++x) acc[x] = make_float2(0.f, 0.f);
+    int kfail = -1;                                  // tile whose copy never completed
 
     for (int k = 0; k < ntile; ++k) {
-        cp_wait<SQ_NST - 1>();
-        __syncwarp();
-        const uint32_t off = (uint32_t)(2 * (k % SQ_NST)) * MQ_TB;
-        const uint8_t* tK = wsm + off;
+        const int s = k % SQ_NST;
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&bar[s], (uint32_t)(k / SQ_NST) & 1u))) {
+            kfail = k;
+            break;
+        }
+        const int nv = min(MQ_TILE, nrun - k * MQ_TILE);
+        const uint8_t* tK = wsm + 2 * s * MQ_TB;
         const uint8_t* tV = tK + MQ_TB;
-        // score of key kr: chunks 4hf .. 4hf+3 of its row
-        float dot = 0.f;
+        float2 dd = make_float2(0.f, 0.f);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const uint4 w = *reinterpret_cast<const uint4*>(tK + swz(kr, 4 * hf + u));
+            const uint4 w = *reinterpret_cast<const uint4*>(tK + kr * 128 +
+                                                            (4 * hf + ((u + kr) & 3)) * 16);
             const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const float2 f = __bfloat1622float2(h2[x]);
-                dot = fmaf(q[8 * u + 2 * x], f.x, dot);
-                dot = fmaf(q[8 * u + 2 * x + 1], f.y, dot);
-            }
+            for (int x = 0; x < 4; ++x) dd = fma2(q2[4 * u + x], __bfloat1622float2(h2[x]), dd);
         }
+        float dot = dd.x + dd.y;
         dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-        const bool vis = k * MQ_TILE + kr < nrun;
-        const float s = vis ? dot : -INFINITY;
-        float tm = s;
+        const bool vis = kr < nv;
+        const float sv = vis ? dot : -INFINITY;
+        float tm = sv;
 #pragma unroll
         for (int o = 2; o < 32; o <<= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, o));
         const float mn = fmaxf(m, tm);               // finite: the tile holds a key
         const float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
-        const float p = vis ? __expf(s - mn) : 0.f;
+        const float p = vis ? __expf(sv - mn) : 0.f;
         lpart = lpart * corr + (hf == 0 ? p : 0.f);
         m = mn;
+        const float2 c2 = make_float2(corr, corr);
 #pragma unroll
-        for (int x = 0; x < 8; ++x) acc[x] *= corr;
+        for (int x = 0; x < 4; ++x) acc[x] = make_float2(acc[x].x * c2.x, acc[x].y * c2.y);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int j = 4 * i + grp;
             const float pj = __shfl_sync(0xffffffffu, p, 2 * j);
-            const uint4 w = *reinterpret_cast<const uint4*>(tV + swz(j, seg));
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+            if (j < nv) {                            // rows past the copy hold stale bytes
+                const uint4 w = *reinterpret_cast<const uint4*>(tV + j * 128 + seg * 16);
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+                const float2 p2 = make_float2(pj, pj);
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const float2 f = __bfloat1622float2(h2[x]);
-                acc[2 * x] = fmaf(pj, f.x, acc[2 * x]);
-                acc[2 * x + 1] = fmaf(pj, f.y, acc[2 * x + 1]);
+                for (int x = 0; x < 4; ++x) acc[x] = fma2(p2, __bfloat1622float2(h2[x]), acc[x]);
             }
         }
-        __syncwarp();
+        __syncwarp();                                // the stage is read: refill it
         issue(k + SQ_NST);
     }
-    cp_wait<0>();
+    if (kfail >= 0) {
+        // a copy never completed: record it, then wait (bounded) for the
+        // copies still in flight -- tiles kfail .. kfail+NST-1 were issued --
+        // so that none lands after the warp is gone
+        if (lane == 0) {
+            atomicExch(&g_mq_error, kDevTimeout);
+            for (int k = kfail; k < min(ntile, kfail + SQ_NST); ++k)
+                tc::mbar_wait(&bar[k % SQ_NST], (uint32_t)(k / SQ_NST) & 1u, 1u << 20);
+        }
+        return;
+    }
     if (SWA && live) {
         // the position itself: every lane pair scores it, lane 0 counts it,
         // group 0 carries its value
-        float dot = 0.f;
+        float2 dd = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-            const float2 f = __bfloat1622float2(
-                *reinterpret_cast<const __nv_bfloat162*>(s_k + 32 * hf + x));
-            dot = fmaf(q[x], f.x, dot);
-            dot = fmaf(q[x + 1], f.y, dot);
+        for (int x = 0; x < 16; ++x) {
+            const float2 kf = __bfloat1622float2(
+                *reinterpret_cast<const __nv_bfloat162*>(s_k + 32 * hf + 2 * x));
+            dd = fma2(make_float2(s_q[32 * hf + 2 * x], s_q[32 * hf + 2 * x + 1]), kf, dd);
         }
+        float dot = dd.x + dd.y;
         dot += __shfl_xor_sync(0xffffffffu, dot, 1);
         const float mn = fmaxf(m, dot);
         const float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
         const float p = __expf(dot - mn);
         lpart = lpart * corr + (lane == 0 ? p : 0.f);
         m = mn;
-        float vf[8];
         const uint4 w = *reinterpret_cast<const uint4*>(s_v + 8 * seg);
         const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-            const float2 f = __bfloat1622float2(h2[x]);
-            vf[2 * x] = f.x;
-            vf[2 * x + 1] = f.y;
+            const float2 vf = __bfloat1622float2(h2[x]);
+            acc[x].x = acc[x].x * corr + (grp == 0 ? p * vf.x : 0.f);
+            acc[x].y = acc[x].y * corr + (grp == 0 ? p * vf.y : 0.f);
         }
-#pragma unroll
-        for (int x = 0; x < 8; ++x) acc[x] = acc[x] * corr + (grp == 0 ? p * vf[x] : 0.f);
     }
     // the normaliser and the output: sums over the lanes and over the groups
     float l = lpart;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
 #pragma unroll
-    for (int x = 0; x < 8; ++x) {
-        acc[x] += __shfl_xor_sync(0xffffffffu, acc[x], 8);
-        acc[x] += __shfl_xor_sync(0xffffffffu, acc[x], 16);
+    for (int x = 0; x < 4; ++x) {
+        acc[x].x += __shfl_xor_sync(0xffffffffu, acc[x].x, 8);
+        acc[x].y += __shfl_xor_sync(0xffffffffu, acc[x].y, 8);
+        acc[x].x += __shfl_xor_sync(0xffffffffu, acc[x].x, 16);
+        acc[x].y += __shfl_xor_sync(0xffffffffu, acc[x].y, 16);
     }
     if (live && grp == 0) {
         const float inv = 1.0f / l;
         uint4 w;
-        w.x = pack_bf16(acc[0] * inv, acc[1] * inv);
-        w.y = pack_bf16(acc[2] * inv, acc[3] * inv);
-        w.z = pack_bf16(acc[4] * inv, acc[5] * inv);
-        w.w = pack_bf16(acc[6] * inv, acc[7] * inv);
+        w.x = pack_bf16(acc[0].x * inv, acc[0].y * inv);
+        w.y = pack_bf16(acc[1].x * inv, acc[1].y * inv);
+        w.z = pack_bf16(acc[2].x * inv, acc[2].y * inv);
+        w.w = pack_bf16(acc[3].x * inv, acc[3].y * inv);
         *reinterpret_cast<uint4*>(A + (size_t)b * d + h * DH + 8 * seg) = w;
         if (SWA && W > 1) {
             // every read of this head's ring is done: the position enters
