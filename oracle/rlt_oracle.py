@@ -83,7 +83,7 @@ ENC_TC_MIN_POSITIONS = 16
 # decoder blocks of this many positions (head size 64, bf16) multiply q and
 # the probabilities as bf16 values (the multi-query tile products)
 DEC_MQ_MIN_POSITIONS = 2
-DEC_MQ_MAX_POSITIONS = 8
+DEC_MQ_MAX_POSITIONS = 16
 
 # ----------------------------------------------------------------------------
 # Scalar helpers (float64)

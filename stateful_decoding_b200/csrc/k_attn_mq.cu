@@ -1,5 +1,5 @@
-// Decoder attention for blocks of NQ = 2..8 positions per row (RLT-2 chunks,
-// short RLT-0 blocks) at d_h = 64: the window self-attention over the ring
+// Decoder attention for blocks of NQ = 2..16 positions per row (RLT-2 chunks,
+// RLT-0 blocks) at d_h = 64: the window self-attention over the ring
 // cache C^D plus the block's own positions, and the cross-attention over the
 // memory prefix M_{<=t} (jiphyeonjeon review "Recurrent Looped Transformer"
 // §2-§3.3; greeksharifa §2.5, §2.7 and App. I.2 for the blocks).
@@ -8,7 +8,8 @@
 // scores of a 16-key tile are the product Q (NQ x 64) . K^T and the output a
 // product P . V: one warp per (row, head) runs both on the warp-level tensor
 // core MMA (m16n8k16, bf16 operands, fp32 accumulation; the NQ queries fill
-// rows 0..NQ-1 of the 16-row operand).  The work stays an HBM stream -- each
+// rows 0..NQ-1 of the 16-row operand, each lane carrying the softmax of rows
+// lane/4 and, past 8 queries, lane/4 + 8).  The work stays an HBM stream -- each
 // key and value is read once -- and the products only cut the per-key
 // instruction count that bounds the CUDA-core form of the same loop.
 //
@@ -199,12 +200,21 @@ k_attn_mq(const bf16* __restrict__ base, size_t row_stride, int span,
     for (int ks = 0; ks < 4; ++ks)
         ldsm4(sQ + swz(r8 + ((mi & 1) << 3), 2 * ks + (mi >> 1)), qa[ks]);
 
-    // this lane's accumulator row (query) and columns
+    // this lane's accumulator rows (queries qi and, for blocks of more than
+    // 8 positions, qi + 8) and columns
+    constexpr int NR = NQ > 8 ? 2 : 1;
     const int qi = lane >> 2, c2 = (lane & 3) * 2;
-    const bool qrow = live && qi < NQ;
-    const int t_i = pd + 1 + qi;
-    const int lo = SWA ? max(1, t_i - W + 1) : 1;    // first visible position
-    float m = -INFINITY, lpart = 0.f;
+    bool qrow[NR];
+    int t_i[NR], lo[NR];
+    float m[NR], lpart[NR];
+#pragma unroll
+    for (int hh = 0; hh < NR; ++hh) {
+        qrow[hh] = live && qi + 8 * hh < NQ;
+        t_i[hh] = pd + 1 + qi + 8 * hh;
+        lo[hh] = SWA ? max(1, t_i[hh] - W + 1) : 1;    // first visible position
+        m[hh] = -INFINITY;
+        lpart[hh] = 0.f;
+    }
     float o[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
@@ -226,56 +236,74 @@ k_attn_mq(const bf16* __restrict__ base, size_t row_stride, int span,
             mma16816(s[0], qa[ks], kb[0], kb[1]);
             mma16816(s[1], qa[ks], kb[2], kb[3]);
         }
-        // visibility of this lane's four keys for query qi
-        float v[4];
-        bool vis[4];
+        // row hh of this lane: scores s[j][2hh], s[j][2hh+1] for keys 8j+c2, 8j+c2+1
+        float p[NR][4], corr[NR];
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int hh = 0; hh < NR; ++hh) {
+            const int qrw = qi + 8 * hh;
+            float v[4];
+            bool vis[4];
 #pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                const int kt = 8 * j + c2 + x;           // key within the tile
-                bool ok = qrow;
-                if (kidx0 < 0) {                         // own position e = kt
-                    ok = ok && kt < NQ && kt <= qi && pd + 1 + kt >= lo;
-                } else {
-                    const int kk = kidx0 + kt;
-                    if (SWA) {
-                        const int p = pd - ((pd - 1 - kk) % span);
-                        ok = ok && kk < nmain && p >= lo;
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    const int kt = 8 * j + c2 + x;       // key within the tile
+                    bool ok = qrow[hh];
+                    if (kidx0 < 0) {                     // own position e = kt
+                        ok = ok && kt < NQ && kt <= qrw && pd + 1 + kt >= lo[hh];
                     } else {
-                        ok = ok && kk < nmain && kk + 1 <= t_i;
+                        const int kk = kidx0 + kt;
+                        if (SWA) {
+                            const int ps = pd - ((pd - 1 - kk) % span);
+                            ok = ok && kk < nmain && ps >= lo[hh];
+                        } else {
+                            ok = ok && kk < nmain && kk + 1 <= t_i[hh];
+                        }
                     }
+                    vis[2 * j + x] = ok;
+                    v[2 * j + x] = s[j][2 * hh + x] * sc;
                 }
-                vis[2 * j + x] = ok;
-                v[2 * j + x] = s[j][x] * sc;
+            float tm = -INFINITY;
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+                if (vis[x]) tm = fmaxf(tm, v[x]);
+            tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 1));
+            tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 2));
+            const float mn = fmaxf(m[hh], tm);
+            corr[hh] = 1.f;
+#pragma unroll
+            for (int x = 0; x < 4; ++x) p[hh][x] = 0.f;
+            if (mn != -INFINITY) {
+                corr[hh] = (m[hh] == -INFINITY) ? 0.f : __expf(m[hh] - mn);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) p[hh][x] = vis[x] ? __expf(v[x] - mn) : 0.f;
+                m[hh] = mn;
             }
-        float tm = -INFINITY;
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-            if (vis[x]) tm = fmaxf(tm, v[x]);
-        tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 1));
-        tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 2));
-        const float mn = fmaxf(m, tm);
-        float corr = 1.f;
-        float p[4] = {0.f, 0.f, 0.f, 0.f};
-        if (mn != -INFINITY) {
-            corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) p[x] = vis[x] ? __expf(v[x] - mn) : 0.f;
-            m = mn;
         }
+        // P as the A operand: rows qi (and qi + 8), keys c2.. and 8+c2..
         uint32_t pa[4];
-        pa[0] = pack_bf16(p[0], p[1]);
-        pa[1] = 0u;
-        pa[2] = pack_bf16(p[2], p[3]);
-        pa[3] = 0u;
-        const float2 r01 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pa[0]));
-        const float2 r23 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pa[2]));
-        lpart = lpart * corr + ((r01.x + r01.y) + (r23.x + r23.y));
+        pa[0] = pack_bf16(p[0][0], p[0][1]);
+        pa[2] = pack_bf16(p[0][2], p[0][3]);
+        if constexpr (NR == 2) {
+            pa[1] = pack_bf16(p[NR - 1][0], p[NR - 1][1]);
+            pa[3] = pack_bf16(p[NR - 1][2], p[NR - 1][3]);
+        } else {
+            pa[1] = 0u;
+            pa[3] = 0u;
+        }
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            o[nt][0] *= corr;
-            o[nt][1] *= corr;
+        for (int hh = 0; hh < NR; ++hh) {
+            // the normaliser sums the rounded probabilities
+            const float2 r01 =
+                __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pa[hh]));
+            const float2 r23 =
+                __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pa[2 + hh]));
+            lpart[hh] = lpart[hh] * corr[hh] + ((r01.x + r01.y) + (r23.x + r23.y));
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                o[nt][2 * hh] *= corr[hh];
+                o[nt][2 * hh + 1] *= corr[hh];
+            }
         }
 #pragma unroll
         for (int np = 0; np < 4; ++np) {
@@ -299,15 +327,19 @@ k_attn_mq(const bf16* __restrict__ base, size_t row_stride, int span,
     if (SWA) fold_tile(sOwnK, sOwnV, -1);
 
     // normaliser: the four lanes of the row hold parts of the sum
-    float l = lpart;
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    if (qrow) {
-        const float inv = 1.0f / l;
-        bf16* arow = A + (size_t)(b * NQ + qi) * d + h * DH + c2;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-            *reinterpret_cast<uint32_t*>(arow + nt * 8) = pack_bf16(o[nt][0] * inv, o[nt][1] * inv);
+    for (int hh = 0; hh < NR; ++hh) {
+        float l = lpart[hh];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        if (qrow[hh]) {
+            const float inv = 1.0f / l;
+            bf16* arow = A + (size_t)(b * NQ + qi + 8 * hh) * d + h * DH + c2;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+                *reinterpret_cast<uint32_t*>(arow + nt * 8) =
+                    pack_bf16(o[nt][2 * hh] * inv, o[nt][2 * hh + 1] * inv);
+        }
     }
     if (SWA && live && W > 1) {
         // every read of this head's ring is done: the block's positions enter
@@ -620,7 +652,7 @@ template bool launch_attn_sq<true>(const bf16*, size_t, int, const int32_t*, int
 template bool launch_attn_sq<false>(const bf16*, size_t, int, const int32_t*, int, bf16*, int,
                                     int, int, const ProjIn&, cudaStream_t);
 
-// RLT_MQ=0 keeps blocks of 2..8 positions on the earlier kernels (read once).
+// RLT_MQ=0 keeps blocks of 2..16 positions on the earlier kernels (read once).
 static bool mq_enabled() {
     static const bool on = [] {
         const char* e = getenv("RLT_MQ");
@@ -632,7 +664,7 @@ static bool mq_enabled() {
 template <bool SWA>
 bool launch_attn_mq(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W,
                     bf16* A, int B, int n, int heads, int dh, const ProjIn& pin, cudaStream_t st) {
-    if (!mq_enabled() || dh != 64 || n < 2 || n > 8 || pin.S > 8) return false;
+    if (!mq_enabled() || dh != 64 || n < 2 || n > 16 || pin.S > 8) return false;
     if (B * n <= 0) return true;
     bool ok = false;
     switch (n) {
@@ -648,6 +680,14 @@ bool launch_attn_mq(const bf16* base, size_t row_stride, int span, const int32_t
         RLT_MQ_CASE(6)
         RLT_MQ_CASE(7)
         RLT_MQ_CASE(8)
+        RLT_MQ_CASE(9)
+        RLT_MQ_CASE(10)
+        RLT_MQ_CASE(11)
+        RLT_MQ_CASE(12)
+        RLT_MQ_CASE(13)
+        RLT_MQ_CASE(14)
+        RLT_MQ_CASE(15)
+        RLT_MQ_CASE(16)
 #undef RLT_MQ_CASE
     }
     if (ok) rlt_count_launch();

@@ -198,7 +198,7 @@ bool launch_attn_cross_proj(const ProjIn& pin, const bf16* mem, size_t row_strid
                             const int32_t* pos_dec, bf16* A, int B, int n, int heads, int dh,
                             cudaStream_t st);
 bool fast_attn_enabled();           // false when RLT_ATTN=warp
-// Blocks of 2..8 positions per row at d_h = 64 (k_attn_mq.cu): one warp per
+// Blocks of 2..16 positions per row at d_h = 64 (k_attn_mq.cu): one warp per
 // (row, head) scores the block's queries against 16-key tiles with the
 // warp-level tensor-core MMA; the window form (SWA) also takes the block's
 // own keys from the slabs and writes them into the ring.  false (nothing

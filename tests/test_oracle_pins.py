@@ -802,7 +802,7 @@ def test_bf16_mode_rounds_every_cache_and_product_input():
 
 
 def test_decoder_blocks_round_attention_inputs_like_the_tile_products():
-    """bf16 mode, head size 64: a decoder block of 2..8 positions (an RLT-2
+    """bf16 mode, head size 64: a decoder block of 2..16 positions (an RLT-2
     chunk) passes rounded q and probabilities to both attentions (the window
     only when W exceeds the block); a one-position transition does not; the
     fp64 mode never does."""

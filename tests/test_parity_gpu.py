@@ -147,11 +147,12 @@ def test_prefill_matches_oracle(sd, name, B, T):
             np.testing.assert_allclose(R_gpu, r.R, atol=max(10 * tol, 1e-3), rtol=0)
 
 
-@pytest.mark.parametrize("chunk", [2, 3, 8])
+@pytest.mark.parametrize("chunk", [2, 3, 8, 16])
 def test_rlt2_chunk_blocks_match_oracle(sd, chunk):
     """RLT-2 at other chunk sizes B_c (greeksharifa App. J.10): rlt_prefill
     runs each chunk as one block of B_c positions -- the multi-query tile
-    products at d_h 64 -- against the oracle's chunked run of the same
+    products at d_h 64, one or two query rows per lane -- against the
+    oracle's chunked run of the same
     blocks; logits, argmax and the held register R."""
     cfg = ri.CONFIGS["rlt2_mod5_bf16"].replace(name=f"rlt2_chunk{chunk}", chunk=chunk)
     B, T = 3, 40
