@@ -179,6 +179,7 @@ int read_and_clear_device_error();  // device error word of the bounded-wait ker
 int read_and_clear_attn_error();
 int read_and_clear_persist_error();  // same, for the persistent GEMM
 int read_and_clear_mq_error();       // same, for the multi-query block attention
+int read_and_clear_sq_error();       // same, for the one-position attention
 // Partial-sum slabs of a projection, consumed directly by an attention kernel.
 struct ProjIn {
     const float* P;   // slab 0 of the fp32 partial sums, [R][ldp]
@@ -203,8 +204,8 @@ bool fast_attn_enabled();           // false when RLT_ATTN=warp
 // warp-level tensor-core MMA; the window form (SWA) also takes the block's
 // own keys from the slabs and writes them into the ring.  false (nothing
 // launched) for other shapes or when RLT_MQ=0.
-// One position per row at d_h = 64 (k_attn_mq.cu): one warp per (row, head)
-// streams 16-key tiles through shared memory by cp.async and scores them on
+// One position per row at d_h = 64 (k_attn_sq.cu): one warp per (row, head)
+// streams 16-key tiles through shared memory by bulk copy and scores them on
 // the CUDA cores (q and p fp32); false when RLT_SQ=0 or for other shapes.
 template <bool SWA>
 bool launch_attn_sq(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W,

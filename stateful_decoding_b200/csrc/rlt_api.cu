@@ -1819,8 +1819,9 @@ extern "C" int rlt_state_check(rlt_state* s, void* stream) {
     const int ga = rlt::read_and_clear_attn_error();
     const int gp = rlt::read_and_clear_persist_error();
     const int gm = rlt::read_and_clear_mq_error();
-    if (g < 0 || ga < 0 || gp < 0 || gm < 0) return RLT_E_DEVICE;
-    if (w == 0) w = g ? g : (ga ? ga : (gp ? gp : gm));
+    const int gs = rlt::read_and_clear_sq_error();
+    if (g < 0 || ga < 0 || gp < 0 || gm < 0 || gs < 0) return RLT_E_DEVICE;
+    if (w == 0) w = g ? g : (ga ? ga : (gp ? gp : (gm ? gm : gs)));
     if (w == rlt::kDevTimeout) return RLT_E_TIMEOUT;
     if (w == rlt::kDevBounds) return RLT_E_ARG;
     if (w == rlt::kDevOrder) return RLT_E_ORDER;
