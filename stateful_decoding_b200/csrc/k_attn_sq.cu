@@ -54,9 +54,10 @@ __device__ __forceinline__ float slab_sum(const float* __restrict__ P, int S, si
 // gives up records a timeout, the warp stops, and it waits (bounded) for the
 // copies it has in flight before it exits.
 constexpr int SQ_WARPS = 4;
-constexpr int SQ_NST = 3;
-constexpr int SQ_WARP_SMEM = SQ_NST * 2 * SQ_TB + 512;   // tiles, q (fp32), own k and v
-constexpr int SQ_SMEM = SQ_WARPS * SQ_WARP_SMEM;
+// NST tiles in flight per warp; per warp NST (K, V) tile pairs, q (fp32)
+// and the own k and v
+constexpr int sq_warp_smem(int nst) { return nst * 2 * SQ_TB + 512; }
+constexpr int sq_smem(int nst) { return SQ_WARPS * sq_warp_smem(nst); }
 
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes,
                                           uint64_t* bar) {
@@ -77,13 +78,13 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
     return d;
 }
 
-template <bool SWA>
+template <bool SWA, int SQ_NST>
 __global__ void __launch_bounds__(SQ_WARPS * 32)
 k_attn_sq(const bf16* __restrict__ base, size_t row_stride, int span,
           const int32_t* __restrict__ pos, int W, bf16* __restrict__ A, int B, int heads,
           ProjIn pin) {
     constexpr int DH = 64, HALF = 32;
-    extern __shared__ __align__(1024) uint8_t sq_smem[];
+    extern __shared__ __align__(1024) uint8_t sq_smem_raw[];
     __shared__ uint64_t bars[SQ_WARPS][SQ_NST];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int it = blockIdx.x * SQ_WARPS + warp;
@@ -98,7 +99,7 @@ k_attn_sq(const bf16* __restrict__ base, size_t row_stride, int span,
     const int ntile = (nrun + SQ_TILE - 1) / SQ_TILE;
     const bf16* kg = base + (size_t)b * row_stride + (size_t)h * span * DH;
     const bf16* vg = kg + (size_t)heads * span * DH;
-    uint8_t* wsm = sq_smem + warp * SQ_WARP_SMEM;
+    uint8_t* wsm = sq_smem_raw + warp * sq_warp_smem(SQ_NST);
     const uint32_t sKV = tc::smem_u32(wsm);
     float* s_q = reinterpret_cast<float*>(wsm + SQ_NST * 2 * SQ_TB);    // 64 floats
     bf16* s_k = reinterpret_cast<bf16*>(s_q + DH);                      // own k, v
@@ -303,16 +304,37 @@ static bool sq_enabled() {
     return on;
 }
 
+// RLT_SQ_STAGES=2|4: key tiles in flight per warp (default 3; read once)
+static int sq_stages() {
+    static const int v = [] {
+        const char* e = getenv("RLT_SQ_STAGES");
+        const int n = e ? atoi(e) : 3;
+        return (n == 2 || n == 4) ? n : 3;
+    }();
+    return v;
+}
+
+template <bool SWA, int NST>
+bool launch_sq_nst(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W,
+                   bf16* A, int B, int heads, const ProjIn& pin, cudaStream_t st) {
+    if (!set_smem_once(reinterpret_cast<const void*>(k_attn_sq<SWA, NST>), sq_smem(NST)))
+        return false;
+    launch(k_attn_sq<SWA, NST>, (B * heads + SQ_WARPS - 1) / SQ_WARPS, SQ_WARPS * 32,
+           sq_smem(NST), st, base, row_stride, span, pos, W, A, B, heads, pin);
+    rlt_count_launch();
+    return true;
+}
+
 template <bool SWA>
 bool launch_attn_sq(const bf16* base, size_t row_stride, int span, const int32_t* pos, int W,
                     bf16* A, int B, int heads, int dh, const ProjIn& pin, cudaStream_t st) {
     if (!sq_enabled() || dh != 64 || pin.S > 8) return false;
     if (B <= 0) return true;
-    if (!set_smem_once(reinterpret_cast<const void*>(k_attn_sq<SWA>), SQ_SMEM)) return false;
-    launch(k_attn_sq<SWA>, (B * heads + SQ_WARPS - 1) / SQ_WARPS, SQ_WARPS * 32, SQ_SMEM, st,
-           base, row_stride, span, pos, W, A, B, heads, pin);
-    rlt_count_launch();
-    return true;
+    switch (sq_stages()) {
+        case 2: return launch_sq_nst<SWA, 2>(base, row_stride, span, pos, W, A, B, heads, pin, st);
+        case 4: return launch_sq_nst<SWA, 4>(base, row_stride, span, pos, W, A, B, heads, pin, st);
+        default: return launch_sq_nst<SWA, 3>(base, row_stride, span, pos, W, A, B, heads, pin, st);
+    }
 }
 template bool launch_attn_sq<true>(const bf16*, size_t, int, const int32_t*, int, bf16*, int, int,
                                    int, const ProjIn&, cudaStream_t);
