@@ -304,14 +304,18 @@ static bool sq_enabled() {
     return on;
 }
 
-// RLT_SQ_STAGES=2|4: key tiles in flight per warp (default 3; read once)
-static int sq_stages() {
+// Key tiles in flight per warp: two for the window (at most four tiles of
+// ring, the first two requested before the previous kernel ends), three for
+// the memory prefix (measured best on the parity and S5 workloads; four
+// leave fewer warps resident than one wave needs).  RLT_SQ_STAGES=2|3|4
+// sets both (read once).
+static int sq_stages(bool swa) {
     static const int v = [] {
         const char* e = getenv("RLT_SQ_STAGES");
-        const int n = e ? atoi(e) : 3;
-        return (n == 2 || n == 4) ? n : 3;
+        const int n = e ? atoi(e) : 0;
+        return (n >= 2 && n <= 4) ? n : 0;
     }();
-    return v;
+    return v ? v : (swa ? 2 : 3);
 }
 
 template <bool SWA, int NST>
@@ -330,7 +334,7 @@ bool launch_attn_sq(const bf16* base, size_t row_stride, int span, const int32_t
                     bf16* A, int B, int heads, int dh, const ProjIn& pin, cudaStream_t st) {
     if (!sq_enabled() || dh != 64 || pin.S > 8) return false;
     if (B <= 0) return true;
-    switch (sq_stages()) {
+    switch (sq_stages(SWA)) {
         case 2: return launch_sq_nst<SWA, 2>(base, row_stride, span, pos, W, A, B, heads, pin, st);
         case 4: return launch_sq_nst<SWA, 4>(base, row_stride, span, pos, W, A, B, heads, pin, st);
         default: return launch_sq_nst<SWA, 3>(base, row_stride, span, pos, W, A, B, heads, pin, st);
