@@ -1127,15 +1127,20 @@ static bool graphs_enabled(cudaStream_t st) {
 // RLT_ROW_GROUPS=g: a captured run splits the rows into g contiguous groups
 // whose chains of kernels run as concurrent branches of the graph (rows never
 // interact; every kernel's result for a row is the same in any group).
-// Read once.  Default: two groups from 512 rows on (each branch then has the
-// shape of a 256-row batch, whose chain leaves the machine idle between
-// dependent kernels), one below.
-static int row_groups(int B) {
+// Read once.  Default, by the product rows R = B*n of a block: one group
+// below 512, R/128 groups (at most 4) up to 1024 -- chains of 128-row
+// products overlap each other's dependent-launch gaps -- and two beyond,
+// where each product already fills the machine (measured: S5, 512 rows,
+// 1.60M -> 1.72M tokens/s with four groups; the RLT-2 chunk workload, 4096
+// product rows, best with two; the parity workload's 256 rows stay one
+// chain).
+static int row_groups(int B, int n) {
     static const int v = [] {
         const char* e = getenv("RLT_ROW_GROUPS");
         return e ? std::max(1, std::min(atoi(e), 8)) : 0;
     }();
-    const int g = v ? v : (B >= 512 ? 2 : 1);
+    const long R = (long)B * n;
+    const int g = v ? v : (R < 512 ? 1 : R <= 1024 ? (int)std::min<long>(4, R / 128) : 2);
     return std::max(1, std::min(g, B));
 }
 
@@ -1174,7 +1179,7 @@ static int run_graph(rlt_state* s, int n, cudaStream_t st) {
         // row groups: branches forked from and joined back into st (the
         // profiling twin issues them one after another on st, so that each
         // timed launch runs alone)
-        int G = row_groups(s->B);
+        int G = row_groups(s->B, n);
         while ((int)s->aux.size() < G - 1) {
             cudaStream_t a = nullptr;
             if (cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking) != cudaSuccess) {
